@@ -1,0 +1,126 @@
+"""CPU fp64 oracle for paged-KV attention (TEST INFRASTRUCTURE ONLY).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it, and the
+two share no code: the C source here (``pkv_oracle.c``) is compiled with gcc
+into ``liboracle.so`` and loaded with ctypes.
+
+The arithmetic and the passages it follows are documented at the top of
+``pkv_oracle.c``.  This module only marshals torch CPU tensors into the C
+calls.  Parity of every function here is pinned by ``tests/test_oracle_pins.py``
+(closed forms, invariants, and a library routine on special cases).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pkv_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile pkv_oracle.c into liboracle.so with gcc (fp64, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+               "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        p = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        i32 = ctypes.c_int
+        lib.oracle_paged_attn.argtypes = [p, p, p, p, p, p, i64, p, i64, p,
+                                          i32, i32, i32, i32, i32, i32,
+                                          ctypes.c_double, i32,
+                                          i32, i32, i32, i32, p, p]
+        lib.oracle_paged_attn.restype = i32
+        lib.oracle_kv_append.argtypes = [p, p, p, p, p, p, p, p, i64, p, i64,
+                                         i32, p, i32, i32, i32, i32, i32]
+        lib.oracle_kv_append.restype = i32
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = i32
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def _strides3(t: torch.Tensor, dims=(0, 1, 2)) -> ctypes.Array:
+    return (ctypes.c_int64 * 3)(*[int(t.stride(d)) for d in dims])
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype != torch.bfloat16 or t.device.type != "cpu":
+        raise TypeError("oracle expects bf16 CPU tensors")
+    if t.stride(-1) != 1:
+        raise ValueError("oracle expects a unit stride on the last (head_dim) axis")
+    return t.view(torch.int16)
+
+
+def paged_attn(q, k_cache, v_cache, block_table, seqlens, scale, causal,
+               b_range=None, kvh_range=None):
+    """fp64 paged attention.
+
+    q:            [B, sq, Hq, D] bf16 (CPU)
+    k_cache/v_cache: [num_blocks, block_size, Hkv, D] bf16 views (any strides,
+                  unit stride on D), e.g. the interleaved views kv[:, 0], kv[:, 1]
+    block_table:  [B, nblk] int32
+    seqlens:      [B] int32, context length including the query tokens
+    Returns (out [B, sq, Hq, D] fp64, lse [B, Hq, sq] fp64).  Rows outside
+    b_range x kvh_range are left as NaN.
+    """
+    lib = _load()
+    B, sq, Hq, D = q.shape
+    nblocks, bs, Hkv, D2 = k_cache.shape
+    assert D2 == D and tuple(v_cache.shape) == tuple(k_cache.shape)
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    bt = block_table.to(torch.int32)
+    if bt.stride(1) != 1:
+        bt = bt.contiguous()
+    sl = seqlens.to(torch.int32).contiguous()
+    out = torch.full((B, sq, Hq, D), float("nan"), dtype=torch.float64)
+    lse = torch.full((B, Hq, sq), float("nan"), dtype=torch.float64)
+    b0, b1 = b_range if b_range is not None else (0, B)
+    h0, h1 = kvh_range if kvh_range is not None else (0, Hkv)
+    rc = lib.oracle_paged_attn(
+        qb.data_ptr(), _strides3(q), kb.data_ptr(), _strides3(k_cache),
+        vb.data_ptr(), _strides3(v_cache), nblocks, bt.data_ptr(), bt.stride(0),
+        sl.data_ptr(), B, sq, Hq, Hkv, D, bs, float(scale), int(bool(causal)),
+        b0, b1, h0, h1, out.data_ptr(), lse.data_ptr())
+    if rc != 0:
+        raise RuntimeError(f"oracle_paged_attn failed with status {rc}")
+    return out, lse
+
+
+def kv_append(k_new, v_new, k_cache, v_cache, block_table, seqlens):
+    """Write k_new/v_new [B, n, Hkv, D] into the caches (in place) at
+    positions seqlens[b] + t, copying bf16 bits unchanged."""
+    lib = _load()
+    B, n, Hkv, D = k_new.shape
+    nblocks, bs, Hkv2, D2 = k_cache.shape
+    assert (Hkv2, D2) == (Hkv, D)
+    bt = block_table.to(torch.int32)
+    if bt.stride(1) != 1:
+        bt = bt.contiguous()
+    sl = seqlens.to(torch.int32).contiguous()
+    rc = lib.oracle_kv_append(
+        _bits(k_new).data_ptr(), _strides3(k_new), _bits(v_new).data_ptr(),
+        _strides3(v_new), _bits(k_cache).data_ptr(), _strides3(k_cache),
+        _bits(v_cache).data_ptr(), _strides3(v_cache), nblocks, bt.data_ptr(),
+        bt.stride(0), bt.shape[1], sl.data_ptr(), B, n, Hkv, D, bs)
+    if rc != 0:
+        raise RuntimeError(f"oracle_kv_append failed with status {rc}")
