@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark: paged decode attention KV-read GB/s and tokens/s on B200.
+
+Workload (one "step" = one pass of the whole hot path over one batch):
+  long-context split-K decode -- batch 4, seqlen_q 1, context 131072 tokens
+  each, Hq 32 / Hkv 8, head_dim 128, bf16 N(0,1) data, contiguous paged cache
+  with block_size 16 and a seeded randperm block table [4, 8192], fixed split
+  chunk 4096 tokens merged in global block order.  A step appends the newest
+  token's K/V (kv_append, position 131071) and runs paged_decode_attn over the
+  131072-token contexts (split kernel + merge kernel).
+
+value   = algorithmic KV bytes (every visible token read once per KV head, K
+          and V, bf16) of all ranks / device time of the K timed steps (max
+          over ranks), in GB/s.  The 2.15 GB cache is larger than L2, so no
+          flush is needed between steps.
+e2e     = the same metric through the public API with pinned host buffers:
+          each step copies q, the new K/V, the sequence lengths and the block
+          table host->device and the output and lse device->host.
+roofline: the decode call's KV bytes / its mean CUDA-event duration, against
+          the measured HBM copy bandwidth.
+cpu_baseline: the CPU fp64 oracle on a bounded sample of the same workload.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: torchrun --nproc-per-node N bench.py --gpus N  (weak scaling: each
+rank runs its own batch; there is no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode attention KV-read GB/s (% of HBM peak) and tokens/s at 1 B200"
+WORKLOAD = ("long-context split-K decode: batch 4, seqlen_q 1, context 131072, Hq 32, Hkv 8, "
+            "head_dim 128, bf16, contiguous paged cache block_size 16, randperm block_table "
+            "[4, 8192], split chunk 4096 tokens")
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_decode_31_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per decode call from the committed ncu summary, or None if
+    the kernels changed since those counters were taken."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            t = json.load(f)
+        if t.get("kernel_digest") == kernel_source_digest():
+            return int(t["dram_bytes_per_call"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML (read-only) while the
+    timed region runs."""
+
+    REASONS = {
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sync_boost": 0x10,
+        "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                self.reasons |= int(n.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"],
+                    "samples": 0}
+        names = [k for k, bit in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def cpu_baseline(di_dev, n_seq: int = 2):
+    """The fp64 oracle on a bounded sample: the first n_seq sequences, every
+    KV head, full context.  Returns the cpu_baseline object."""
+    import oracle
+    from paged_kv_decode_31_b200 import inputs as I
+    cores = max(1, min(os.cpu_count() or 1, n_seq * di_dev.Hkv))
+    oracle.set_num_threads(cores)
+    host = I.DecodeInputs(di_dev.q[:n_seq].cpu(), di_dev.cache.to("cpu"),
+                          di_dev.block_table[:n_seq].cpu(), di_dev.seqlens[:n_seq].cpu(),
+                          di_dev.Hq, di_dev.Hkv, di_dev.D, di_dev.scale, di_dev.causal)
+    t0 = time.perf_counter()
+    oracle.paged_attn(host.q, host.cache.k, host.cache.v, host.block_table, host.seqlens,
+                      host.scale, host.causal)
+    dt = time.perf_counter() - t0
+    gbs = host.kv_bytes() / dt / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n_seq} of 4 sequences, all {di_dev.Hkv} KV heads, full 131072-token "
+                      f"context ({host.kv_bytes()} KV bytes) in {dt:.2f} s",
+            "tokens_per_s": round(n_seq / dt, 4)}
+
+
+def run_ours(args):
+    import torch.distributed as dist
+    import paged_kv_decode_31_b200 as pkv
+    from paged_kv_decode_31_b200 import inputs as I
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    di = I.config_long_context(seed=1000 + rank, device=dev)
+    B, ctx, Hq, Hkv, D = di.batch, int(di.seqlens[0].item()), di.Hq, di.Hkv, di.D
+    gen = torch.Generator(device=dev).manual_seed(2000 + rank)
+    k_new = torch.randn(B, 1, Hkv, D, generator=gen, device=dev).to(torch.bfloat16)
+    v_new = torch.randn(B, 1, Hkv, D, generator=gen, device=dev).to(torch.bfloat16)
+    seq_prev = torch.full((B,), ctx - 1, dtype=torch.int32, device=dev)
+    seq = di.seqlens
+    out = torch.empty(B, 1, Hq, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, Hq, 1, dtype=torch.float32, device=dev)
+    ws = torch.empty(pkv.workspace_size(B, 1, Hq, D, ctx), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    kv_bytes = di.kv_bytes()
+
+    def step(ev0=None, ev1=None):
+        pkv.kv_append(k_new, v_new, di.cache.k, di.cache.v, di.block_table, seq_prev, err=err)
+        if ev0 is not None:
+            ev0.record(stream)
+        pkv.paged_decode_attn(di.q, di.cache.k, di.cache.v, di.block_table, seq,
+                              max_seqlen_k=ctx, scale=di.scale, causal=False, out=out, lse=lse,
+                              workspace=ws, err=err)
+        if ev1 is not None:
+            ev1.record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(err.item())}")
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for k in range(args.steps):
+            step(*evs[k])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    decode_ms = [a.elapsed_time(b) for a, b in evs]
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(err.item())}")
+
+    # e2e through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_q = di.q.cpu().pin_memory()
+        h_kn, h_vn = k_new.cpu().pin_memory(), v_new.cpu().pin_memory()
+        h_sp, h_s = seq_prev.cpu().pin_memory(), seq.cpu().pin_memory()
+        h_bt = di.block_table.cpu().pin_memory()
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        d_q, d_kn, d_vn = torch.empty_like(di.q), torch.empty_like(k_new), torch.empty_like(v_new)
+        d_sp, d_s, d_bt = torch.empty_like(seq_prev), torch.empty_like(seq), torch.empty_like(di.block_table)
+        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_sp, h_s, h_bt))
+        d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+
+        def e2e_step():
+            for d, h in ((d_q, h_q), (d_kn, h_kn), (d_vn, h_vn), (d_sp, h_sp), (d_s, h_s), (d_bt, h_bt)):
+                d.copy_(h, non_blocking=True)
+            pkv.kv_append(d_kn, d_vn, di.cache.k, di.cache.v, d_bt, d_sp, err=err)
+            pkv.paged_decode_attn(d_q, di.cache.k, di.cache.v, d_bt, d_s, max_seqlen_k=ctx,
+                                  scale=di.scale, causal=False, out=out, lse=lse, workspace=ws,
+                                  err=err)
+            h_out.copy_(out, non_blocking=True)
+            h_lse.copy_(lse, non_blocking=True)
+
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": round(kv_bytes * world * args.steps / (e2e_ms / 1e3) / 1e9, 2),
+               "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(e2e_ms / args.steps, 5)}
+
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    peak, peak_kind = measured_peaks()
+    ms_step = ms_total / args.steps
+    value = kv_bytes * world * args.steps / (ms_total / 1e3) / 1e9
+    dec_ms = statistics.mean(decode_ms)
+    achieved = kv_bytes / (dec_ms / 1e3) / 1e9
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "batch": B, "seqlen_q": 1, "seqlen_k": ctx,
+                   "Hq": Hq, "Hkv": Hkv, "head_dim": D, "block_size": 16,
+                   "split_tokens": pkv.SPLIT_TOKENS,
+                   "step": "kv_append (1 token/sequence) + paged_decode_attn",
+                   "l2": "inputs larger than L2 (2.15 GB of K/V per rank), no flush",
+                   "parallelism": f"dp{world}"},
+        "tokens_per_s": round(B * world * args.steps / (ms_total / 1e3), 1),
+        "hbm_frac": round(value / world / peak, 4),
+        "hbm_frac_basis": f"{peak_kind} HBM copy bandwidth {peak} GB/s",
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(),
+                     "kernel": "paged_decode_attn (attn_split_kernel<128,16,3> + merge_kernel<128>)",
+                     "algorithmic_bytes_per_launch": kv_bytes,
+                     "launch_ms_mean": round(dec_ms, 5),
+                     "launch_ms_min": round(min(decode_ms), 5),
+                     "peak_basis": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        result["cpu_baseline"] = cpu_baseline(di)
+    print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The CPU fp64 oracle, timed on the host cores, on this workload's config
+    and metric: each step is a bounded sample (one sequence, every KV head, the
+    full 131072-token context)."""
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from paged_kv_decode_31_b200 import inputs as I
+    di = I.config_long_context(seed=1000, device="cpu")
+    Hkv = di.Hkv
+    cores = max(1, min(os.cpu_count() or 1, Hkv))
+    oracle.set_num_threads(cores)
+    b = 0
+    q = di.q[b:b + 1].contiguous()
+    bt = di.block_table[b:b + 1].contiguous()
+    sl = di.seqlens[b:b + 1].contiguous()
+    sample_bytes = int(sl.sum()) * Hkv * di.D * 4
+
+    def step():
+        oracle.paged_attn(q, di.cache.k, di.cache.v, bt, sl, di.scale, False)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = sample_bytes * args.steps / dt / 1e9
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "batch": 4, "seqlen_q": 1, "seqlen_k": 131072,
+                   "Hq": 32, "Hkv": 8, "head_dim": 128, "block_size": 16,
+                   "split_tokens": 4096, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: sequence 0 of 4, all {Hkv} KV heads, full "
+                                   f"131072-token context ({sample_bytes} KV bytes)"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,184 @@
+/*
+ * pagedkv.h -- C ABI of the B200 (sm_100a) paged-KV attention library
+ * (libpagedkv.so).
+ *
+ * Three operations, all enqueued on the caller's CUDA stream:
+ *
+ *   pkv_kv_append          write new K/V tokens into cache blocks;
+ *   pkv_paged_decode_attn  attention of one or a few query tokens against a
+ *                          paged KV cache (split-K / flash-decoding over a
+ *                          block table), returning out and lse;
+ *   pkv_paged_prefill_attn causal or chunked prefill over the same cache,
+ *                          under the same reduction contract.
+ *
+ * The call shape follows flash_attn_with_kvcache(q, k_cache, v_cache,
+ * cache_seqlens=, page_table=, causal=) as exercised by ROCm/aiter commit
+ * d293d61 "test(triton/decode): pin non-contiguous paged KV block stride"
+ * (test_flash_attn_kvcache_noncontiguous_paged), extended with lse, an
+ * explicit softmax scale, the real per-component cache strides and kv_append.
+ *
+ * Reduction contract (shared by decode and prefill).  The KV context of every
+ * query row is cut into fixed chunks ("splits") of PKV_SPLIT_TOKENS tokens
+ * starting at absolute position 0, each split into tiles of PKV_TILE_TOKENS
+ * tokens.  Within a split, tiles are folded in ascending order with an online
+ * softmax in fp32 (scores, P.V and the row sums on the tensor cores with fp32
+ * accumulation; each probability enters them as a bf16 hi part plus a bf16
+ * remainder, ~16 significant bits).  Split partials are
+ * merged in ascending split index (= global block index) order in fp32, and
+ * out is rounded to bf16 once, at the final write.  Source: RL-Kernel PR #284
+ * "feat(attention): add CP backward drift validation", Changes ("fixed
+ * global_block_index merge order, fp32 accumulation, final-write downcast"),
+ * and the [WS1] "KV-cache path consistency (prefill & decode)" issue, Notes
+ * ("share one reduction-order contract across prefill and decode").  None of
+ * the constants depends on the batch, the SM count or the block size, so a
+ * row's result is bitwise independent of batch composition, padding, cache
+ * layout and of which entry point computed it.
+ *
+ * Conventions shared by all calls
+ * -------------------------------
+ * - All pointers except the stride arrays are DEVICE pointers on the current
+ *   device.  Stride arrays are HOST arrays of element (not byte) strides.
+ * - q, K, V, k_new, v_new and out are bf16 (IEEE bfloat16 bits); lse is fp32;
+ *   block_table and seqlens are int32.
+ * - The last axis (head_dim D) of every bf16 tensor has unit stride.  Every
+ *   other stride of q, K, V, k_new and v_new must be a multiple of 8 elements
+ *   (16 bytes) and their base pointers 16-byte aligned (128-bit loads, TMA).
+ * - Cache views are [num_blocks, block_size, Hkv, D] with element strides
+ *   (block, slot, head) given per component, so the non-contiguous K = kv[:,0]
+ *   and V = kv[:,1] views of an interleaved [num_blocks, 2, block_size, Hkv, D]
+ *   buffer work as is (block stride 2*block_size*Hkv*D).
+ * - block_table row b lists the cache block of tokens
+ *   [j*block_size, (j+1)*block_size) of sequence b at column j; the row stride
+ *   is bt_stride elements and at most max_blocks_per_seq columns are read.
+ * - seqlens[b] (device) is the context length of sequence b INCLUDING the
+ *   query tokens: the caller appends the queries' K/V with pkv_kv_append
+ *   first.  Query row i of seqlen_q sits at absolute position
+ *   seqlens[b] - seqlen_q + i (bottom-right alignment); under causal it sees
+ *   keys 0..position, otherwise keys 0..seqlens[b]-1.  A row that sees no key
+ *   gets out = 0 and lse = -inf.
+ * - GQA: query head h reads KV head h / (Hq / Hkv).
+ * - The library allocates nothing, never synchronises the device and only
+ *   enqueues work on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   The caller owns every buffer, including the workspace.
+ * - err (optional, may be NULL) is a device int32 the kernels OR error bits
+ *   into (PKV_DEVERR_*).  It is never read or cleared by the library, so the
+ *   hot path never synchronises; the caller zeroes it and reads it when it
+ *   wants to check.  Out-of-range table entries are skipped, never read.
+ * - Every call returns PKV_OK or a PKV_ERR_* code and launches nothing when
+ *   it returns an error.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Fixed constants of the reduction contract. */
+#define PKV_SPLIT_TOKENS 4096
+#define PKV_TILE_TOKENS 128
+
+/* Return codes. */
+#define PKV_OK 0
+#define PKV_ERR_ARG 1        /* a size, stride, alignment or pointer is invalid */
+#define PKV_ERR_WORKSPACE 2  /* workspace NULL or smaller than pkv_workspace_size() */
+#define PKV_ERR_CUDA 3       /* a CUDA runtime call or kernel launch failed */
+#define PKV_ERR_LAYOUT 4     /* the cache strides cannot be described to the TMA unit */
+
+/* Device error bits OR-ed into *err by the kernels. */
+#define PKV_DEVERR_BAD_BLOCK 1   /* block_table entry outside [0, num_blocks) */
+#define PKV_DEVERR_TABLE_WIDTH 2 /* a position needs a column >= max_blocks_per_seq */
+#define PKV_DEVERR_TIMEOUT 4     /* an internal pipeline wait gave up (no result) */
+
+/*
+ * pkv_kv_append: for every sequence b and new token t < n_new, copy the bf16
+ * bits of k_new[b, t, :, :] and v_new[b, t, :, :] (shape [batch, n_new, Hkv, D],
+ * element strides kn_strides / vn_strides = (batch, token, head)) to cache
+ * position p = seqlens[b] + t: block block_table[b][p / block_size], slot
+ * p % block_size.  The bits are stored unchanged, so the reader sees exactly
+ * what the writer produced ([WS1] KV-cache path consistency, Scope: stored-KV
+ * dtype/layout must add no drift).  seqlens are NOT modified: the caller
+ * advances them (put-then-advance, as jouleclaw's in-place KV cache does).
+ * block_size: a power of two in [16, 256]; D: 64 or 128.
+ */
+int pkv_kv_append(const void *k_new, const int64_t kn_strides[3],
+                  const void *v_new, const int64_t vn_strides[3],
+                  void *k_cache, const int64_t k_strides[3],
+                  void *v_cache, const int64_t v_strides[3],
+                  int64_t num_blocks,
+                  const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                  const int32_t *seqlens, int batch, int n_new, int Hkv, int D,
+                  int block_size, int32_t *err, void *stream);
+
+/*
+ * pkv_paged_decode_attn: out[b, i, h, :] = softmax(scale * q K^T) V over the
+ * keys visible to query row i (see Conventions), lse[b, h, i] = natural-log
+ * log-sum-exp of scale * q.k over those keys.
+ *
+ *   q            [batch, seqlen_q, Hq, D] bf16, element strides q_strides = (b, s, h)
+ *   k_cache/v_cache  cache views, element strides (block, slot, head)
+ *   num_blocks   number of blocks in the cache (table entries are checked against it)
+ *   seqlens      [batch] int32 device, context lengths incl. the query tokens
+ *   max_seqlen_k host upper bound of seqlens (sizes the split grid); a sequence
+ *                longer than it is an error of the caller (its tail is ignored)
+ *   scale        softmax scale applied to q.k (e.g. 1/sqrt(D))
+ *   causal       0 or 1 (bottom-right aligned)
+ *   out          [batch, seqlen_q, Hq, D] bf16, element strides out_strides = (b, s, h)
+ *   lse          [batch, Hq, seqlen_q] fp32, contiguous
+ *   workspace    >= pkv_workspace_size(batch, seqlen_q, Hq, D, max_seqlen_k) bytes,
+ *                16-byte aligned, no initialisation needed
+ * D: 64 or 128; Hq % Hkv == 0; block_size: power of two in [16, 256].
+ * Split-K decode over the block table (aiter d293d61 commit message), honouring
+ * the real k/v_cache.stride(0) instead of assuming block_size * slot_stride.
+ */
+int pkv_paged_decode_attn(const void *q, const int64_t q_strides[3],
+                          const void *k_cache, const int64_t k_strides[3],
+                          const void *v_cache, const int64_t v_strides[3],
+                          int64_t num_blocks,
+                          const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                          const int32_t *seqlens, int max_seqlen_k,
+                          int batch, int seqlen_q, int Hq, int Hkv, int D, int block_size,
+                          float scale, int causal,
+                          void *out, const int64_t out_strides[3], float *lse,
+                          void *workspace, size_t workspace_bytes,
+                          int32_t *err, void *stream);
+
+/*
+ * pkv_paged_prefill_attn: same arguments and semantics as
+ * pkv_paged_decode_attn, for many query rows per sequence (a causal prefill,
+ * or one chunk of a chunked prefill: append the chunk's K/V, then call with
+ * seqlen_q = chunk length and seqlens = tokens cached so far).  Every row is
+ * reduced under the same contract as a decode row at the same position, so
+ * decode row t equals prefill row t bit for bit ([WS1] KV-cache path
+ * consistency, Acceptance criteria).
+ */
+int pkv_paged_prefill_attn(const void *q, const int64_t q_strides[3],
+                           const void *k_cache, const int64_t k_strides[3],
+                           const void *v_cache, const int64_t v_strides[3],
+                           int64_t num_blocks,
+                           const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                           const int32_t *seqlens, int max_seqlen_k,
+                           int batch, int seqlen_q, int Hq, int Hkv, int D, int block_size,
+                           float scale, int causal,
+                           void *out, const int64_t out_strides[3], float *lse,
+                           void *workspace, size_t workspace_bytes,
+                           int32_t *err, void *stream);
+
+/* Workspace bytes the attention calls need: fp32 split partials
+ * (m, l, acc[D]) for every (batch, query row, query head, split). */
+size_t pkv_workspace_size(int batch, int seqlen_q, int Hq, int D, int max_seqlen_k);
+
+/* Static description of a return code (never NULL). */
+const char *pkv_strerror(int code);
+
+/* PKV_SPLIT_TOKENS, for bindings that cannot read the macro. */
+int pkv_split_tokens(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

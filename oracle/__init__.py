@@ -49,6 +49,8 @@ def _load():
         lib.oracle_kv_append.argtypes = [p, p, p, p, p, p, p, p, i64, p, i64,
                                          i32, p, i32, i32, i32, i32, i32]
         lib.oracle_kv_append.restype = i32
+        lib.oracle_set_num_threads.argtypes = [i32]
+        lib.oracle_set_num_threads.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i32
         _lib = lib
@@ -57,6 +59,10 @@ def _load():
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    _load().oracle_set_num_threads(int(n))
 
 
 def _strides3(t: torch.Tensor, dims=(0, 1, 2)) -> ctypes.Array:

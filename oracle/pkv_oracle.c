@@ -232,6 +232,18 @@ int oracle_kv_append(const uint16_t *k_new, const int64_t kn_st[3],
     return ORACLE_OK;
 }
 
+/* Cap the number of OpenMP threads (each task holds a dense fp64 copy of one
+ * KV head of one sequence, so the cap bounds host memory). */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* Number of OpenMP threads the oracle runs on (1 without OpenMP). */
 int oracle_num_threads(void)
 {

@@ -1,1 +1,18 @@
-"""B200-native paged-KV decode / prefill attention (sm_100a)."""
+"""B200-native paged-KV decode / prefill attention (sm_100a).
+
+The computation lives in libpagedkv.so (CUDA, C ABI in include/pagedkv.h);
+this package is a thin ctypes binding plus seeded input generators.  Importing
+the package does not load the library; the first call does, and raises if the
+library has not been built -- there is no CPU fallback.
+"""
+from .binding import (  # noqa: F401
+    PagedKVError,
+    SPLIT_TOKENS,
+    TILE_TOKENS,
+    kv_append,
+    library_path,
+    paged_decode_attn,
+    paged_prefill_attn,
+    strerror,
+    workspace_size,
+)

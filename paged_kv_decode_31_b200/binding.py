@@ -1,0 +1,180 @@
+"""ctypes binding of libpagedkv.so (C ABI in include/pagedkv.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI.  torch provides device memory and the current
+stream.  If the library is not built, every call raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedkv.so")
+_lib = None
+
+# Mirrors of the constants in include/pagedkv.h
+SPLIT_TOKENS = 4096
+TILE_TOKENS = 128
+DEVERR_BAD_BLOCK = 1
+DEVERR_TABLE_WIDTH = 2
+DEVERR_TIMEOUT = 4
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+_ATTN_ARGS = [_P, _P, _P, _P, _P, _P, _I64, _P, _I64, _I, _P, _I,
+              _I, _I, _I, _I, _I, _I, ctypes.c_float, _I,
+              _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
+
+
+class PagedKVError(RuntimeError):
+    """A C-ABI call returned an error status."""
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with `python -m paged_kv_decode_31_b200.build` "
+                "(there is no CPU fallback)")
+        L = ctypes.CDLL(_LIB_PATH)
+        L.pkv_kv_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I64, _I, _P,
+                                    _I, _I, _I, _I, _I, _P, _P]
+        L.pkv_kv_append.restype = _I
+        L.pkv_paged_decode_attn.argtypes = _ATTN_ARGS
+        L.pkv_paged_decode_attn.restype = _I
+        L.pkv_paged_prefill_attn.argtypes = _ATTN_ARGS
+        L.pkv_paged_prefill_attn.restype = _I
+        L.pkv_workspace_size.argtypes = [_I, _I, _I, _I, _I]
+        L.pkv_workspace_size.restype = ctypes.c_size_t
+        L.pkv_strerror.argtypes = [_I]
+        L.pkv_strerror.restype = ctypes.c_char_p
+        L.pkv_split_tokens.argtypes = []
+        L.pkv_split_tokens.restype = _I
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().pkv_strerror(int(code)).decode()
+
+
+def _check(name: str, rc: int) -> None:
+    if rc != 0:
+        raise PagedKVError(f"{name}: {strerror(rc)} (status {rc})")
+
+
+def _st3(t: torch.Tensor) -> ctypes.Array:
+    return (ctypes.c_int64 * 3)(int(t.stride(0)), int(t.stride(1)), int(t.stride(2)))
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need_cuda_bf16(name: str, t: torch.Tensor) -> None:
+    if not t.is_cuda or t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be a bf16 CUDA tensor (got {t.dtype} on {t.device})")
+    if t.dim() != 4 or t.stride(-1) != 1:
+        raise ValueError(f"{name} must be 4-D with a unit stride on the last axis")
+
+
+def _need_cuda_i32(name: str, t: torch.Tensor) -> None:
+    if not t.is_cuda or t.dtype != torch.int32:
+        raise TypeError(f"{name} must be an int32 CUDA tensor")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def workspace_size(batch: int, seqlen_q: int, Hq: int, D: int, max_seqlen_k: int) -> int:
+    return int(lib().pkv_workspace_size(batch, seqlen_q, Hq, D, max_seqlen_k))
+
+
+def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
+              v_cache: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor, *,
+              err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Write k_new/v_new [B, n, Hkv, D] into the caches at positions
+    seqlens[b] + t (bits unchanged).  seqlens is not advanced."""
+    for name, t in (("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _need_cuda_bf16(name, t)
+    _need_cuda_i32("block_table", block_table)
+    _need_cuda_i32("seqlens", seqlens)
+    if block_table.stride(1) != 1:
+        raise ValueError("block_table must have a unit column stride")
+    B, n, Hkv, D = k_new.shape
+    rc = lib().pkv_kv_append(
+        k_new.data_ptr(), _st3(k_new), v_new.data_ptr(), _st3(v_new),
+        k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(), _st3(v_cache),
+        int(k_cache.shape[0]), block_table.data_ptr(), int(block_table.stride(0)),
+        int(block_table.shape[1]), seqlens.data_ptr(), B, n, Hkv, D, int(k_cache.shape[1]),
+        _ptr(err), _stream_handle(stream))
+    _check("pkv_kv_append", rc)
+
+
+def _attn(fn_name: str, q, k_cache, v_cache, block_table, seqlens, max_seqlen_k, scale,
+          causal, out, lse, workspace, err, stream) -> Tuple[torch.Tensor, torch.Tensor]:
+    _need_cuda_bf16("q", q)
+    _need_cuda_bf16("k_cache", k_cache)
+    _need_cuda_bf16("v_cache", v_cache)
+    _need_cuda_i32("block_table", block_table)
+    _need_cuda_i32("seqlens", seqlens)
+    if block_table.stride(1) != 1:
+        raise ValueError("block_table must have a unit column stride")
+    B, sq, Hq, D = q.shape
+    num_blocks, bs, Hkv, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("q / k_cache / v_cache shapes disagree")
+    if max_seqlen_k is None:
+        max_seqlen_k = int(seqlens.max().item()) if seqlens.numel() else 0
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(B, sq, Hq, D, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, Hq, sq, dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, sq):
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, seqlen_q] tensor")
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != (B, sq, Hq, D) or out.stride(-1) != 1:
+        raise ValueError("out must be bf16 [B, seqlen_q, Hq, D] with a unit last stride")
+    need = workspace_size(B, sq, Hq, D, max_seqlen_k)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = getattr(lib(), fn_name)(
+        q.data_ptr(), _st3(q), k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(),
+        _st3(v_cache), num_blocks, block_table.data_ptr(), int(block_table.stride(0)),
+        int(block_table.shape[1]), seqlens.data_ptr(), int(max_seqlen_k), B, sq, Hq, Hkv, D, bs,
+        float(scale), int(bool(causal)), out.data_ptr(), _st3(out), lse.data_ptr(),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(), _ptr(err),
+        _stream_handle(stream))
+    _check(fn_name, rc)
+    return out, lse
+
+
+def paged_decode_attn(q, k_cache, v_cache, block_table, seqlens, *, max_seqlen_k=None,
+                      scale=None, causal=False, out=None, lse=None, workspace=None, err=None,
+                      stream=None):
+    """Attention of q [B, sq, Hq, D] against the paged cache; returns
+    (out [B, sq, Hq, D] bf16, lse [B, Hq, sq] fp32).  See include/pagedkv.h."""
+    return _attn("pkv_paged_decode_attn", q, k_cache, v_cache, block_table, seqlens,
+                 max_seqlen_k, scale, causal, out, lse, workspace, err, stream)
+
+
+def paged_prefill_attn(q, k_cache, v_cache, block_table, seqlens, *, max_seqlen_k=None,
+                       scale=None, causal=True, out=None, lse=None, workspace=None, err=None,
+                       stream=None):
+    """Causal or chunked prefill over the paged cache; same contract as decode."""
+    return _attn("pkv_paged_prefill_attn", q, k_cache, v_cache, block_table, seqlens,
+                 max_seqlen_k, scale, causal, out, lse, workspace, err, stream)

@@ -1,0 +1,61 @@
+// kv_append.cuh -- write new K/V tokens into paged cache blocks.
+//
+// Token t of sequence b goes to position p = seqlens[b] + t: block
+// block_table[b][p / block_size], slot p % block_size, addressed with the
+// cache's real element strides.  The bf16 bits are copied unchanged with
+// 128-bit loads and stores ([WS1] "KV-cache path consistency (prefill &
+// decode)", Scope: the stored-KV dtype and layout must add no difference
+// between the path that wrote the cache and the path that reads it).
+#pragma once
+
+#include <cstdint>
+
+namespace pkv {
+
+struct AppendParams {
+  const uint16_t *k_new, *v_new;
+  int64_t kn_sb, kn_st, kn_sh, vn_sb, vn_st, vn_sh;
+  uint16_t *k_cache, *v_cache;
+  int64_t k_sb, k_ss, k_sh, v_sb, v_ss, v_sh;
+  int64_t num_blocks;
+  const int32_t *block_table;
+  int64_t bt_stride;
+  int max_blocks_per_seq;
+  const int32_t *seqlens;
+  int batch, n_new, Hkv, chunks;  // chunks = D / 8 (16-byte pieces per head row)
+  int block_shift;
+  int32_t *err;
+};
+
+__global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ AppendParams p) {
+  const int64_t total = static_cast<int64_t>(p.batch) * p.n_new * p.Hkv * p.chunks;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(idx % p.chunks);
+    int64_t r = idx / p.chunks;
+    const int h = static_cast<int>(r % p.Hkv);
+    r /= p.Hkv;
+    const int t = static_cast<int>(r % p.n_new);
+    const int b = static_cast<int>(r / p.n_new);
+    const int64_t pos = static_cast<int64_t>(__ldg(p.seqlens + b)) + t;
+    const int64_t bi = pos >> p.block_shift;
+    if (pos < 0 || bi >= p.max_blocks_per_seq) {
+      if (p.err) atomicOr(p.err, 2);
+      continue;
+    }
+    const int32_t blk = __ldg(p.block_table + b * p.bt_stride + bi);
+    if (blk < 0 || static_cast<int64_t>(blk) >= p.num_blocks) {
+      if (p.err) atomicOr(p.err, 1);
+      continue;
+    }
+    const int64_t slot = pos & ((int64_t{1} << p.block_shift) - 1);
+    const uint4 kv = __ldg(reinterpret_cast<const uint4 *>(p.k_new + b * p.kn_sb + t * p.kn_st +
+                                                           h * p.kn_sh) + c);
+    const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(p.v_new + b * p.vn_sb + t * p.vn_st +
+                                                           h * p.vn_sh) + c);
+    reinterpret_cast<uint4 *>(p.k_cache + blk * p.k_sb + slot * p.k_ss + h * p.k_sh)[c] = kv;
+    reinterpret_cast<uint4 *>(p.v_cache + blk * p.v_sb + slot * p.v_ss + h * p.v_sh)[c] = vv;
+  }
+}
+
+}  // namespace pkv

@@ -1,0 +1,69 @@
+// merge.cuh -- deterministic merge of split partials and final write.
+//
+// For one output row (batch b, query token i, query head h) the partials
+// (m_s, l_s, acc_s[D]) of splits s = 0, 1, ... are folded in ascending split
+// order -- the fixed global_block_index merge order, fp32 accumulation and
+// final-write downcast named in RL-Kernel PR #284 "feat(attention): add CP
+// backward drift validation", Changes:
+//
+//   M' = max(M, m_s), a = 2^(M - M'), c = 2^(m_s - M')
+//   L  = fma(l_s, c, L * a),  A = fma(acc_s, c, A * a),  M = M'
+//   out = bf16_rn(A / L),     lse = (M + log2 L) * ln 2
+//
+// m_s is in base-2 scaled units (scale * log2(e) * q.k), so lse comes out in
+// the natural-log, scale * q.k domain.  The same code merges every row of
+// every entry point, and a single split goes through it too.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace pkv {
+
+struct MergeParams {
+  const int32_t *seqlens;
+  int seqlen_q, Hq, n_splits, causal;
+  const float *ws_acc;
+  const float *ws_ml;
+  __nv_bfloat16 *out;
+  int64_t o_sb, o_ss, o_sh;
+  float *lse;
+};
+
+template <int D>
+__global__ void __launch_bounds__(D) merge_kernel(const __grid_constant__ MergeParams p) {
+  const int64_t row = blockIdx.x;  // (b * seqlen_q + i) * Hq + h
+  const int h = static_cast<int>(row % p.Hq);
+  const int64_t bi = row / p.Hq;
+  const int i = static_cast<int>(bi % p.seqlen_q);
+  const int b = static_cast<int>(bi / p.seqlen_q);
+  const int n = max(__ldg(p.seqlens + b), 0);
+  int lim = n;
+  if (p.causal) lim = min(lim, n - p.seqlen_q + i + 1);
+  lim = max(lim, 0);
+  const int n_s = min((lim + 4095) / 4096, p.n_splits);
+  const int d = threadIdx.x;
+  const float NEG_INF = __int_as_float(0xff800000);
+  float M = NEG_INF, L = 0.f, A = 0.f;
+  for (int s = 0; s < n_s; ++s) {
+    const int64_t k = row * p.n_splits + s;
+    const float ms = p.ws_ml[2 * k];
+    const float ls = p.ws_ml[2 * k + 1];
+    if (ms == NEG_INF) continue;  // the row sees no key of this split
+    const float Mn = fmaxf(M, ms);
+    const float a = ex2(__fsub_rn(M, Mn));
+    const float c = ex2(__fsub_rn(ms, Mn));
+    L = __fmaf_rn(ls, c, __fmul_rn(L, a));
+    A = __fmaf_rn(p.ws_acc[k * D + d], c, __fmul_rn(A, a));
+    M = Mn;
+  }
+  const bool any = L > 0.f;
+  const float o = any ? __fdiv_rn(A, L) : 0.f;
+  p.out[b * p.o_sb + i * p.o_ss + h * p.o_sh + d] = __float2bfloat16_rn(o);
+  if (d == 0)
+    p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.seqlen_q + i] =
+        any ? __fmul_rn(__fadd_rn(M, log2f(L)), 0.69314718055994531f) : NEG_INF;
+}
+
+}  // namespace pkv

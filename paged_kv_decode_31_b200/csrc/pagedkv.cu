@@ -1,0 +1,367 @@
+// pagedkv.cu -- C ABI of libpagedkv.so (declarations and contract in
+// include/pagedkv.h): argument validation, TMA tensor maps over the caller's
+// cache views, and the kernel launches.  No allocation, no synchronisation.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "pagedkv.h"
+#include "attn_split.cuh"
+#include "kv_append.cuh"
+#include "merge.cuh"
+
+static_assert(PKV_SPLIT_TOKENS == pkv::kSplitTokens, "split size");
+static_assert(PKV_TILE_TOKENS == pkv::kTileTokens, "tile size");
+static_assert(PKV_DEVERR_BAD_BLOCK == pkv::kErrBadBlock, "error bits");
+static_assert(PKV_DEVERR_TABLE_WIDTH == pkv::kErrTableWidth, "error bits");
+static_assert(PKV_DEVERR_TIMEOUT == pkv::kErrTimeout, "error bits");
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+int sm_count(int dev) {
+  static std::atomic<int> cache[kMaxDevices];
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    v = 148;
+  cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+int log2i(int v) {
+  int s = 0;
+  while ((1 << s) < v) ++s;
+  return s;
+}
+
+// Element strides usable for 128-bit access: positive multiples of 8.
+bool strides_ok(const int64_t *st) {
+  if (!st) return false;
+  for (int i = 0; i < 3; ++i)
+    if (st[i] <= 0 || st[i] % 8 != 0) return false;
+  return true;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+size_t ws_acc_bytes(int64_t rows, int64_t splits, int D) {
+  const size_t b = static_cast<size_t>(rows) * splits * D * sizeof(float);
+  return (b + 255) & ~static_cast<size_t>(255);
+}
+
+size_t ws_bytes(int batch, int seqlen_q, int Hq, int D, int max_seqlen_k) {
+  const int64_t rows = static_cast<int64_t>(batch) * seqlen_q * Hq;
+  const int64_t splits = max_seqlen_k > 0 ? ceil_div(max_seqlen_k, pkv::kSplitTokens) : 1;
+  return ws_acc_bytes(rows, splits, D) + static_cast<size_t>(rows) * splits * 2 * sizeof(float);
+}
+
+// TMA map over one cache view [num_blocks, block_size, Hkv, D] with the given
+// element strides (block, slot, head).  Dimension 0 is head_dim; the head and
+// slot dimensions are ordered by stride; the last is the block.  The box is
+// 64 head_dim elements x box_slots slots of one head of one block, 128-byte
+// swizzled, so every box lands as box_slots rows of 128 bytes.
+int make_kv_map(CUtensorMap *map, const void *base, const int64_t st[3], int64_t num_blocks,
+                int block_size, int Hkv, int D, int box_slots, int *head_first) {
+  auto enc = encode_fn();
+  if (!enc) return PKV_ERR_CUDA;
+  const bool hf = st[2] <= st[1];
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4], estr[4] = {1, 1, 1, 1};
+  dims[0] = static_cast<cuuint64_t>(D);
+  box[0] = 64;
+  if (hf) {
+    dims[1] = Hkv;
+    dims[2] = block_size;
+    strides[0] = st[2] * 2;
+    strides[1] = st[1] * 2;
+    box[1] = 1;
+    box[2] = box_slots;
+  } else {
+    dims[1] = block_size;
+    dims[2] = Hkv;
+    strides[0] = st[1] * 2;
+    strides[1] = st[2] * 2;
+    box[1] = box_slots;
+    box[2] = 1;
+  }
+  dims[3] = static_cast<cuuint64_t>(num_blocks);
+  strides[2] = st[0] * 2;
+  box[3] = 1;
+  std::memset(map, 0, sizeof(*map));
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return PKV_ERR_LAYOUT;
+  *head_first = hf ? 1 : 0;
+  return PKV_OK;
+}
+
+// Pipeline depth (K/V stages) and Q buffers per instance, sized to the
+// 227 KB of shared memory one CTA may use.
+template <int D, int N>
+constexpr int stages() {
+  return D == 128 ? (N == 16 ? 3 : 2) : (N == 16 ? 6 : 4);
+}
+template <int D, int N>
+constexpr int q_buffers() {
+  return (D == 128 && N == 64) ? 1 : 2;
+}
+
+template <int D, int N>
+int launch_split(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensorMap &mv,
+                 cudaStream_t s, int dev) {
+  constexpr int NS = stages<D, N>();
+  constexpr int QB = q_buffers<D, N>();
+  using C = pkv::Cfg<D, N, NS, QB>;
+  static_assert(C::kSmemBytes <= 232448, "shared memory budget");
+  static std::atomic<bool> attr_set[kMaxDevices];
+  auto kern = pkv::attn_split_kernel<D, N, NS, QB>;
+  if (dev < 0 || dev >= kMaxDevices || !attr_set[dev].load(std::memory_order_acquire)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+      return PKV_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices) attr_set[dev].store(true, std::memory_order_release);
+  }
+  const int grid = p.n_units < sm_count(dev) ? p.n_units : sm_count(dev);
+  kern<<<grid, pkv::kThreads, C::kSmemBytes, s>>>(p, mk, mv);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+template <int D>
+int launch_merge(const pkv::MergeParams &m, int64_t rows, cudaStream_t s) {
+  pkv::merge_kernel<D><<<static_cast<unsigned>(rows), D, 0, s>>>(m);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+// Rows of query heads x tokens per tile: 16 when a KV head's whole query
+// group fits (decode), else 64.  Both sizes run the same arithmetic per row.
+int rows_per_tile(int rows) { return rows <= 16 ? 16 : 64; }
+
+int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
+               const int64_t k_strides[3], const void *v_cache, const int64_t v_strides[3],
+               int64_t num_blocks, const int32_t *block_table, int64_t bt_stride,
+               int max_blocks_per_seq, const int32_t *seqlens, int max_seqlen_k, int batch,
+               int seqlen_q, int Hq, int Hkv, int D, int block_size, float scale, int causal,
+               void *out, const int64_t out_strides[3], float *lse, void *workspace,
+               size_t workspace_bytes, int32_t *err, void *stream) {
+  if (!q || !k_cache || !v_cache || !block_table || !seqlens || !out || !lse) return PKV_ERR_ARG;
+  if (batch <= 0 || seqlen_q <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return PKV_ERR_ARG;
+  if (D != 64 && D != 128) return PKV_ERR_ARG;
+  if (!pow2_in(block_size, 16, 256)) return PKV_ERR_ARG;
+  if (num_blocks <= 0 || num_blocks > INT32_MAX || max_blocks_per_seq <= 0 || bt_stride < max_blocks_per_seq)
+    return PKV_ERR_ARG;
+  if (max_seqlen_k < 0) return PKV_ERR_ARG;
+  if (!strides_ok(q_strides) || !strides_ok(k_strides) || !strides_ok(v_strides)) return PKV_ERR_ARG;
+  if (!out_strides || out_strides[0] <= 0 || out_strides[1] <= 0 || out_strides[2] <= 0)
+    return PKV_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_ERR_ARG;
+  if (!(scale > 0.f) || !(scale < 3.0e38f)) return PKV_ERR_ARG;
+  const int G = Hq / Hkv;
+  const int64_t R = static_cast<int64_t>(G) * seqlen_q;
+  const int64_t rows = static_cast<int64_t>(batch) * seqlen_q * Hq;
+  if (R > INT32_MAX / 2 || rows > INT32_MAX) return PKV_ERR_ARG;
+  const int N = rows_per_tile(static_cast<int>(R));
+  const int64_t S = max_seqlen_k > 0 ? ceil_div(max_seqlen_k, pkv::kSplitTokens) : 1;
+  const int64_t RT = ceil_div(R, N);
+  const int64_t units = static_cast<int64_t>(batch) * S * Hkv * RT;
+  if (units > INT32_MAX) return PKV_ERR_ARG;
+  const size_t need = ws_bytes(batch, seqlen_q, Hq, D, max_seqlen_k);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  const int box_slots = block_size < pkv::kTileTokens ? block_size : pkv::kTileTokens;
+  alignas(64) CUtensorMap mk, mv;
+  int hf_k = 0, hf_v = 0;
+  int rc = make_kv_map(&mk, k_cache, k_strides, num_blocks, block_size, Hkv, D, box_slots, &hf_k);
+  if (rc != PKV_OK) return rc;
+  rc = make_kv_map(&mv, v_cache, v_strides, num_blocks, block_size, Hkv, D, box_slots, &hf_v);
+  if (rc != PKV_OK) return rc;
+  if (hf_k != hf_v) return PKV_ERR_LAYOUT;  // K and V must order head/slot alike
+
+  float *ws_acc = static_cast<float *>(workspace);
+  float *ws_ml = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                           ws_acc_bytes(rows, S, D));
+  pkv::AttnParams p{};
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.q_sb = q_strides[0];
+  p.q_ss = q_strides[1];
+  p.q_sh = q_strides[2];
+  p.block_table = block_table;
+  p.bt_stride = bt_stride;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
+  p.seqlens = seqlens;
+  p.batch = batch;
+  p.seqlen_q = seqlen_q;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.block_shift = log2i(block_size);
+  p.box_slots = box_slots;
+  p.map_head_first = hf_k;
+  p.n_row_tiles = static_cast<int>(RT);
+  p.n_splits = static_cast<int>(S);
+  p.n_units = static_cast<int>(units);
+  p.cscale = scale * 1.4426950408889634f;  // host IEEE multiply, one rounding
+  p.causal = causal ? 1 : 0;
+  p.ws_acc = ws_acc;
+  p.ws_ml = ws_ml;
+  p.err = err;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (D == 128)
+    rc = N == 16 ? launch_split<128, 16>(p, mk, mv, s, dev) : launch_split<128, 64>(p, mk, mv, s, dev);
+  else
+    rc = N == 16 ? launch_split<64, 16>(p, mk, mv, s, dev) : launch_split<64, 64>(p, mk, mv, s, dev);
+  if (rc != PKV_OK) return rc;
+
+  pkv::MergeParams m{};
+  m.seqlens = seqlens;
+  m.seqlen_q = seqlen_q;
+  m.Hq = Hq;
+  m.n_splits = static_cast<int>(S);
+  m.causal = p.causal;
+  m.ws_acc = ws_acc;
+  m.ws_ml = ws_ml;
+  m.out = static_cast<__nv_bfloat16 *>(out);
+  m.o_sb = out_strides[0];
+  m.o_ss = out_strides[1];
+  m.o_sh = out_strides[2];
+  m.lse = lse;
+  return D == 128 ? launch_merge<128>(m, rows, s) : launch_merge<64>(m, rows, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int pkv_kv_append(const void *k_new, const int64_t kn_strides[3], const void *v_new,
+                  const int64_t vn_strides[3], void *k_cache, const int64_t k_strides[3],
+                  void *v_cache, const int64_t v_strides[3], int64_t num_blocks,
+                  const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                  const int32_t *seqlens, int batch, int n_new, int Hkv, int D, int block_size,
+                  int32_t *err, void *stream) {
+  if (!k_new || !v_new || !k_cache || !v_cache || !block_table || !seqlens) return PKV_ERR_ARG;
+  if (batch <= 0 || n_new < 0 || Hkv <= 0 || (D != 64 && D != 128)) return PKV_ERR_ARG;
+  if (!pow2_in(block_size, 16, 256)) return PKV_ERR_ARG;
+  if (num_blocks <= 0 || num_blocks > INT32_MAX || max_blocks_per_seq <= 0 || bt_stride < max_blocks_per_seq)
+    return PKV_ERR_ARG;
+  if (!strides_ok(kn_strides) || !strides_ok(vn_strides) || !strides_ok(k_strides) ||
+      !strides_ok(v_strides))
+    return PKV_ERR_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PKV_ERR_ARG;
+  if (n_new == 0) return PKV_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  pkv::AppendParams p{};
+  p.k_new = static_cast<const uint16_t *>(k_new);
+  p.v_new = static_cast<const uint16_t *>(v_new);
+  p.kn_sb = kn_strides[0];
+  p.kn_st = kn_strides[1];
+  p.kn_sh = kn_strides[2];
+  p.vn_sb = vn_strides[0];
+  p.vn_st = vn_strides[1];
+  p.vn_sh = vn_strides[2];
+  p.k_cache = static_cast<uint16_t *>(k_cache);
+  p.v_cache = static_cast<uint16_t *>(v_cache);
+  p.k_sb = k_strides[0];
+  p.k_ss = k_strides[1];
+  p.k_sh = k_strides[2];
+  p.v_sb = v_strides[0];
+  p.v_ss = v_strides[1];
+  p.v_sh = v_strides[2];
+  p.num_blocks = num_blocks;
+  p.block_table = block_table;
+  p.bt_stride = bt_stride;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.seqlens = seqlens;
+  p.batch = batch;
+  p.n_new = n_new;
+  p.Hkv = Hkv;
+  p.chunks = D / 8;
+  p.block_shift = log2i(block_size);
+  p.err = err;
+  const int64_t total = static_cast<int64_t>(batch) * n_new * Hkv * (D / 8);
+  const int64_t want = ceil_div(total, 256);
+  const int64_t cap = static_cast<int64_t>(sm_count(dev)) * 8;
+  const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
+  pkv::kv_append_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int pkv_paged_decode_attn(const void *q, const int64_t q_strides[3], const void *k_cache,
+                          const int64_t k_strides[3], const void *v_cache,
+                          const int64_t v_strides[3], int64_t num_blocks,
+                          const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                          const int32_t *seqlens, int max_seqlen_k, int batch, int seqlen_q,
+                          int Hq, int Hkv, int D, int block_size, float scale, int causal,
+                          void *out, const int64_t out_strides[3], float *lse, void *workspace,
+                          size_t workspace_bytes, int32_t *err, void *stream) {
+  return attn_entry(q, q_strides, k_cache, k_strides, v_cache, v_strides, num_blocks, block_table,
+                    bt_stride, max_blocks_per_seq, seqlens, max_seqlen_k, batch, seqlen_q, Hq, Hkv,
+                    D, block_size, scale, causal, out, out_strides, lse, workspace,
+                    workspace_bytes, err, stream);
+}
+
+int pkv_paged_prefill_attn(const void *q, const int64_t q_strides[3], const void *k_cache,
+                           const int64_t k_strides[3], const void *v_cache,
+                           const int64_t v_strides[3], int64_t num_blocks,
+                           const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                           const int32_t *seqlens, int max_seqlen_k, int batch, int seqlen_q,
+                           int Hq, int Hkv, int D, int block_size, float scale, int causal,
+                           void *out, const int64_t out_strides[3], float *lse, void *workspace,
+                           size_t workspace_bytes, int32_t *err, void *stream) {
+  return attn_entry(q, q_strides, k_cache, k_strides, v_cache, v_strides, num_blocks, block_table,
+                    bt_stride, max_blocks_per_seq, seqlens, max_seqlen_k, batch, seqlen_q, Hq, Hkv,
+                    D, block_size, scale, causal, out, out_strides, lse, workspace,
+                    workspace_bytes, err, stream);
+}
+
+size_t pkv_workspace_size(int batch, int seqlen_q, int Hq, int D, int max_seqlen_k) {
+  if (batch <= 0 || seqlen_q <= 0 || Hq <= 0 || D <= 0 || max_seqlen_k < 0) return 0;
+  return ws_bytes(batch, seqlen_q, Hq, D, max_seqlen_k);
+}
+
+const char *pkv_strerror(int code) {
+  switch (code) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_ARG: return "invalid argument (size, stride, alignment or pointer)";
+    case PKV_ERR_WORKSPACE: return "workspace missing, misaligned or smaller than pkv_workspace_size()";
+    case PKV_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
+    case PKV_ERR_LAYOUT: return "cache strides cannot be described to the TMA unit";
+    default: return "unknown pagedkv status";
+  }
+}
+
+int pkv_split_tokens(void) { return PKV_SPLIT_TOKENS; }
+
+}  // extern "C"

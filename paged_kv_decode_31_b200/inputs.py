@@ -69,6 +69,14 @@ class PagedCache:
         v = self.backing[1].to(device)
         return PagedCache(k, v, (k, v), self.layout)
 
+    def clone(self) -> "PagedCache":
+        """A deep copy with the same layout (same device)."""
+        if self.layout == "interleaved":
+            kv = self.backing[0].clone()
+            return PagedCache(kv[:, 0], kv[:, 1], (kv,), self.layout)
+        k, v = self.k.clone(), self.v.clone()
+        return PagedCache(k, v, (k, v), self.layout)
+
     def as_contiguous(self) -> "PagedCache":
         """The same data in a contiguous two-buffer layout (bitwise copy)."""
         k = self.k.contiguous().clone()

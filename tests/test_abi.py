@@ -1,0 +1,125 @@
+"""The C ABI without a GPU: libpagedkv.so builds, loads, exports every
+function include/pagedkv.h declares, and rejects bad arguments before any CUDA
+call (so none of these tests launches anything)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_decode_31_b200 import binding
+from paged_kv_decode_31_b200 import build as pkv_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pkv_build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", text)))
+
+
+def header_macros():
+    return dict((k, int(v)) for k, v in re.findall(r"#define\s+(PKV_\w+)\s+(-?\d+)", open(HEADER).read()))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"pkv_kv_append", "pkv_paged_decode_attn", "pkv_paged_prefill_attn",
+            "pkv_workspace_size", "pkv_strerror"} <= set(names)
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in pagedkv.h but not exported"
+
+
+def test_constants_agree_with_header(lib):
+    m = header_macros()
+    assert lib.pkv_split_tokens() == m["PKV_SPLIT_TOKENS"] == binding.SPLIT_TOKENS
+    assert m["PKV_TILE_TOKENS"] == binding.TILE_TOKENS
+    assert m["PKV_DEVERR_BAD_BLOCK"] == binding.DEVERR_BAD_BLOCK
+    assert m["PKV_DEVERR_TABLE_WIDTH"] == binding.DEVERR_TABLE_WIDTH
+    assert m["PKV_DEVERR_TIMEOUT"] == binding.DEVERR_TIMEOUT
+
+
+def test_strerror_covers_every_status(lib):
+    m = header_macros()
+    for key in ("PKV_OK", "PKV_ERR_ARG", "PKV_ERR_WORKSPACE", "PKV_ERR_CUDA", "PKV_ERR_LAYOUT"):
+        s = binding.strerror(m[key])
+        assert s and s != "unknown pagedkv status"
+    assert binding.strerror(12345) == "unknown pagedkv status"
+
+
+def test_workspace_size_formula(lib):
+    # fp32 acc[D] per (row, split), padded to 256 B, then (m, l) per (row, split)
+    rows, S, D = 4 * 1 * 32, 131072 // 4096, 128
+    acc = rows * S * D * 4
+    acc = (acc + 255) // 256 * 256
+    assert binding.workspace_size(4, 1, 32, 128, 131072) == acc + rows * S * 2 * 4
+    assert binding.workspace_size(1, 1, 1, 64, 0) == 256 + 8
+    assert binding.workspace_size(0, 1, 1, 64, 10) == 0
+
+
+def _attn_args(**over):
+    """Arguments of pkv_paged_decode_attn with plausible (never dereferenced)
+    pointers; `over` replaces fields by name."""
+    st = (ctypes.c_int64 * 3)(2048, 2048, 128)
+    kst = (ctypes.c_int64 * 3)(16 * 8 * 128, 8 * 128, 128)
+    ost = (ctypes.c_int64 * 3)(4096, 4096, 128)
+    a = dict(q=0x10000, q_st=st, k=0x20000, k_st=kst, v=0x30000, v_st=kst, num_blocks=64,
+             table=0x40000, bt_stride=16, max_blocks=16, seqlens=0x50000, max_seqlen_k=256,
+             batch=2, sq=1, Hq=32, Hkv=8, D=128, bs=16, scale=0.088, causal=0,
+             out=0x60000, o_st=ost, lse=0x70000, ws=0x80000, ws_bytes=1 << 30, err=None,
+             stream=None)
+    a.update(over)
+    return list(a.values())
+
+
+@pytest.mark.parametrize("over", [
+    dict(D=96), dict(Hq=30), dict(bs=24), dict(bs=8), dict(bs=512), dict(batch=0),
+    dict(sq=0), dict(num_blocks=0), dict(max_blocks=0), dict(bt_stride=4),
+    dict(q=0x10008), dict(k=0x20002), dict(scale=0.0), dict(scale=float("nan")),
+    dict(q=None), dict(max_seqlen_k=-1),
+    dict(k_st=(ctypes.c_int64 * 3)(16 * 8 * 128, 8 * 128, 100)),
+])
+def test_invalid_arguments_rejected_before_any_launch(lib, over):
+    rc = lib.pkv_paged_decode_attn(*_attn_args(**over))
+    assert rc == header_macros()["PKV_ERR_ARG"]
+    rc = lib.pkv_paged_prefill_attn(*_attn_args(**over))
+    assert rc == header_macros()["PKV_ERR_ARG"]
+
+
+def test_small_workspace_rejected_before_any_launch(lib):
+    rc = lib.pkv_paged_decode_attn(*_attn_args(ws_bytes=100))
+    assert rc == header_macros()["PKV_ERR_WORKSPACE"]
+    rc = lib.pkv_paged_decode_attn(*_attn_args(ws=None))
+    assert rc == header_macros()["PKV_ERR_WORKSPACE"]
+
+
+def test_kv_append_rejects_bad_arguments(lib):
+    st = (ctypes.c_int64 * 3)(1024, 1024, 128)
+    kst = (ctypes.c_int64 * 3)(16 * 8 * 128, 8 * 128, 128)
+    good = [0x10000, st, 0x20000, st, 0x30000, kst, 0x40000, kst, 64, 0x50000, 16, 16,
+            0x60000, 2, 1, 8, 128, 16, None, None]
+    for idx, bad in ((16, 96), (17, 20), (13, 0), (14, -1), (8, 0), (0, 0x10004)):
+        args = list(good)
+        args[idx] = bad
+        assert lib.pkv_kv_append(*args) == header_macros()["PKV_ERR_ARG"], (idx, bad)
+    args = list(good)
+    args[14] = 0                                     # n_new = 0: nothing to do
+    assert lib.pkv_kv_append(*args) == 0
+
+
+def test_product_path_has_no_cpu_fallback():
+    """The binding loads only the CUDA library; it never imports the oracle."""
+    import paged_kv_decode_31_b200 as pkg
+    pkg_dir = os.path.dirname(pkg.__file__)
+    for fn in os.listdir(pkg_dir):
+        if fn.endswith(".py"):
+            src = open(os.path.join(pkg_dir, fn)).read()
+            assert "import oracle" not in src and "from oracle" not in src, fn

@@ -1,0 +1,160 @@
+"""GPU parity of the CUDA path against the CPU fp64 oracle, through the C ABI.
+
+Grid: the aiter test "test(triton/decode): pin non-contiguous paged KV block
+stride" (mha/gqa x causal x block_size {16, 256} x (seqlen_q, seqlen_k) in
+{(1, 339), (3, 1024), (17, 156)} x D {64, 128}, batch 2, Hq 6, Hkv 3 for gqa),
+on the interleaved non-contiguous cache with every unused slot NaN, through
+both entry points.  Edge cases: one-token contexts, split boundaries, rows with
+no visible key, empty sequences, many splits with a ragged tail.
+"""
+import pytest
+import torch
+
+import paged_kv_decode_31_b200 as pkv
+from paged_kv_decode_31_b200 import inputs as I
+
+from gpu_helpers import assert_close_to_oracle, oracle_of, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+GRID = [(mha, causal, bs, sqk, d)
+        for mha in ("mha", "gqa") for causal in (False, True) for bs in (16, 256)
+        for sqk in ((1, 339), (3, 1024), (17, 156)) for d in (64, 128)]
+
+
+def test_tiny_config_matches_oracle():
+    di = I.config_tiny()
+    assert not di.cache.k.is_contiguous() and di.cache.k.stride(0) == 2 * 16 * 2 * 64
+    out, lse = run_gpu(di)
+    ref_out, ref_lse = oracle_of(di)
+    assert_close_to_oracle(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("entry", ["decode", "prefill"])
+@pytest.mark.parametrize("mha,causal,bs,sqk,d", GRID)
+def test_p2_grid_matches_oracle(mha, causal, bs, sqk, d, entry):
+    sq, sk = sqk
+    Hkv = 6 if mha == "mha" else 3
+    di = I.p2_case(2, sq, sk, 6, Hkv, d, bs, causal=causal, layout="interleaved",
+                   seed=hash((mha, causal, bs, sq, d)) % 1000, poison=True)
+    fn = pkv.paged_decode_attn if entry == "decode" else pkv.paged_prefill_attn
+    out, lse = run_gpu(di, entry=fn)
+    ref_out, ref_lse = oracle_of(di)
+    assert_close_to_oracle(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("seqlens", [[1, 1], [4096, 4095], [4097, 8192], [8193, 129],
+                                     [12345, 3], [0, 5]])
+@pytest.mark.parametrize("d", [64, 128])
+def test_split_boundaries_and_edge_lengths(seqlens, d):
+    di = I.p2_case(2, 1, max(max(seqlens), 1), 8, 2, d, 16, causal=False, layout="contiguous",
+                   seed=sum(seqlens) % 997, seqlens=seqlens, poison=True)
+    out, lse = run_gpu(di)
+    ref_out, ref_lse = oracle_of(di)
+    assert_close_to_oracle(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("sq,n", [(17, 5), (40, 40), (3, 2), (64, 4097)])
+def test_causal_rows_without_keys_and_long_multi_query(sq, n):
+    di = I.p2_case(2, sq, n, 4, 1, 128, 16, causal=True, layout="interleaved", seed=sq + n,
+                   seqlens=[n, max(n - 1, 1)], poison=True)
+    out, lse = run_gpu(di, entry=pkv.paged_prefill_attn)
+    ref_out, ref_lse = oracle_of(di)
+    assert_close_to_oracle(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+def test_query_group_sizes(G):
+    Hkv = 2
+    di = I.p2_case(3, 1, 700, G * Hkv, Hkv, 128, 32, causal=False, layout="interleaved",
+                   seed=G, poison=True)
+    out, lse = run_gpu(di)
+    ref_out, ref_lse = oracle_of(di)
+    assert_close_to_oracle(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("bs", [16, 32, 64, 128, 256])
+def test_block_sizes(bs):
+    di = I.p2_case(2, 2, 1500, 8, 4, 128, bs, causal=True, layout="interleaved", seed=bs,
+                   poison=True)
+    out, lse = run_gpu(di)
+    ref_out, ref_lse = oracle_of(di)
+    assert_close_to_oracle(out, lse, ref_out, ref_lse)
+
+
+def test_head_major_cache_layout():
+    """A cache laid out [num_blocks, Hkv, block_size, D] (head stride larger
+    than slot stride) viewed as [num_blocks, block_size, Hkv, D]."""
+    di = I.p2_case(2, 1, 600, 8, 4, 128, 16, causal=False, layout="contiguous", seed=21,
+                   poison=True)
+    k_hm = di.cache.k.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+    v_hm = di.cache.v.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+    assert k_hm.stride(2) > k_hm.stride(1)
+    di2 = I.DecodeInputs(di.q, I.PagedCache(k_hm, v_hm, (k_hm, v_hm), "contiguous"),
+                         di.block_table, di.seqlens, di.Hq, di.Hkv, di.D, di.scale, di.causal)
+    out, lse = run_gpu(di2)
+    ref_out, ref_lse = oracle_of(di)
+    assert_close_to_oracle(out, lse, ref_out, ref_lse)
+
+
+def test_strided_query_and_output():
+    """q taken from a fused [B, s, (Hq + 2 Hkv) * D] projection output, out
+    written into a wider buffer: only the strides change."""
+    di = I.p2_case(2, 3, 300, 8, 2, 128, 16, causal=True, layout="interleaved", seed=22)
+    qkv = torch.zeros(2, 3, 12, 128, dtype=torch.bfloat16)
+    qkv[:, :, :8] = di.q
+    d = di.to("cuda")
+    q_view = qkv.cuda()[:, :, :8]
+    assert not q_view.is_contiguous()
+    out_buf = torch.full((2, 3, 10, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    out_view = out_buf[:, :, 1:9]
+    lse = torch.empty(2, 8, 3, dtype=torch.float32, device="cuda")
+    pkv.paged_decode_attn(q_view, d.cache.k, d.cache.v, d.block_table, d.seqlens,
+                          max_seqlen_k=300, scale=di.scale, causal=True, out=out_view, lse=lse)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = oracle_of(di)
+    out = out_buf.cpu()
+    assert torch.all(out[:, :, 0] == 7.0) and torch.all(out[:, :, 9] == 7.0)
+    assert_close_to_oracle(out[:, :, 1:9].contiguous(), lse.cpu(), ref_out, ref_lse)
+
+
+def test_argument_errors_raise_and_launch_nothing():
+    di = I.p2_case(1, 1, 64, 4, 2, 128, 16, causal=False, seed=23).to("cuda")
+    with pytest.raises(pkv.PagedKVError):  # workspace too small
+        pkv.paged_decode_attn(di.q, di.cache.k, di.cache.v, di.block_table, di.seqlens,
+                              max_seqlen_k=64, workspace=torch.empty(16, dtype=torch.uint8,
+                                                                     device="cuda"))
+    with pytest.raises(pkv.PagedKVError):  # Hq % Hkv != 0
+        q3 = torch.zeros(1, 1, 3, 128, dtype=torch.bfloat16, device="cuda")
+        pkv.paged_decode_attn(q3, di.cache.k, di.cache.v, di.block_table, di.seqlens,
+                              max_seqlen_k=64)
+    with pytest.raises(pkv.PagedKVError):  # head_dim 96
+        kc = torch.zeros(8, 16, 2, 96, dtype=torch.bfloat16, device="cuda")
+        q96 = torch.zeros(1, 1, 4, 96, dtype=torch.bfloat16, device="cuda")
+        pkv.paged_decode_attn(q96, kc, kc, di.block_table, di.seqlens, max_seqlen_k=64)
+
+
+def test_bad_block_ids_set_the_error_flag_and_do_not_fault():
+    di = I.p2_case(2, 1, 300, 4, 2, 128, 16, causal=False, seed=24, seqlens=[300, 200])
+    di.block_table[0, 3] = di.cache.num_blocks + 100
+    di.block_table[1, 5] = -7
+    d = di.to("cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.paged_decode_attn(d.q, d.cache.k, d.cache.v, d.block_table, d.seqlens, max_seqlen_k=300,
+                          err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & pkv.binding.DEVERR_BAD_BLOCK
+    # the context is still usable
+    out, lse = run_gpu(I.config_tiny())
+    assert torch.isfinite(out.float()).all()
+
+
+def test_table_too_narrow_sets_the_error_flag():
+    di = I.p2_case(1, 1, 300, 4, 2, 128, 16, causal=False, seed=25, seqlens=[300])
+    d = di.to("cuda")
+    narrow = d.block_table[:, :10].contiguous()        # covers 160 tokens only
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.paged_decode_attn(d.q, d.cache.k, d.cache.v, narrow, d.seqlens, max_seqlen_k=300,
+                          err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & pkv.binding.DEVERR_TABLE_WIDTH
