@@ -58,6 +58,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--context", type=int, default=131072,
+                    help="tokens per sequence (a smaller workload for profiling captures)")
+    ap.add_argument("--batch", type=int, default=4)
     return ap.parse_args()
 
 
@@ -189,7 +192,8 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    di = I.config_long_context(seed=1000 + rank, device=dev)
+    di = I.config_long_context(seed=1000 + rank, device=dev, batch=args.batch,
+                               seqlen=args.context)
     B, ctx, Hq, Hkv, D = di.batch, int(di.seqlens[0].item()), di.Hq, di.Hkv, di.D
     gen = torch.Generator(device=dev).manual_seed(2000 + rank)
     k_new = torch.randn(B, 1, Hkv, D, generator=gen, device=dev).to(torch.bfloat16)
@@ -331,6 +335,9 @@ def run_ours(args):
         "clocks": clocks.summary(),
         "e2e": e2e,
     }
+    if (args.context, args.batch) != (131072, 4):
+        result["config"]["workload"] = (f"profiling size: batch {B}, context {ctx} "
+                                        "(otherwise as the long-context workload)")
     if not args.no_cpu_baseline and world == 1:
         result["cpu_baseline"] = cpu_baseline(di)
     print(json.dumps(result), flush=True)
