@@ -177,6 +177,47 @@ const char *pkv_strerror(int code);
 /* PKV_SPLIT_TOKENS, for bindings that cannot read the macro. */
 int pkv_split_tokens(void);
 
+/*
+ * pkv_paged_decode_attn_static_ws: pkv_paged_decode_attn for callers that
+ * cannot allocate device memory when they call, and have no buffer to lend as
+ * workspace -- for example a host framework that owns the whole device-memory
+ * budget and forbids cudaMalloc after start-up, or a latency-bound serving
+ * loop that cannot afford cudaMalloc's implicit device synchronisation.  The
+ * pages have no counterpart of this call; it exists only for such callers.
+ *
+ * Same arguments and results as pkv_paged_decode_attn, minus the workspace:
+ * the split partials go to a scratch array of PKV_STATIC_WORKSPACE_BYTES that
+ * the library keeps in device memory (a file-scope __device__ array, so every
+ * GPU that loads the library holds it until the process exits).  The call
+ * itself allocates nothing.
+ *
+ * - Limit: returns PKV_ERR_WORKSPACE, launching nothing, when
+ *   pkv_workspace_size(batch, seqlen_q, Hq, D, max_seqlen_k) exceeds
+ *   PKV_STATIC_WORKSPACE_BYTES.
+ * - Set-up: the first call on each device (with that device current) looks up
+ *   the array's device address once; make that first call before any stream
+ *   capture begins.  A failed look-up returns PKV_ERR_CUDA.
+ * - Sharing: every call on a device uses the same array and leaves its
+ *   partials there.  Nothing in it needs to start at zero (each call writes
+ *   every partial it reads), but two calls whose kernels overlap on the GPU --
+ *   on different streams, or from different host threads -- race on it and
+ *   give undefined results.  Serialise them (one stream) or use
+ *   pkv_paged_decode_attn with a workspace per stream.
+ */
+#define PKV_STATIC_WORKSPACE_BYTES (8u << 20)
+
+int pkv_paged_decode_attn_static_ws(const void *q, const int64_t q_strides[3],
+                                    const void *k_cache, const int64_t k_strides[3],
+                                    const void *v_cache, const int64_t v_strides[3],
+                                    int64_t num_blocks,
+                                    const int32_t *block_table, int64_t bt_stride,
+                                    int max_blocks_per_seq,
+                                    const int32_t *seqlens, int max_seqlen_k,
+                                    int batch, int seqlen_q, int Hq, int Hkv, int D,
+                                    int block_size, float scale, int causal,
+                                    void *out, const int64_t out_strides[3], float *lse,
+                                    int32_t *err, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

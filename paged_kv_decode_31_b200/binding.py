@@ -178,3 +178,43 @@ def paged_prefill_attn(q, k_cache, v_cache, block_table, seqlens, *, max_seqlen_
     """Causal or chunked prefill over the paged cache; same contract as decode."""
     return _attn("pkv_paged_prefill_attn", q, k_cache, v_cache, block_table, seqlens,
                  max_seqlen_k, scale, causal, out, lse, workspace, err, stream)
+
+
+# Allocation-free decode (see pkv_paged_decode_attn_static_ws in pagedkv.h).
+STATIC_WORKSPACE_BYTES = 8 << 20
+
+
+def paged_decode_attn_static_ws(q, k_cache, v_cache, block_table, seqlens, *, max_seqlen_k,
+                                scale=None, causal=False, out, lse, err=None, stream=None):
+    """Decode attention whose scratch lives in a device array the library owns,
+    for callers that cannot allocate device memory when they call: the caller
+    passes every input and output (out, lse, and max_seqlen_k as a host int),
+    and nothing is allocated here or in the library.  Calls on one device
+    share that array, so calls that overlap on the GPU race; serialise them.
+    The first call on a device looks up the array's address: make it before
+    any stream capture."""
+    L = lib()
+    fn = L.pkv_paged_decode_attn_static_ws
+    if not fn.argtypes:
+        fn.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _P, _I64, _I, _P, _I,
+                       _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P, _P, _P, _P, _P]
+        fn.restype = _I
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("out", out)):
+        _need_cuda_bf16(name, t)
+    _need_cuda_i32("block_table", block_table)
+    _need_cuda_i32("seqlens", seqlens)
+    B, sq, Hq, D = q.shape
+    num_blocks, bs, Hkv, _ = k_cache.shape
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, sq):
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, seqlen_q] tensor")
+    need = workspace_size(B, sq, Hq, D, max_seqlen_k)
+    if need > STATIC_WORKSPACE_BYTES:
+        raise PagedKVError(f"this problem needs {need} bytes of scratch; the library's static "
+                           f"workspace holds {STATIC_WORKSPACE_BYTES} (use paged_decode_attn)")
+    rc = fn(q.data_ptr(), _st3(q), k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(),
+            _st3(v_cache), num_blocks, block_table.data_ptr(), int(block_table.stride(0)),
+            int(block_table.shape[1]), seqlens.data_ptr(), int(max_seqlen_k), B, sq, Hq, Hkv, D,
+            bs, float(1.0 / math.sqrt(D) if scale is None else scale), int(bool(causal)),
+            out.data_ptr(), _st3(out), lse.data_ptr(), _ptr(err), _stream_handle(stream))
+    _check("pkv_paged_decode_attn_static_ws", rc)
+    return out, lse

@@ -365,3 +365,58 @@ const char *pkv_strerror(int code) {
 int pkv_split_tokens(void) { return PKV_SPLIT_TOKENS; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode: scratch in a library-owned device array.
+// ---------------------------------------------------------------------------
+// For callers that may not allocate device memory at call time (see
+// pkv_paged_decode_attn_static_ws in pagedkv.h).  In host code
+// g_static_workspace is only a host-side stand-in for the device array: its
+// device address comes from cudaGetSymbolAddress, once per device, and only
+// that address is handed to the kernels.
+static __device__ __align__(256) unsigned char g_static_workspace[PKV_STATIC_WORKSPACE_BYTES];
+
+namespace {
+
+void *static_workspace_address(int dev) {
+  static std::mutex mu;
+  static void *addr[kMaxDevices] = {};
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || !p) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int pkv_paged_decode_attn_static_ws(const void *q, const int64_t q_strides[3],
+                                    const void *k_cache, const int64_t k_strides[3],
+                                    const void *v_cache, const int64_t v_strides[3],
+                                    int64_t num_blocks, const int32_t *block_table,
+                                    int64_t bt_stride, int max_blocks_per_seq,
+                                    const int32_t *seqlens, int max_seqlen_k, int batch,
+                                    int seqlen_q, int Hq, int Hkv, int D, int block_size,
+                                    float scale, int causal, void *out,
+                                    const int64_t out_strides[3], float *lse, int32_t *err,
+                                    void *stream) {
+  if (batch <= 0 || seqlen_q <= 0 || Hq <= 0 || (D != 64 && D != 128) || max_seqlen_k < 0)
+    return PKV_ERR_ARG;
+  if (ws_bytes(batch, seqlen_q, Hq, D, max_seqlen_k) > PKV_STATIC_WORKSPACE_BYTES)
+    return PKV_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  void *ws = static_workspace_address(dev);
+  if (!ws) return PKV_ERR_CUDA;
+  return attn_entry(q, q_strides, k_cache, k_strides, v_cache, v_strides, num_blocks, block_table,
+                    bt_stride, max_blocks_per_seq, seqlens, max_seqlen_k, batch, seqlen_q, Hq, Hkv,
+                    D, block_size, scale, causal, out, out_strides, lse, ws,
+                    PKV_STATIC_WORKSPACE_BYTES, err, stream);
+}
+
+}  // extern "C"
