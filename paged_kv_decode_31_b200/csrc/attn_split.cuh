@@ -20,23 +20,24 @@
 //            N = rows, K = head_dim, fp32 accumulation in TMEM);
 //   softmax  one thread per token: mask (key < row limit), scale to base 2,
 //            column max over the 128 tokens (exact, order-free), running max,
-//            p = 2^(s - m) stored as P^T in two bf16 parts, hi = bf16(p) and
-//            lo = bf16(p - hi), so the tensor cores see p to ~16 bits;
-//   O^T      = V^T * (P_hi + P_lo)^T and L = 1 * (P_hi + P_lo)^T on the tensor
-//            cores (fresh accumulators each tile): the weighted values and the
-//            row sums of the very weights used;
-//   update   acc = fma(acc, alpha, O), l = fma(l, alpha, L), alpha = 2^(m_old - m_new),
-//            skipped for rows the tile does not reach.
+//            p = 2^(s - m); P^T holds p as two bf16 parts side by side, hi =
+//            bf16(p) and lo = bf16(p - hi), so the tensor cores see p to ~16
+//            bits; the fp32 p of each row are summed in one fixed shuffle tree;
+//   O^T      = V^T * [P_hi | P_lo]^T on the tensor cores (fresh accumulator
+//            each tile), O = O_hi + O_lo;
+//   update   acc = fma(acc, alpha, O), l = fma(l, alpha, sum p), alpha =
+//            2^(m_old - m_new), skipped for rows the tile does not reach.
 // Tiles start at absolute multiples of 128 and rows never influence each
 // other, so a row's arithmetic depends only on its own query, its visible
 // keys and the fixed constants: decode row t and prefill row t, batch 1 and
 // batch N, contiguous and interleaved caches all give the same bits.
 //
-// Roles (192 threads): warps 0-3 softmax + correction + epilogue (thread t =
-// TMEM lane t = token t of the tile = output column d), warp 4 TMA producer
-// (+ Q staging), warp 5 MMA issuer (+ TMEM owner).  The kernel is persistent:
-// CTA k takes units k, k + gridDim.x, ...; the producer and the MMA issuer
-// run ahead across unit boundaries.
+// Roles (224 threads): warps 0-3 softmax + correction + epilogue (thread t =
+// TMEM lane t = token t of the tile = output column d), warp 4 K producer
+// (+ Q staging), warp 5 V producer, warp 6 MMA issuer (+ TMEM owner).  K and V
+// have their own stage rings, so a K stage is refilled as soon as its S^T is
+// computed.  The kernel is persistent: CTA k takes units k, k + gridDim.x,
+// ...; producers and the MMA issuer run ahead across unit boundaries.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -47,9 +48,10 @@ namespace pkv {
 
 constexpr int kSplitTokens = 4096;
 constexpr int kTileTokens = 128;
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kThreads = 224;  // 7 warps
+constexpr int kKWarp = 4;      // K producer (+ Q staging)
+constexpr int kVWarp = 5;      // V producer
+constexpr int kMmaWarp = 6;    // MMA issuer + TMEM owner
 
 constexpr int kErrBadBlock = 1;
 constexpr int kErrTableWidth = 2;
@@ -92,6 +94,32 @@ __device__ __forceinline__ bool softmax_bar_or(bool pred) {
   return r != 0;
 }
 
+// Cross-lane reductions over the 32 tokens of a warp, four columns at a time
+// so the shuffles of the four columns overlap.  Each column's tree is fixed.
+// Maximum: xor butterfly (max is exact, every lane ends with the same value).
+__device__ __forceinline__ void warp_max4(float (&v)[4]) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    float o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = __shfl_xor_sync(0xffffffffu, v[i], off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = fmaxf(v[i], o[i]);
+  }
+}
+
+// Sum: shift-down tree; lane 0 holds the result.
+__device__ __forceinline__ void warp_sum4_lane0(float (&v)[4]) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    float o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = __shfl_down_sync(0xffffffffu, v[i], off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __fadd_rn(v[i], o[i]);
+  }
+}
+
 // Shared-memory plan.  Every operand region is 1024-byte aligned (the 128-byte
 // swizzle pattern repeats every 8 rows of 128 bytes).
 template <int D, int N, int NS, int QB>
@@ -101,30 +129,33 @@ struct Cfg {
   static_assert(QB == 1 || QB == 2, "Q buffers");
   static constexpr int kHalfBytes = kTileTokens * 128;   // 128 tokens x 64 head_dim x bf16
   static constexpr int kKVBytes = (D / 64) * kHalfBytes;  // one K (or V) tile
-  static constexpr int kStageBytes = 2 * kKVBytes;        // K tile then V tile
   static constexpr int kQHalfBytes = N * 128;
   static constexpr int kQBytes = (D / 64) * kQHalfBytes;
-  static constexpr int kPBytes = kTileTokens * N * 2;     // one bf16 P^T (hi or lo part)
-  static constexpr int kPKGroup = (N / 8) * 128;          // P^T stride between 8-token groups
-  static constexpr int kOnesBytes = 4096;                 // 128 x 16 bf16 ones
-  static constexpr int kOffStage = 0;
-  static constexpr int kOffQ = NS * kStageBytes;
-  static constexpr int kOffP = kOffQ + QB * kQBytes;      // 2 buffers x (hi, lo)
-  static constexpr int kOffOnes = kOffP + 4 * kPBytes;
-  static constexpr int kOffSmall = kOffOnes + kOnesBytes;
+  static constexpr int kPCols = 2 * N;                    // P^T columns: N hi, then N lo
+  static constexpr int kPBytes = kTileTokens * kPCols * 2;
+  static constexpr int kPKGroup = (kPCols / 8) * 128;     // P^T stride between 8-token groups
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = NS * kKVBytes;
+  static constexpr int kOffQ = 2 * NS * kKVBytes;
+  static constexpr int kOffP = kOffQ + QB * kQBytes;
+  static constexpr int kOffSmall = kOffP + 2 * kPBytes;
   struct Small {
-    uint64_t full[NS], empty[NS];
+    uint64_t full_k[NS], empty_k[NS], full_v[NS], empty_v[NS];
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
     uint64_t q_full[QB], q_empty[QB], drain;
     uint32_t tmem_base;
     int abort_any;
-    float wmax[4][N];
+    __align__(16) float wmax[4][N];
+    __align__(16) float wsum[2][4][N];
     float mnew[2][N];
     float alpha[2][N];
     int skip[2][N];
     int lim[N];
+    int tab_k[kSplitTokens / 16];  // block-table entries of each producer's current split
+    int tab_v[kSplitTokens / 16];
   };
   static constexpr int kSmemBytes = kOffSmall + static_cast<int>(sizeof(Small)) + 1024;
+  // TMEM: S^T (N columns) x 2 buffers, then O^T (hi and lo, 2N columns) x 2 buffers
   static constexpr int kTmemCols = (6 * N <= 128) ? 128 : (6 * N <= 256) ? 256 : 512;
 };
 
@@ -162,71 +193,30 @@ __device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
   return x;
 }
 
+// One producer warp: stages the split's block-table entries in `tab` (all
+// lanes), then per tile lane k issues the TMA boxes of the tile's k-th box of
+// cache rows into the ring `dst`, lane 0 arrives on `full`.  With `stage_q`
+// the warp also stages each unit's Q rows (the B operand of S^T = K Q^T).
 template <int D, int N, int NS, int QB>
-__global__ void __launch_bounds__(kThreads, 1)
-    attn_split_kernel(const __grid_constant__ AttnParams p,
-                      const __grid_constant__ CUtensorMap map_k,
-                      const __grid_constant__ CUtensorMap map_v) {
+__device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *map, uint8_t *smem,
+                                        typename Cfg<D, N, NS, QB>::Small *sm, uint64_t *full,
+                                        uint64_t *empty, int *tab, uint32_t dst_off, bool stage_q,
+                                        int lane, volatile int *abort_any) {
   using C = Cfg<D, N, NS, QB>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  auto *sm = reinterpret_cast<typename C::Small *>(smem + C::kOffSmall);
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  volatile int *abort_any = &sm->abort_any;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&sm->full[i], 1);
-      mbar_init(&sm->empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm->s_full[i], 1);
-      mbar_init(&sm->p_full[i], 128);
-      mbar_init(&sm->o_full[i], 1);
-      mbar_init(&sm->o_free[i], 128);
-    }
-    for (int i = 0; i < QB; ++i) {
-      mbar_init(&sm->q_full[i], 1);
-      mbar_init(&sm->q_empty[i], 1);
-    }
-    mbar_init(&sm->drain, 1);
-    sm->abort_any = 0;
-    fence_barrier_init();
-  }
-  {  // the all-ones A operand that turns the row sum of P into an MMA
-    uint4 ones = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-    for (int i = threadIdx.x; i < C::kOnesBytes / 16; i += kThreads)
-      reinterpret_cast<uint4 *>(smem + C::kOffOnes)[i] = ones;
-    fence_proxy_async_smem();
-  }
-  if (warp == kMmaWarp) tmem_alloc(&sm->tmem_base, C::kTmemCols);
-  tc_fence_before_sync();
-  __syncthreads();
-  tc_fence_after_sync();
-  const uint32_t tmem = sm->tmem_base;
-  const uint32_t sbase = smem_u32(smem);
-
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------------
-    // Producer: Q rows of each unit (all 32 lanes), K/V tiles via TMA (lane 0)
-    // ------------------------------------------------------------------
-    if (lane == 0) {
-      tma_prefetch_desc(&map_k);
-      tma_prefetch_desc(&map_v);
-    }
-    int gi = 0, ui = 0;
-    bool failed = false;
-    int last_gi[NS];
+  constexpr int kPastWidth = static_cast<int>(0x80000000u);
+  if (lane == 0) tma_prefetch_desc(map);
+  int gi = 0, ui = 0;
+  bool failed = false;
+  int last_gi[NS];
 #pragma unroll
-    for (int i = 0; i < NS; ++i) last_gi[i] = -1;
-    const int R = p.G * p.seqlen_q;
-    for (int u = blockIdx.x; u < p.n_units && !failed; u += gridDim.x) {
-      const Unit x = unit_at<N>(p, u);
-      if (x.n_tiles == 0) continue;
+  for (int i = 0; i < NS; ++i) last_gi[i] = -1;
+  const int bmask = (1 << p.block_shift) - 1;
+  for (int u = blockIdx.x; u < p.n_units && !failed; u += gridDim.x) {
+    const Unit x = unit_at<N>(p, u);
+    if (x.n_tiles == 0) continue;
+    if (stage_q) {
       const int qb = ui % QB;
-      bool ok = mbar_wait(&sm->q_empty[qb], ((ui / QB) & 1) ^ 1, abort_any);
+      const bool ok = mbar_wait(&sm->q_empty[qb], ((ui / QB) & 1) ^ 1, abort_any);
       if (__any_sync(0xffffffffu, !ok)) {
         failed = true;
         break;
@@ -245,100 +235,148 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = ch >> 3, cc = ch & 7;
         *reinterpret_cast<uint4 *>(qdst + h * C::kQHalfBytes + c * 128 + ((cc ^ (c & 7)) << 4)) = v;
       }
-      (void)R;
       fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sm->q_full[qb]);
-        for (int j = 0; j < x.n_tiles; ++j, ++gi) {
-          const int st = gi % NS;
-          if (!mbar_wait(&sm->empty[st], ((gi / NS) & 1) ^ 1, abort_any)) {
-            failed = true;
-            break;
-          }
-          const int tok0 = x.tok0 + j * kTileTokens;
-          const int nvalid = min(kTileTokens, x.lim_max - tok0);
-          uint8_t *kdst = smem + C::kOffStage + st * C::kStageBytes;
-          uint8_t *vdst = kdst + C::kKVBytes;
-          int errs = 0;
-          for (int k = 0; k * p.box_slots < nvalid; ++k) {
-            const int tok = tok0 + k * p.box_slots;
-            const int bi = tok >> p.block_shift;
-            const int slot = tok & ((1 << p.block_shift) - 1);
-            if (bi >= p.max_blocks_per_seq) {
-              errs |= kErrTableWidth;
-              continue;
-            }
-            const int blk = __ldg(p.block_table + x.b * p.bt_stride + bi);
-            if (blk < 0 || static_cast<int64_t>(blk) >= p.num_blocks) {
-              errs |= kErrBadBlock;
-              continue;
-            }
-            mbar_expect_tx(&sm->full[st], 2u * (D / 64) * p.box_slots * 128u);
-            const int c1 = p.map_head_first ? x.kvh : slot;
-            const int c2 = p.map_head_first ? slot : x.kvh;
+    }
+    {
+      const int ntok = min(kSplitTokens, x.lim_max - x.tok0);
+      const int first = x.tok0 >> p.block_shift;
+      const int nent = (ntok + bmask) >> p.block_shift;
+      for (int e = lane; e < nent; e += 32) {
+        const int col = first + e;
+        tab[e] = col < p.max_blocks_per_seq ? __ldg(p.block_table + x.b * p.bt_stride + col)
+                                            : kPastWidth;
+      }
+    }
+    __syncwarp();
+    if (stage_q && lane == 0) mbar_arrive(&sm->q_full[ui % QB]);
+    for (int j = 0; j < x.n_tiles; ++j, ++gi) {
+      const int st = gi % NS;
+      bool okw = true;
+      if (lane == 0) okw = mbar_wait(&empty[st], ((gi / NS) & 1) ^ 1, abort_any);
+      if (!__shfl_sync(0xffffffffu, okw ? 1 : 0, 0)) {
+        failed = true;
+        break;
+      }
+      const int tok0 = x.tok0 + j * kTileTokens;
+      const int nvalid = min(kTileTokens, x.lim_max - tok0);
+      const int nbox = (nvalid + p.box_slots - 1) / p.box_slots;
+      int errs = 0;
+      if (lane < nbox) {
+        const int tok = tok0 + lane * p.box_slots;
+        const int blk = tab[(tok - x.tok0) >> p.block_shift];
+        if (blk == kPastWidth) {
+          errs = kErrTableWidth;
+        } else if (blk < 0 || static_cast<int64_t>(blk) >= p.num_blocks) {
+          errs = kErrBadBlock;
+        } else {
+          uint8_t *d0 = smem + dst_off + st * C::kKVBytes + lane * p.box_slots * 128;
+          const int slot = tok & bmask;
+          const int c1 = p.map_head_first ? x.kvh : slot;
+          const int c2 = p.map_head_first ? slot : x.kvh;
+          mbar_expect_tx(&full[st], static_cast<uint32_t>((D / 64) * p.box_slots * 128));
 #pragma unroll
-            for (int h = 0; h < D / 64; ++h) {
-              const int off = h * C::kHalfBytes + k * p.box_slots * 128;
-              tma_load_4d(kdst + off, &map_k, &sm->full[st], h * 64, c1, c2, blk);
-              tma_load_4d(vdst + off, &map_v, &sm->full[st], h * 64, c1, c2, blk);
-            }
-          }
-          mbar_arrive(&sm->full[st]);
-          last_gi[st] = gi;
-          if (errs && p.err) atomicOr(p.err, errs);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(d0 + h * C::kHalfBytes, map, &full[st], h * 64, c1, c2, blk);
         }
       }
-      failed = __any_sync(0xffffffffu, failed);
-      ++ui;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&full[st]);
+        last_gi[st] = gi;
+      }
+      if (errs && p.err) atomicOr(p.err, errs);
     }
-    if (failed && lane == 0) {
-      // wait (bounded, ignoring the abort flag) for our own copies in flight
-      volatile int no_abort = 0;
+    ++ui;
+  }
+  if (failed && lane == 0) {
+    // wait (bounded, ignoring the abort flag) for this warp's copies in flight
+    volatile int no_abort = 0;
 #pragma unroll
-      for (int i = 0; i < NS; ++i)
-        if (last_gi[i] >= 0) mbar_wait(&sm->full[i], (last_gi[i] / NS) & 1, &no_abort);
+    for (int i = 0; i < NS; ++i)
+      if (last_gi[i] >= 0) mbar_wait(&full[i], (last_gi[i] / NS) & 1, &no_abort);
+  }
+}
+
+template <int D, int N, int NS, int QB>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_split_kernel(const __grid_constant__ AttnParams p,
+                      const __grid_constant__ CUtensorMap map_k,
+                      const __grid_constant__ CUtensorMap map_v) {
+  using C = Cfg<D, N, NS, QB>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  auto *sm = reinterpret_cast<typename C::Small *>(smem + C::kOffSmall);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  volatile int *abort_any = &sm->abort_any;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&sm->full_k[i], 1);
+      mbar_init(&sm->empty_k[i], 1);
+      mbar_init(&sm->full_v[i], 1);
+      mbar_init(&sm->empty_v[i], 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm->s_full[i], 1);
+      mbar_init(&sm->p_full[i], 4);   // one arrival per softmax warp
+      mbar_init(&sm->o_full[i], 1);
+      mbar_init(&sm->o_free[i], 4);
+    }
+    for (int i = 0; i < QB; ++i) {
+      mbar_init(&sm->q_full[i], 1);
+      mbar_init(&sm->q_empty[i], 1);
+    }
+    mbar_init(&sm->drain, 1);
+    sm->abort_any = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) tmem_alloc(&sm->tmem_base, C::kTmemCols);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = sm->tmem_base;
+  const uint32_t sbase = smem_u32(smem);
+
+  if (warp == kKWarp) {
+    produce<D, N, NS, QB>(p, &map_k, smem, sm, sm->full_k, sm->empty_k, sm->tab_k, C::kOffK,
+                          true, lane, abort_any);
+  } else if (warp == kVWarp) {
+    produce<D, N, NS, QB>(p, &map_v, smem, sm, sm->full_v, sm->empty_v, sm->tab_v, C::kOffV,
+                          false, lane, abort_any);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------
     // MMA issuer (one thread)
     // ------------------------------------------------------------------
     if (lane == 0) {
-      constexpr uint32_t kIdescQK = idesc_bf16(128, N, 0, 0);  // A = K tile, B = Q, both K-major
-      constexpr uint32_t kIdescPV = idesc_bf16(128, N, 1, 1);  // A = V^T, B = P^T, both MN-major
-      constexpr uint32_t kIdescL = idesc_bf16(128, N, 0, 1);   // A = ones, B = P^T
-      const uint32_t tS = tmem, tO = tmem + 2 * N, tL = tmem + 4 * N;
-      const uint64_t d_ones = smem_desc(sbase + C::kOffOnes, 128, 256, kLayoutInterleave);
+      constexpr uint32_t kIdescQK = idesc_bf16(128, N, 0, 0);           // A = K tile, B = Q (K-major)
+      constexpr uint32_t kIdescPV = idesc_bf16(128, C::kPCols, 1, 1);  // A = V^T, B = P^T (MN-major)
+      const uint32_t tS = tmem, tO = tmem + 2 * N;
       int gi = 0, ui = 0, prev = -1;
       bool failed = false;
       auto pv_step = [&](int g) -> bool {
         const int st = g % NS, bb = g & 1;
         if (!mbar_wait(&sm->p_full[bb], (g >> 1) & 1, abort_any)) return false;
         if (!mbar_wait(&sm->o_free[bb], ((g >> 1) & 1) ^ 1, abort_any)) return false;
+        if (!mbar_wait(&sm->full_v[st], (g / NS) & 1, abort_any)) return false;
         tc_fence_after_sync();
-        const uint32_t vaddr = sbase + C::kOffStage + st * C::kStageBytes + C::kKVBytes;
-        const uint32_t paddr = sbase + C::kOffP + bb * 2 * C::kPBytes;
-        // P = P_hi + P_lo (two bf16 parts, ~16 significant bits): both the
-        // weighted values and the row sums accumulate the hi part, then the lo
-        // part, k-step by k-step, in one fixed order.
+        const uint32_t vaddr = sbase + C::kOffV + st * C::kKVBytes;
+        const uint32_t paddr = sbase + C::kOffP + bb * C::kPBytes;
 #pragma unroll
         for (int kk = 0; kk < kTileTokens / 16; ++kk) {
-          // V^T: MN-major, 128-byte swizzle; 64-wide d groups C::kHalfBytes apart
+          // V^T: MN-major, 128-byte swizzle, 64-wide d groups C::kHalfBytes apart
           // (D = 64: both M halves read the same 64 columns; lanes 64..127 are unused).
           const uint64_t a = smem_desc(vaddr + kk * 2048, D == 128 ? C::kHalfBytes : 0, 1024,
                                        kLayoutSw128);
-#pragma unroll
-          for (int part = 0; part < 2; ++part) {
-            // P^T: MN-major, no swizzle; 8-row groups at 128 B (N), 8-token groups at kPKGroup (K).
-            const uint64_t bd = smem_desc(paddr + part * C::kPBytes + kk * 2 * C::kPKGroup,
-                                          C::kPKGroup, 128, kLayoutInterleave);
-            const uint32_t acc = (kk > 0 || part > 0) ? 1u : 0u;
-            umma_bf16(tO + bb * N, a, bd, kIdescPV, acc);
-            umma_bf16(tL + bb * N, d_ones, bd, kIdescL, acc);
-          }
+          // P^T = [P_hi | P_lo]: MN-major, no swizzle; 8-column groups 128 B apart,
+          // 8-token groups kPKGroup apart.
+          const uint64_t b = smem_desc(paddr + kk * 2 * C::kPKGroup, C::kPKGroup, 128,
+                                       kLayoutInterleave);
+          umma_bf16(tO + bb * C::kPCols, a, b, kIdescPV, kk > 0 ? 1u : 0u);
         }
         umma_commit(&sm->o_full[bb]);
-        umma_commit(&sm->empty[st]);
+        umma_commit(&sm->empty_v[st]);
         return true;
       };
       for (int u = blockIdx.x; u < p.n_units && !failed; u += gridDim.x) {
@@ -352,12 +390,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t qaddr = sbase + C::kOffQ + qb * C::kQBytes;
         for (int j = 0; j < x.n_tiles; ++j, ++gi) {
           const int st = gi % NS, bb = gi & 1;
-          if (!mbar_wait(&sm->full[st], (gi / NS) & 1, abort_any)) {
+          if (!mbar_wait(&sm->full_k[st], (gi / NS) & 1, abort_any)) {
             failed = true;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t kaddr = sbase + C::kOffStage + st * C::kStageBytes;
+          const uint32_t kaddr = sbase + C::kOffK + st * C::kKVBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const int h = kk >> 2, off = (kk & 3) * 32;
@@ -366,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16(tS + bb * N, a, b, kIdescQK, kk > 0 ? 1u : 0u);
           }
           umma_commit(&sm->s_full[bb]);
+          umma_commit(&sm->empty_k[st]);
           if (j == x.n_tiles - 1) umma_commit(&sm->q_empty[qb]);
           if (prev >= 0 && !pv_step(prev)) {
             failed = true;
@@ -416,64 +455,84 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
 
-      // correction of tile g: fold O_g, L_g into acc, l
-      auto correction = [&](int g) -> bool {
+      // correction of tile g: acc = fma(acc, alpha, O_hi + O_lo),
+      // l = fma(l, alpha, sum of the tile's probabilities), rows the tile reaches only
+      auto correction = [&](int g) {
         const int bb = g & 1;
-        const bool ok = mbar_wait(&sm->o_full[bb], (g >> 1) & 1, abort_any);
+        mbar_wait(&sm->o_full[bb], (g >> 1) & 1, abort_any);
         tc_fence_after_sync();
 #pragma unroll
         for (int ch = 0; ch < N / 16; ++ch) {
-          float o16[16], l16[16];
-          tmem_ld16(tmem + lane_off + 2 * N + bb * N + ch * 16, o16);
-          tmem_ld16(tmem + lane_off + 4 * N + bb * N + ch * 16, l16);
-          tmem_ld_wait();
+          if (ch * 16 < x.rows) {  // warp-uniform
+            float hi[16], lo[16];
+            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + ch * 16, hi);
+            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + N + ch * 16, lo);
+            tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c = ch * 16 + e;
-            if (!sm->skip[bb][c]) acc[c] = __fmaf_rn(acc[c], sm->alpha[bb][c], o16[e]);
-            if (c == t && !sm->skip[bb][c]) l_run = __fmaf_rn(l_run, sm->alpha[bb][c], l16[e]);
+            for (int e = 0; e < 16; ++e) {
+              const int c = ch * 16 + e;
+              if (c < x.rows && !sm->skip[bb][c])
+                acc[c] = __fmaf_rn(acc[c], sm->alpha[bb][c], __fadd_rn(hi[e], lo[e]));
+            }
           }
         }
+        if (t < x.rows && !sm->skip[bb][t]) {
+          const float lt = __fadd_rn(__fadd_rn(sm->wsum[bb][0][t], sm->wsum[bb][1][t]),
+                                     __fadd_rn(sm->wsum[bb][2][t], sm->wsum[bb][3][t]));
+          l_run = __fmaf_rn(l_run, sm->alpha[bb][t], lt);
+        }
         tc_fence_before_sync();
-        mbar_arrive(&sm->o_free[bb]);
-        return ok;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->o_free[bb]);
       };
 
       bool fail = false;
       for (int j = 0; j < x.n_tiles; ++j, ++gi) {
-        const int bb = gi & 1;
-        const bool ok = mbar_wait(&sm->s_full[bb], (gi >> 1) & 1, abort_any);
+        const int bb = gi & 1, st = gi % NS;
+        bool ok = mbar_wait(&sm->s_full[bb], (gi >> 1) & 1, abort_any);
         tc_fence_after_sync();
         float sv[N];
 #pragma unroll
         for (int ch = 0; ch < N / 16; ++ch)
-          tmem_ld16(tmem + lane_off + bb * N + ch * 16, *reinterpret_cast<float(*)[16]>(&sv[ch * 16]));
+          if (ch * 16 < x.rows)
+            tmem_ld16(tmem + lane_off + bb * N + ch * 16, *reinterpret_cast<float(*)[16]>(&sv[ch * 16]));
         tmem_ld_wait();
-        const int tok = x.tok0 + j * kTileTokens + t;
+        const int tok0 = x.tok0 + j * kTileTokens;
+        const int tok = tok0 + t;
 #pragma unroll
-        for (int c = 0; c < N; ++c) sv[c] = (tok < sm->lim[c]) ? __fmul_rn(sv[c], p.cscale) : NEG_INF;
-        if (tok >= x.lim_max) {
-          // keys past the loaded range: their V rows hold stale bytes (or the
-          // cache's NaN tails); zero them so 0 * V stays 0 in P.V.
-          uint8_t *vrow = smem + C::kOffStage + (gi % NS) * C::kStageBytes + C::kKVBytes + t * 128;
+        for (int c = 0; c < N; ++c)
+          sv[c] = (c < x.rows && tok < sm->lim[c]) ? __fmul_rn(sv[c], p.cscale) : NEG_INF;
+        if (tok0 + kTileTokens > x.lim_max) {
+          // The last tile: keys past the loaded range hold stale bytes or the
+          // cache's NaN tails; once V has landed, zero those V rows so that
+          // 0 * V stays 0 in P.V.
+          ok = mbar_wait(&sm->full_v[st], (gi / NS) & 1, abort_any) && ok;
+          if (tok >= x.lim_max) {
+            uint8_t *vrow = smem + C::kOffV + st * C::kKVBytes + t * 128;
 #pragma unroll
-          for (int h = 0; h < D / 64; ++h)
+            for (int h = 0; h < D / 64; ++h)
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              *reinterpret_cast<uint4 *>(vrow + h * C::kHalfBytes + k * 16) = make_uint4(0u, 0u, 0u, 0u);
+              for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<uint4 *>(vrow + h * C::kHalfBytes + k * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
         }
 #pragma unroll
-        for (int c = 0; c < N; ++c) {
-          const float wm = warp_max(sv[c]);
-          if (lane == 0) sm->wmax[warp][c] = wm;
+        for (int q4 = 0; q4 < N / 4; ++q4) {
+          if (q4 * 4 < x.rows) {  // warp-uniform: padded rows need no reduction
+            float v[4] = {sv[4 * q4], sv[4 * q4 + 1], sv[4 * q4 + 2], sv[4 * q4 + 3]};
+            warp_max4(v);
+            if (lane == 0)
+              *reinterpret_cast<float4 *>(&sm->wmax[warp][4 * q4]) = make_float4(v[0], v[1], v[2], v[3]);
+          }
         }
         if (softmax_bar_or(!ok)) {
           fail = true;
           break;
         }
         if (t < N) {
-          const float tmax = fmaxf(fmaxf(sm->wmax[0][t], sm->wmax[1][t]),
-                                   fmaxf(sm->wmax[2][t], sm->wmax[3][t]));
+          const float tmax = t < x.rows ? fmaxf(fmaxf(sm->wmax[0][t], sm->wmax[1][t]),
+                                                fmaxf(sm->wmax[2][t], sm->wmax[3][t]))
+                                        : NEG_INF;
           const int skip = (tmax == NEG_INF) ? 1 : 0;
           const float mnew = skip ? m_run : fmaxf(m_run, tmax);
           const float alpha = skip ? 1.f : ex2(__fsub_rn(m_run, mnew));
@@ -483,31 +542,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           sm->skip[bb][t] = skip;
         }
         softmax_bar_or(false);
-        // P^T row t (MN-major, no swizzle: one 16-byte chunk per 8 rows), as a
-        // bf16 hi part and the bf16 rounding of the remainder (lo part).
-        uint8_t *prow = smem + C::kOffP + bb * 2 * C::kPBytes + (t >> 3) * C::kPKGroup + (t & 7) * 16;
+        // P^T row t (MN-major, no swizzle: one 16-byte chunk per 8 columns):
+        // p in the hi columns as bf16, the bf16 rounding of p - hi in the lo
+        // columns; the fp32 p are also summed per row (fixed tree) for l.
+        uint8_t *prow = smem + C::kOffP + bb * C::kPBytes + (t >> 3) * C::kPKGroup + (t & 7) * 16;
 #pragma unroll
         for (int grp = 0; grp < N / 8; ++grp) {
-          uint32_t whi[4], wlo[4];
+          uint32_t whi[4] = {0u, 0u, 0u, 0u}, wlo[4] = {0u, 0u, 0u, 0u};
+          if (grp * 8 < x.rows) {  // groups of padded rows keep p = 0
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c0 = grp * 8 + 2 * e;
-            const float p0 = (sv[c0] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0], sm->mnew[bb][c0]));
-            const float p1 =
-                (sv[c0 + 1] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0 + 1], sm->mnew[bb][c0 + 1]));
-            __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
-            __nv_bfloat162 lo = __floats2bfloat162_rn(__fsub_rn(p0, __low2float(hi)),
-                                                      __fsub_rn(p1, __high2float(hi)));
-            whi[e] = *reinterpret_cast<uint32_t *>(&hi);
-            wlo[e] = *reinterpret_cast<uint32_t *>(&lo);
+            for (int e = 0; e < 4; ++e) {
+              const int c0 = grp * 8 + 2 * e;
+              const float p0 = (sv[c0] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0], sm->mnew[bb][c0]));
+              const float p1 =
+                  (sv[c0 + 1] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0 + 1], sm->mnew[bb][c0 + 1]));
+              sv[c0] = p0;
+              sv[c0 + 1] = p1;
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+              __nv_bfloat162 l2 = __floats2bfloat162_rn(__fsub_rn(p0, __low2float(h2)),
+                                                        __fsub_rn(p1, __high2float(h2)));
+              whi[e] = *reinterpret_cast<uint32_t *>(&h2);
+              wlo[e] = *reinterpret_cast<uint32_t *>(&l2);
+            }
           }
           *reinterpret_cast<uint4 *>(prow + grp * 128) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
-          *reinterpret_cast<uint4 *>(prow + C::kPBytes + grp * 128) =
+          *reinterpret_cast<uint4 *>(prow + (N / 8 + grp) * 128) =
               make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < N / 4; ++q4) {
+          if (q4 * 4 < x.rows) {
+            float v[4] = {sv[4 * q4], sv[4 * q4 + 1], sv[4 * q4 + 2], sv[4 * q4 + 3]};
+            warp_sum4_lane0(v);
+            if (lane == 0)
+              *reinterpret_cast<float4 *>(&sm->wsum[bb][warp][4 * q4]) = make_float4(v[0], v[1], v[2], v[3]);
+          }
         }
         fence_proxy_async_smem();
         tc_fence_before_sync();
-        mbar_arrive(&sm->p_full[bb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->p_full[bb]);
         if (j > 0) correction(gi - 1);
       }
       if (fail) {
