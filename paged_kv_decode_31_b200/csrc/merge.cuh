@@ -45,18 +45,31 @@ __global__ void __launch_bounds__(D) merge_kernel(const __grid_constant__ MergeP
   const int n_s = min((lim + 4095) / 4096, p.n_splits);
   const int d = threadIdx.x;
   const float NEG_INF = __int_as_float(0xff800000);
+  const float *ml = p.ws_ml + row * p.n_splits * 2;
+  const float *ap = p.ws_acc + row * p.n_splits * D + d;
   float M = NEG_INF, L = 0.f, A = 0.f;
-  for (int s = 0; s < n_s; ++s) {
-    const int64_t k = row * p.n_splits + s;
-    const float ms = p.ws_ml[2 * k];
-    const float ls = p.ws_ml[2 * k + 1];
-    if (ms == NEG_INF) continue;  // the row sees no key of this split
-    const float Mn = fmaxf(M, ms);
-    const float a = ex2(__fsub_rn(M, Mn));
-    const float c = ex2(__fsub_rn(ms, Mn));
-    L = __fmaf_rn(ls, c, __fmul_rn(L, a));
-    A = __fmaf_rn(p.ws_acc[k * D + d], c, __fmul_rn(A, a));
-    M = Mn;
+  // Partials are fetched kBatch splits at a time (independent loads in
+  // flight together) and folded strictly in ascending split order.
+  constexpr int kBatch = 16;
+  for (int s0 = 0; s0 < n_s; s0 += kBatch) {
+    float ms[kBatch], ls[kBatch], as[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int s = s0 + k;
+      ms[k] = s < n_s ? ml[2 * s] : NEG_INF;
+      ls[k] = s < n_s ? ml[2 * s + 1] : 0.f;
+      as[k] = s < n_s ? ap[static_cast<int64_t>(s) * D] : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      if (ms[k] == NEG_INF) continue;  // the row sees no key of this split
+      const float Mn = fmaxf(M, ms[k]);
+      const float a = ex2(__fsub_rn(M, Mn));
+      const float c = ex2(__fsub_rn(ms[k], Mn));
+      L = __fmaf_rn(ls[k], c, __fmul_rn(L, a));
+      A = __fmaf_rn(as[k], c, __fmul_rn(A, a));
+      M = Mn;
+    }
   }
   const bool any = L > 0.f;
   const float o = any ? __fdiv_rn(A, L) : 0.f;
