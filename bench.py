@@ -27,7 +27,6 @@ rank runs its own batch; there is no collective on the data path).
 from __future__ import annotations
 
 import argparse
-import datetime
 import json
 import math
 import os
@@ -65,10 +64,8 @@ def parse_args():
 
 
 def dist_env():
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return rank, world, local
+    from paged_kv_decode_31_b200 import dist as pdist
+    return pdist.rank_env()
 
 
 def measured_peaks():
@@ -184,14 +181,14 @@ def cpu_baseline(di_dev, n_seq: int = 2):
 def run_ours(args):
     import torch.distributed as dist
     import paged_kv_decode_31_b200 as pkv
+    from paged_kv_decode_31_b200 import dist as pdist
     from paged_kv_decode_31_b200 import inputs as I
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        pdist.init("nccl", device=dev)
     di = I.config_long_context(seed=1000 + rank, device=dev, batch=args.batch,
                                seqlen=args.context)
     B, ctx, Hq, Hkv, D = di.batch, int(di.seqlens[0].item()), di.Hq, di.Hkv, di.D
@@ -278,19 +275,12 @@ def run_ours(args):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": round(kv_bytes * world * args.steps / (e2e_ms / 1e3) / 1e9, 2),
+        e2e_ms = pdist.max_over_ranks(e0.elapsed_time(e1), device=dev)
+        e2e = {"value": round(pdist.weak_scaling_rate(kv_bytes, world, args.steps, e2e_ms) / 1e9, 2),
                "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(e2e_ms / args.steps, 5)}
 
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = pdist.max_over_ranks(ms_total, device=dev)
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
@@ -298,7 +288,7 @@ def run_ours(args):
 
     peak, peak_kind = measured_peaks()
     ms_step = ms_total / args.steps
-    value = kv_bytes * world * args.steps / (ms_total / 1e3) / 1e9
+    value = pdist.weak_scaling_rate(kv_bytes, world, args.steps, ms_total) / 1e9
     dec_ms = statistics.mean(decode_ms)
     achieved = kv_bytes / (dec_ms / 1e3) / 1e9
     result = {
