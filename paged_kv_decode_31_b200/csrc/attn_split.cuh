@@ -48,10 +48,12 @@ namespace pkv {
 
 constexpr int kSplitTokens = 4096;
 constexpr int kTileTokens = 128;
-constexpr int kThreads = 224;  // 7 warps
-constexpr int kKWarp = 4;      // K producer (+ Q staging)
-constexpr int kVWarp = 5;      // V producer
-constexpr int kMmaWarp = 6;    // MMA issuer + TMEM owner
+constexpr int kThreads = 480;  // 15 warps
+// warps 0-3 and 4-7: softmax warpgroups (even / odd tiles of the CTA's sequence)
+constexpr int kCorrWarp0 = 8;  // warps 8-11: correction + epilogue warpgroup
+constexpr int kKWarp = 12;     // K producer (+ Q staging)
+constexpr int kVWarp = 13;     // V producer
+constexpr int kMmaWarp = 14;   // MMA issuer + TMEM owner
 
 constexpr int kErrBadBlock = 1;
 constexpr int kErrTableWidth = 2;
@@ -79,17 +81,18 @@ struct AttnParams {
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
 
-// Named barrier over the 128 softmax threads that also ORs a predicate across
-// them, so an abort decision is taken by all of them at the same barrier.
-__device__ __forceinline__ bool softmax_bar_or(bool pred) {
+// Named barrier `id` over one warpgroup (128 threads) that also ORs a
+// predicate across it, so an abort decision is taken by the whole warpgroup
+// at the same barrier.
+__device__ __forceinline__ bool wg_bar_or(uint32_t id, bool pred) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred))
+      : "r"(static_cast<uint32_t>(pred)), "r"(id)
       : "memory");
   return r != 0;
 }
@@ -141,16 +144,16 @@ struct Cfg {
   static constexpr int kOffSmall = kOffP + 2 * kPBytes;
   struct Small {
     uint64_t full_k[NS], empty_k[NS], full_v[NS], empty_v[NS];
-    uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+    uint64_t s_full[2], p_full[2], o_full[2], o_free[2], stat_free[2];
     uint64_t q_full[QB], q_empty[QB], drain;
     uint32_t tmem_base;
     int abort_any;
-    __align__(16) float wmax[4][N];
-    __align__(16) float wsum[2][4][N];
-    float mnew[2][N];
-    float alpha[2][N];
-    int skip[2][N];
-    int lim[N];
+    __align__(16) float wmax[2][2][4][N];  // [softmax warpgroup][tile parity][warp][row]
+    __align__(16) float wsum[2][4][N];     // [buffer][warp][row]: per-warp sums of p
+    float tmax[2][N];                      // [buffer][row]: the tile's max (base-2 units)
+    float coef_a[N], coef_b[N];            // correction factors of the current tile
+    int coef_skip[N];
+    int lim[2][N];                         // [softmax warpgroup][row]: key limit
     int tab_k[kSplitTokens / 16];  // block-table entries of each producer's current split
     int tab_v[kSplitTokens / 16];
   };
@@ -320,9 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm->s_full[i], 1);
-      mbar_init(&sm->p_full[i], 4);   // one arrival per softmax warp
+      mbar_init(&sm->p_full[i], 4);   // one arrival per warp of a softmax warpgroup
       mbar_init(&sm->o_full[i], 1);
-      mbar_init(&sm->o_free[i], 4);
+      mbar_init(&sm->o_free[i], 4);   // one arrival per correction warp
+      mbar_init(&sm->stat_free[i], 4);
     }
     for (int i = 0; i < QB; ++i) {
       mbar_init(&sm->q_full[i], 1);
@@ -421,18 +425,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&sm->drain, 0, &no_abort);
       }
     }
-  } else {
+  } else if (warp < kCorrWarp0) {
     // ------------------------------------------------------------------
-    // Softmax + correction + epilogue: 128 threads, thread t <-> TMEM lane t
+    // Softmax warpgroups: warpgroup wg takes the tiles with gi % 2 == wg.
+    // Thread t <-> TMEM lane t <-> token t of the tile.  Per tile and row:
+    // tmax = exact max of the masked scores, p = 2^(s - tmax) written as
+    // P^T = [bf16(p) | bf16(p - bf16(p))], per-warp sums of the fp32 p.
     // ------------------------------------------------------------------
-    const int t = threadIdx.x;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int wg = warp >> 2, wq = warp & 3, t = threadIdx.x & 127;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t bar_id = 1 + wg;
     const float NEG_INF = neg_inf();
-    float acc[N];
-    float m_run = NEG_INF, l_run = 0.f;
-    int gi = 0;
+    int gbase = 0;
     bool stop = false;
-
     for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
       const Unit x = unit_at<N>(p, u);
       if (x.n_tiles == 0) continue;
@@ -444,52 +449,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (p.causal) lim = min(lim, x.seqlen - p.seqlen_q + i + 1);
           lim = lim > 0 ? lim : 0;
         }
-        sm->lim[t] = lim;
+        sm->lim[wg][t] = lim;
       }
-#pragma unroll
-      for (int c = 0; c < N; ++c) acc[c] = 0.f;
-      m_run = NEG_INF;
-      l_run = 0.f;
-      if (softmax_bar_or(false)) {
+      if (wg_bar_or(bar_id, false)) {
         stop = true;
         break;
       }
-
-      // correction of tile g: acc = fma(acc, alpha, O_hi + O_lo),
-      // l = fma(l, alpha, sum of the tile's probabilities), rows the tile reaches only
-      auto correction = [&](int g) {
-        const int bb = g & 1;
-        mbar_wait(&sm->o_full[bb], (g >> 1) & 1, abort_any);
-        tc_fence_after_sync();
-#pragma unroll
-        for (int ch = 0; ch < N / 16; ++ch) {
-          if (ch * 16 < x.rows) {  // warp-uniform
-            float hi[16], lo[16];
-            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + ch * 16, hi);
-            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + N + ch * 16, lo);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int c = ch * 16 + e;
-              if (c < x.rows && !sm->skip[bb][c])
-                acc[c] = __fmaf_rn(acc[c], sm->alpha[bb][c], __fadd_rn(hi[e], lo[e]));
-            }
-          }
-        }
-        if (t < x.rows && !sm->skip[bb][t]) {
-          const float lt = __fadd_rn(__fadd_rn(sm->wsum[bb][0][t], sm->wsum[bb][1][t]),
-                                     __fadd_rn(sm->wsum[bb][2][t], sm->wsum[bb][3][t]));
-          l_run = __fmaf_rn(l_run, sm->alpha[bb][t], lt);
-        }
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->o_free[bb]);
-      };
-
-      bool fail = false;
-      for (int j = 0; j < x.n_tiles; ++j, ++gi) {
-        const int bb = gi & 1, st = gi % NS;
-        bool ok = mbar_wait(&sm->s_full[bb], (gi >> 1) & 1, abort_any);
+      for (int j = 0; j < x.n_tiles; ++j) {
+        const int gi = gbase + j;
+        if ((gi & 1) != wg) continue;
+        const int bb = wg, st = gi % NS, par = (gi >> 1) & 1;
+        bool ok = mbar_wait(&sm->s_full[bb], par, abort_any);
+        // P^T[bb] is free once P.V of tile gi - 2 is done, the row statistics
+        // once the correction of tile gi - 2 has read them
+        ok = mbar_wait(&sm->o_full[bb], par ^ 1, abort_any) && ok;
+        ok = mbar_wait(&sm->stat_free[bb], par ^ 1, abort_any) && ok;
         tc_fence_after_sync();
         float sv[N];
 #pragma unroll
@@ -501,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tok = tok0 + t;
 #pragma unroll
         for (int c = 0; c < N; ++c)
-          sv[c] = (c < x.rows && tok < sm->lim[c]) ? __fmul_rn(sv[c], p.cscale) : NEG_INF;
+          sv[c] = (c < x.rows && tok < sm->lim[wg][c]) ? __fmul_rn(sv[c], p.cscale) : NEG_INF;
         if (tok0 + kTileTokens > x.lim_max) {
           // The last tile: keys past the loaded range hold stale bytes or the
           // cache's NaN tails; once V has landed, zero those V rows so that
@@ -516,35 +490,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint4 *>(vrow + h * C::kHalfBytes + k * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
         }
+        float(*wmax)[N] = sm->wmax[wg][par];
 #pragma unroll
         for (int q4 = 0; q4 < N / 4; ++q4) {
           if (q4 * 4 < x.rows) {  // warp-uniform: padded rows need no reduction
             float v[4] = {sv[4 * q4], sv[4 * q4 + 1], sv[4 * q4 + 2], sv[4 * q4 + 3]};
             warp_max4(v);
             if (lane == 0)
-              *reinterpret_cast<float4 *>(&sm->wmax[warp][4 * q4]) = make_float4(v[0], v[1], v[2], v[3]);
+              *reinterpret_cast<float4 *>(&wmax[wq][4 * q4]) = make_float4(v[0], v[1], v[2], v[3]);
           }
         }
-        if (softmax_bar_or(!ok)) {
-          fail = true;
+        if (wg_bar_or(bar_id, !ok)) {
+          stop = true;
           break;
         }
-        if (t < N) {
-          const float tmax = t < x.rows ? fmaxf(fmaxf(sm->wmax[0][t], sm->wmax[1][t]),
-                                                fmaxf(sm->wmax[2][t], sm->wmax[3][t]))
-                                        : NEG_INF;
-          const int skip = (tmax == NEG_INF) ? 1 : 0;
-          const float mnew = skip ? m_run : fmaxf(m_run, tmax);
-          const float alpha = skip ? 1.f : ex2(__fsub_rn(m_run, mnew));
-          m_run = mnew;
-          sm->mnew[bb][t] = mnew;
-          sm->alpha[bb][t] = alpha;
-          sm->skip[bb][t] = skip;
-        }
-        softmax_bar_or(false);
-        // P^T row t (MN-major, no swizzle: one 16-byte chunk per 8 columns):
-        // p in the hi columns as bf16, the bf16 rounding of p - hi in the lo
-        // columns; the fp32 p are also summed per row (fixed tree) for l.
+        // P^T row t (MN-major, no swizzle: one 16-byte chunk per 8 columns).
         uint8_t *prow = smem + C::kOffP + bb * C::kPBytes + (t >> 3) * C::kPKGroup + (t & 7) * 16;
 #pragma unroll
         for (int grp = 0; grp < N / 8; ++grp) {
@@ -553,9 +513,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int c0 = grp * 8 + 2 * e;
-              const float p0 = (sv[c0] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0], sm->mnew[bb][c0]));
-              const float p1 =
-                  (sv[c0 + 1] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0 + 1], sm->mnew[bb][c0 + 1]));
+              const float m0 = fmaxf(fmaxf(wmax[0][c0], wmax[1][c0]), fmaxf(wmax[2][c0], wmax[3][c0]));
+              const float m1 = fmaxf(fmaxf(wmax[0][c0 + 1], wmax[1][c0 + 1]),
+                                     fmaxf(wmax[2][c0 + 1], wmax[3][c0 + 1]));
+              const float p0 = (sv[c0] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0], m0));
+              const float p1 = (sv[c0 + 1] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0 + 1], m1));
               sv[c0] = p0;
               sv[c0 + 1] = p1;
               __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
@@ -575,24 +537,93 @@ __global__ void __launch_bounds__(kThreads, 1)
             float v[4] = {sv[4 * q4], sv[4 * q4 + 1], sv[4 * q4 + 2], sv[4 * q4 + 3]};
             warp_sum4_lane0(v);
             if (lane == 0)
-              *reinterpret_cast<float4 *>(&sm->wsum[bb][warp][4 * q4]) = make_float4(v[0], v[1], v[2], v[3]);
+              *reinterpret_cast<float4 *>(&sm->wsum[bb][wq][4 * q4]) = make_float4(v[0], v[1], v[2], v[3]);
           }
         }
+        if (t < x.rows)
+          sm->tmax[bb][t] = fmaxf(fmaxf(wmax[0][t], wmax[1][t]), fmaxf(wmax[2][t], wmax[3][t]));
         fence_proxy_async_smem();
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->p_full[bb]);
-        if (j > 0) correction(gi - 1);
       }
-      if (fail) {
-        stop = true;
-        break;
+      gbase += x.n_tiles;
+    }
+    (void)stop;
+  } else if (warp < kCorrWarp0 + 4) {
+    // ------------------------------------------------------------------
+    // Correction + epilogue warpgroup: thread t <-> TMEM lane t <-> output
+    // column d of O^T; thread r (< rows) owns row r's running (m, l).
+    // Per tile, in order: m' = max(m, tmax), a = 2^(m - m'), b = 2^(tmax - m'),
+    // acc = fma(O_hi + O_lo, b, acc * a), l = fma(sum p, b, l * a); a tile a
+    // row does not reach (tmax = -inf) leaves the row untouched.
+    // ------------------------------------------------------------------
+    const int wq = warp & 3, t = threadIdx.x & 127;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    constexpr uint32_t bar_id = 3;
+    const float NEG_INF = neg_inf();
+    float acc[N];
+    float m_run = NEG_INF, l_run = 0.f;
+    int gbase = 0;
+    bool stop = false;
+    for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
+      const Unit x = unit_at<N>(p, u);
+      if (x.n_tiles == 0) continue;
+#pragma unroll
+      for (int c = 0; c < N; ++c) acc[c] = 0.f;
+      m_run = NEG_INF;
+      l_run = 0.f;
+      for (int j = 0; j < x.n_tiles; ++j) {
+        const int gi = gbase + j, bb = gi & 1, par = (gi >> 1) & 1;
+        bool ok = mbar_wait(&sm->p_full[bb], par, abort_any);  // the tile's row statistics
+        ok = mbar_wait(&sm->o_full[bb], par, abort_any) && ok;  // its P.V
+        tc_fence_after_sync();
+        if (t < x.rows) {
+          const float tm = sm->tmax[bb][t];
+          const int skip = (tm == NEG_INF) ? 1 : 0;
+          float a = 1.f, b = 0.f;
+          if (!skip) {
+            const float mn = fmaxf(m_run, tm);
+            a = ex2(__fsub_rn(m_run, mn));
+            b = ex2(__fsub_rn(tm, mn));
+            const float lt = __fadd_rn(__fadd_rn(sm->wsum[bb][0][t], sm->wsum[bb][1][t]),
+                                       __fadd_rn(sm->wsum[bb][2][t], sm->wsum[bb][3][t]));
+            l_run = __fmaf_rn(lt, b, __fmul_rn(l_run, a));
+            m_run = mn;
+          }
+          sm->coef_a[t] = a;
+          sm->coef_b[t] = b;
+          sm->coef_skip[t] = skip;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->stat_free[bb]);  // the tile's statistics are read
+        if (wg_bar_or(bar_id, !ok)) {
+          stop = true;
+          break;
+        }
+#pragma unroll
+        for (int ch = 0; ch < N / 16; ++ch) {
+          if (ch * 16 < x.rows) {  // warp-uniform
+            float hi[16], lo[16];
+            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + ch * 16, hi);
+            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + N + ch * 16, lo);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c = ch * 16 + e;
+              if (c < x.rows && !sm->coef_skip[c])
+                acc[c] = __fmaf_rn(__fadd_rn(hi[e], lo[e]), sm->coef_b[c],
+                                   __fmul_rn(acc[c], sm->coef_a[c]));
+            }
+          }
+        }
+        tc_fence_before_sync();
+        // coef_* are rewritten for the next tile only after this barrier
+        wg_bar_or(bar_id, false);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->o_free[bb]);
       }
-      correction(gi - 1);
-      if (softmax_bar_or(false)) {
-        stop = true;
-        break;
-      }
+      if (stop) break;
       // epilogue: unnormalised split partial of every real row
       const int64_t S = p.n_splits;
 #pragma unroll
@@ -612,6 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.ws_ml[(row_id * S + x.s) * 2 + 0] = m_run;
         p.ws_ml[(row_id * S + x.s) * 2 + 1] = l_run;
       }
+      gbase += x.n_tiles;
     }
     (void)stop;
   }
