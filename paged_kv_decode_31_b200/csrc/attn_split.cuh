@@ -154,8 +154,7 @@ struct Cfg {
     float coef_a[N], coef_b[N];            // correction factors of the current tile
     int coef_skip[N];
     int lim[2][N];                         // [softmax warpgroup][row]: key limit
-    int tab_k[kSplitTokens / 16];  // block-table entries of each producer's current split
-    int tab_v[kSplitTokens / 16];
+    int tab[2][2][kSplitTokens / 16];      // [producer][unit parity]: block-table entries
   };
   static constexpr int kSmemBytes = kOffSmall + static_cast<int>(sizeof(Small)) + 1024;
   // TMEM: S^T (N columns) x 2 buffers, then O^T (hi and lo, 2N columns) x 2 buffers
@@ -196,100 +195,157 @@ __device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
   return x;
 }
 
-// One producer warp: stages the split's block-table entries in `tab` (all
-// lanes), then per tile lane k issues the TMA boxes of the tile's k-th box of
-// cache rows into the ring `dst`, lane 0 arrives on `full`.  With `stage_q`
-// the warp also stages each unit's Q rows (the B operand of S^T = K Q^T).
+constexpr int kPastWidth = static_cast<int>(0x80000000u);
+
+// First unit at or after `from` (stride gridDim.x) with work, or -1.
+template <int N>
+__device__ __forceinline__ int next_unit(const AttnParams &p, int from, Unit &out) {
+  for (int v = from; v < p.n_units; v += gridDim.x) {
+    out = unit_at<N>(p, v);
+    if (out.n_tiles > 0) return v;
+  }
+  return -1;
+}
+
+// Stage the Q rows of unit x (the B operand of S^T = K Q^T, 128-byte
+// swizzled); padded rows are zero.  Plain loads: cp.async here measurably
+// slowed the TMA issue of the same warp.
+template <int D, int N>
+__device__ __forceinline__ void stage_q(const AttnParams &p, const Unit &x, uint8_t *qdst, int lane) {
+  constexpr int kQHalf = N * 128;
+  for (int idx = lane; idx < N * (D / 8); idx += 32) {
+    const int c = idx / (D / 8), ch = idx % (D / 8);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (c < x.rows) {
+      const int r = x.row0 + c;
+      const int i = r / p.G, g = r - i * p.G;
+      v = __ldg(reinterpret_cast<const uint4 *>(p.q + x.b * p.q_sb + static_cast<int64_t>(i) * p.q_ss +
+                                                static_cast<int64_t>(x.kvh * p.G + g) * p.q_sh +
+                                                ch * 8));
+    }
+    const int h = ch >> 3, cc = ch & 7;
+    *reinterpret_cast<uint4 *>(qdst + h * kQHalf + c * 128 + ((cc ^ (c & 7)) << 4)) = v;
+  }
+}
+
+// Stage the block-table entries of unit x's split (columns past the table are
+// marked kPastWidth).
+__device__ __forceinline__ void stage_tab(const AttnParams &p, const Unit &x, int *tab, int lane) {
+  const int ntok = min(kSplitTokens, x.lim_max - x.tok0);
+  const int first = x.tok0 >> p.block_shift;
+  const int nent = (ntok + (1 << p.block_shift) - 1) >> p.block_shift;
+  for (int e = lane; e < nent; e += 32) {
+    const int col = first + e;
+    tab[e] = col < p.max_blocks_per_seq ? __ldg(p.block_table + x.b * p.bt_stride + col)
+                                        : kPastWidth;
+  }
+}
+
+// One producer warp.  The current unit's block-table entries (and, for the K
+// warp, its Q rows) are already in shared memory when its first tile is
+// issued: the warp stages the NEXT unit's entries at the start of every unit
+// and (two Q buffers) the next unit's Q just before the current unit's last
+// tile -- points where its stage ring is full and it would wait anyway.  Per tile, lane k issues the TMA boxes of the tile's k-th box of cache
+// rows, all lanes in parallel; lane 0 arrives on `full`.
 template <int D, int N, int NS, int QB>
 __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *map, uint8_t *smem,
                                         typename Cfg<D, N, NS, QB>::Small *sm, uint64_t *full,
-                                        uint64_t *empty, int *tab, uint32_t dst_off, bool stage_q,
-                                        int lane, volatile int *abort_any) {
+                                        uint64_t *empty, int (*tabs)[kSplitTokens / 16],
+                                        uint32_t dst_off, bool with_q, int lane,
+                                        volatile int *abort_any) {
   using C = Cfg<D, N, NS, QB>;
-  constexpr int kPastWidth = static_cast<int>(0x80000000u);
   if (lane == 0) tma_prefetch_desc(map);
-  int gi = 0, ui = 0;
-  bool failed = false;
   int last_gi[NS];
 #pragma unroll
   for (int i = 0; i < NS; ++i) last_gi[i] = -1;
-  const int bmask = (1 << p.block_shift) - 1;
-  for (int u = blockIdx.x; u < p.n_units && !failed; u += gridDim.x) {
-    const Unit x = unit_at<N>(p, u);
-    if (x.n_tiles == 0) continue;
-    if (stage_q) {
-      const int qb = ui % QB;
-      const bool ok = mbar_wait(&sm->q_empty[qb], ((ui / QB) & 1) ^ 1, abort_any);
-      if (__any_sync(0xffffffffu, !ok)) {
-        failed = true;
-        break;
-      }
-      uint8_t *qdst = smem + C::kOffQ + qb * C::kQBytes;
-      for (int idx = lane; idx < N * (D / 8); idx += 32) {
-        const int c = idx / (D / 8), ch = idx % (D / 8);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (c < x.rows) {
-          const int r = x.row0 + c;
-          const int i = r / p.G, g = r - i * p.G;
-          const __nv_bfloat16 *src = p.q + x.b * p.q_sb + static_cast<int64_t>(i) * p.q_ss +
-                                     static_cast<int64_t>(x.kvh * p.G + g) * p.q_sh + ch * 8;
-          v = __ldg(reinterpret_cast<const uint4 *>(src));
-        }
-        const int h = ch >> 3, cc = ch & 7;
-        *reinterpret_cast<uint4 *>(qdst + h * C::kQHalfBytes + c * 128 + ((cc ^ (c & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
-    }
-    {
-      const int ntok = min(kSplitTokens, x.lim_max - x.tok0);
-      const int first = x.tok0 >> p.block_shift;
-      const int nent = (ntok + bmask) >> p.block_shift;
-      for (int e = lane; e < nent; e += 32) {
-        const int col = first + e;
-        tab[e] = col < p.max_blocks_per_seq ? __ldg(p.block_table + x.b * p.bt_stride + col)
-                                            : kPastWidth;
-      }
-    }
+  bool failed = false;
+  Unit cur;
+  int cu = next_unit<N>(p, blockIdx.x, cur);
+  if (cu >= 0) {
+    const int bmask = (1 << p.block_shift) - 1;
+    int ui = 0, gi = 0;
+    // the first unit (Q buffer 0 is free)
+    stage_tab(p, cur, tabs[0], lane);
+    if (with_q) stage_q<D, N>(p, cur, smem + C::kOffQ, lane);
+    if (with_q) fence_proxy_async_smem();
     __syncwarp();
-    if (stage_q && lane == 0) mbar_arrive(&sm->q_full[ui % QB]);
-    for (int j = 0; j < x.n_tiles; ++j, ++gi) {
-      const int st = gi % NS;
-      bool okw = true;
-      if (lane == 0) okw = mbar_wait(&empty[st], ((gi / NS) & 1) ^ 1, abort_any);
-      if (!__shfl_sync(0xffffffffu, okw ? 1 : 0, 0)) {
-        failed = true;
-        break;
-      }
-      const int tok0 = x.tok0 + j * kTileTokens;
-      const int nvalid = min(kTileTokens, x.lim_max - tok0);
-      const int nbox = (nvalid + p.box_slots - 1) / p.box_slots;
-      int errs = 0;
-      if (lane < nbox) {
-        const int tok = tok0 + lane * p.box_slots;
-        const int blk = tab[(tok - x.tok0) >> p.block_shift];
-        if (blk == kPastWidth) {
-          errs = kErrTableWidth;
-        } else if (blk < 0 || static_cast<int64_t>(blk) >= p.num_blocks) {
-          errs = kErrBadBlock;
-        } else {
-          uint8_t *d0 = smem + dst_off + st * C::kKVBytes + lane * p.box_slots * 128;
-          const int slot = tok & bmask;
-          const int c1 = p.map_head_first ? x.kvh : slot;
-          const int c2 = p.map_head_first ? slot : x.kvh;
-          mbar_expect_tx(&full[st], static_cast<uint32_t>((D / 64) * p.box_slots * 128));
-#pragma unroll
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(d0 + h * C::kHalfBytes, map, &full[st], h * 64, c1, c2, blk);
+    if (with_q && lane == 0) mbar_arrive(&sm->q_full[0]);
+    while (true) {
+      // stage the next unit while this one's tiles are issued
+      Unit nxt;
+      const int nu = next_unit<N>(p, cu + gridDim.x, nxt);
+      bool q_early = false;
+      if (nu >= 0) stage_tab(p, nxt, tabs[(ui + 1) & 1], lane);
+      const int *tab = tabs[ui & 1];
+      for (int j = 0; j < cur.n_tiles && !failed; ++j, ++gi) {
+        if (with_q && QB == 2 && nu >= 0 && j == cur.n_tiles - 1) {
+          // the next unit's Q goes to the buffer of the previous unit, whose
+          // QKs are done by the time this unit's last tile is issued
+          const int qb = (ui + 1) % QB;
+          bool okq = true;
+          if (lane == 0) okq = mbar_wait(&sm->q_empty[qb], (((ui + 1) / QB) & 1) ^ 1, abort_any);
+          if (!__shfl_sync(0xffffffffu, okq ? 1 : 0, 0)) {
+            failed = true;
+            break;
+          }
+          stage_q<D, N>(p, nxt, smem + C::kOffQ + qb * C::kQBytes, lane);
+          q_early = true;
         }
+        const int st = gi % NS;
+        bool okw = true;
+        if (lane == 0) okw = mbar_wait(&empty[st], ((gi / NS) & 1) ^ 1, abort_any);
+        if (!__shfl_sync(0xffffffffu, okw ? 1 : 0, 0)) {
+          failed = true;
+          break;
+        }
+        const int tok0 = cur.tok0 + j * kTileTokens;
+        const int nvalid = min(kTileTokens, cur.lim_max - tok0);
+        const int nbox = (nvalid + p.box_slots - 1) / p.box_slots;
+        int errs = 0;
+        if (lane < nbox) {
+          const int tok = tok0 + lane * p.box_slots;
+          const int blk = tab[(tok - cur.tok0) >> p.block_shift];
+          if (blk == kPastWidth) {
+            errs = kErrTableWidth;
+          } else if (blk < 0 || static_cast<int64_t>(blk) >= p.num_blocks) {
+            errs = kErrBadBlock;
+          } else {
+            uint8_t *d0 = smem + dst_off + st * C::kKVBytes + lane * p.box_slots * 128;
+            const int slot = tok & bmask;
+            const int c1 = p.map_head_first ? cur.kvh : slot;
+            const int c2 = p.map_head_first ? slot : cur.kvh;
+            mbar_expect_tx(&full[st], static_cast<uint32_t>((D / 64) * p.box_slots * 128));
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_4d(d0 + h * C::kHalfBytes, map, &full[st], h * 64, c1, c2, blk);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&full[st]);
+          last_gi[st] = gi;
+        }
+        if (errs && p.err) atomicOr(p.err, errs);
       }
+      if (failed || nu < 0) break;
+      // unit boundary: the next unit's entries (and Q) are in shared memory
+      if (with_q && !q_early) {  // one Q buffer: wait until this unit's QKs are done
+        const int qb = (ui + 1) % QB;
+        bool okq = true;
+        if (lane == 0) okq = mbar_wait(&sm->q_empty[qb], (((ui + 1) / QB) & 1) ^ 1, abort_any);
+        if (!__shfl_sync(0xffffffffu, okq ? 1 : 0, 0)) {
+          failed = true;
+          break;
+        }
+        stage_q<D, N>(p, nxt, smem + C::kOffQ + qb * C::kQBytes, lane);
+      }
+      if (with_q) fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&full[st]);
-        last_gi[st] = gi;
-      }
-      if (errs && p.err) atomicOr(p.err, errs);
+      if (with_q && lane == 0) mbar_arrive(&sm->q_full[(ui + 1) % QB]);
+      ++ui;
+      cur = nxt;
+      cu = nu;
     }
-    ++ui;
   }
   if (failed && lane == 0) {
     // wait (bounded, ignoring the abort flag) for this warp's copies in flight
@@ -344,10 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
 
   if (warp == kKWarp) {
-    produce<D, N, NS, QB>(p, &map_k, smem, sm, sm->full_k, sm->empty_k, sm->tab_k, C::kOffK,
+    produce<D, N, NS, QB>(p, &map_k, smem, sm, sm->full_k, sm->empty_k, sm->tab[0], C::kOffK,
                           true, lane, abort_any);
   } else if (warp == kVWarp) {
-    produce<D, N, NS, QB>(p, &map_v, smem, sm, sm->full_v, sm->empty_v, sm->tab_v, C::kOffV,
+    produce<D, N, NS, QB>(p, &map_v, smem, sm, sm->full_v, sm->empty_v, sm->tab[1], C::kOffV,
                           false, lane, abort_any);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------
