@@ -6,8 +6,9 @@ Workload (one "step" = one pass of the whole hot path over one batch):
   each, Hq 32 / Hkv 8, head_dim 128, bf16 N(0,1) data, contiguous paged cache
   with block_size 16 and a seeded randperm block table [4, 8192], fixed split
   chunk 4096 tokens merged in global block order.  A step appends the newest
-  token's K/V (kv_append, position 131071) and runs paged_decode_attn over the
-  131072-token contexts (split kernel + merge kernel).
+  token's K/V (position 131071) and runs decode attention over the
+  131072-token contexts (split kernel + merge kernel), the append fused into
+  the same call (paged_decode_attn_append).
 
 value   = algorithmic KV bytes (every visible token read once per KV head, K
           and V, bf16) of all ranks / device time of the K timed steps (max
@@ -195,7 +196,6 @@ def run_ours(args):
     gen = torch.Generator(device=dev).manual_seed(2000 + rank)
     k_new = torch.randn(B, 1, Hkv, D, generator=gen, device=dev).to(torch.bfloat16)
     v_new = torch.randn(B, 1, Hkv, D, generator=gen, device=dev).to(torch.bfloat16)
-    seq_prev = torch.full((B,), ctx - 1, dtype=torch.int32, device=dev)
     seq = di.seqlens
     out = torch.empty(B, 1, Hq, D, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(B, Hq, 1, dtype=torch.float32, device=dev)
@@ -205,12 +205,12 @@ def run_ours(args):
     kv_bytes = di.kv_bytes()
 
     def step(ev0=None, ev1=None):
-        pkv.kv_append(k_new, v_new, di.cache.k, di.cache.v, di.block_table, seq_prev, err=err)
+        # kv_append of the newest token fused into the decode call
         if ev0 is not None:
             ev0.record(stream)
-        pkv.paged_decode_attn(di.q, di.cache.k, di.cache.v, di.block_table, seq,
-                              max_seqlen_k=ctx, scale=di.scale, causal=False, out=out, lse=lse,
-                              workspace=ws, err=err)
+        pkv.paged_decode_attn_append(di.q, k_new, v_new, di.cache.k, di.cache.v, di.block_table,
+                                     seq, max_seqlen_k=ctx, scale=di.scale, causal=False, out=out,
+                                     lse=lse, workspace=ws, err=err)
         if ev1 is not None:
             ev1.record(stream)
 
@@ -245,22 +245,21 @@ def run_ours(args):
     if not args.no_e2e:
         h_q = di.q.cpu().pin_memory()
         h_kn, h_vn = k_new.cpu().pin_memory(), v_new.cpu().pin_memory()
-        h_sp, h_s = seq_prev.cpu().pin_memory(), seq.cpu().pin_memory()
+        h_s = seq.cpu().pin_memory()
         h_bt = di.block_table.cpu().pin_memory()
         h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
         d_q, d_kn, d_vn = torch.empty_like(di.q), torch.empty_like(k_new), torch.empty_like(v_new)
-        d_sp, d_s, d_bt = torch.empty_like(seq_prev), torch.empty_like(seq), torch.empty_like(di.block_table)
-        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_sp, h_s, h_bt))
+        d_s, d_bt = torch.empty_like(seq), torch.empty_like(di.block_table)
+        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_s, h_bt))
         d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
 
         def e2e_step():
-            for d, h in ((d_q, h_q), (d_kn, h_kn), (d_vn, h_vn), (d_sp, h_sp), (d_s, h_s), (d_bt, h_bt)):
+            for d, h in ((d_q, h_q), (d_kn, h_kn), (d_vn, h_vn), (d_s, h_s), (d_bt, h_bt)):
                 d.copy_(h, non_blocking=True)
-            pkv.kv_append(d_kn, d_vn, di.cache.k, di.cache.v, d_bt, d_sp, err=err)
-            pkv.paged_decode_attn(d_q, di.cache.k, di.cache.v, d_bt, d_s, max_seqlen_k=ctx,
-                                  scale=di.scale, causal=False, out=out, lse=lse, workspace=ws,
-                                  err=err)
+            pkv.paged_decode_attn_append(d_q, d_kn, d_vn, di.cache.k, di.cache.v, d_bt, d_s,
+                                         max_seqlen_k=ctx, scale=di.scale, causal=False, out=out,
+                                         lse=lse, workspace=ws, err=err)
             h_out.copy_(out, non_blocking=True)
             h_lse.copy_(lse, non_blocking=True)
 
@@ -307,7 +306,7 @@ def run_ours(args):
         "config": {"workload": WORKLOAD, "batch": B, "seqlen_q": 1, "seqlen_k": ctx,
                    "Hq": Hq, "Hkv": Hkv, "head_dim": D, "block_size": 16,
                    "split_tokens": pkv.SPLIT_TOKENS,
-                   "step": "kv_append (1 token/sequence) + paged_decode_attn",
+                   "step": "paged_decode_attn_append: kv_append of 1 token/sequence fused into the decode call",
                    "l2": "inputs larger than L2 (2.15 GB of K/V per rank), no flush",
                    "parallelism": f"dp{world}"},
         "tokens_per_s": round(B * world * args.steps / (ms_total / 1e3), 1),
@@ -316,12 +315,12 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": profiled_traffic(),
-                     "kernel": "paged_decode_attn (attn_split_kernel<128,16,3> + merge_kernel<128>)",
+                     "kernel": "paged_decode_attn_append (attn_split_kernel<128,16,3,2> + merge_kernel<128>)",
                      "algorithmic_bytes_per_launch": kv_bytes,
                      "launch_ms_mean": round(dec_ms, 5),
                      "launch_ms_min": round(min(decode_ms), 5),
                      "peak_basis": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s"},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 2 * args.steps,
         "clocks": clocks.summary(),
         "e2e": e2e,
     }

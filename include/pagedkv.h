@@ -167,6 +167,35 @@ int pkv_paged_prefill_attn(const void *q, const int64_t q_strides[3],
                            void *workspace, size_t workspace_bytes,
                            int32_t *err, void *stream);
 
+/*
+ * pkv_paged_decode_attn_append: kv_append fused into the attention call --
+ * the "new_kv" form of flash_attn_with_kvcache in the aiter test grid.  The
+ * n_new tokens of k_new/v_new ([batch, n_new, Hkv, D] bf16, element strides
+ * kn_strides / vn_strides = (batch, token, head)) are written to cache
+ * positions seqlens[b] - n_new + t (seqlens count them: the context length
+ * AFTER the append, as in pkv_paged_decode_attn), and the attention then reads
+ * them.  On return the cache holds exactly the bits pkv_kv_append would have
+ * written (with seqlens - n_new), and out / lse are bitwise those of
+ * pkv_kv_append followed by pkv_paged_decode_attn: one launch fewer per
+ * decode step.  Requires 1 <= n_new <= PKV_SPLIT_TOKENS and n_new <=
+ * seqlens[b] (positions below 0 are not written).  Other arguments as for
+ * pkv_paged_decode_attn; the cache views must be writable.
+ */
+int pkv_paged_decode_attn_append(const void *q, const int64_t q_strides[3],
+                                 const void *k_new, const int64_t kn_strides[3],
+                                 const void *v_new, const int64_t vn_strides[3], int n_new,
+                                 void *k_cache, const int64_t k_strides[3],
+                                 void *v_cache, const int64_t v_strides[3],
+                                 int64_t num_blocks,
+                                 const int32_t *block_table, int64_t bt_stride,
+                                 int max_blocks_per_seq,
+                                 const int32_t *seqlens, int max_seqlen_k,
+                                 int batch, int seqlen_q, int Hq, int Hkv, int D, int block_size,
+                                 float scale, int causal,
+                                 void *out, const int64_t out_strides[3], float *lse,
+                                 void *workspace, size_t workspace_bytes,
+                                 int32_t *err, void *stream);
+
 /* Workspace bytes the attention calls need: fp32 split partials
  * (m, l, acc[D]) for every (batch, query row, query head, split). */
 size_t pkv_workspace_size(int batch, int seqlen_q, int Hq, int D, int max_seqlen_k);

@@ -12,6 +12,7 @@ from .binding import (  # noqa: F401
     kv_append,
     library_path,
     paged_decode_attn,
+    paged_decode_attn_append,
     paged_prefill_attn,
     strerror,
     workspace_size,

@@ -172,6 +172,52 @@ def paged_decode_attn(q, k_cache, v_cache, block_table, seqlens, *, max_seqlen_k
                  max_seqlen_k, scale, causal, out, lse, workspace, err, stream)
 
 
+def paged_decode_attn_append(q, k_new, v_new, k_cache, v_cache, block_table, seqlens, *,
+                             max_seqlen_k=None, scale=None, causal=False, out=None, lse=None,
+                             workspace=None, err=None, stream=None):
+    """kv_append fused into decode: writes k_new/v_new [B, n_new, Hkv, D] at
+    positions seqlens[b] - n_new + t (seqlens already count them), then attends.
+    Bitwise equal to kv_append(seqlens - n_new) followed by paged_decode_attn."""
+    _need_cuda_bf16("k_new", k_new)
+    _need_cuda_bf16("v_new", v_new)
+    L = lib()
+    fn = L.pkv_paged_decode_attn_append
+    if not fn.argtypes:
+        fn.argtypes = [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I64, _P, _I64, _I, _P, _I,
+                       _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P, _P, _P, _P,
+                       ctypes.c_size_t, _P, _P]
+        fn.restype = _I
+    _need_cuda_bf16("q", q)
+    _need_cuda_bf16("k_cache", k_cache)
+    _need_cuda_bf16("v_cache", v_cache)
+    _need_cuda_i32("block_table", block_table)
+    _need_cuda_i32("seqlens", seqlens)
+    if block_table.stride(1) != 1:
+        raise ValueError("block_table must have a unit column stride")
+    B, sq, Hq, D = q.shape
+    num_blocks, bs, Hkv, _ = k_cache.shape
+    if max_seqlen_k is None:
+        max_seqlen_k = int(seqlens.max().item()) if seqlens.numel() else 0
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(B, sq, Hq, D, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, Hq, sq, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_size(B, sq, Hq, D, max_seqlen_k), dtype=torch.uint8,
+                                device=q.device)
+    rc = fn(q.data_ptr(), _st3(q), k_new.data_ptr(), _st3(k_new), v_new.data_ptr(), _st3(v_new),
+            int(k_new.shape[1]), k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(),
+            _st3(v_cache), num_blocks, block_table.data_ptr(), int(block_table.stride(0)),
+            int(block_table.shape[1]), seqlens.data_ptr(), int(max_seqlen_k), B, sq, Hq, Hkv, D, bs,
+            float(scale), int(bool(causal)), out.data_ptr(), _st3(out), lse.data_ptr(),
+            workspace.data_ptr(), workspace.numel() * workspace.element_size(), _ptr(err),
+            _stream_handle(stream))
+    _check("pkv_paged_decode_attn_append", rc)
+    return out, lse
+
+
 def paged_prefill_attn(q, k_cache, v_cache, block_table, seqlens, *, max_seqlen_k=None,
                        scale=None, causal=True, out=None, lse=None, workspace=None, err=None,
                        stream=None):

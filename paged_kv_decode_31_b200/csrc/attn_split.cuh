@@ -77,6 +77,13 @@ struct AttnParams {
   float *ws_acc;        // [rows][n_splits][D]
   float *ws_ml;         // [rows][n_splits][2] (max in base-2 scaled units, sum)
   int32_t *err;
+  // Fused append (n_new > 0): token t of k_new/v_new [batch, n_new, Hkv, D] is
+  // written to position seqlens[b] - n_new + t before it is read.
+  int n_new;
+  const uint16_t *k_new, *v_new;
+  int64_t kn_sb, kn_st, kn_sh, vn_sb, vn_st, vn_sh;
+  uint16_t *k_cache, *v_cache;
+  int64_t k_sb, k_ss, k_sh, v_sb, v_ss, v_sh;
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -241,6 +248,39 @@ __device__ __forceinline__ void stage_tab(const AttnParams &p, const Unit &x, in
   }
 }
 
+// Fused append: write the new tokens that fall inside this unit's loaded key
+// range [tok0, min(tok0 + 4096, lim_max)) for this unit's KV head -- K from the
+// K producer, V from the V producer -- then order those generic writes before
+// the warp's TMA reads of the same rows.  Every unit that loads a new position
+// writes it itself (the same bits), so no unit depends on another.
+template <int D>
+__device__ __forceinline__ void append_new_tokens(const AttnParams &p, const Unit &x,
+                                                  const int *tab, bool is_k, int lane) {
+  const int first_new = x.seqlen - p.n_new;
+  const int lo = max(first_new, x.tok0);
+  const int hi = min(x.lim_max, x.tok0 + kSplitTokens);
+  if (lo < hi) {
+    const uint16_t *src = is_k ? p.k_new : p.v_new;
+    uint16_t *cache = is_k ? p.k_cache : p.v_cache;
+    const int64_t nb = is_k ? p.kn_sb : p.vn_sb, nt = is_k ? p.kn_st : p.vn_st,
+                  nh = is_k ? p.kn_sh : p.vn_sh;
+    const int64_t cb = is_k ? p.k_sb : p.v_sb, cs = is_k ? p.k_ss : p.v_ss,
+                  ch_ = is_k ? p.k_sh : p.v_sh;
+    const int bmask = (1 << p.block_shift) - 1;
+    for (int idx = lane; idx < (hi - lo) * (D / 8); idx += 32) {
+      const int tok = lo + idx / (D / 8), c = idx % (D / 8);
+      const int blk = tab[(tok - x.tok0) >> p.block_shift];
+      if (blk == kPastWidth || blk < 0 || static_cast<int64_t>(blk) >= p.num_blocks) continue;
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
+          src + x.b * nb + static_cast<int64_t>(tok - first_new) * nt + x.kvh * nh) + c);
+      reinterpret_cast<uint4 *>(cache + blk * cb + static_cast<int64_t>(tok & bmask) * cs +
+                                x.kvh * ch_)[c] = v;
+    }
+    fence_proxy_async_global();
+  }
+  __syncwarp();
+}
+
 // One producer warp.  The current unit's block-table entries (and, for the K
 // warp, its Q rows) are already in shared memory when its first tile is
 // issued: the warp stages the NEXT unit's entries at the start of every unit
@@ -276,7 +316,8 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
       const int nu = next_unit<N>(p, cu + gridDim.x, nxt);
       bool q_early = false;
       if (nu >= 0) stage_tab(p, nxt, tabs[(ui + 1) & 1], lane);
-      const int *tab = tabs[ui & 1];
+        const int *tab = tabs[ui & 1];
+      if (p.n_new > 0) append_new_tokens<D>(p, cur, tab, with_q, lane);
       for (int j = 0; j < cur.n_tiles && !failed; ++j, ++gi) {
         if (with_q && QB == 2 && nu >= 0 && j == cur.n_tiles - 1) {
           // the next unit's Q goes to the buffer of the previous unit, whose

@@ -164,13 +164,21 @@ int launch_merge(const pkv::MergeParams &m, int64_t rows, cudaStream_t s) {
 // group fits (decode), else 64.  Both sizes run the same arithmetic per row.
 int rows_per_tile(int rows) { return rows <= 16 ? 16 : 64; }
 
+// New tokens written into the cache by the attention call itself.
+struct FusedAppend {
+  const void *k_new, *v_new;
+  const int64_t *kn_strides, *vn_strides;
+  int n_new;
+};
+
 int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
                const int64_t k_strides[3], const void *v_cache, const int64_t v_strides[3],
                int64_t num_blocks, const int32_t *block_table, int64_t bt_stride,
                int max_blocks_per_seq, const int32_t *seqlens, int max_seqlen_k, int batch,
                int seqlen_q, int Hq, int Hkv, int D, int block_size, float scale, int causal,
                void *out, const int64_t out_strides[3], float *lse, void *workspace,
-               size_t workspace_bytes, int32_t *err, void *stream) {
+               size_t workspace_bytes, int32_t *err, void *stream,
+               const FusedAppend *app = nullptr) {
   if (!q || !k_cache || !v_cache || !block_table || !seqlens || !out || !lse) return PKV_ERR_ARG;
   if (batch <= 0 || seqlen_q <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return PKV_ERR_ARG;
   if (D != 64 && D != 128) return PKV_ERR_ARG;
@@ -235,6 +243,29 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   p.ws_acc = ws_acc;
   p.ws_ml = ws_ml;
   p.err = err;
+  if (app && app->n_new > 0) {
+    if (!app->k_new || !app->v_new || !strides_ok(app->kn_strides) ||
+        !strides_ok(app->vn_strides) || !aligned16(app->k_new) || !aligned16(app->v_new) ||
+        app->n_new > pkv::kSplitTokens)
+      return PKV_ERR_ARG;
+    p.n_new = app->n_new;
+    p.k_new = static_cast<const uint16_t *>(app->k_new);
+    p.v_new = static_cast<const uint16_t *>(app->v_new);
+    p.kn_sb = app->kn_strides[0];
+    p.kn_st = app->kn_strides[1];
+    p.kn_sh = app->kn_strides[2];
+    p.vn_sb = app->vn_strides[0];
+    p.vn_st = app->vn_strides[1];
+    p.vn_sh = app->vn_strides[2];
+    p.k_cache = static_cast<uint16_t *>(const_cast<void *>(k_cache));
+    p.v_cache = static_cast<uint16_t *>(const_cast<void *>(v_cache));
+    p.k_sb = k_strides[0];
+    p.k_ss = k_strides[1];
+    p.k_sh = k_strides[2];
+    p.v_sb = v_strides[0];
+    p.v_ss = v_strides[1];
+    p.v_sh = v_strides[2];
+  }
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (D == 128)
@@ -344,6 +375,25 @@ int pkv_paged_prefill_attn(const void *q, const int64_t q_strides[3], const void
                     bt_stride, max_blocks_per_seq, seqlens, max_seqlen_k, batch, seqlen_q, Hq, Hkv,
                     D, block_size, scale, causal, out, out_strides, lse, workspace,
                     workspace_bytes, err, stream);
+}
+
+int pkv_paged_decode_attn_append(const void *q, const int64_t q_strides[3], const void *k_new,
+                                 const int64_t kn_strides[3], const void *v_new,
+                                 const int64_t vn_strides[3], int n_new, void *k_cache,
+                                 const int64_t k_strides[3], void *v_cache,
+                                 const int64_t v_strides[3], int64_t num_blocks,
+                                 const int32_t *block_table, int64_t bt_stride,
+                                 int max_blocks_per_seq, const int32_t *seqlens, int max_seqlen_k,
+                                 int batch, int seqlen_q, int Hq, int Hkv, int D, int block_size,
+                                 float scale, int causal, void *out, const int64_t out_strides[3],
+                                 float *lse, void *workspace, size_t workspace_bytes, int32_t *err,
+                                 void *stream) {
+  if (n_new < 1) return PKV_ERR_ARG;
+  const FusedAppend app{k_new, v_new, kn_strides, vn_strides, n_new};
+  return attn_entry(q, q_strides, k_cache, k_strides, v_cache, v_strides, num_blocks, block_table,
+                    bt_stride, max_blocks_per_seq, seqlens, max_seqlen_k, batch, seqlen_q, Hq, Hkv,
+                    D, block_size, scale, causal, out, out_strides, lse, workspace,
+                    workspace_bytes, err, stream, &app);
 }
 
 size_t pkv_workspace_size(int batch, int seqlen_q, int Hq, int D, int max_seqlen_k) {

@@ -91,6 +91,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Make this thread's generic-proxy global-memory writes visible to its later
+// async-proxy (TMA) reads of the same addresses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // TMA: 4-D tiled tensor load global -> shared, completion on an mbarrier.
 // No multicast.
