@@ -84,6 +84,12 @@ struct AttnParams {
   int64_t kn_sb, kn_st, kn_sh, vn_sb, vn_st, vn_sh;
   uint16_t *k_cache, *v_cache;
   int64_t k_sb, k_ss, k_sh, v_sb, v_ss, v_sh;
+  // Direct final write (row-major kernel, one split per row): out / lse are
+  // written by the split kernel itself with the merge's arithmetic.
+  int direct, out_vec;
+  __nv_bfloat16 *out;
+  int64_t o_sb, o_ss, o_sh;
+  float *lse;
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -137,6 +143,8 @@ struct Cfg {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(N == 16 || N == 32 || N == 64, "rows per tile");
   static_assert(QB == 1 || QB == 2, "Q buffers");
+  static constexpr int kD = D, kN = N, kNS = NS, kQB = QB;
+  static constexpr bool kQTma = false;  // Q rows staged with plain loads
   static constexpr int kHalfBytes = kTileTokens * 128;   // 128 tokens x 64 head_dim x bf16
   static constexpr int kKVBytes = (D / 64) * kHalfBytes;  // one K (or V) tile
   static constexpr int kQHalfBytes = N * 128;
@@ -287,14 +295,30 @@ __device__ __forceinline__ void append_new_tokens(const AttnParams &p, const Uni
 // and (two Q buffers) the next unit's Q just before the current unit's last
 // tile -- points where its stage ring is full and it would wait anyway.  Per tile, lane k issues the TMA boxes of the tile's k-th box of cache
 // rows, all lanes in parallel; lane 0 arrives on `full`.
-template <int D, int N, int NS, int QB>
-__device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *map, uint8_t *smem,
-                                        typename Cfg<D, N, NS, QB>::Small *sm, uint64_t *full,
-                                        uint64_t *empty, int (*tabs)[kSplitTokens / 16],
-                                        uint32_t dst_off, bool with_q, int lane,
-                                        volatile int *abort_any) {
-  using C = Cfg<D, N, NS, QB>;
+template <class C>
+__device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *map,
+                                        const CUtensorMap *map_q, uint8_t *smem,
+                                        typename C::Small *sm, uint64_t *full, uint64_t *empty,
+                                        int (*tabs)[kSplitTokens / 16], uint32_t dst_off,
+                                        bool with_q, int lane, volatile int *abort_any) {
+  constexpr int D = C::kD, N = C::kN, NS = C::kNS, QB = C::kQB;
+  // Q of unit u into buffer qb: TMA (completing on q_full[qb]) or plain loads
+  auto put_q = [&](const Unit &u, int qb) {
+    if constexpr (C::kQTma) {
+      if (lane == 0) {
+        mbar_expect_tx(&sm->q_full[qb], static_cast<uint32_t>(C::kQBytes));
+        const int i0 = u.row0 / p.G;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_4d(smem + C::kOffQ + qb * C::kQBytes + h * C::kQHalfBytes, map_q,
+                      &sm->q_full[qb], h * 64, u.kvh * p.G, i0, u.b);
+      }
+    } else {
+      stage_q<D, N>(p, u, smem + C::kOffQ + qb * C::kQBytes, lane);
+    }
+  };
   if (lane == 0) tma_prefetch_desc(map);
+  if (C::kQTma && with_q && lane == 0) tma_prefetch_desc(map_q);
   int last_gi[NS];
 #pragma unroll
   for (int i = 0; i < NS; ++i) last_gi[i] = -1;
@@ -306,7 +330,7 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
     int ui = 0, gi = 0;
     // the first unit (Q buffer 0 is free)
     stage_tab(p, cur, tabs[0], lane);
-    if (with_q) stage_q<D, N>(p, cur, smem + C::kOffQ, lane);
+    if (with_q) put_q(cur, 0);
     if (with_q) fence_proxy_async_smem();
     __syncwarp();
     if (with_q && lane == 0) mbar_arrive(&sm->q_full[0]);
@@ -316,7 +340,7 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
       const int nu = next_unit<N>(p, cu + gridDim.x, nxt);
       bool q_early = false;
       if (nu >= 0) stage_tab(p, nxt, tabs[(ui + 1) & 1], lane);
-        const int *tab = tabs[ui & 1];
+      const int *tab = tabs[ui & 1];
       if (p.n_new > 0) append_new_tokens<D>(p, cur, tab, with_q, lane);
       for (int j = 0; j < cur.n_tiles && !failed; ++j, ++gi) {
         if (with_q && QB == 2 && nu >= 0 && j == cur.n_tiles - 1) {
@@ -329,7 +353,7 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
             failed = true;
             break;
           }
-          stage_q<D, N>(p, nxt, smem + C::kOffQ + qb * C::kQBytes, lane);
+          put_q(nxt, qb);
           q_early = true;
         }
         const int st = gi % NS;
@@ -378,7 +402,7 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
           failed = true;
           break;
         }
-        stage_q<D, N>(p, nxt, smem + C::kOffQ + qb * C::kQBytes, lane);
+        put_q(nxt, qb);
       }
       if (with_q) fence_proxy_async_smem();
       __syncwarp();
@@ -441,11 +465,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
 
   if (warp == kKWarp) {
-    produce<D, N, NS, QB>(p, &map_k, smem, sm, sm->full_k, sm->empty_k, sm->tab[0], C::kOffK,
-                          true, lane, abort_any);
+    produce<C>(p, &map_k, nullptr, smem, sm, sm->full_k, sm->empty_k, sm->tab[0], C::kOffK, true,
+               lane, abort_any);
   } else if (warp == kVWarp) {
-    produce<D, N, NS, QB>(p, &map_v, smem, sm, sm->full_v, sm->empty_v, sm->tab[1], C::kOffV,
-                          false, lane, abort_any);
+    produce<C>(p, &map_v, nullptr, smem, sm, sm->full_v, sm->empty_v, sm->tab[1], C::kOffV, false,
+               lane, abort_any);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------
     // MMA issuer (one thread)

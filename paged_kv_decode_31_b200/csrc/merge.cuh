@@ -8,7 +8,7 @@
 //
 //   M' = max(M, m_s), a = 2^(M - M'), c = 2^(m_s - M')
 //   L  = fma(l_s, c, L * a),  A = fma(acc_s, c, A * a),  M = M'
-//   out = bf16_rn(A / L),     lse = (M + log2 L) * ln 2
+//   out = bf16_rn(A / L),     lse = (M + log2 L) * ln 2   (L = 0: out 0, lse -inf)
 //
 // m_s is in base-2 scaled units (scale * log2(e) * q.k), so lse comes out in
 // the natural-log, scale * q.k domain.  The same code merges every row of
@@ -30,6 +30,26 @@ struct MergeParams {
   int64_t o_sb, o_ss, o_sh;
   float *lse;
 };
+
+// One step of the ascending fold: partial (m_s, l_s, x_s) into (M, L, X).
+struct FoldCoef {
+  float Mn, a, c;
+};
+__device__ __forceinline__ FoldCoef fold_coef(float M, float m_s) {
+  const float Mn = fmaxf(M, m_s);
+  return FoldCoef{Mn, ex2(__fsub_rn(M, Mn)), ex2(__fsub_rn(m_s, Mn))};
+}
+__device__ __forceinline__ float fold_val(float X, float x_s, const FoldCoef &k) {
+  return __fmaf_rn(x_s, k.c, __fmul_rn(X, k.a));
+}
+// Final write of a folded row: out element and lse.
+__device__ __forceinline__ float final_out(float A, float L) {
+  return L > 0.f ? __fdiv_rn(A, L) : 0.f;
+}
+__device__ __forceinline__ float final_lse(float M, float L) {
+  return L > 0.f ? __fmul_rn(__fadd_rn(M, log2f(L)), 0.69314718055994531f)
+                 : __int_as_float(0xff800000);
+}
 
 template <int D>
 __global__ void __launch_bounds__(D) merge_kernel(const __grid_constant__ MergeParams p) {
@@ -63,20 +83,14 @@ __global__ void __launch_bounds__(D) merge_kernel(const __grid_constant__ MergeP
 #pragma unroll
     for (int k = 0; k < kBatch; ++k) {
       if (ms[k] == NEG_INF) continue;  // the row sees no key of this split
-      const float Mn = fmaxf(M, ms[k]);
-      const float a = ex2(__fsub_rn(M, Mn));
-      const float c = ex2(__fsub_rn(ms[k], Mn));
-      L = __fmaf_rn(ls[k], c, __fmul_rn(L, a));
-      A = __fmaf_rn(as[k], c, __fmul_rn(A, a));
-      M = Mn;
+      const FoldCoef kc = fold_coef(M, ms[k]);
+      L = fold_val(L, ls[k], kc);
+      A = fold_val(A, as[k], kc);
+      M = kc.Mn;
     }
   }
-  const bool any = L > 0.f;
-  const float o = any ? __fdiv_rn(A, L) : 0.f;
-  p.out[b * p.o_sb + i * p.o_ss + h * p.o_sh + d] = __float2bfloat16_rn(o);
-  if (d == 0)
-    p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.seqlen_q + i] =
-        any ? __fmul_rn(__fadd_rn(M, log2f(L)), 0.69314718055994531f) : NEG_INF;
+  p.out[b * p.o_sb + i * p.o_ss + h * p.o_sh + d] = __float2bfloat16_rn(final_out(A, L));
+  if (d == 0) p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.seqlen_q + i] = final_lse(M, L);
 }
 
 }  // namespace pkv

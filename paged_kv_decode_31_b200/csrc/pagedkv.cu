@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "pagedkv.h"
+#include "attn_rows.cuh"
 #include "attn_split.cuh"
 #include "kv_append.cuh"
 #include "merge.cuh"
@@ -123,6 +124,28 @@ int make_kv_map(CUtensorMap *map, const void *base, const int64_t st[3], int64_t
   return PKV_OK;
 }
 
+// TMA map over q [batch, seqlen_q, Hq, D] with element strides (b, s, h).
+// The box is 64 head_dim x G heads x 128 / G tokens of one sequence: it lands
+// as the 128 rows r = i * G + g of one row tile (row r at r * 128 bytes,
+// 128-byte swizzled); tokens past seqlen_q read as zeros.
+int make_q_map(CUtensorMap *map, const void *q, const int64_t st[3], int batch, int seqlen_q,
+               int Hq, int D, int G) {
+  auto enc = encode_fn();
+  if (!enc) return PKV_ERR_CUDA;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hq),
+                        static_cast<cuuint64_t>(seqlen_q), static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(st[2] * 2), static_cast<cuuint64_t>(st[1] * 2),
+                           static_cast<cuuint64_t>(st[0] * 2)};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(G),
+                       static_cast<cuuint32_t>(pkv::kRowsPerTile / G), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  std::memset(map, 0, sizeof(*map));
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_LAYOUT;
+}
+
 // Pipeline depth (K/V stages) and Q buffers per instance, sized to the
 // 227 KB of shared memory one CTA may use.
 template <int D, int N>
@@ -154,6 +177,31 @@ int launch_split(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensor
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// The row-major kernel rebalances registers between warpgroups; the shares
+// add up to exactly the allocation of a launch built with kRowsLaunchRegs
+// registers per thread, so the launch is refused if the build differs.
+template <int D>
+int launch_rows(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensorMap &mv,
+                const CUtensorMap &mq, cudaStream_t s, int dev) {
+  constexpr int NS = D == 128 ? 2 : 4;
+  using C = pkv::RowCfg<D, NS>;
+  static_assert(C::kSmemBytes <= 232448, "shared memory budget");
+  static std::atomic<bool> attr_set[kMaxDevices];
+  auto kern = pkv::attn_rows_kernel<D, NS>;
+  if (dev < 0 || dev >= kMaxDevices || !attr_set[dev].load(std::memory_order_acquire)) {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return PKV_ERR_CUDA;
+    if (fa.numRegs != pkv::kRowsLaunchRegs) return PKV_ERR_CUDA;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+      return PKV_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices) attr_set[dev].store(true, std::memory_order_release);
+  }
+  const int grid = p.n_units < sm_count(dev) ? p.n_units : sm_count(dev);
+  kern<<<grid, pkv::kRowThreads, C::kSmemBytes, s>>>(p, mk, mv, mq);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 template <int D>
 int launch_merge(const pkv::MergeParams &m, int64_t rows, cudaStream_t s) {
   pkv::merge_kernel<D><<<static_cast<unsigned>(rows), D, 0, s>>>(m);
@@ -161,8 +209,15 @@ int launch_merge(const pkv::MergeParams &m, int64_t rows, cudaStream_t s) {
 }
 
 // Rows of query heads x tokens per tile: 16 when a KV head's whole query
-// group fits (decode), else 64.  Both sizes run the same arithmetic per row.
-int rows_per_tile(int rows) { return rows <= 16 ? 16 : 64; }
+// group fits (decode), 64 up to 64 rows, else 128 rows in the row-major
+// kernel -- when G divides 128 (a Q box is whole tokens) and the box's
+// 128 / G tokens fit inside seqlen_q (no TMA box is ever larger than the
+// tensor it reads); otherwise 64.  Every size runs the same arithmetic per row.
+int rows_per_tile(int64_t rows, int G, int seqlen_q) {
+  if (rows <= 16) return 16;
+  if (rows <= 64 || pkv::kRowsPerTile % G != 0 || pkv::kRowsPerTile / G > seqlen_q) return 64;
+  return pkv::kRowsPerTile;
+}
 
 // New tokens written into the cache by the attention call itself.
 struct FusedAppend {
@@ -195,7 +250,11 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   const int64_t R = static_cast<int64_t>(G) * seqlen_q;
   const int64_t rows = static_cast<int64_t>(batch) * seqlen_q * Hq;
   if (R > INT32_MAX / 2 || rows > INT32_MAX) return PKV_ERR_ARG;
-  const int N = rows_per_tile(static_cast<int>(R));
+  alignas(64) CUtensorMap mq;
+  int N = rows_per_tile(R, G, seqlen_q);
+  if (N == pkv::kRowsPerTile &&
+      make_q_map(&mq, q, q_strides, batch, seqlen_q, Hq, D, G) != PKV_OK)
+    N = 64;  // q's strides cannot be described to the TMA unit: transposed kernel
   const int64_t S = max_seqlen_k > 0 ? ceil_div(max_seqlen_k, pkv::kSplitTokens) : 1;
   const int64_t RT = ceil_div(R, N);
   const int64_t units = static_cast<int64_t>(batch) * S * Hkv * RT;
@@ -268,10 +327,25 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   }
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (D == 128)
+  if (N == pkv::kRowsPerTile) {
+    // one split per row: the split kernel writes out / lse itself
+    p.direct = S == 1 ? 1 : 0;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.o_sb = out_strides[0];
+    p.o_ss = out_strides[1];
+    p.o_sh = out_strides[2];
+    p.lse = lse;
+    p.out_vec = (aligned16(out) && out_strides[0] % 8 == 0 && out_strides[1] % 8 == 0 &&
+                 out_strides[2] % 8 == 0)
+                    ? 1
+                    : 0;
+    rc = D == 128 ? launch_rows<128>(p, mk, mv, mq, s, dev) : launch_rows<64>(p, mk, mv, mq, s, dev);
+    if (rc != PKV_OK || p.direct) return rc;
+  } else if (D == 128) {
     rc = N == 16 ? launch_split<128, 16>(p, mk, mv, s, dev) : launch_split<128, 64>(p, mk, mv, s, dev);
-  else
+  } else {
     rc = N == 16 ? launch_split<64, 16>(p, mk, mv, s, dev) : launch_split<64, 64>(p, mk, mv, s, dev);
+  }
   if (rc != PKV_OK) return rc;
 
   pkv::MergeParams m{};
