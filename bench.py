@@ -61,6 +61,9 @@ def parse_args():
     ap.add_argument("--context", type=int, default=131072,
                     help="tokens per sequence (a smaller workload for profiling captures)")
     ap.add_argument("--batch", type=int, default=4)
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only the chunked causal prefill (--steps repetitions, "
+                         "2 warm-up passes) and print its result object")
     return ap.parse_args()
 
 
@@ -181,8 +184,9 @@ def cpu_baseline(di_dev, n_seq: int = 2):
 
 def prefill_secondary(dev, reps: int = 5):
     """Chunked causal prefill of the parity workload (batch 8, Hq 16 / Hkv 4,
-    D 128, block_size 16): 4 chunks of 512 tokens, each appended with the
-    fused call.  Algorithmic flops: 4 * D per (query row, visible key) for
+    D 128, block_size 16): 4 chunks of 512 tokens, each appended and attended
+    by one paged_decode_attn_append call (an append launch, then the row-major
+    attention kernel).  Algorithmic flops: 4 * D per (query row, visible key) for
     Q K^T and P V.  Returns the secondary result object."""
     import paged_kv_decode_31_b200 as pkv
     from paged_kv_decode_31_b200 import inputs as I
@@ -193,29 +197,35 @@ def prefill_secondary(dev, reps: int = 5):
     ws = torch.empty(pkv.workspace_size(B, chunk, Hq, D, 2048), dtype=torch.uint8, device=dev)
     seqs = [torch.full((B,), chunk * (c + 1), dtype=torch.int32, device=dev) for c in range(4)]
 
-    def prefill():
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(reps)]
+
+    def prefill(marks=None):
         for c in range(4):
+            if marks is not None:
+                marks[c].record()
             s, e = chunk * c, chunk * (c + 1)
             pkv.paged_decode_attn_append(q_all[:, s:e], k_all[:, s:e], v_all[:, s:e], cache.k,
                                          cache.v, table, seqs[c], max_seqlen_k=e, causal=True,
                                          out=outs[c], lse=lses[c], workspace=ws)
+        if marks is not None:
+            marks[4].record()
 
     for _ in range(2):
         prefill()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    a.record()
-    for _ in range(reps):
-        prefill()
-    b.record()
+    for r in range(reps):
+        prefill(ev[r])
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / reps
+    chunk_ms = [sum(ev[r][c].elapsed_time(ev[r][c + 1]) for r in range(reps)) / reps
+                for c in range(4)]
+    ms = sum(ev[r][0].elapsed_time(ev[r][4]) for r in range(reps)) / reps
     pairs = sum(p + 1 for p in range(4 * chunk))          # (query token, visible key)
     flops = 4.0 * D * pairs * B * Hq
     tflops = flops / (ms / 1e3) / 1e12
     return {"workload": "chunked causal prefill, batch 8 x 2048 tokens in 4 chunks of 512, "
-                        "Hq 16, Hkv 4, D 128, block_size 16 (append fused)",
+                        "Hq 16, Hkv 4, D 128, block_size 16 (append + attention per chunk)",
             "ms_per_prefill": round(ms, 4), "tflops": round(tflops, 2),
+            "chunk_us": [round(1e3 * x, 1) for x in chunk_ms],
             "algorithmic_flops": flops}
 
 
@@ -435,6 +445,10 @@ def run_reference(args):
 
 def main():
     args = parse_args()
+    if args.prefill_only:
+        torch.cuda.set_device(0)
+        print(json.dumps(prefill_secondary(torch.device("cuda", 0), reps=max(args.steps, 1))))
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -21,9 +21,10 @@
  * query row is cut into fixed chunks ("splits") of PKV_SPLIT_TOKENS tokens
  * starting at absolute position 0, each split into tiles of PKV_TILE_TOKENS
  * tokens.  Within a split, tiles are folded in ascending order with an online
- * softmax in fp32 (scores, P.V and the row sums on the tensor cores with fp32
- * accumulation; each probability enters them as a bf16 hi part plus a bf16
- * remainder, ~16 significant bits).  Split partials are
+ * softmax in fp32: scores and P.V on the tensor cores with fp32 accumulation
+ * (P entering P.V as bf16), each tile's max and row sums of the fp32
+ * probabilities on the CUDA cores in fixed reduction trees, and the running
+ * rescale in fp32 with the tile's own max.  Split partials are
  * merged in ascending split index (= global block index) order in fp32, and
  * out is rounded to bf16 once, at the final write.  Source: RL-Kernel PR #284
  * "feat(attention): add CP backward drift validation", Changes ("fixed
@@ -176,9 +177,12 @@ int pkv_paged_prefill_attn(const void *q, const int64_t q_strides[3],
  * AFTER the append, as in pkv_paged_decode_attn), and the attention then reads
  * them.  On return the cache holds exactly the bits pkv_kv_append would have
  * written (with seqlens - n_new), and out / lse are bitwise those of
- * pkv_kv_append followed by pkv_paged_decode_attn: one launch fewer per
- * decode step.  Requires 1 <= n_new <= PKV_SPLIT_TOKENS and n_new <=
- * seqlens[b] (positions below 0 are not written).  Other arguments as for
+ * pkv_kv_append followed by pkv_paged_decode_attn.  With at most 16 new
+ * tokens and at most one tile of query rows per KV head (decode steps) the
+ * attention kernel writes them itself, one launch fewer per step; otherwise
+ * (prefill chunks) an append launch precedes the attention on the same
+ * stream.  Requires 1 <= n_new <= PKV_SPLIT_TOKENS and n_new <= seqlens[b]
+ * (positions below 0 are not written).  Other arguments as for
  * pkv_paged_decode_attn; the cache views must be writable.
  */
 int pkv_paged_decode_attn_append(const void *q, const int64_t q_strides[3],

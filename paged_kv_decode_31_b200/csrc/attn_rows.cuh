@@ -10,16 +10,15 @@
 //   softmax one thread per ROW: all of a row's reductions are in-thread
 //           (the row sum replays the 32-key shuffle-down trees and the
 //           four-warp combine of attn_split.cuh element for element),
-//   P      = [bf16(p) | bf16(p - bf16(p))] written back over S in TMEM,
-//   O      = P_hi * V + P_lo * V with P read from TMEM (A operand) and V from
-//           shared memory (MN-major),
-//   update acc = fma(O_hi + O_lo, b, acc * a) per row in the correction
-//           warpgroup, which owns the row's (m, l, acc[D]) in registers.
+//   P      = bf16(p) written back over the front of the S buffer in TMEM,
+//   O      = P * V with P read from TMEM (A operand) and V from shared memory
+//           (MN-major),
+//   update acc = fma(O, b, acc * a) per row in the correction warpgroup,
+//           which owns the row's (m, l, acc[D]) in registers.
 // The tensor cores give every output element the same bits whichever operand
 // is A and whichever is B (the per-element dot products do not depend on the
-// orientation or on N), so S, O_hi and O_lo here equal the transposed
-// kernel's S^T, O_hi^T and O_lo^T bit for bit, and so does every row's
-// result.
+// orientation or on N), so S and O here equal the transposed kernel's S^T and
+// O^T bit for bit, and so does every row's result.
 //
 // Roles (512 threads): warps 0-3 / 4-7 softmax warpgroups (even / odd tiles;
 // thread t = TMEM lane t = row t of the tile), 8-11 correction + epilogue,
@@ -27,9 +26,10 @@
 // 15 idle.  Registers are rebalanced per warpgroup (setmaxnreg): the
 // correction warpgroup holds a row's D fp32 accumulators.
 //
-// TMEM (512 columns): S/P buffer 0 at column 0, buffer 1 at 128 (P of 32 keys
-// sits over the S columns of those keys: hi in the first 16, lo in the next
-// 16), O_hi at 256, O_lo at 256 + D.
+// TMEM (512 columns): three S/P buffers at columns 0, 128 and 256 (tile gi
+// uses buffer gi % 3, so the QK of tile gi waits only for the P.V of tile
+// gi - 3; P of keys [32 g, 32 g + 32) goes to columns [16 g, 16 g + 16), whose
+// scores are already read), O at 384.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -65,17 +65,17 @@ struct RowCfg {
   static constexpr int kOffSmall = kOffQ + kQB * kQBytes;
   struct Small {
     uint64_t full_k[NS], empty_k[NS], full_v[NS], empty_v[NS];
-    uint64_t s_full[2], p_full[2], s_free[2], stat_free[2], o_full, o_free;
+    uint64_t s_full[3], p_full[3], s_free[3], stat_free[3], o_full, o_free;
     uint64_t q_full[2], q_empty[2], drain;
     uint32_t tmem_base;
     int abort_any;
-    float tmax[2][kRowsPerTile];  // [buffer][row]: the tile's max (base-2 units)
-    float lsum[2][kRowsPerTile];  // [buffer][row]: the tile's sum of p
+    float tmax[3][kRowsPerTile];  // [buffer][row]: the tile's max (base-2 units)
+    float lsum[3][kRowsPerTile];  // [buffer][row]: the tile's sum of p
     int tab[2][2][kSplitTokens / 16];
   };
   static constexpr int kSmemBytes = kOffSmall + static_cast<int>(sizeof(Small)) + 1024;
   static constexpr int kTmemCols = 512;
-  static constexpr uint32_t kColOhi = 256, kColOlo = 256 + D;
+  static constexpr uint32_t kColO = 384;
 };
 
 // Row t of a 128-row tile: out / lse through the merge's fold of one split.
@@ -140,11 +140,13 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       mbar_init(&sm->full_v[i], 1);
       mbar_init(&sm->empty_v[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 3; ++i) {
       mbar_init(&sm->s_full[i], 1);
       mbar_init(&sm->p_full[i], 4);     // one arrival per softmax warp
       mbar_init(&sm->s_free[i], 1);
       mbar_init(&sm->stat_free[i], 4);  // one arrival per correction warp
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sm->q_full[i], 1);
       mbar_init(&sm->q_empty[i], 1);
     }
@@ -172,17 +174,19 @@ __global__ void __launch_bounds__(kRowThreads, 1)
                  false, lane, abort_any);
     } else if (warp == kMmaWarp && lane == 0) {
       // ----------------------------------------------------------------
-      // MMA issuer.  Per tile gi: S[gi & 1] = Q K^T once the K stage has
-      // landed and P.V of tile gi - 2 (which read P from the same columns)
-      // is done; then P.V of the previous tile.
+      // MMA issuer.  Per tile gi: S[gi % 3] = Q K^T once the K stage has
+      // landed and P.V of tile gi - 3 (which read P from the same columns)
+      // is done; then P.V of tile gi - 2, so that the softmax of two tiles
+      // can run while the tensor cores work.
       // ----------------------------------------------------------------
       constexpr uint32_t kIdescQK = idesc_bf16(128, 128, 0, 0);  // A = Q, B = K (K-major)
       constexpr uint32_t kIdescPV = idesc_bf16(128, D, 0, 1);    // A = P (TMEM), B = V (MN-major)
-      int gi = 0, ui = 0, prev = -1;
+      // (phase parity of the k-th use of buffer gi % 3 is k & 1, k = gi / 3)
+      int gi = 0, ui = 0, pend0 = -1, pend1 = -1;  // tiles whose P.V is not issued yet
       bool failed = false;
       auto pv_step = [&](int g) -> bool {
-        const int st = g % NS, bb = g & 1;
-        if (!mbar_wait(&sm->p_full[bb], (g >> 1) & 1, abort_any)) return false;
+        const int st = g % NS, bb = g % 3;
+        if (!mbar_wait(&sm->p_full[bb], (g / 3) & 1, abort_any)) return false;
         if (!mbar_wait(&sm->o_free, (g & 1) ^ 1, abort_any)) return false;
         if (!mbar_wait(&sm->full_v[st], (g / NS) & 1, abort_any)) return false;
         tc_fence_after_sync();
@@ -191,11 +195,10 @@ __global__ void __launch_bounds__(kRowThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kTileTokens / 16; ++kk) {
           // V: MN-major (N = head_dim), 128-byte swizzle; 64-wide d groups
-          // kHalfBytes apart, 8-key groups 1024 bytes apart.
+          // kHalfBytes apart, 8-key groups 1024 bytes apart.  P of keys
+          // [16 kk, 16 kk + 16): TMEM columns [8 kk, 8 kk + 8).
           const uint64_t b = smem_desc(vaddr + kk * 2048, C::kHalfBytes, 1024, kLayoutSw128);
-          const uint32_t a = pcol + (kk >> 1) * 32 + (kk & 1) * 8;
-          umma_bf16_ts(tmem + C::kColOhi, a, b, kIdescPV, kk > 0 ? 1u : 0u);
-          umma_bf16_ts(tmem + C::kColOlo, a + 16, b, kIdescPV, kk > 0 ? 1u : 0u);
+          umma_bf16_ts(tmem + C::kColO, pcol + kk * 8, b, kIdescPV, kk > 0 ? 1u : 0u);
         }
         umma_commit(&sm->o_full);
         umma_commit(&sm->empty_v[st]);
@@ -212,9 +215,9 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         }
         const uint32_t qaddr = sbase + C::kOffQ + qb * C::kQBytes;
         for (int j = 0; j < x.n_tiles; ++j, ++gi) {
-          const int st = gi % NS, bb = gi & 1;
+          const int st = gi % NS, bb = gi % 3;
           if (!mbar_wait(&sm->full_k[st], (gi / NS) & 1, abort_any) ||
-              !mbar_wait(&sm->s_free[bb], ((gi >> 1) & 1) ^ 1, abort_any)) {
+              !mbar_wait(&sm->s_free[bb], ((gi / 3) & 1) ^ 1, abort_any)) {
             failed = true;
             break;
           }
@@ -230,15 +233,23 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           umma_commit(&sm->s_full[bb]);
           umma_commit(&sm->empty_k[st]);
           if (j == x.n_tiles - 1) umma_commit(&sm->q_empty[qb]);
-          if (prev >= 0 && !pv_step(prev)) {
-            failed = true;
-            break;
+          if (pend1 >= 0) {
+            if (!pv_step(pend0)) {
+              failed = true;
+              break;
+            }
+            pend0 = pend1;
+            pend1 = gi;
+          } else if (pend0 >= 0) {
+            pend1 = gi;
+          } else {
+            pend0 = gi;
           }
-          prev = gi;
         }
         ++ui;
       }
-      if (!failed && prev >= 0) failed = !pv_step(prev);
+      if (!failed && pend0 >= 0) failed = !pv_step(pend0);
+      if (!failed && pend1 >= 0) failed = !pv_step(pend1);
       if (failed) {
         umma_commit(&sm->drain);
         volatile int no_abort = 0;
@@ -249,8 +260,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     // ------------------------------------------------------------------
     // Softmax warpgroups: warpgroup wg takes the tiles with gi % 2 == wg;
     // thread t owns row t.  tmax = exact max of the row's masked scores,
-    // p = 2^(s - tmax), P = [bf16(p) | bf16(p - bf16(p))] over S in TMEM,
-    // L = the row's sum of the fp32 p in the contract's fixed tree.
+    // p = 2^(s - tmax), P = bf16(p) over S in TMEM, L = the row's sum of the
+    // fp32 p in the contract's fixed tree.
     // ------------------------------------------------------------------
     regs_dec<kRowsSoftmaxRegs>();
     const int wg = warp >> 2, wq = warp & 3, t = threadIdx.x & 127;
@@ -271,22 +282,23 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       for (int j = 0; j < x.n_tiles; ++j) {
         const int gi = gbase + j;
         if ((gi & 1) != wg) continue;
-        const int bb = wg, st = gi % NS, par = (gi >> 1) & 1;
+        const int bb = gi % 3, st = gi % NS, par = (gi / 3) & 1;
         bool ok = mbar_wait(&sm->s_full[bb], par, abort_any);
         ok = mbar_wait(&sm->stat_free[bb], par ^ 1, abort_any) && ok;
         tc_fence_after_sync();
         const int tok0 = x.tok0 + j * kTileTokens;
         const int nvis = min(max(nlim - tok0, 0), kTileTokens);
-        const uint32_t srow = tmem + lane_off + bb * 128;
+        const uint32_t srow = tmem + lane_off + bb * 128;  // S of this tile, then its P
         // pass 1: the row's max.  Scaling by cscale > 0 rounds monotonically,
         // so on a fully visible tile max(s) * cscale is the max of the scaled
         // scores exactly.  The branch is taken per WARP (tcgen05.ld is
         // .sync.aligned: all 32 lanes must issue the same load together).
         __syncwarp();
+        const bool full = __all_sync(0xffffffffu, nvis == kTileTokens);  // warp-uniform
         float mx = NEG_INF;
-        if (__all_sync(0xffffffffu, nvis == kTileTokens)) {
+        if (full) {
           float raw = NEG_INF;
-#pragma unroll
+#pragma unroll 1
           for (int ch = 0; ch < 8; ch += 2) {
             float v0[16], v1[16];
             tmem_ld16(srow + ch * 16, v0);
@@ -298,7 +310,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           }
           mx = __fmul_rn(raw, p.cscale);
         } else {
-#pragma unroll
+#pragma unroll 1
           for (int ch = 0; ch < 8; ch += 2) {
             float v0[16], v1[16];
             tmem_ld16(srow + ch * 16, v0);
@@ -314,35 +326,42 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           }
         }
         // pass 2: p, P_hi / P_lo back into TMEM, and the row sum, 32 keys at
-        // a time (one warp's keys in the transposed kernel)
-        float wsum[4];
-#pragma unroll
+        // a time (one warp's keys in the transposed kernel); the four 32-key
+        // sums combine as (w0 + w1) + (w2 + w3)
+        float w_even = 0.f, s01 = 0.f, s23 = 0.f;
+#pragma unroll 1
         for (int grp = 0; grp < 4; ++grp) {
           float va[16], vb[16];  // keys 32 grp + [0, 16) and + [16, 32)
           tmem_ld16(srow + grp * 32, va);
           tmem_ld16(srow + grp * 32 + 16, vb);
           tmem_ld_wait_for(va);
           tmem_ld_wait_for(vb);
+          if (full) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float sa = (grp * 32 + e < nvis) ? __fmul_rn(va[e], p.cscale) : NEG_INF;
-            const float sb = (grp * 32 + 16 + e < nvis) ? __fmul_rn(vb[e], p.cscale) : NEG_INF;
-            va[e] = (sa == NEG_INF) ? 0.f : ex2(__fsub_rn(sa, mx));
-            vb[e] = (sb == NEG_INF) ? 0.f : ex2(__fsub_rn(sb, mx));
+            for (int e = 0; e < 16; ++e) {
+              const float sa = __fmul_rn(va[e], p.cscale);
+              const float sb = __fmul_rn(vb[e], p.cscale);
+              va[e] = (sa == NEG_INF) ? 0.f : ex2(__fsub_rn(sa, mx));
+              vb[e] = (sb == NEG_INF) ? 0.f : ex2(__fsub_rn(sb, mx));
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float sa = (grp * 32 + e < nvis) ? __fmul_rn(va[e], p.cscale) : NEG_INF;
+              const float sb = (grp * 32 + 16 + e < nvis) ? __fmul_rn(vb[e], p.cscale) : NEG_INF;
+              va[e] = (sa == NEG_INF) ? 0.f : ex2(__fsub_rn(sa, mx));
+              vb[e] = (sb == NEG_INF) ? 0.f : ex2(__fsub_rn(sb, mx));
+            }
           }
-          uint32_t whi[16], wlo[16];
+          uint32_t w[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             const float x0 = k < 8 ? va[2 * k] : vb[2 * k - 16];
             const float x1 = k < 8 ? va[2 * k + 1] : vb[2 * k - 15];
             __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
-            __nv_bfloat162 l2 = __floats2bfloat162_rn(__fsub_rn(x0, __low2float(h2)),
-                                                      __fsub_rn(x1, __high2float(h2)));
-            whi[k] = *reinterpret_cast<uint32_t *>(&h2);
-            wlo[k] = *reinterpret_cast<uint32_t *>(&l2);
+            w[k] = *reinterpret_cast<uint32_t *>(&h2);
           }
-          tmem_st16(srow + grp * 32, whi);
-          tmem_st16(srow + grp * 32 + 16, wlo);
+          tmem_st16(srow + grp * 16, w);
           // the shuffle-down tree of one warp's 32 keys: offsets 16, 8, 4, 2, 1
 #pragma unroll
           for (int e = 0; e < 16; ++e) va[e] = __fadd_rn(va[e], vb[e]);
@@ -350,7 +369,13 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           for (int off = 8; off >= 1; off >>= 1)
 #pragma unroll
             for (int e = 0; e < off; ++e) va[e] = __fadd_rn(va[e], va[e + off]);
-          wsum[grp] = va[0];
+          if (grp & 1) {
+            const float pair = __fadd_rn(w_even, va[0]);
+            s01 = grp == 1 ? pair : s01;
+            s23 = grp == 3 ? pair : s23;
+          } else {
+            w_even = va[0];
+          }
         }
         if (tok0 + kTileTokens > x.lim_max) {
           // The last tile: keys past the loaded range hold stale bytes or the
@@ -367,7 +392,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           }
         }
         sm->tmax[bb][t] = mx;
-        sm->lsum[bb][t] = __fadd_rn(__fadd_rn(wsum[0], wsum[1]), __fadd_rn(wsum[2], wsum[3]));
+        sm->lsum[bb][t] = __fadd_rn(s01, s23);
         if (wg_bar_or(bar_id, !ok)) {
           stop = true;
           break;
@@ -386,9 +411,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     // ------------------------------------------------------------------
     // Correction + epilogue warpgroup: thread t owns row t's running
     // (m, l, acc[D]).  Per tile, in order: m' = max(m, tmax), a = 2^(m - m'),
-    // b = 2^(tmax - m'), acc = fma(O_hi + O_lo, b, acc * a),
-    // l = fma(L, b, l * a); a tile the row does not reach (tmax = -inf)
-    // leaves it untouched.
+    // b = 2^(tmax - m'), acc = fma(O, b, acc * a), l = fma(L, b, l * a); a
+    // tile the row does not reach (tmax = -inf) leaves it untouched.
     // ------------------------------------------------------------------
     regs_inc<kRowsCorrRegs>();
     const int wq = warp & 3, t = threadIdx.x & 127;
@@ -413,7 +437,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       for (int c = 0; c < D; ++c) acc[c] = 0.f;
       float m_run = NEG_INF, l_run = 0.f;
       for (int j = 0; j < x.n_tiles; ++j) {
-        const int gi = gbase + j, bb = gi & 1, par = (gi >> 1) & 1;
+        const int gi = gbase + j, bb = gi % 3, par = (gi / 3) & 1;
         bool ok = mbar_wait(&sm->p_full[bb], par, abort_any);  // the tile's row statistics
         ok = mbar_wait(&sm->o_full, gi & 1, abort_any) && ok;    // its P.V
         tc_fence_after_sync();
@@ -438,16 +462,18 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         const uint32_t orow = tmem + lane_off;
         __syncwarp();
 #pragma unroll
-        for (int ch = 0; ch < D / 16; ++ch) {
-          float hi[16], lo[16];
-          tmem_ld16(orow + C::kColOhi + ch * 16, hi);
-          tmem_ld16(orow + C::kColOlo + ch * 16, lo);
-          tmem_ld_wait_for(hi);
-          tmem_ld_wait_for(lo);
+        for (int ch = 0; ch < D / 16; ch += 2) {
+          float o0[16], o1[16];
+          tmem_ld16(orow + C::kColO + ch * 16, o0);
+          tmem_ld16(orow + C::kColO + ch * 16 + 16, o1);
+          tmem_ld_wait_for(o0);
+          tmem_ld_wait_for(o1);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {  // branch-free: the loop's TMEM loads are warp-wide
-            const float nv = __fmaf_rn(__fadd_rn(hi[e], lo[e]), b, __fmul_rn(acc[ch * 16 + e], a));
-            acc[ch * 16 + e] = skip ? acc[ch * 16 + e] : nv;
+            const float n0 = __fmaf_rn(o0[e], b, __fmul_rn(acc[ch * 16 + e], a));
+            const float n1 = __fmaf_rn(o1[e], b, __fmul_rn(acc[ch * 16 + 16 + e], a));
+            acc[ch * 16 + e] = skip ? acc[ch * 16 + e] : n0;
+            acc[ch * 16 + 16 + e] = skip ? acc[ch * 16 + 16 + e] : n1;
           }
         }
         tc_fence_before_sync();

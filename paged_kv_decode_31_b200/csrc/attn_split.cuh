@@ -19,14 +19,14 @@
 //   S^T      = K_tile * Q^T on the tensor cores (tcgen05, M = 128 tokens,
 //            N = rows, K = head_dim, fp32 accumulation in TMEM);
 //   softmax  one thread per token: mask (key < row limit), scale to base 2,
-//            column max over the 128 tokens (exact, order-free), running max,
-//            p = 2^(s - m); P^T holds p as two bf16 parts side by side, hi =
-//            bf16(p) and lo = bf16(p - hi), so the tensor cores see p to ~16
-//            bits; the fp32 p of each row are summed in one fixed shuffle tree;
-//   O^T      = V^T * [P_hi | P_lo]^T on the tensor cores (fresh accumulator
-//            each tile), O = O_hi + O_lo;
-//   update   acc = fma(acc, alpha, O), l = fma(l, alpha, sum p), alpha =
-//            2^(m_old - m_new), skipped for rows the tile does not reach.
+//            the tile's column max over its 128 tokens (exact, order-free),
+//            p = 2^(s - tmax); P^T = bf16(p); the fp32 p of each row are summed
+//            in one fixed shuffle tree (so the row sum l never sees the bf16
+//            rounding of P);
+//   O^T      = V^T * P^T on the tensor cores (fresh accumulator each tile);
+//   update   m' = max(m, tmax), acc = fma(O, 2^(tmax - m'), acc * 2^(m - m')),
+//            l likewise with the tile's row sum; skipped for rows the tile
+//            does not reach.
 // Tiles start at absolute multiples of 128 and rows never influence each
 // other, so a row's arithmetic depends only on its own query, its visible
 // keys and the fixed constants: decode row t and prefill row t, batch 1 and
@@ -149,7 +149,7 @@ struct Cfg {
   static constexpr int kKVBytes = (D / 64) * kHalfBytes;  // one K (or V) tile
   static constexpr int kQHalfBytes = N * 128;
   static constexpr int kQBytes = (D / 64) * kQHalfBytes;
-  static constexpr int kPCols = 2 * N;                    // P^T columns: N hi, then N lo
+  static constexpr int kPCols = N;                        // P^T columns: one per row
   static constexpr int kPBytes = kTileTokens * kPCols * 2;
   static constexpr int kPKGroup = (kPCols / 8) * 128;     // P^T stride between 8-token groups
   static constexpr int kOffK = 0;
@@ -172,8 +172,8 @@ struct Cfg {
     int tab[2][2][kSplitTokens / 16];      // [producer][unit parity]: block-table entries
   };
   static constexpr int kSmemBytes = kOffSmall + static_cast<int>(sizeof(Small)) + 1024;
-  // TMEM: S^T (N columns) x 2 buffers, then O^T (hi and lo, 2N columns) x 2 buffers
-  static constexpr int kTmemCols = (6 * N <= 128) ? 128 : (6 * N <= 256) ? 256 : 512;
+  // TMEM: S^T (N columns) x 2 buffers, then O^T (N columns) x 2 buffers
+  static constexpr int kTmemCols = (4 * N <= 128) ? 128 : (4 * N <= 256) ? 256 : 512;
 };
 
 struct Unit {
@@ -476,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------
     if (lane == 0) {
       constexpr uint32_t kIdescQK = idesc_bf16(128, N, 0, 0);           // A = K tile, B = Q (K-major)
-      constexpr uint32_t kIdescPV = idesc_bf16(128, C::kPCols, 1, 1);  // A = V^T, B = P^T (MN-major)
+      constexpr uint32_t kIdescPV = idesc_bf16(128, N, 1, 1);  // A = V^T, B = P^T (MN-major)
       const uint32_t tS = tmem, tO = tmem + 2 * N;
       int gi = 0, ui = 0, prev = -1;
       bool failed = false;
@@ -494,11 +494,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // (D = 64: both M halves read the same 64 columns; lanes 64..127 are unused).
           const uint64_t a = smem_desc(vaddr + kk * 2048, D == 128 ? C::kHalfBytes : 0, 1024,
                                        kLayoutSw128);
-          // P^T = [P_hi | P_lo]: MN-major, no swizzle; 8-column groups 128 B apart,
-          // 8-token groups kPKGroup apart.
+          // P^T: MN-major, no swizzle; 8-column groups 128 B apart, 8-token
+          // groups kPKGroup apart.
           const uint64_t b = smem_desc(paddr + kk * 2 * C::kPKGroup, C::kPKGroup, 128,
                                        kLayoutInterleave);
-          umma_bf16(tO + bb * C::kPCols, a, b, kIdescPV, kk > 0 ? 1u : 0u);
+          umma_bf16(tO + bb * N, a, b, kIdescPV, kk > 0 ? 1u : 0u);
         }
         umma_commit(&sm->o_full[bb]);
         umma_commit(&sm->empty_v[st]);
@@ -551,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Softmax warpgroups: warpgroup wg takes the tiles with gi % 2 == wg.
     // Thread t <-> TMEM lane t <-> token t of the tile.  Per tile and row:
     // tmax = exact max of the masked scores, p = 2^(s - tmax) written as
-    // P^T = [bf16(p) | bf16(p - bf16(p))], per-warp sums of the fp32 p.
+    // P^T = bf16(p), per-warp sums of the fp32 p.
     // ------------------------------------------------------------------
     const int wg = warp >> 2, wq = warp & 3, t = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -629,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *prow = smem + C::kOffP + bb * C::kPBytes + (t >> 3) * C::kPKGroup + (t & 7) * 16;
 #pragma unroll
         for (int grp = 0; grp < N / 8; ++grp) {
-          uint32_t whi[4] = {0u, 0u, 0u, 0u}, wlo[4] = {0u, 0u, 0u, 0u};
+          uint32_t w[4] = {0u, 0u, 0u, 0u};
           if (grp * 8 < x.rows) {  // groups of padded rows keep p = 0
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -642,15 +642,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               sv[c0] = p0;
               sv[c0 + 1] = p1;
               __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-              __nv_bfloat162 l2 = __floats2bfloat162_rn(__fsub_rn(p0, __low2float(h2)),
-                                                        __fsub_rn(p1, __high2float(h2)));
-              whi[e] = *reinterpret_cast<uint32_t *>(&h2);
-              wlo[e] = *reinterpret_cast<uint32_t *>(&l2);
+              w[e] = *reinterpret_cast<uint32_t *>(&h2);
             }
           }
-          *reinterpret_cast<uint4 *>(prow + grp * 128) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
-          *reinterpret_cast<uint4 *>(prow + (N / 8 + grp) * 128) =
-              make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
+          *reinterpret_cast<uint4 *>(prow + grp * 128) = make_uint4(w[0], w[1], w[2], w[3]);
         }
 #pragma unroll
         for (int q4 = 0; q4 < N / 4; ++q4) {
@@ -676,8 +671,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Correction + epilogue warpgroup: thread t <-> TMEM lane t <-> output
     // column d of O^T; thread r (< rows) owns row r's running (m, l).
     // Per tile, in order: m' = max(m, tmax), a = 2^(m - m'), b = 2^(tmax - m'),
-    // acc = fma(O_hi + O_lo, b, acc * a), l = fma(sum p, b, l * a); a tile a
-    // row does not reach (tmax = -inf) leaves the row untouched.
+    // acc = fma(O, b, acc * a), l = fma(sum p, b, l * a); a tile a row does
+    // not reach (tmax = -inf) leaves the row untouched.
     // ------------------------------------------------------------------
     const int wq = warp & 3, t = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -725,16 +720,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int ch = 0; ch < N / 16; ++ch) {
           if (ch * 16 < x.rows) {  // warp-uniform
-            float hi[16], lo[16];
-            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + ch * 16, hi);
-            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + N + ch * 16, lo);
-            tmem_ld_wait();
+            float o[16];
+            tmem_ld16(tmem + lane_off + 2 * N + bb * N + ch * 16, o);
+            tmem_ld_wait_for(o);
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int c = ch * 16 + e;
               if (c < x.rows && !sm->coef_skip[c])
-                acc[c] = __fmaf_rn(__fadd_rn(hi[e], lo[e]), sm->coef_b[c],
-                                   __fmul_rn(acc[c], sm->coef_a[c]));
+                acc[c] = __fmaf_rn(o[e], sm->coef_b[c], __fmul_rn(acc[c], sm->coef_a[c]));
             }
           }
         }

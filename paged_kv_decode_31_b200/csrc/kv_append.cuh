@@ -1,6 +1,6 @@
 // kv_append.cuh -- write new K/V tokens into paged cache blocks.
 //
-// Token t of sequence b goes to position p = seqlens[b] + t: block
+// Token t of sequence b goes to position p = seqlens[b] - seq_bias + t: block
 // block_table[b][p / block_size], slot p % block_size, addressed with the
 // cache's real element strides.  The bf16 bits are copied unchanged with
 // 128-bit loads and stores ([WS1] "KV-cache path consistency (prefill &
@@ -24,6 +24,10 @@ struct AppendParams {
   const int32_t *seqlens;
   int batch, n_new, Hkv, chunks;  // chunks = D / 8 (16-byte pieces per head row)
   int block_shift;
+  // 0 for pkv_kv_append (seqlens before the append); n_new when the attention
+  // call appends (seqlens after it): then positions below 0 are skipped
+  // without an error, as the fused path does.
+  int seq_bias;
   int32_t *err;
 };
 
@@ -37,8 +41,9 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ 
     r /= p.Hkv;
     const int t = static_cast<int>(r % p.n_new);
     const int b = static_cast<int>(r / p.n_new);
-    const int64_t pos = static_cast<int64_t>(__ldg(p.seqlens + b)) + t;
+    const int64_t pos = static_cast<int64_t>(__ldg(p.seqlens + b)) - p.seq_bias + t;
     const int64_t bi = pos >> p.block_shift;
+    if (pos < 0 && p.seq_bias > 0) continue;
     if (pos < 0 || bi >= p.max_blocks_per_seq) {
       if (p.err) atomicOr(p.err, 2);
       continue;

@@ -219,7 +219,56 @@ int rows_per_tile(int64_t rows, int G, int seqlen_q) {
   return pkv::kRowsPerTile;
 }
 
-// New tokens written into the cache by the attention call itself.
+// The append kernel: token t of sequence b to position seqlens[b] - seq_bias + t.
+int launch_append(const void *k_new, const int64_t kn_strides[3], const void *v_new,
+                  const int64_t vn_strides[3], void *k_cache, const int64_t k_strides[3],
+                  void *v_cache, const int64_t v_strides[3], int64_t num_blocks,
+                  const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                  const int32_t *seqlens, int batch, int n_new, int Hkv, int D, int block_size,
+                  int seq_bias, int32_t *err, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  pkv::AppendParams p{};
+  p.k_new = static_cast<const uint16_t *>(k_new);
+  p.v_new = static_cast<const uint16_t *>(v_new);
+  p.kn_sb = kn_strides[0];
+  p.kn_st = kn_strides[1];
+  p.kn_sh = kn_strides[2];
+  p.vn_sb = vn_strides[0];
+  p.vn_st = vn_strides[1];
+  p.vn_sh = vn_strides[2];
+  p.k_cache = static_cast<uint16_t *>(k_cache);
+  p.v_cache = static_cast<uint16_t *>(v_cache);
+  p.k_sb = k_strides[0];
+  p.k_ss = k_strides[1];
+  p.k_sh = k_strides[2];
+  p.v_sb = v_strides[0];
+  p.v_ss = v_strides[1];
+  p.v_sh = v_strides[2];
+  p.num_blocks = num_blocks;
+  p.block_table = block_table;
+  p.bt_stride = bt_stride;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.seqlens = seqlens;
+  p.batch = batch;
+  p.n_new = n_new;
+  p.Hkv = Hkv;
+  p.chunks = D / 8;
+  p.block_shift = log2i(block_size);
+  p.seq_bias = seq_bias;
+  p.err = err;
+  const int64_t total = static_cast<int64_t>(batch) * n_new * Hkv * (D / 8);
+  const int64_t want = ceil_div(total, 256);
+  const int64_t cap = static_cast<int64_t>(sm_count(dev)) * 8;
+  const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
+  pkv::kv_append_kernel<<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+// New tokens written into the cache by the attention call itself.  The
+// producers write them just before loading the tiles that hold them when
+// there are few (decode steps) and one row tile reads them.
+constexpr int kFuseMaxNew = 16;
 struct FusedAppend {
   const void *k_new, *v_new;
   const int64_t *kn_strides, *vn_strides;
@@ -302,11 +351,22 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   p.ws_acc = ws_acc;
   p.ws_ml = ws_ml;
   p.err = err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (app && app->n_new > 0) {
     if (!app->k_new || !app->v_new || !strides_ok(app->kn_strides) ||
         !strides_ok(app->vn_strides) || !aligned16(app->k_new) || !aligned16(app->v_new) ||
         app->n_new > pkv::kSplitTokens)
       return PKV_ERR_ARG;
+  }
+  if (app && app->n_new > 0 && (app->n_new > kFuseMaxNew || RT > 1)) {
+    // Many new tokens, or several row tiles that would each write them: one
+    // append launch first (the same bits in the cache), then plain attention.
+    rc = launch_append(app->k_new, app->kn_strides, app->v_new, app->vn_strides,
+                       const_cast<void *>(k_cache), k_strides, const_cast<void *>(v_cache),
+                       v_strides, num_blocks, block_table, bt_stride, max_blocks_per_seq, seqlens,
+                       batch, app->n_new, Hkv, D, block_size, app->n_new, err, s);
+    if (rc != PKV_OK) return rc;
+  } else if (app && app->n_new > 0) {
     p.n_new = app->n_new;
     p.k_new = static_cast<const uint16_t *>(app->k_new);
     p.v_new = static_cast<const uint16_t *>(app->v_new);
@@ -326,7 +386,6 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
     p.v_sh = v_strides[2];
   }
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (N == pkv::kRowsPerTile) {
     // one split per row: the split kernel writes out / lse itself
     p.direct = S == 1 ? 1 : 0;
@@ -385,42 +444,9 @@ int pkv_kv_append(const void *k_new, const int64_t kn_strides[3], const void *v_
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
     return PKV_ERR_ARG;
   if (n_new == 0) return PKV_OK;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
-  pkv::AppendParams p{};
-  p.k_new = static_cast<const uint16_t *>(k_new);
-  p.v_new = static_cast<const uint16_t *>(v_new);
-  p.kn_sb = kn_strides[0];
-  p.kn_st = kn_strides[1];
-  p.kn_sh = kn_strides[2];
-  p.vn_sb = vn_strides[0];
-  p.vn_st = vn_strides[1];
-  p.vn_sh = vn_strides[2];
-  p.k_cache = static_cast<uint16_t *>(k_cache);
-  p.v_cache = static_cast<uint16_t *>(v_cache);
-  p.k_sb = k_strides[0];
-  p.k_ss = k_strides[1];
-  p.k_sh = k_strides[2];
-  p.v_sb = v_strides[0];
-  p.v_ss = v_strides[1];
-  p.v_sh = v_strides[2];
-  p.num_blocks = num_blocks;
-  p.block_table = block_table;
-  p.bt_stride = bt_stride;
-  p.max_blocks_per_seq = max_blocks_per_seq;
-  p.seqlens = seqlens;
-  p.batch = batch;
-  p.n_new = n_new;
-  p.Hkv = Hkv;
-  p.chunks = D / 8;
-  p.block_shift = log2i(block_size);
-  p.err = err;
-  const int64_t total = static_cast<int64_t>(batch) * n_new * Hkv * (D / 8);
-  const int64_t want = ceil_div(total, 256);
-  const int64_t cap = static_cast<int64_t>(sm_count(dev)) * 8;
-  const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
-  pkv::kv_append_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
-  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+  return launch_append(k_new, kn_strides, v_new, vn_strides, k_cache, k_strides, v_cache,
+                       v_strides, num_blocks, block_table, bt_stride, max_blocks_per_seq, seqlens,
+                       batch, n_new, Hkv, D, block_size, 0, err, static_cast<cudaStream_t>(stream));
 }
 
 int pkv_paged_decode_attn(const void *q, const int64_t q_strides[3], const void *k_cache,

@@ -21,6 +21,8 @@ CASES = [
     (2, 3, 4097, 8, 2, 128, 16, "interleaved", True),    # new tokens straddle a split boundary
     (2, 17, 1500, 16, 4, 128, 32, "contiguous", True),    # 68 rows: two row tiles
     (5, 1, 9000, 8, 8, 128, 64, "contiguous", False),     # G = 1
+    (2, 200, 3000, 16, 4, 128, 16, "interleaved", True),  # prefill chunk: append launch first
+    (3, 40, 6000, 8, 2, 64, 32, "contiguous", True),      # 160 rows, two splits
 ]
 
 
