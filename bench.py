@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--context", type=int, default=131072,
                     help="tokens per sequence (a smaller workload for profiling captures)")
     ap.add_argument("--batch", type=int, default=4)
+    ap.add_argument("--varlen-only", action="store_true",
+                    help="time only the packed mixed-batch call and print its result object")
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the chunked causal prefill (--steps repetitions, "
                          "2 warm-up passes) and print its result object")
@@ -229,6 +231,77 @@ def prefill_secondary(dev, reps: int = 5):
             "algorithmic_flops": flops}
 
 
+# Packed mixed batch for the varlen measurement: (requests, queries each, context)
+VARLEN_MIX = [(16, 1, 16384), (8, 4, 8192), (6, 256, 2048), (2, 1024, 4096)]
+
+
+def varlen_secondary(dev, reps: int = 10):
+    """One packed multi-request call (paged_varlen_attn) over a mix of decode
+    steps, multi-token steps and prefill chunks (VARLEN_MIX; Hq 32 / Hkv 8,
+    D 128, block_size 16, causal), with each request's final row selected as
+    well.  Reports the call time, queries/s, the unique K/V bytes / time and
+    the algorithmic flops (4 * D per (query row, visible key)) / time."""
+    import paged_kv_decode_31_b200 as pkv
+    from paged_kv_decode_31_b200 import inputs as I
+    Hq, Hkv, D, bs = 32, 8, 128, 16
+    lengths, ctx = [], []
+    for count, n, c in VARLEN_MIX:
+        lengths += [n] * count
+        ctx += [c] * count
+    B = len(ctx)
+    gen = torch.Generator().manual_seed(2024)
+    nblk = [(c + bs - 1) // bs for c in ctx]
+    gen_d = torch.Generator(device=dev).manual_seed(2025)
+    cache = I.make_cache(sum(nblk) + 64, bs, Hkv, D, "contiguous", gen_d, device=dev)
+    perm = torch.randperm(sum(nblk) + 64, generator=gen)[:sum(nblk)].to(torch.int32)
+    table = torch.zeros(B, max(nblk), dtype=torch.int32)
+    o = 0
+    for b, k in enumerate(nblk):
+        table[b, :k] = perm[o:o + k]
+        o += k
+    table = table.to(dev)
+    seqlens = torch.tensor(ctx, dtype=torch.int32, device=dev)
+    cu = torch.tensor([0] + torch.tensor(lengths).cumsum(0).tolist(), dtype=torch.int32,
+                      device=dev)
+    total_q = int(sum(lengths))
+    q = I.randn_bf16((total_q, Hq, D), gen).to(dev)
+    out = torch.empty(total_q, Hq, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(Hq, total_q, dtype=torch.float32, device=dev)
+    fo = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    fl = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    ws = torch.empty(pkv.varlen_workspace_size(total_q, Hq, D, max(ctx)), dtype=torch.uint8,
+                     device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def call():
+        pkv.paged_varlen_attn(q, cache.k, cache.v, table, seqlens, cu, max(lengths),
+                              max_seqlen_k=max(ctx), causal=True, out=out, lse=lse,
+                              final_out=fo, final_lse=fl, workspace=ws, err=err)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        call()
+    b_.record()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"varlen call set device error bits {int(err.item())}")
+    ms = a.elapsed_time(b_) / reps
+    kv_bytes = sum(c * Hkv * 2 * D * 2 for c in ctx)
+    pairs = sum(sum(c - n + i + 1 for i in range(n)) for n, c in zip(lengths, ctx))
+    flops = 4.0 * D * pairs * Hq
+    return {"workload": "packed causal batch of " + ", ".join(
+                f"{k} x {n} queries at context {c}" for k, n, c in VARLEN_MIX) +
+                f" ({B} requests, {total_q} query tokens), Hq 32, Hkv 8, D 128, block_size 16, "
+                "final rows selected",
+            "ms_per_call": round(ms, 4), "queries_per_s": round(total_q / (ms / 1e3), 1),
+            "kv_gbs": round(kv_bytes / (ms / 1e3) / 1e9, 2), "kv_bytes": kv_bytes,
+            "tflops": round(flops / (ms / 1e3) / 1e12, 2), "algorithmic_flops": flops}
+
+
 def run_ours(args):
     import torch.distributed as dist
     import paged_kv_decode_31_b200 as pkv
@@ -388,6 +461,10 @@ def run_ours(args):
         pre["tensor_peak_tflops"] = bf16_peak
         pre["frac_of_tensor_peak"] = round(pre["tflops"] / bf16_peak, 4)
         result["prefill"] = pre
+        vl = varlen_secondary(dev)
+        vl["hbm_frac"] = round(vl["kv_gbs"] / peak, 4)
+        vl["frac_of_tensor_peak"] = round(vl["tflops"] / bf16_peak, 4)
+        result["varlen"] = vl
     if not args.no_cpu_baseline and world == 1:
         result["cpu_baseline"] = cpu_baseline(di)
     print(json.dumps(result), flush=True)
@@ -445,6 +522,10 @@ def run_reference(args):
 
 def main():
     args = parse_args()
+    if args.varlen_only:
+        torch.cuda.set_device(0)
+        print(json.dumps(varlen_secondary(torch.device("cuda", 0), reps=max(args.steps, 1))))
+        return
     if args.prefill_only:
         torch.cuda.set_device(0)
         print(json.dumps(prefill_secondary(torch.device("cuda", 0), reps=max(args.steps, 1))))

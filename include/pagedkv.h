@@ -93,6 +93,9 @@ extern "C" {
 #define PKV_DEVERR_BAD_BLOCK 1   /* block_table entry outside [0, num_blocks) */
 #define PKV_DEVERR_TABLE_WIDTH 2 /* a position needs a column >= max_blocks_per_seq */
 #define PKV_DEVERR_TIMEOUT 4     /* an internal pipeline wait gave up (no result) */
+#define PKV_DEVERR_QUERY_LEN 8   /* packed call: a sequence has more than max_seqlen_q
+                                    queries (or cu_seqlens_q decreases); rows past the
+                                    bound are not written */
 
 /*
  * pkv_kv_append: for every sequence b and new token t < n_new, copy the bf16
@@ -199,6 +202,64 @@ int pkv_paged_decode_attn_append(const void *q, const int64_t q_strides[3],
                                  void *out, const int64_t out_strides[3], float *lse,
                                  void *workspace, size_t workspace_bytes,
                                  int32_t *err, void *stream);
+
+/*
+ * pkv_paged_varlen_attn: packed multi-request attention -- the "cumulative
+ * query lengths" form of a packed forward (AstrAI commit search page: "Pack
+ * prompts ... into one forward", "Select per-request final logits from
+ * cumulative query lengths").  Request b owns the packed query tokens
+ * cu_seqlens_q[b] .. cu_seqlens_q[b+1] - 1 (device int32 [batch + 1],
+ * non-decreasing, cu_seqlens_q[0] = 0, cu_seqlens_q[batch] = total_q; empty
+ * requests allowed); its n_b queries are the last n_b positions of its
+ * context, exactly as seqlen_q = n_b in pkv_paged_decode_attn (bottom-right,
+ * causal or not, seqlens[b] counts them).  Every row is bitwise the row the
+ * dense call on that request alone returns.
+ *   q        [total_q, Hq, D] bf16, element strides q_strides = (token, head)
+ *   out      [total_q, Hq, D] bf16, strides out_strides = (token, head)
+ *   lse      [Hq, total_q] fp32, contiguous
+ *   max_seqlen_q  host bound on every n_b (sizes the grid; a larger n_b sets
+ *                 PKV_DEVERR_QUERY_LEN and its rows past the bound stay unwritten)
+ *   final_out / final_lse  optional (both null, or both given): each
+ *                 request's last query row (token cu_seqlens_q[b+1] - 1) is also
+ *                 written to final_out [batch, Hq, D] (strides final_strides =
+ *                 (batch, head)) and final_lse [batch, Hq]; requests with no
+ *                 query leave their final row untouched
+ *   workspace     >= pkv_varlen_workspace_size(total_q, Hq, D, max_seqlen_k)
+ * Other arguments and all error codes as for pkv_paged_decode_attn.
+ */
+int pkv_paged_varlen_attn(const void *q, const int64_t q_strides[2], const int32_t *cu_seqlens_q,
+                          int total_q, int max_seqlen_q,
+                          const void *k_cache, const int64_t k_strides[3],
+                          const void *v_cache, const int64_t v_strides[3],
+                          int64_t num_blocks,
+                          const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                          const int32_t *seqlens, int max_seqlen_k,
+                          int batch, int Hq, int Hkv, int D, int block_size,
+                          float scale, int causal,
+                          void *out, const int64_t out_strides[2], float *lse,
+                          void *final_out, const int64_t final_strides[2], float *final_lse,
+                          void *workspace, size_t workspace_bytes,
+                          int32_t *err, void *stream);
+
+/* Workspace bytes pkv_paged_varlen_attn needs (0 on invalid arguments). */
+size_t pkv_varlen_workspace_size(int total_q, int Hq, int D, int max_seqlen_k);
+
+/*
+ * pkv_kv_append_varlen: pkv_kv_append for packed new tokens.  Sequence b's
+ * new tokens are rows cu_seqlens_new[b] .. cu_seqlens_new[b+1] - 1 of k_new /
+ * v_new ([total_new, Hkv, D] bf16, element strides (token, head)); token t of
+ * sequence b goes to position seqlens[b] + t (seqlens BEFORE the append).
+ * Bits, errors and device error bits as for pkv_kv_append.
+ */
+int pkv_kv_append_varlen(const void *k_new, const int64_t kn_strides[2],
+                         const void *v_new, const int64_t vn_strides[2],
+                         const int32_t *cu_seqlens_new, int total_new,
+                         void *k_cache, const int64_t k_strides[3],
+                         void *v_cache, const int64_t v_strides[3],
+                         int64_t num_blocks,
+                         const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                         const int32_t *seqlens, int batch, int Hkv, int D, int block_size,
+                         int32_t *err, void *stream);
 
 /* Workspace bytes the attention calls need: fp32 split partials
  * (m, l, acc[D]) for every (batch, query row, query head, split). */

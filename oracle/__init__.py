@@ -130,3 +130,47 @@ def kv_append(k_new, v_new, k_cache, v_cache, block_table, seqlens):
         bt.stride(0), bt.shape[1], sl.data_ptr(), B, n, Hkv, D, bs)
     if rc != 0:
         raise RuntimeError(f"oracle_kv_append failed with status {rc}")
+
+
+def paged_attn_varlen(q, k_cache, v_cache, block_table, seqlens, cu_seqlens_q, scale, causal):
+    """fp64 attention of packed multi-request queries (the cumulative query
+    lengths of a packed forward, AstrAI commit search page: "Pack prompts ...
+    into one forward", "Select per-request final logits from cumulative query
+    lengths").  Packing is only an indexing convention: request b is the dense
+    problem of its own n_b = cu[b+1] - cu[b] queries (the last n_b positions of
+    its context), so each request is handed to paged_attn on its own.
+
+    q: [total_q, Hq, D] bf16; cu_seqlens_q: [B + 1] int.  Returns (out
+    [total_q, Hq, D] fp64, lse [Hq, total_q] fp64, final_out [B, Hq, D] fp64,
+    final_lse [B, Hq] fp64); the final row of request b is its packed token
+    cu[b+1] - 1 (NaN for a request with no query)."""
+    total_q, Hq, D = q.shape
+    cu = [int(x) for x in cu_seqlens_q.tolist()]
+    B = len(cu) - 1
+    out = torch.full((total_q, Hq, D), float("nan"), dtype=torch.float64)
+    lse = torch.full((Hq, total_q), float("nan"), dtype=torch.float64)
+    fin_out = torch.full((B, Hq, D), float("nan"), dtype=torch.float64)
+    fin_lse = torch.full((B, Hq), float("nan"), dtype=torch.float64)
+    for b in range(B):
+        a, e = cu[b], cu[b + 1]
+        if e <= a:
+            continue
+        o_b, l_b = paged_attn(q[a:e].unsqueeze(0), k_cache, v_cache, block_table[b:b + 1],
+                              seqlens[b:b + 1], scale, causal)
+        out[a:e] = o_b[0]
+        lse[:, a:e] = l_b[0]
+        fin_out[b] = o_b[0, -1]
+        fin_lse[b] = l_b[0, :, -1]
+    return out, lse, fin_out, fin_lse
+
+
+def kv_append_varlen(k_new, v_new, k_cache, v_cache, block_table, seqlens, cu_seqlens_new):
+    """kv_append for packed new tokens [total_new, Hkv, D]: sequence b's are
+    rows cu[b] .. cu[b+1] - 1, written at positions seqlens[b] + t."""
+    cu = [int(x) for x in cu_seqlens_new.tolist()]
+    for b in range(len(cu) - 1):
+        a, e = cu[b], cu[b + 1]
+        if e <= a:
+            continue
+        kv_append(k_new[a:e].unsqueeze(0), v_new[a:e].unsqueeze(0), k_cache, v_cache,
+                  block_table[b:b + 1], seqlens[b:b + 1])

@@ -10,10 +10,13 @@ from .binding import (  # noqa: F401
     SPLIT_TOKENS,
     TILE_TOKENS,
     kv_append,
+    kv_append_varlen,
     library_path,
     paged_decode_attn,
     paged_decode_attn_append,
     paged_prefill_attn,
+    paged_varlen_attn,
     strerror,
+    varlen_workspace_size,
     workspace_size,
 )

@@ -22,6 +22,7 @@ TILE_TOKENS = 128
 DEVERR_BAD_BLOCK = 1
 DEVERR_TABLE_WIDTH = 2
 DEVERR_TIMEOUT = 4
+DEVERR_QUERY_LEN = 8
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -60,6 +61,15 @@ def lib() -> ctypes.CDLL:
         L.pkv_strerror.restype = ctypes.c_char_p
         L.pkv_split_tokens.argtypes = []
         L.pkv_split_tokens.restype = _I
+        L.pkv_paged_varlen_attn.argtypes = [_P, _P, _P, _I, _I, _P, _P, _P, _P, _I64, _P, _I64,
+                                            _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I,
+                                            _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
+        L.pkv_paged_varlen_attn.restype = _I
+        L.pkv_varlen_workspace_size.argtypes = [_I, _I, _I, _I]
+        L.pkv_varlen_workspace_size.restype = ctypes.c_size_t
+        L.pkv_kv_append_varlen.argtypes = [_P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I64, _P,
+                                           _I64, _I, _P, _I, _I, _I, _I, _P, _P]
+        L.pkv_kv_append_varlen.restype = _I
         _lib = L
     return _lib
 
@@ -224,6 +234,109 @@ def paged_prefill_attn(q, k_cache, v_cache, block_table, seqlens, *, max_seqlen_
     """Causal or chunked prefill over the paged cache; same contract as decode."""
     return _attn("pkv_paged_prefill_attn", q, k_cache, v_cache, block_table, seqlens,
                  max_seqlen_k, scale, causal, out, lse, workspace, err, stream)
+
+
+def _st2(t: torch.Tensor) -> ctypes.Array:
+    return (ctypes.c_int64 * 2)(int(t.stride(0)), int(t.stride(1)))
+
+
+def _need_packed_bf16(name: str, t: torch.Tensor) -> None:
+    if not t.is_cuda or t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be a bf16 CUDA tensor (got {t.dtype} on {t.device})")
+    if t.dim() != 3 or t.stride(-1) != 1:
+        raise ValueError(f"{name} must be 3-D [tokens, heads, D] with a unit last stride")
+
+
+def varlen_workspace_size(total_q: int, Hq: int, D: int, max_seqlen_k: int) -> int:
+    return int(lib().pkv_varlen_workspace_size(total_q, Hq, D, max_seqlen_k))
+
+
+def paged_varlen_attn(q, k_cache, v_cache, block_table, seqlens, cu_seqlens_q, max_seqlen_q, *,
+                      max_seqlen_k=None, scale=None, causal=True, out=None, lse=None,
+                      final=False, final_out=None, final_lse=None, workspace=None, err=None,
+                      stream=None):
+    """Packed multi-request attention: request b's queries are rows
+    cu_seqlens_q[b] .. cu_seqlens_q[b+1] - 1 of q [total_q, Hq, D] (the last
+    n_b positions of its context).  Returns (out [total_q, Hq, D], lse
+    [Hq, total_q]); with final=True also (final_out [B, Hq, D], final_lse
+    [B, Hq]), each request's last query row.  See include/pagedkv.h."""
+    _need_packed_bf16("q", q)
+    _need_cuda_bf16("k_cache", k_cache)
+    _need_cuda_bf16("v_cache", v_cache)
+    _need_cuda_i32("block_table", block_table)
+    _need_cuda_i32("seqlens", seqlens)
+    _need_cuda_i32("cu_seqlens_q", cu_seqlens_q)
+    if block_table.stride(1) != 1:
+        raise ValueError("block_table must have a unit column stride")
+    total_q, Hq, D = q.shape
+    B = int(seqlens.shape[0])
+    if tuple(cu_seqlens_q.shape) != (B + 1,):
+        raise ValueError("cu_seqlens_q must have batch + 1 entries")
+    num_blocks, bs, Hkv, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("q / k_cache / v_cache shapes disagree")
+    if max_seqlen_k is None:
+        max_seqlen_k = int(seqlens.max().item()) if seqlens.numel() else 0
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(total_q, Hq, D, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(Hq, total_q, dtype=torch.float32, device=q.device)
+    _need_packed_bf16("out", out)
+    if tuple(out.shape) != (total_q, Hq, D):
+        raise ValueError("out must be [total_q, Hq, D]")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (Hq, total_q):
+        raise ValueError("lse must be a contiguous fp32 [Hq, total_q] tensor")
+    if final and final_out is None:
+        final_out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=q.device)
+    if final and final_lse is None:
+        final_lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    if final_out is not None:
+        _need_packed_bf16("final_out", final_out)
+        if tuple(final_out.shape) != (B, Hq, D) or final_lse is None or \
+                tuple(final_lse.shape) != (B, Hq) or not final_lse.is_contiguous():
+            raise ValueError("final_out must be [B, Hq, D] and final_lse a contiguous [B, Hq]")
+    need = varlen_workspace_size(total_q, Hq, D, max_seqlen_k)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = lib().pkv_paged_varlen_attn(
+        q.data_ptr(), _st2(q), cu_seqlens_q.data_ptr(), total_q, int(max_seqlen_q),
+        k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(), _st3(v_cache), num_blocks,
+        block_table.data_ptr(), int(block_table.stride(0)), int(block_table.shape[1]),
+        seqlens.data_ptr(), int(max_seqlen_k), B, Hq, Hkv, D, bs, float(scale),
+        int(bool(causal)), out.data_ptr(), _st2(out), lse.data_ptr(), _ptr(final_out),
+        None if final_out is None else _st2(final_out), _ptr(final_lse), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _ptr(err), _stream_handle(stream))
+    _check("pkv_paged_varlen_attn", rc)
+    if final_out is not None:
+        return out, lse, final_out, final_lse
+    return out, lse
+
+
+def kv_append_varlen(k_new, v_new, k_cache, v_cache, block_table, seqlens, cu_seqlens_new, *,
+                     err=None, stream=None) -> None:
+    """Write packed k_new/v_new [total_new, Hkv, D] (sequence b's tokens are
+    rows cu_seqlens_new[b] .. cu_seqlens_new[b+1] - 1) at positions
+    seqlens[b] + t.  seqlens is not advanced."""
+    _need_packed_bf16("k_new", k_new)
+    _need_packed_bf16("v_new", v_new)
+    _need_cuda_bf16("k_cache", k_cache)
+    _need_cuda_bf16("v_cache", v_cache)
+    _need_cuda_i32("block_table", block_table)
+    _need_cuda_i32("seqlens", seqlens)
+    _need_cuda_i32("cu_seqlens_new", cu_seqlens_new)
+    if block_table.stride(1) != 1:
+        raise ValueError("block_table must have a unit column stride")
+    total, Hkv, D = k_new.shape
+    B = int(seqlens.shape[0])
+    rc = lib().pkv_kv_append_varlen(
+        k_new.data_ptr(), _st2(k_new), v_new.data_ptr(), _st2(v_new), cu_seqlens_new.data_ptr(),
+        total, k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(), _st3(v_cache),
+        int(k_cache.shape[0]), block_table.data_ptr(), int(block_table.stride(0)),
+        int(block_table.shape[1]), seqlens.data_ptr(), B, Hkv, D, int(k_cache.shape[1]),
+        _ptr(err), _stream_handle(stream))
+    _check("pkv_kv_append_varlen", rc)
 
 
 # Allocation-free decode (see pkv_paged_decode_attn_static_ws in pagedkv.h).

@@ -96,7 +96,9 @@ __device__ __forceinline__ void write_final_row(const AttnParams &p, const Unit 
     k_c = kc.c;
   }
   const bool seen = m != NEG_INF;
-  __nv_bfloat16 *o = p.out + x.b * p.o_sb + i * p.o_ss + h * p.o_sh;
+  __nv_bfloat16 *o = p.out + o_tok_off(p, x, i) + h * p.o_sh;
+  const bool fin = p.fin_out != nullptr && i == x.nq - 1;  // the sequence's last query row
+  __nv_bfloat16 *fo = fin ? p.fin_out + x.b * p.fo_sb + h * p.fo_sh : nullptr;
 #pragma unroll
   for (int c8 = 0; c8 < D / 8; ++c8) {
     float v[8];
@@ -114,8 +116,14 @@ __device__ __forceinline__ void write_final_row(const AttnParams &p, const Unit 
 #pragma unroll
       for (int e = 0; e < 8; ++e) o[c8 * 8 + e] = __float2bfloat16_rn(v[e]);
     }
+    if (fin) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) fo[c8 * 8 + e] = __float2bfloat16_rn(v[e]);
+    }
   }
-  p.lse[(static_cast<int64_t>(x.b) * p.Hq + h) * p.seqlen_q + i] = final_lse(M, L);
+  const float ls = final_lse(M, L);
+  p.lse[lse_index(p, x, i, h)] = ls;
+  if (fin) p.fin_lse[static_cast<int64_t>(x.b) * p.Hq + h] = ls;
 }
 
 template <int D, int NS>
@@ -276,7 +284,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       if (t < x.rows) {
         const int i = (x.row0 + t) / p.G;
         int lim = x.seqlen;
-        if (p.causal) lim = min(lim, x.seqlen - p.seqlen_q + i + 1);
+        if (p.causal) lim = min(lim, x.seqlen - x.nq + i + 1);
         nlim = lim > 0 ? lim : 0;
       }
       for (int j = 0; j < x.n_tiles; ++j) {
@@ -423,10 +431,11 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     bool stop = false;
     for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
       const Unit x = unit_at<kRowsPerTile>(p, u);
+      if (t == 0) check_query_count(p, x);
       if (x.n_tiles == 0) {
-        // rows that see no key: out = 0, lse = -inf (written here only when
-        // there is no merge to write them)
-        if (p.direct && t < x.rows) {
+        // rows that see no key: out = 0, lse = -inf (written by the unit of
+        // split 0; the merge skips rows of at most one split)
+        if (x.s == 0 && t < x.rows) {
 #pragma unroll
           for (int c = 0; c < D; ++c) acc[c] = 0.f;
           write_final_row<D>(p, x, t, NEG_INF, 0.f, acc);
@@ -482,15 +491,19 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       }
       if (stop) break;
       if (t < x.rows) {
-        if (p.direct) {
-          write_final_row<D>(p, x, t, m_run, l_run, acc);
+        // A row whose visible keys all lie in split 0 is finished here, with
+        // the merge's fold of one split; other rows leave a partial.
+        const int i = (x.row0 + t) / p.G;
+        int lim = x.seqlen;
+        if (p.causal) lim = min(lim, x.seqlen - x.nq + i + 1);
+        const bool single = lim <= kSplitTokens;
+        if (single) {
+          if (x.s == 0) write_final_row<D>(p, x, t, m_run, l_run, acc);
         } else {
           // unnormalised split partial of the row
-          const int r = x.row0 + t;
-          const int i = r / p.G, g = r - i * p.G;
+          const int g = x.row0 + t - i * p.G;
           const int64_t S = p.n_splits;
-          const int64_t row_id =
-              (static_cast<int64_t>(x.b) * p.seqlen_q + i) * p.Hq + x.kvh * p.G + g;
+          const int64_t row_id = (x.q0 + i) * p.Hq + x.kvh * p.G + g;
           float4 *dst = reinterpret_cast<float4 *>(p.ws_acc + (row_id * S + x.s) * D);
 #pragma unroll
           for (int c4 = 0; c4 < D / 4; ++c4)

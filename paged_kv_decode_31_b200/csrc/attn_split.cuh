@@ -58,6 +58,7 @@ constexpr int kMmaWarp = 14;   // MMA issuer + TMEM owner
 constexpr int kErrBadBlock = 1;
 constexpr int kErrTableWidth = 2;
 constexpr int kErrTimeout = 4;
+constexpr int kErrQueryLen = 8;
 
 struct AttnParams {
   const __nv_bfloat16 *q;
@@ -84,12 +85,25 @@ struct AttnParams {
   int64_t kn_sb, kn_st, kn_sh, vn_sb, vn_st, vn_sh;
   uint16_t *k_cache, *v_cache;
   int64_t k_sb, k_ss, k_sh, v_sb, v_ss, v_sh;
-  // Direct final write (row-major kernel, one split per row): out / lse are
-  // written by the split kernel itself with the merge's arithmetic.
+  // Final write by the row-major kernel (rows of at most one split): out /
+  // lse written with the merge's arithmetic.  direct: every row of the call
+  // has at most one split (host side: no merge launch).
   int direct, out_vec;
   __nv_bfloat16 *out;
   int64_t o_sb, o_ss, o_sh;
   float *lse;
+  // Packed (varlen) queries, cu_q != null: sequence b's query tokens are the
+  // tokens cu_q[b] .. cu_q[b+1] - 1 of q and out (token stride q_ss / o_ss),
+  // lse is [Hq, total_q], and seqlen_q is the host bound on every sequence's
+  // query count.  Dense (cu_q == null): q / out are [batch, seqlen_q, ...],
+  // lse [batch, Hq, seqlen_q].
+  const int32_t *cu_q;
+  int total_q;
+  // Optional copy of each sequence's last query row (its "final" row):
+  // fin_out [batch, Hq, D] (strides fo_sb, fo_sh), fin_lse [batch, Hq].
+  __nv_bfloat16 *fin_out;
+  int64_t fo_sb, fo_sh;
+  float *fin_lse;
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -178,30 +192,43 @@ struct Cfg {
 
 struct Unit {
   int b, kvh, rt, s;
+  int nq;       // query tokens of sequence b
+  int64_t q0;   // flat index of its first query token (row id = (q0 + i) * Hq + h)
   int seqlen, row0, rows;
   int tok0;     // first token of the split
   int lim_max;  // keys [0, lim_max) cover every row of the tile
   int n_tiles;  // tiles of this split holding keys < lim_max
 };
 
+// Unit u = kvh + Hkv * (s + n_splits * (b + batch * rt)): the row tile varies
+// slowest, so the first row tiles of every sequence (all the work of decode
+// steps in a packed batch) spread over all CTAs of the strided assignment.
 template <int N>
 __device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
   Unit x;
-  x.rt = u % p.n_row_tiles;
-  u /= p.n_row_tiles;
   x.kvh = u % p.Hkv;
   u /= p.Hkv;
   x.s = u % p.n_splits;
-  x.b = u / p.n_splits;
+  u /= p.n_splits;
+  x.b = u % p.batch;
+  x.rt = u / p.batch;
   const int sl = __ldg(p.seqlens + x.b);
   x.seqlen = sl > 0 ? sl : 0;
-  const int R = p.G * p.seqlen_q;
+  if (p.cu_q) {
+    const int a = __ldg(p.cu_q + x.b), e = __ldg(p.cu_q + x.b + 1);
+    x.q0 = a;
+    x.nq = min(max(e - a, 0), p.seqlen_q);  // more than the bound: flagged, rows past it unwritten
+  } else {
+    x.q0 = static_cast<int64_t>(x.b) * p.seqlen_q;
+    x.nq = p.seqlen_q;
+  }
+  const int R = p.G * x.nq;
   x.row0 = x.rt * N;
-  x.rows = min(N, R - x.row0);
-  int lim = x.seqlen;
-  if (p.causal) {
+  x.rows = max(min(N, R - x.row0), 0);
+  int lim = x.rows > 0 ? x.seqlen : 0;
+  if (p.causal && x.rows > 0) {
     const int i_last = (x.row0 + x.rows - 1) / p.G;
-    lim = min(lim, x.seqlen - p.seqlen_q + i_last + 1);
+    lim = min(lim, x.seqlen - x.nq + i_last + 1);
   }
   x.lim_max = lim > 0 ? lim : 0;
   x.tok0 = x.s * kSplitTokens;
@@ -211,6 +238,28 @@ __device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
 }
 
 constexpr int kPastWidth = static_cast<int>(0x80000000u);
+
+// Element offsets of query token i of unit x's sequence in q and out, and the
+// lse index of (token i, head h).
+__device__ __forceinline__ int64_t q_tok_off(const AttnParams &p, const Unit &x, int i) {
+  return p.cu_q ? (x.q0 + i) * p.q_ss : x.b * p.q_sb + static_cast<int64_t>(i) * p.q_ss;
+}
+__device__ __forceinline__ int64_t o_tok_off(const AttnParams &p, const Unit &x, int i) {
+  return p.cu_q ? (x.q0 + i) * p.o_ss : x.b * p.o_sb + static_cast<int64_t>(i) * p.o_ss;
+}
+__device__ __forceinline__ int64_t lse_index(const AttnParams &p, const Unit &x, int i, int h) {
+  return p.cu_q ? static_cast<int64_t>(h) * p.total_q + x.q0 + i
+                : (static_cast<int64_t>(x.b) * p.Hq + h) * p.seqlen_q + i;
+}
+
+// Sequences whose query count exceeds the host bound are flagged once (by
+// the unit of their first row tile, KV head 0, split 0).
+__device__ __forceinline__ void check_query_count(const AttnParams &p, const Unit &x) {
+  if (p.cu_q && x.rt == 0 && x.kvh == 0 && x.s == 0 && p.err) {
+    const int n = __ldg(p.cu_q + x.b + 1) - __ldg(p.cu_q + x.b);
+    if (n < 0 || n > p.seqlen_q) atomicOr(p.err, kErrQueryLen);
+  }
+}
 
 // First unit at or after `from` (stride gridDim.x) with work, or -1.
 template <int N>
@@ -234,7 +283,7 @@ __device__ __forceinline__ void stage_q(const AttnParams &p, const Unit &x, uint
     if (c < x.rows) {
       const int r = x.row0 + c;
       const int i = r / p.G, g = r - i * p.G;
-      v = __ldg(reinterpret_cast<const uint4 *>(p.q + x.b * p.q_sb + static_cast<int64_t>(i) * p.q_ss +
+      v = __ldg(reinterpret_cast<const uint4 *>(p.q + q_tok_off(p, x, i) +
                                                 static_cast<int64_t>(x.kvh * p.G + g) * p.q_sh +
                                                 ch * 8));
     }
@@ -308,10 +357,13 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
       if (lane == 0) {
         mbar_expect_tx(&sm->q_full[qb], static_cast<uint32_t>(C::kQBytes));
         const int i0 = u.row0 / p.G;
+        // dense map (D, Hq, seqlen_q, batch); packed map (D, Hq, total_q, 1)
+        const int c2 = p.cu_q ? static_cast<int>(u.q0) + i0 : i0;
+        const int c3 = p.cu_q ? 0 : u.b;
 #pragma unroll
         for (int h = 0; h < D / 64; ++h)
           tma_load_4d(smem + C::kOffQ + qb * C::kQBytes + h * C::kQHalfBytes, map_q,
-                      &sm->q_full[qb], h * 64, u.kvh * p.G, i0, u.b);
+                      &sm->q_full[qb], h * 64, u.kvh * p.G, c2, c3);
       }
     } else {
       stage_q<D, N>(p, u, smem + C::kOffQ + qb * C::kQBytes, lane);
@@ -567,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t < x.rows) {
           const int i = (x.row0 + t) / p.G;
           lim = x.seqlen;
-          if (p.causal) lim = min(lim, x.seqlen - p.seqlen_q + i + 1);
+          if (p.causal) lim = min(lim, x.seqlen - x.nq + i + 1);
           lim = lim > 0 ? lim : 0;
         }
         sm->lim[wg][t] = lim;
@@ -684,6 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool stop = false;
     for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
       const Unit x = unit_at<N>(p, u);
+      if (t == 0) check_query_count(p, x);
       if (x.n_tiles == 0) continue;
 #pragma unroll
       for (int c = 0; c < N; ++c) acc[c] = 0.f;
@@ -745,15 +798,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c < x.rows && t < D) {
           const int r = x.row0 + c;
           const int i = r / p.G, g = r - i * p.G;
-          const int64_t row_id =
-              (static_cast<int64_t>(x.b) * p.seqlen_q + i) * p.Hq + x.kvh * p.G + g;
+          const int64_t row_id = (x.q0 + i) * p.Hq + x.kvh * p.G + g;
           p.ws_acc[(row_id * S + x.s) * D + t] = acc[c];
         }
       }
       if (t < x.rows) {
         const int r = x.row0 + t;
         const int i = r / p.G, g = r - i * p.G;
-        const int64_t row_id = (static_cast<int64_t>(x.b) * p.seqlen_q + i) * p.Hq + x.kvh * p.G + g;
+        const int64_t row_id = (x.q0 + i) * p.Hq + x.kvh * p.G + g;
         p.ws_ml[(row_id * S + x.s) * 2 + 0] = m_run;
         p.ws_ml[(row_id * S + x.s) * 2 + 1] = l_run;
       }

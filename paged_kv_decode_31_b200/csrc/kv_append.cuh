@@ -10,6 +10,8 @@
 
 #include <cstdint>
 
+#include "packed.cuh"
+
 namespace pkv {
 
 struct AppendParams {
@@ -28,19 +30,37 @@ struct AppendParams {
   // call appends (seqlens after it): then positions below 0 are skipped
   // without an error, as the fused path does.
   int seq_bias;
+  // Packed new tokens (cu_new != null): k_new / v_new are [total_new, Hkv, D]
+  // (token stride kn_st / vn_st) and token tf belongs to sequence
+  // b = seq_of_token(cu_new, batch, tf) at t = tf - cu_new[b].
+  const int32_t *cu_new;
+  int total_new;
   int32_t *err;
 };
 
 __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ AppendParams p) {
-  const int64_t total = static_cast<int64_t>(p.batch) * p.n_new * p.Hkv * p.chunks;
+  const int64_t tokens = p.cu_new ? static_cast<int64_t>(p.total_new)
+                                  : static_cast<int64_t>(p.batch) * p.n_new;
+  const int64_t total = tokens * p.Hkv * p.chunks;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int c = static_cast<int>(idx % p.chunks);
     int64_t r = idx / p.chunks;
     const int h = static_cast<int>(r % p.Hkv);
-    r /= p.Hkv;
-    const int t = static_cast<int>(r % p.n_new);
-    const int b = static_cast<int>(r / p.n_new);
+    r /= p.Hkv;  // token: b * n_new + t, or the packed index
+    int b, t;
+    int64_t kn_off, vn_off;
+    if (p.cu_new) {
+      b = seq_of_token(p.cu_new, p.batch, r);
+      t = static_cast<int>(r - __ldg(p.cu_new + b));
+      kn_off = r * p.kn_st;
+      vn_off = r * p.vn_st;
+    } else {
+      t = static_cast<int>(r % p.n_new);
+      b = static_cast<int>(r / p.n_new);
+      kn_off = b * p.kn_sb + t * p.kn_st;
+      vn_off = b * p.vn_sb + t * p.vn_st;
+    }
     const int64_t pos = static_cast<int64_t>(__ldg(p.seqlens + b)) - p.seq_bias + t;
     const int64_t bi = pos >> p.block_shift;
     if (pos < 0 && p.seq_bias > 0) continue;
@@ -54,10 +74,8 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ 
       continue;
     }
     const int64_t slot = pos & ((int64_t{1} << p.block_shift) - 1);
-    const uint4 kv = __ldg(reinterpret_cast<const uint4 *>(p.k_new + b * p.kn_sb + t * p.kn_st +
-                                                           h * p.kn_sh) + c);
-    const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(p.v_new + b * p.vn_sb + t * p.vn_st +
-                                                           h * p.vn_sh) + c);
+    const uint4 kv = __ldg(reinterpret_cast<const uint4 *>(p.k_new + kn_off + h * p.kn_sh) + c);
+    const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(p.v_new + vn_off + h * p.vn_sh) + c);
     reinterpret_cast<uint4 *>(p.k_cache + blk * p.k_sb + slot * p.k_ss + h * p.k_sh)[c] = kv;
     reinterpret_cast<uint4 *>(p.v_cache + blk * p.v_sb + slot * p.v_ss + h * p.v_sh)[c] = vv;
   }

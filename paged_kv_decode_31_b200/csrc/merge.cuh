@@ -17,6 +17,7 @@
 
 #include <cuda_bf16.h>
 
+#include "packed.cuh"
 #include "ptx.cuh"
 
 namespace pkv {
@@ -29,7 +30,19 @@ struct MergeParams {
   __nv_bfloat16 *out;
   int64_t o_sb, o_ss, o_sh;
   float *lse;
+  // packed queries (as AttnParams): rows are token-major over the packed
+  // tokens, lse [Hq, total_q]; the last query row of each sequence is also
+  // written to fin_out / fin_lse when they are given
+  const int32_t *cu_q;
+  int batch, total_q;
+  __nv_bfloat16 *fin_out;
+  int64_t fo_sb, fo_sh;
+  float *fin_lse;
+  int64_t rows;     // output rows (tokens x Hq)
+  int skip_single;  // rows of at most one split were finished by the split kernel
 };
+
+constexpr int kMergeRowsPerBlock = 8;  // one warp per row
 
 // One step of the ascending fold: partial (m_s, l_s, x_s) into (M, L, X).
 struct FoldCoef {
@@ -51,46 +64,91 @@ __device__ __forceinline__ float final_lse(float M, float L) {
                  : __int_as_float(0xff800000);
 }
 
+// One warp per output row; lane l owns head_dim elements [l V, l V + V),
+// V = D / 32.  Every element runs the fold above in ascending split order.
 template <int D>
-__global__ void __launch_bounds__(D) merge_kernel(const __grid_constant__ MergeParams p) {
-  const int64_t row = blockIdx.x;  // (b * seqlen_q + i) * Hq + h
+__global__ void __launch_bounds__(32 * kMergeRowsPerBlock)
+    merge_kernel(const __grid_constant__ MergeParams p) {
+  constexpr int V = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kMergeRowsPerBlock + warp;
+  if (row >= p.rows) return;  // row = token * Hq + h; token = b * seqlen_q + i, or packed
   const int h = static_cast<int>(row % p.Hq);
-  const int64_t bi = row / p.Hq;
-  const int i = static_cast<int>(bi % p.seqlen_q);
-  const int b = static_cast<int>(bi / p.seqlen_q);
+  const int64_t tok = row / p.Hq;
+  int b, i, nq;
+  if (p.cu_q) {
+    b = seq_of_token(p.cu_q, p.batch, tok);
+    const int a = __ldg(p.cu_q + b);
+    i = static_cast<int>(tok - a);
+    nq = __ldg(p.cu_q + b + 1) - a;
+    if (i >= p.seqlen_q) return;  // past the host bound: flagged by the split kernel
+  } else {
+    i = static_cast<int>(tok % p.seqlen_q);
+    b = static_cast<int>(tok / p.seqlen_q);
+    nq = p.seqlen_q;
+  }
   const int n = max(__ldg(p.seqlens + b), 0);
   int lim = n;
-  if (p.causal) lim = min(lim, n - p.seqlen_q + i + 1);
+  if (p.causal) lim = min(lim, n - nq + i + 1);
   lim = max(lim, 0);
   const int n_s = min((lim + 4095) / 4096, p.n_splits);
-  const int d = threadIdx.x;
+  if (p.skip_single && n_s <= 1) return;
+  const int d0 = lane * V;
   const float NEG_INF = __int_as_float(0xff800000);
   const float *ml = p.ws_ml + row * p.n_splits * 2;
-  const float *ap = p.ws_acc + row * p.n_splits * D + d;
-  float M = NEG_INF, L = 0.f, A = 0.f;
+  const float *ap = p.ws_acc + row * p.n_splits * D + d0;
+  float M = NEG_INF, L = 0.f, A[V];
+#pragma unroll
+  for (int j = 0; j < V; ++j) A[j] = 0.f;
   // Partials are fetched kBatch splits at a time (independent loads in
   // flight together) and folded strictly in ascending split order.
-  constexpr int kBatch = 16;
+  constexpr int kBatch = 8;
   for (int s0 = 0; s0 < n_s; s0 += kBatch) {
-    float ms[kBatch], ls[kBatch], as[kBatch];
+    float ms[kBatch], ls[kBatch], as[kBatch][V];
 #pragma unroll
     for (int k = 0; k < kBatch; ++k) {
       const int s = s0 + k;
       ms[k] = s < n_s ? ml[2 * s] : NEG_INF;
       ls[k] = s < n_s ? ml[2 * s + 1] : 0.f;
-      as[k] = s < n_s ? ap[static_cast<int64_t>(s) * D] : 0.f;
+#pragma unroll
+      for (int j = 0; j < V; ++j) as[k][j] = 0.f;
+      if (s < n_s) {
+        if constexpr (V == 4) {
+          const float4 v = *reinterpret_cast<const float4 *>(ap + static_cast<int64_t>(s) * D);
+          as[k][0] = v.x; as[k][1] = v.y; as[k][2] = v.z; as[k][3] = v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2 *>(ap + static_cast<int64_t>(s) * D);
+          as[k][0] = v.x; as[k][1] = v.y;
+        }
+      }
     }
 #pragma unroll
     for (int k = 0; k < kBatch; ++k) {
       if (ms[k] == NEG_INF) continue;  // the row sees no key of this split
       const FoldCoef kc = fold_coef(M, ms[k]);
       L = fold_val(L, ls[k], kc);
-      A = fold_val(A, as[k], kc);
+#pragma unroll
+      for (int j = 0; j < V; ++j) A[j] = fold_val(A[j], as[k][j], kc);
       M = kc.Mn;
     }
   }
-  p.out[b * p.o_sb + i * p.o_ss + h * p.o_sh + d] = __float2bfloat16_rn(final_out(A, L));
-  if (d == 0) p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.seqlen_q + i] = final_lse(M, L);
+  const float ls = final_lse(M, L);
+  __nv_bfloat16 *o = p.cu_q ? p.out + tok * p.o_ss + h * p.o_sh
+                            : p.out + b * p.o_sb + i * p.o_ss + h * p.o_sh;
+  const bool fin = p.fin_out != nullptr && i == nq - 1;
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    const __nv_bfloat16 ob = __float2bfloat16_rn(final_out(A[j], L));
+    o[d0 + j] = ob;
+    if (fin) p.fin_out[b * p.fo_sb + h * p.fo_sh + d0 + j] = ob;
+  }
+  if (lane == 0) {
+    if (p.cu_q)
+      p.lse[static_cast<int64_t>(h) * p.total_q + tok] = ls;
+    else
+      p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.seqlen_q + i] = ls;
+    if (fin) p.fin_lse[static_cast<int64_t>(b) * p.Hq + h] = ls;
+  }
 }
 
 }  // namespace pkv

@@ -22,6 +22,7 @@ static_assert(PKV_TILE_TOKENS == pkv::kTileTokens, "tile size");
 static_assert(PKV_DEVERR_BAD_BLOCK == pkv::kErrBadBlock, "error bits");
 static_assert(PKV_DEVERR_TABLE_WIDTH == pkv::kErrTableWidth, "error bits");
 static_assert(PKV_DEVERR_TIMEOUT == pkv::kErrTimeout, "error bits");
+static_assert(PKV_DEVERR_QUERY_LEN == pkv::kErrQueryLen, "error bits");
 
 namespace {
 
@@ -128,6 +129,7 @@ int make_kv_map(CUtensorMap *map, const void *base, const int64_t st[3], int64_t
 // The box is 64 head_dim x G heads x 128 / G tokens of one sequence: it lands
 // as the 128 rows r = i * G + g of one row tile (row r at r * 128 bytes,
 // 128-byte swizzled); tokens past seqlen_q read as zeros.
+// Packed queries use the same box over dims (D, Hq, total_q, 1).
 int make_q_map(CUtensorMap *map, const void *q, const int64_t st[3], int batch, int seqlen_q,
                int Hq, int D, int G) {
   auto enc = encode_fn();
@@ -204,7 +206,8 @@ int launch_rows(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensorM
 
 template <int D>
 int launch_merge(const pkv::MergeParams &m, int64_t rows, cudaStream_t s) {
-  pkv::merge_kernel<D><<<static_cast<unsigned>(rows), D, 0, s>>>(m);
+  const int64_t blocks = ceil_div(rows, pkv::kMergeRowsPerBlock);
+  pkv::merge_kernel<D><<<static_cast<unsigned>(blocks), 32 * pkv::kMergeRowsPerBlock, 0, s>>>(m);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -225,7 +228,8 @@ int launch_append(const void *k_new, const int64_t kn_strides[3], const void *v_
                   void *v_cache, const int64_t v_strides[3], int64_t num_blocks,
                   const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
                   const int32_t *seqlens, int batch, int n_new, int Hkv, int D, int block_size,
-                  int seq_bias, int32_t *err, cudaStream_t stream) {
+                  int seq_bias, int32_t *err, cudaStream_t stream,
+                  const int32_t *cu_new = nullptr, int total_new = 0) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
   pkv::AppendParams p{};
@@ -256,8 +260,11 @@ int launch_append(const void *k_new, const int64_t kn_strides[3], const void *v_
   p.chunks = D / 8;
   p.block_shift = log2i(block_size);
   p.seq_bias = seq_bias;
+  p.cu_new = cu_new;
+  p.total_new = total_new;
   p.err = err;
-  const int64_t total = static_cast<int64_t>(batch) * n_new * Hkv * (D / 8);
+  const int64_t tokens = cu_new ? static_cast<int64_t>(total_new) : static_cast<int64_t>(batch) * n_new;
+  const int64_t total = tokens * Hkv * (D / 8);
   const int64_t want = ceil_div(total, 256);
   const int64_t cap = static_cast<int64_t>(sm_count(dev)) * 8;
   const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
@@ -275,6 +282,16 @@ struct FusedAppend {
   int n_new;
 };
 
+// Packed (varlen) queries: cu_q [batch + 1] on the device, total_q tokens;
+// optional copies of each sequence's last query row.
+struct PackedQ {
+  const int32_t *cu_q;
+  int total_q;
+  void *fin_out;
+  const int64_t *fin_strides;  // (batch, head)
+  float *fin_lse;
+};
+
 int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
                const int64_t k_strides[3], const void *v_cache, const int64_t v_strides[3],
                int64_t num_blocks, const int32_t *block_table, int64_t bt_stride,
@@ -282,7 +299,7 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
                int seqlen_q, int Hq, int Hkv, int D, int block_size, float scale, int causal,
                void *out, const int64_t out_strides[3], float *lse, void *workspace,
                size_t workspace_bytes, int32_t *err, void *stream,
-               const FusedAppend *app = nullptr) {
+               const FusedAppend *app = nullptr, const PackedQ *pq = nullptr) {
   if (!q || !k_cache || !v_cache || !block_table || !seqlens || !out || !lse) return PKV_ERR_ARG;
   if (batch <= 0 || seqlen_q <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return PKV_ERR_ARG;
   if (D != 64 && D != 128) return PKV_ERR_ARG;
@@ -297,18 +314,27 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   if (!(scale > 0.f) || !(scale < 3.0e38f)) return PKV_ERR_ARG;
   const int G = Hq / Hkv;
   const int64_t R = static_cast<int64_t>(G) * seqlen_q;
-  const int64_t rows = static_cast<int64_t>(batch) * seqlen_q * Hq;
+  if (pq && (!pq->cu_q || pq->total_q <= 0 || (app && app->n_new > 0))) return PKV_ERR_ARG;
+  if (pq && pq->fin_out && (!pq->fin_lse || !pq->fin_strides || pq->fin_strides[0] <= 0 ||
+                            pq->fin_strides[1] <= 0))
+    return PKV_ERR_ARG;
+  const int64_t tokens = pq ? static_cast<int64_t>(pq->total_q) : static_cast<int64_t>(batch) * seqlen_q;
+  const int64_t rows = tokens * Hq;
   if (R > INT32_MAX / 2 || rows > INT32_MAX) return PKV_ERR_ARG;
   alignas(64) CUtensorMap mq;
-  int N = rows_per_tile(R, G, seqlen_q);
+  // (a Q box spans 128 / G tokens: of one sequence when dense, of the packed
+  // token axis otherwise)
+  int N = rows_per_tile(R, G, pq ? pq->total_q : seqlen_q);
   if (N == pkv::kRowsPerTile &&
-      make_q_map(&mq, q, q_strides, batch, seqlen_q, Hq, D, G) != PKV_OK)
+      (pq ? make_q_map(&mq, q, q_strides, 1, pq->total_q, Hq, D, G)
+          : make_q_map(&mq, q, q_strides, batch, seqlen_q, Hq, D, G)) != PKV_OK)
     N = 64;  // q's strides cannot be described to the TMA unit: transposed kernel
   const int64_t S = max_seqlen_k > 0 ? ceil_div(max_seqlen_k, pkv::kSplitTokens) : 1;
   const int64_t RT = ceil_div(R, N);
   const int64_t units = static_cast<int64_t>(batch) * S * Hkv * RT;
   if (units > INT32_MAX) return PKV_ERR_ARG;
-  const size_t need = ws_bytes(batch, seqlen_q, Hq, D, max_seqlen_k);
+  const size_t need = pq ? ws_bytes(1, pq->total_q, Hq, D, max_seqlen_k)
+                        : ws_bytes(batch, seqlen_q, Hq, D, max_seqlen_k);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
 
   int dev = 0;
@@ -351,6 +377,16 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   p.ws_acc = ws_acc;
   p.ws_ml = ws_ml;
   p.err = err;
+  if (pq) {
+    p.cu_q = pq->cu_q;
+    p.total_q = pq->total_q;
+    if (pq->fin_out) {
+      p.fin_out = static_cast<__nv_bfloat16 *>(pq->fin_out);
+      p.fo_sb = pq->fin_strides[0];
+      p.fo_sh = pq->fin_strides[1];
+      p.fin_lse = pq->fin_lse;
+    }
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (app && app->n_new > 0) {
     if (!app->k_new || !app->v_new || !strides_ok(app->kn_strides) ||
@@ -387,7 +423,8 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   }
 
   if (N == pkv::kRowsPerTile) {
-    // one split per row: the split kernel writes out / lse itself
+    // rows of at most one split are finished by the split kernel itself; the
+    // merge (needed only with more than one split) skips them
     p.direct = S == 1 ? 1 : 0;
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.o_sb = out_strides[0];
@@ -420,6 +457,15 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   m.o_ss = out_strides[1];
   m.o_sh = out_strides[2];
   m.lse = lse;
+  m.cu_q = p.cu_q;
+  m.batch = batch;
+  m.total_q = p.total_q;
+  m.fin_out = p.fin_out;
+  m.fo_sb = p.fo_sb;
+  m.fo_sh = p.fo_sh;
+  m.fin_lse = p.fin_lse;
+  m.rows = rows;
+  m.skip_single = N == pkv::kRowsPerTile ? 1 : 0;
   return D == 128 ? launch_merge<128>(m, rows, s) : launch_merge<64>(m, rows, s);
 }
 
@@ -494,6 +540,60 @@ int pkv_paged_decode_attn_append(const void *q, const int64_t q_strides[3], cons
                     bt_stride, max_blocks_per_seq, seqlens, max_seqlen_k, batch, seqlen_q, Hq, Hkv,
                     D, block_size, scale, causal, out, out_strides, lse, workspace,
                     workspace_bytes, err, stream, &app);
+}
+
+int pkv_paged_varlen_attn(const void *q, const int64_t q_strides[2], const int32_t *cu_seqlens_q,
+                          int total_q, int max_seqlen_q, const void *k_cache,
+                          const int64_t k_strides[3], const void *v_cache,
+                          const int64_t v_strides[3], int64_t num_blocks,
+                          const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                          const int32_t *seqlens, int max_seqlen_k, int batch, int Hq, int Hkv,
+                          int D, int block_size, float scale, int causal, void *out,
+                          const int64_t out_strides[2], float *lse, void *final_out,
+                          const int64_t final_strides[2], float *final_lse, void *workspace,
+                          size_t workspace_bytes, int32_t *err, void *stream) {
+  if (!q_strides || !out_strides || !cu_seqlens_q || total_q <= 0 || max_seqlen_q <= 0)
+    return PKV_ERR_ARG;
+  // the batch stride of the packed views is never used; repeat the token stride
+  const int64_t qs[3] = {q_strides[0], q_strides[0], q_strides[1]};
+  const int64_t os[3] = {out_strides[0], out_strides[0], out_strides[1]};
+  const PackedQ pq{cu_seqlens_q, total_q, final_out, final_strides, final_lse};
+  return attn_entry(q, qs, k_cache, k_strides, v_cache, v_strides, num_blocks, block_table,
+                    bt_stride, max_blocks_per_seq, seqlens, max_seqlen_k, batch, max_seqlen_q, Hq,
+                    Hkv, D, block_size, scale, causal, out, os, lse, workspace, workspace_bytes,
+                    err, stream, nullptr, &pq);
+}
+
+size_t pkv_varlen_workspace_size(int total_q, int Hq, int D, int max_seqlen_k) {
+  if (total_q <= 0 || Hq <= 0 || D <= 0 || max_seqlen_k < 0) return 0;
+  return ws_bytes(1, total_q, Hq, D, max_seqlen_k);
+}
+
+int pkv_kv_append_varlen(const void *k_new, const int64_t kn_strides[2], const void *v_new,
+                         const int64_t vn_strides[2], const int32_t *cu_seqlens_new, int total_new,
+                         void *k_cache, const int64_t k_strides[3], void *v_cache,
+                         const int64_t v_strides[3], int64_t num_blocks,
+                         const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                         const int32_t *seqlens, int batch, int Hkv, int D, int block_size,
+                         int32_t *err, void *stream) {
+  if (!k_new || !v_new || !k_cache || !v_cache || !block_table || !seqlens || !cu_seqlens_new ||
+      !kn_strides || !vn_strides)
+    return PKV_ERR_ARG;
+  if (batch <= 0 || total_new < 0 || Hkv <= 0 || (D != 64 && D != 128)) return PKV_ERR_ARG;
+  if (!pow2_in(block_size, 16, 256)) return PKV_ERR_ARG;
+  if (num_blocks <= 0 || num_blocks > INT32_MAX || max_blocks_per_seq <= 0 || bt_stride < max_blocks_per_seq)
+    return PKV_ERR_ARG;
+  const int64_t kn[3] = {kn_strides[0], kn_strides[0], kn_strides[1]};
+  const int64_t vn[3] = {vn_strides[0], vn_strides[0], vn_strides[1]};
+  if (!strides_ok(kn) || !strides_ok(vn) || !strides_ok(k_strides) || !strides_ok(v_strides))
+    return PKV_ERR_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PKV_ERR_ARG;
+  if (total_new == 0) return PKV_OK;
+  return launch_append(k_new, kn, v_new, vn, k_cache, k_strides, v_cache, v_strides, num_blocks,
+                       block_table, bt_stride, max_blocks_per_seq, seqlens, batch, 0, Hkv, D,
+                       block_size, 0, err, static_cast<cudaStream_t>(stream), cu_seqlens_new,
+                       total_new);
 }
 
 size_t pkv_workspace_size(int batch, int seqlen_q, int Hq, int D, int max_seqlen_k) {
