@@ -261,6 +261,59 @@ int pkv_kv_append_varlen(const void *k_new, const int64_t kn_strides[2],
                          const int32_t *seqlens, int batch, int Hkv, int D, int block_size,
                          int32_t *err, void *stream);
 
+/*
+ * Context parallelism (CP) over the KV context -- the CP forward of RL-Kernel
+ * PR #284 "feat(attention): add CP backward drift validation" (Changes: CP
+ * world size, KV chunk size, fixed global_block_index merge order, fp32
+ * accumulation, final-write downcast).  Rank r of W owns the contiguous
+ * splits [split_begin, split_begin + n_splits_local) of every sequence (its
+ * slice of the context; its cache and block table need only hold those
+ * tokens), computes their partials with pkv_paged_attn_partials, the ranks
+ * all-gather the partial buffers (any transport; each rank's buffer is one
+ * block of pkv_partials_size bytes), and every rank calls pkv_merge_partials
+ * on the gathered blocks.  A split's partial does not depend on which rank or
+ * call computed it and the merge folds splits in ascending global index, so
+ * out / lse are bitwise those of one pkv_paged_decode_attn /
+ * pkv_paged_prefill_attn call over the whole context.
+ *
+ * pkv_paged_attn_partials: arguments as pkv_paged_decode_attn (dense q,
+ * seqlens = the FULL context lengths) without out / lse / max_seqlen_k; writes
+ * into `partials` (>= pkv_partials_size(batch, seqlen_q, Hq, D,
+ * n_splits_local) bytes, 16-byte aligned) the fp32 partials (m, l, acc[D]) of
+ * every (row, local split): acc [rows][n_local][D] (256-byte padded), then
+ * (m, l) [rows][n_local][2], rows = batch * seqlen_q * Hq.  Partials of
+ * (row, split) pairs the row does not reach are left unwritten (the merge
+ * never reads them).  Errors as pkv_paged_decode_attn (PKV_ERR_WORKSPACE if
+ * partials is too small).
+ */
+int pkv_paged_attn_partials(const void *q, const int64_t q_strides[3],
+                            const void *k_cache, const int64_t k_strides[3],
+                            const void *v_cache, const int64_t v_strides[3],
+                            int64_t num_blocks,
+                            const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                            const int32_t *seqlens,
+                            int batch, int seqlen_q, int Hq, int Hkv, int D, int block_size,
+                            float scale, int causal,
+                            int split_begin, int n_splits_local,
+                            void *partials, size_t partials_bytes,
+                            int32_t *err, void *stream);
+
+/* Bytes of one rank's partial buffer (0 on invalid arguments). */
+size_t pkv_partials_size(int batch, int seqlen_q, int Hq, int D, int n_splits_local);
+
+/*
+ * pkv_merge_partials: the ascending-split merge and final write over
+ * `world` partial buffers laid side by side (block r, rank_bytes bytes from
+ * block r - 1, holds global splits [r * n_splits_local, (r + 1) *
+ * n_splits_local)).  rank_bytes >= pkv_partials_size(...) and a multiple of
+ * 16; seqlens are the full context lengths; out [batch, seqlen_q, Hq, D]
+ * bf16 (strides as pkv_paged_decode_attn), lse [batch, Hq, seqlen_q] fp32.
+ */
+int pkv_merge_partials(const void *partials, int world, int n_splits_local, size_t rank_bytes,
+                       const int32_t *seqlens, int batch, int seqlen_q, int Hq, int D,
+                       int causal, void *out, const int64_t out_strides[3], float *lse,
+                       void *stream);
+
 /* Workspace bytes the attention calls need: fp32 split partials
  * (m, l, acc[D]) for every (batch, query row, query head, split). */
 size_t pkv_workspace_size(int batch, int seqlen_q, int Hq, int D, int max_seqlen_k);

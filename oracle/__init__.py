@@ -174,3 +174,48 @@ def kv_append_varlen(k_new, v_new, k_cache, v_cache, block_table, seqlens, cu_se
             continue
         kv_append(k_new[a:e].unsqueeze(0), v_new[a:e].unsqueeze(0), k_cache, v_cache,
                   block_table[b:b + 1], seqlens[b:b + 1])
+
+
+def split_partials(q, k_cache, v_cache, block_table, seqlens, scale, causal, split_begin,
+                   n_splits_local, split_tokens=4096):
+    """fp64 unnormalised partials of the splits [split_begin, split_begin +
+    n_splits_local): for every (b, i, h, local split), over the row's visible
+    keys j in [split_tokens * s, split_tokens * (s + 1)): m = max_j s_j (natural
+    units, s_j = scale * q.k_j), l = sum_j exp(s_j - m), acc = sum_j exp(s_j -
+    m) v_j; m = -inf, l = 0, acc = 0 where the row sees no key of the split.
+    The KV chunks of the CP forward (RL-Kernel PR #284, Changes: KV chunk
+    size, fixed global_block_index merge order).  Plain torch fp64 on the CPU.
+
+    Returns (m [B, sq, Hq, n], l [B, sq, Hq, n], acc [B, sq, Hq, n, D])."""
+    B, sq, Hq, D = q.shape
+    nb, bs, Hkv, _ = k_cache.shape
+    G = Hq // Hkv
+    m = torch.full((B, sq, Hq, n_splits_local), float("-inf"), dtype=torch.float64)
+    l = torch.zeros((B, sq, Hq, n_splits_local), dtype=torch.float64)
+    acc = torch.zeros((B, sq, Hq, n_splits_local, D), dtype=torch.float64)
+    for b in range(B):
+        n = max(int(seqlens[b]), 0)
+        if n == 0:
+            continue
+        j = torch.arange(n)
+        blk = block_table[b, j // bs].long()
+        K = k_cache[blk, j % bs].double()    # [n, Hkv, D]
+        V = v_cache[blk, j % bs].double()
+        for i in range(sq):
+            lim = min(n, n - sq + i + 1) if causal else n
+            for h in range(Hq):
+                if lim <= 0:
+                    continue
+                s_all = scale * (K[:lim, h // G] @ q[b, i, h].double())
+                for ls in range(n_splits_local):
+                    a = (split_begin + ls) * split_tokens
+                    e = min(a + split_tokens, lim)
+                    if e <= a:
+                        continue
+                    sc = s_all[a:e]
+                    mm = float(sc.max())
+                    w = torch.exp(sc - mm)
+                    m[b, i, h, ls] = mm
+                    l[b, i, h, ls] = w.sum()
+                    acc[b, i, h, ls] = w @ V[a:e, h // G]
+    return m, l, acc

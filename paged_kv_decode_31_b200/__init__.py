@@ -12,6 +12,9 @@ from .binding import (  # noqa: F401
     kv_append,
     kv_append_varlen,
     library_path,
+    merge_partials,
+    paged_attn_partials,
+    partials_size,
     paged_decode_attn,
     paged_decode_attn_append,
     paged_prefill_attn,

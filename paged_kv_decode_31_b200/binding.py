@@ -339,6 +339,75 @@ def kv_append_varlen(k_new, v_new, k_cache, v_cache, block_table, seqlens, cu_se
     _check("pkv_kv_append_varlen", rc)
 
 
+def partials_size(batch: int, seqlen_q: int, Hq: int, D: int, n_splits_local: int) -> int:
+    L = lib()
+    fn = L.pkv_partials_size
+    if not fn.argtypes:
+        fn.argtypes = [_I, _I, _I, _I, _I]
+        fn.restype = ctypes.c_size_t
+    return int(fn(batch, seqlen_q, Hq, D, n_splits_local))
+
+
+def paged_attn_partials(q, k_cache, v_cache, block_table, seqlens, split_begin, n_splits_local,
+                        *, scale=None, causal=False, partials=None, err=None, stream=None):
+    """Split partials of absolute splits [split_begin, split_begin +
+    n_splits_local) for every row of q [B, sq, Hq, D] (one context-parallel
+    rank's share).  Returns the partial buffer (uint8, pkv_partials_size
+    bytes).  seqlens are the full context lengths."""
+    L = lib()
+    fn = L.pkv_paged_attn_partials
+    if not fn.argtypes:
+        fn.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _P, _I64, _I, _P, _I, _I, _I, _I, _I, _I,
+                       ctypes.c_float, _I, _I, _I, _P, ctypes.c_size_t, _P, _P]
+        fn.restype = _I
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _need_cuda_bf16(name, t)
+    _need_cuda_i32("block_table", block_table)
+    _need_cuda_i32("seqlens", seqlens)
+    if block_table.stride(1) != 1:
+        raise ValueError("block_table must have a unit column stride")
+    B, sq, Hq, D = q.shape
+    num_blocks, bs, Hkv, _ = k_cache.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    need = partials_size(B, sq, Hq, D, n_splits_local)
+    if partials is None:
+        partials = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = fn(q.data_ptr(), _st3(q), k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(),
+            _st3(v_cache), num_blocks, block_table.data_ptr(), int(block_table.stride(0)),
+            int(block_table.shape[1]), seqlens.data_ptr(), B, sq, Hq, Hkv, D, bs, float(scale),
+            int(bool(causal)), int(split_begin), int(n_splits_local), partials.data_ptr(),
+            partials.numel() * partials.element_size(), _ptr(err), _stream_handle(stream))
+    _check("pkv_paged_attn_partials", rc)
+    return partials
+
+
+def merge_partials(gathered, world, n_splits_local, seqlens, q_shape, *, causal=False, out=None,
+                   lse=None, stream=None):
+    """Merge `world` partial buffers laid side by side in `gathered` (uint8,
+    world x partials_size bytes, rank r's block holding global splits
+    [r n_local, (r + 1) n_local)) into (out, lse) for q_shape (B, sq, Hq, D)."""
+    L = lib()
+    fn = L.pkv_merge_partials
+    if not fn.argtypes:
+        fn.argtypes = [_P, _I, _I, ctypes.c_size_t, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]
+        fn.restype = _I
+    _need_cuda_i32("seqlens", seqlens)
+    B, sq, Hq, D = q_shape
+    nbytes = gathered.numel() * gathered.element_size()
+    if nbytes % world != 0:
+        raise ValueError("gathered buffer is not world equal blocks")
+    if out is None:
+        out = torch.empty(B, sq, Hq, D, dtype=torch.bfloat16, device=gathered.device)
+    if lse is None:
+        lse = torch.empty(B, Hq, sq, dtype=torch.float32, device=gathered.device)
+    rc = fn(gathered.data_ptr(), int(world), int(n_splits_local), nbytes // world,
+            seqlens.data_ptr(), B, sq, Hq, D, int(bool(causal)), out.data_ptr(), _st3(out),
+            lse.data_ptr(), _stream_handle(stream))
+    _check("pkv_merge_partials", rc)
+    return out, lse
+
+
 # Allocation-free decode (see pkv_paged_decode_attn_static_ws in pagedkv.h).
 STATIC_WORKSPACE_BYTES = 8 << 20
 

@@ -435,7 +435,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       if (x.n_tiles == 0) {
         // rows that see no key: out = 0, lse = -inf (written by the unit of
         // split 0; the merge skips rows of at most one split)
-        if (x.s == 0 && t < x.rows) {
+        if (!p.part_only && x.s == 0 && t < x.rows) {
 #pragma unroll
           for (int c = 0; c < D; ++c) acc[c] = 0.f;
           write_final_row<D>(p, x, t, NEG_INF, 0.f, acc);
@@ -496,7 +496,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         const int i = (x.row0 + t) / p.G;
         int lim = x.seqlen;
         if (p.causal) lim = min(lim, x.seqlen - x.nq + i + 1);
-        const bool single = lim <= kSplitTokens;
+        const bool single = !p.part_only && lim <= kSplitTokens;
         if (single) {
           if (x.s == 0) write_final_row<D>(p, x, t, m_run, l_run, acc);
         } else {

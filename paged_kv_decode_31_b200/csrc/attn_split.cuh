@@ -104,6 +104,11 @@ struct AttnParams {
   __nv_bfloat16 *fin_out;
   int64_t fo_sb, fo_sh;
   float *fin_lse;
+  // Split range: the units cover absolute splits split_base .. split_base +
+  // n_splits - 1 (one rank's share under context parallelism; 0 otherwise);
+  // partials are stored by local split.  part_only: every row leaves
+  // partials, none is finished in the split kernel.
+  int split_base, part_only;
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -231,7 +236,7 @@ __device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
     lim = min(lim, x.seqlen - x.nq + i_last + 1);
   }
   x.lim_max = lim > 0 ? lim : 0;
-  x.tok0 = x.s * kSplitTokens;
+  x.tok0 = (p.split_base + x.s) * kSplitTokens;
   const int ntok = min(kSplitTokens, x.lim_max - x.tok0);
   x.n_tiles = ntok > 0 ? (ntok + kTileTokens - 1) / kTileTokens : 0;
   return x;

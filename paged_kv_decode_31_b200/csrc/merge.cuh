@@ -40,6 +40,12 @@ struct MergeParams {
   float *fin_lse;
   int64_t rows;     // output rows (tokens x Hq)
   int skip_single;  // rows of at most one split were finished by the split kernel
+  // Partials of global split s live in block r = s / n_local (local split
+  // s % n_local) -- one block per context-parallel rank, gathered side by
+  // side rank_floats floats apart; a single call has one block (n_local =
+  // n_splits).  Within a block: acc [rows][n_local][D], ml [rows][n_local][2].
+  int n_local;
+  int64_t rank_floats;
 };
 
 constexpr int kMergeRowsPerBlock = 8;  // one warp per row
@@ -95,8 +101,6 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerBlock)
   if (p.skip_single && n_s <= 1) return;
   const int d0 = lane * V;
   const float NEG_INF = __int_as_float(0xff800000);
-  const float *ml = p.ws_ml + row * p.n_splits * 2;
-  const float *ap = p.ws_acc + row * p.n_splits * D + d0;
   float M = NEG_INF, L = 0.f, A[V];
 #pragma unroll
   for (int j = 0; j < V; ++j) A[j] = 0.f;
@@ -108,16 +112,22 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerBlock)
 #pragma unroll
     for (int k = 0; k < kBatch; ++k) {
       const int s = s0 + k;
-      ms[k] = s < n_s ? ml[2 * s] : NEG_INF;
-      ls[k] = s < n_s ? ml[2 * s + 1] : 0.f;
+      ms[k] = NEG_INF;
+      ls[k] = 0.f;
 #pragma unroll
       for (int j = 0; j < V; ++j) as[k][j] = 0.f;
       if (s < n_s) {
+        const int r = s / p.n_local;
+        const int64_t e = r * p.rank_floats;  // this rank's block, in floats
+        const int64_t slot = row * p.n_local + (s - r * p.n_local);
+        ms[k] = p.ws_ml[e + slot * 2];
+        ls[k] = p.ws_ml[e + slot * 2 + 1];
+        const float *ap = p.ws_acc + e + slot * D + d0;
         if constexpr (V == 4) {
-          const float4 v = *reinterpret_cast<const float4 *>(ap + static_cast<int64_t>(s) * D);
+          const float4 v = *reinterpret_cast<const float4 *>(ap);
           as[k][0] = v.x; as[k][1] = v.y; as[k][2] = v.z; as[k][3] = v.w;
         } else {
-          const float2 v = *reinterpret_cast<const float2 *>(ap + static_cast<int64_t>(s) * D);
+          const float2 v = *reinterpret_cast<const float2 *>(ap);
           as[k][0] = v.x; as[k][1] = v.y;
         }
       }

@@ -292,6 +292,13 @@ struct PackedQ {
   float *fin_lse;
 };
 
+// Context-parallel share: partials of absolute splits [split_begin,
+// split_begin + n_local) into `partials` (acc then ml, local split order);
+// nothing is merged or written to out / lse.
+struct SplitShare {
+  int split_begin, n_local;
+};
+
 int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
                const int64_t k_strides[3], const void *v_cache, const int64_t v_strides[3],
                int64_t num_blocks, const int32_t *block_table, int64_t bt_stride,
@@ -299,8 +306,11 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
                int seqlen_q, int Hq, int Hkv, int D, int block_size, float scale, int causal,
                void *out, const int64_t out_strides[3], float *lse, void *workspace,
                size_t workspace_bytes, int32_t *err, void *stream,
-               const FusedAppend *app = nullptr, const PackedQ *pq = nullptr) {
-  if (!q || !k_cache || !v_cache || !block_table || !seqlens || !out || !lse) return PKV_ERR_ARG;
+               const FusedAppend *app = nullptr, const PackedQ *pq = nullptr,
+               const SplitShare *share = nullptr) {
+  if (!q || !k_cache || !v_cache || !block_table || !seqlens) return PKV_ERR_ARG;
+  if (!share && (!out || !lse)) return PKV_ERR_ARG;
+  if (share && (pq || app || share->split_begin < 0 || share->n_local <= 0)) return PKV_ERR_ARG;
   if (batch <= 0 || seqlen_q <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return PKV_ERR_ARG;
   if (D != 64 && D != 128) return PKV_ERR_ARG;
   if (!pow2_in(block_size, 16, 256)) return PKV_ERR_ARG;
@@ -308,7 +318,7 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
     return PKV_ERR_ARG;
   if (max_seqlen_k < 0) return PKV_ERR_ARG;
   if (!strides_ok(q_strides) || !strides_ok(k_strides) || !strides_ok(v_strides)) return PKV_ERR_ARG;
-  if (!out_strides || out_strides[0] <= 0 || out_strides[1] <= 0 || out_strides[2] <= 0)
+  if (!share && (!out_strides || out_strides[0] <= 0 || out_strides[1] <= 0 || out_strides[2] <= 0))
     return PKV_ERR_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_ERR_ARG;
   if (!(scale > 0.f) || !(scale < 3.0e38f)) return PKV_ERR_ARG;
@@ -329,12 +339,14 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
       (pq ? make_q_map(&mq, q, q_strides, 1, pq->total_q, Hq, D, G)
           : make_q_map(&mq, q, q_strides, batch, seqlen_q, Hq, D, G)) != PKV_OK)
     N = 64;  // q's strides cannot be described to the TMA unit: transposed kernel
-  const int64_t S = max_seqlen_k > 0 ? ceil_div(max_seqlen_k, pkv::kSplitTokens) : 1;
+  const int64_t S = share ? share->n_local
+                          : (max_seqlen_k > 0 ? ceil_div(max_seqlen_k, pkv::kSplitTokens) : 1);
   const int64_t RT = ceil_div(R, N);
   const int64_t units = static_cast<int64_t>(batch) * S * Hkv * RT;
   if (units > INT32_MAX) return PKV_ERR_ARG;
-  const size_t need = pq ? ws_bytes(1, pq->total_q, Hq, D, max_seqlen_k)
-                        : ws_bytes(batch, seqlen_q, Hq, D, max_seqlen_k);
+  const size_t need = share ? ws_bytes(batch, seqlen_q, Hq, D, static_cast<int>(S) * pkv::kSplitTokens)
+                     : pq ? ws_bytes(1, pq->total_q, Hq, D, max_seqlen_k)
+                          : ws_bytes(batch, seqlen_q, Hq, D, max_seqlen_k);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
 
   int dev = 0;
@@ -377,6 +389,10 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   p.ws_acc = ws_acc;
   p.ws_ml = ws_ml;
   p.err = err;
+  if (share) {
+    p.split_base = share->split_begin;
+    p.part_only = 1;
+  }
   if (pq) {
     p.cu_q = pq->cu_q;
     p.total_q = pq->total_q;
@@ -425,24 +441,26 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   if (N == pkv::kRowsPerTile) {
     // rows of at most one split are finished by the split kernel itself; the
     // merge (needed only with more than one split) skips them
-    p.direct = S == 1 ? 1 : 0;
-    p.out = static_cast<__nv_bfloat16 *>(out);
-    p.o_sb = out_strides[0];
-    p.o_ss = out_strides[1];
-    p.o_sh = out_strides[2];
-    p.lse = lse;
-    p.out_vec = (aligned16(out) && out_strides[0] % 8 == 0 && out_strides[1] % 8 == 0 &&
-                 out_strides[2] % 8 == 0)
-                    ? 1
-                    : 0;
+    p.direct = (S == 1 && !share) ? 1 : 0;
+    if (!share) {
+      p.out = static_cast<__nv_bfloat16 *>(out);
+      p.o_sb = out_strides[0];
+      p.o_ss = out_strides[1];
+      p.o_sh = out_strides[2];
+      p.lse = lse;
+      p.out_vec = (aligned16(out) && out_strides[0] % 8 == 0 && out_strides[1] % 8 == 0 &&
+                   out_strides[2] % 8 == 0)
+                      ? 1
+                      : 0;
+    }
     rc = D == 128 ? launch_rows<128>(p, mk, mv, mq, s, dev) : launch_rows<64>(p, mk, mv, mq, s, dev);
-    if (rc != PKV_OK || p.direct) return rc;
+    if (rc != PKV_OK || p.direct || share) return rc;
   } else if (D == 128) {
     rc = N == 16 ? launch_split<128, 16>(p, mk, mv, s, dev) : launch_split<128, 64>(p, mk, mv, s, dev);
   } else {
     rc = N == 16 ? launch_split<64, 16>(p, mk, mv, s, dev) : launch_split<64, 64>(p, mk, mv, s, dev);
   }
-  if (rc != PKV_OK) return rc;
+  if (rc != PKV_OK || share) return rc;
 
   pkv::MergeParams m{};
   m.seqlens = seqlens;
@@ -466,6 +484,8 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   m.fin_lse = p.fin_lse;
   m.rows = rows;
   m.skip_single = N == pkv::kRowsPerTile ? 1 : 0;
+  m.n_local = static_cast<int>(S);
+  m.rank_floats = 0;
   return D == 128 ? launch_merge<128>(m, rows, s) : launch_merge<64>(m, rows, s);
 }
 
@@ -594,6 +614,63 @@ int pkv_kv_append_varlen(const void *k_new, const int64_t kn_strides[2], const v
                        block_table, bt_stride, max_blocks_per_seq, seqlens, batch, 0, Hkv, D,
                        block_size, 0, err, static_cast<cudaStream_t>(stream), cu_seqlens_new,
                        total_new);
+}
+
+int pkv_paged_attn_partials(const void *q, const int64_t q_strides[3], const void *k_cache,
+                            const int64_t k_strides[3], const void *v_cache,
+                            const int64_t v_strides[3], int64_t num_blocks,
+                            const int32_t *block_table, int64_t bt_stride, int max_blocks_per_seq,
+                            const int32_t *seqlens, int batch, int seqlen_q, int Hq, int Hkv,
+                            int D, int block_size, float scale, int causal, int split_begin,
+                            int n_splits_local, void *partials, size_t partials_bytes,
+                            int32_t *err, void *stream) {
+  const SplitShare share{split_begin, n_splits_local};
+  return attn_entry(q, q_strides, k_cache, k_strides, v_cache, v_strides, num_blocks, block_table,
+                    bt_stride, max_blocks_per_seq, seqlens,
+                    (split_begin + n_splits_local) * pkv::kSplitTokens, batch, seqlen_q, Hq, Hkv,
+                    D, block_size, scale, causal, nullptr, nullptr, nullptr, partials,
+                    partials_bytes, err, stream, nullptr, nullptr, &share);
+}
+
+size_t pkv_partials_size(int batch, int seqlen_q, int Hq, int D, int n_splits_local) {
+  if (batch <= 0 || seqlen_q <= 0 || Hq <= 0 || D <= 0 || n_splits_local <= 0) return 0;
+  return ws_bytes(batch, seqlen_q, Hq, D, n_splits_local * pkv::kSplitTokens);
+}
+
+int pkv_merge_partials(const void *partials, int world, int n_splits_local, size_t rank_bytes,
+                       const int32_t *seqlens, int batch, int seqlen_q, int Hq, int D, int causal,
+                       void *out, const int64_t out_strides[3], float *lse, void *stream) {
+  if (!partials || !seqlens || !out || !lse || !out_strides) return PKV_ERR_ARG;
+  if (world <= 0 || n_splits_local <= 0 || batch <= 0 || seqlen_q <= 0 || Hq <= 0 ||
+      (D != 64 && D != 128))
+    return PKV_ERR_ARG;
+  if (out_strides[0] <= 0 || out_strides[1] <= 0 || out_strides[2] <= 0) return PKV_ERR_ARG;
+  const int64_t rows = static_cast<int64_t>(batch) * seqlen_q * Hq;
+  if (rows > INT32_MAX) return PKV_ERR_ARG;
+  const size_t acc_bytes = ws_acc_bytes(rows, n_splits_local, D);
+  if (rank_bytes < acc_bytes + static_cast<size_t>(rows) * n_splits_local * 2 * sizeof(float) ||
+      rank_bytes % 16 != 0 || !aligned16(partials))
+    return PKV_ERR_WORKSPACE;
+  pkv::MergeParams m{};
+  m.seqlens = seqlens;
+  m.seqlen_q = seqlen_q;
+  m.Hq = Hq;
+  m.n_splits = world * n_splits_local;
+  m.causal = causal ? 1 : 0;
+  m.ws_acc = static_cast<const float *>(partials);
+  m.ws_ml = reinterpret_cast<const float *>(static_cast<const uint8_t *>(partials) + acc_bytes);
+  m.out = static_cast<__nv_bfloat16 *>(out);
+  m.o_sb = out_strides[0];
+  m.o_ss = out_strides[1];
+  m.o_sh = out_strides[2];
+  m.lse = lse;
+  m.batch = batch;
+  m.rows = rows;
+  m.skip_single = 0;
+  m.n_local = n_splits_local;
+  m.rank_floats = static_cast<int64_t>(rank_bytes / sizeof(float));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch_merge<128>(m, rows, s) : launch_merge<64>(m, rows, s);
 }
 
 size_t pkv_workspace_size(int batch, int seqlen_q, int Hq, int D, int max_seqlen_k) {

@@ -3,7 +3,13 @@
 The decode path partitions into independent (sequence, KV head, split) units,
 so ranks shard sequences and need no collective on the data path; the only
 collectives are the timing barrier and the max-over-ranks reduction of the
-timed region.  Everything here also runs on the `gloo` backend on CPU.
+timed region.  Context parallelism over one long context has one exchange
+step: each rank computes the partials of its contiguous share of the 4096-token
+splits, the partial buffers are all-gathered, and every rank runs the same
+ascending-split merge (RL-Kernel PR #284 "feat(attention): add CP backward
+drift validation", Changes: CP world size, KV chunk size, fixed
+global_block_index merge order).  Everything here also runs on the `gloo`
+backend on CPU.
 """
 from __future__ import annotations
 
@@ -49,3 +55,47 @@ def max_over_ranks(value: float, device=None) -> float:
 def weak_scaling_rate(units_per_rank: float, world: int, steps: int, max_ms: float) -> float:
     """Whole-job throughput: the units all ranks processed / the slowest rank's time."""
     return units_per_rank * world * steps / (max_ms / 1e3)
+
+
+SPLIT_TOKENS = 4096
+
+
+def cp_split_share(max_seqlen_k: int, rank: int, world: int) -> Tuple[int, int]:
+    """(split_begin, n_splits_local) of this rank: the S = ceil(max_seqlen_k /
+    4096) splits cut into `world` contiguous blocks of n_local = ceil(S / world)
+    splits (the last blocks may run past S; their extra splits see no key)."""
+    S = max(1, -(-int(max_seqlen_k) // SPLIT_TOKENS))
+    n_local = -(-S // world)
+    return rank * n_local, n_local
+
+
+def cp_exchange(partials: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gather every rank's partial buffer (equal sizes) side by side, rank
+    0's first: the layout pkv_merge_partials reads."""
+    world = dist.get_world_size(group)
+    if world == 1:
+        return partials
+    flat = partials.reshape(-1)
+    if dist.get_backend(group) == "nccl":
+        out = torch.empty(world * flat.numel(), dtype=flat.dtype, device=flat.device)
+        dist.all_gather_into_tensor(out, flat, group=group)
+        return out
+    parts = [torch.empty_like(flat) for _ in range(world)]
+    dist.all_gather(parts, flat, group=group)
+    return torch.cat(parts)
+
+
+def cp_attention(q, k_cache, v_cache, block_table, seqlens, max_seqlen_k, *, scale=None,
+                 causal=False, group=None):
+    """Context-parallel attention on this rank: partials of its split share,
+    the exchange, and the merge.  Every rank returns the same (out, lse), bitwise
+    those of one paged_decode_attn call over the whole context.  This rank's
+    cache and block table need only hold the tokens of its splits."""
+    from . import binding
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    begin, n_local = cp_split_share(max_seqlen_k, rank, world)
+    part = binding.paged_attn_partials(q, k_cache, v_cache, block_table, seqlens, begin, n_local,
+                                       scale=scale, causal=causal)
+    gathered = cp_exchange(part, group)
+    return binding.merge_partials(gathered, world, n_local, seqlens, tuple(q.shape),
+                                  causal=causal)

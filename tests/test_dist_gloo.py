@@ -56,3 +56,83 @@ def test_shard_sizes_and_rate():
             assert [x for p in parts for x in p] == list(range(n))
     assert pdist.weak_scaling_rate(100.0, 4, 10, 1000.0) == 4000.0
     assert pdist.max_over_ranks(3.5) == 3.5                          # no process group
+
+
+def _cp_worker(rank, world, port, q):
+    """One CP rank on CPU: fp64 partials of its split share (the oracle's), the
+    gloo exchange of the packed buffers, then the ascending fold over all
+    global splits from the gathered blocks."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import math
+    import torch
+    import torch.distributed as dist
+    import oracle
+    from paged_kv_decode_31_b200 import inputs as I
+    pdist.init("gloo", timeout_s=60)
+    split = 64   # small splits so a short context spans several
+    di = I.p2_case(2, 3, 300, 4, 2, 64, 16, causal=True, seed=31, seqlens=[300, 141])
+    S = -(-300 // split)
+    n_local = -(-S // world)
+    begin = rank * n_local
+    m, l, acc = oracle.split_partials(di.q, di.cache.k, di.cache.v, di.block_table, di.seqlens,
+                                      di.scale, True, begin, n_local, split_tokens=split)
+    block = torch.cat([acc.reshape(-1), m.reshape(-1), l.reshape(-1)])
+    gathered = pdist.cp_exchange(block, None).reshape(world, -1)
+    B, sq, Hq, D = di.q.shape
+    na = B * sq * Hq * n_local * D
+    nm = B * sq * Hq * n_local
+    out = torch.zeros(B, sq, Hq, D, dtype=torch.float64)
+    lse = torch.zeros(B, Hq, sq, dtype=torch.float64)
+    for b in range(B):
+        for i in range(sq):
+            for h in range(Hq):
+                M, Lsum, A = -math.inf, 0.0, torch.zeros(D, dtype=torch.float64)
+                for s in range(world * n_local):          # ascending global split
+                    r, ls = divmod(s, n_local)
+                    blk = gathered[r]
+                    idx = ((b * sq + i) * Hq + h) * n_local + ls
+                    ms, lsv = float(blk[na + idx]), float(blk[na + nm + idx])
+                    if ms == -math.inf:
+                        continue
+                    a_s = blk[idx * D:(idx + 1) * D]
+                    Mn = max(M, ms)
+                    ca, cs = math.exp(M - Mn) if M > -math.inf else 0.0, math.exp(ms - Mn)
+                    Lsum = Lsum * ca + lsv * cs
+                    A = A * ca + a_s * cs
+                    M = Mn
+                out[b, i, h] = A / Lsum if Lsum > 0 else 0.0
+                lse[b, h, i] = M + math.log(Lsum) if Lsum > 0 else -math.inf
+    ro, rl = oracle.paged_attn(di.q, di.cache.k, di.cache.v, di.block_table, di.seqlens,
+                               di.scale, True)
+    ok_out = float((out - ro).abs().max())
+    fin = torch.isfinite(rl)
+    ok_lse = float((lse[fin] - rl[fin]).abs().max())
+    same_empty = bool(torch.equal(torch.isneginf(lse), torch.isneginf(rl)))
+    shares = (begin, n_local)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, ok_out, ok_lse, same_empty, shares))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_context_parallel_exchange_and_ascending_merge_with_gloo(world):
+    """The split shares cover every split once, in rank order; the exchanged
+    blocks land side by side; folding them in ascending global split order
+    reproduces the whole-context attention (fp64, CPU)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    S = -(-300 // 64)
+    n_local = -(-S // world)
+    for rank, d_out, d_lse, same_empty, shares in res:
+        assert shares == (rank * n_local, n_local)
+        assert d_out < 1e-12 and d_lse < 1e-12 and same_empty
+    assert pdist.cp_split_share(20000, 2, 3) == (4, 2)
