@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--context", type=int, default=131072,
                     help="tokens per sequence (a smaller workload for profiling captures)")
     ap.add_argument("--batch", type=int, default=4)
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the prefill backward and print its result object")
     ap.add_argument("--varlen-only", action="store_true",
                     help="time only the packed mixed-batch call and print its result object")
     ap.add_argument("--prefill-only", action="store_true",
@@ -302,6 +304,54 @@ def varlen_secondary(dev, reps: int = 10):
             "tflops": round(flops / (ms / 1e3) / 1e12, 2), "algorithmic_flops": flops}
 
 
+def backward_secondary(dev, reps: int = 5):
+    """Deterministic backward of the full causal prefill of the parity
+    workload (batch 8 x 2048 tokens, Hq 16 / Hkv 4, D 128, block_size 16):
+    one forward for out / lse, then paged_prefill_attn_bwd timed alone.
+    Algorithmic flops: 10 * D per (query row, visible key) -- the five
+    products S, dP, dV, dK, dQ; the kernels' recompute of S and dP for dQ is
+    not counted."""
+    import paged_kv_decode_31_b200 as pkv
+    from paged_kv_decode_31_b200 import inputs as I
+    cache, table, q_all, k_all, v_all = I.config_parity_cache(device=dev)
+    B, Hq, D, T = 8, 16, 128, 2048
+    seq = torch.full((B,), T, dtype=torch.int32, device=dev)
+    pkv.kv_append(k_all[:, :T], v_all[:, :T], cache.k, cache.v, table, seq - T)
+    q = q_all[:, :T].contiguous()
+    out, lse = pkv.paged_prefill_attn(q, cache.k, cache.v, table, seq, max_seqlen_k=T,
+                                      causal=True)
+    gen = torch.Generator(device=dev).manual_seed(77)
+    dout = torch.randn(B, T, Hq, D, generator=gen, device=dev).to(torch.bfloat16)
+    dq = torch.empty_like(q)
+    dk = torch.zeros(tuple(cache.k.shape), dtype=torch.bfloat16, device=dev)
+    dv = torch.zeros(tuple(cache.v.shape), dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def bwd():
+        pkv.paged_prefill_attn_bwd(q, cache.k, cache.v, table, seq, out, lse, dout,
+                                   max_seqlen_k=T, causal=True, dq=dq, dk_cache=dk, dv_cache=dv,
+                                   err=err)
+
+    for _ in range(2):
+        bwd()
+    torch.cuda.synchronize()
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        bwd()
+    b_.record()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"backward set device error bits {int(err.item())}")
+    ms = a.elapsed_time(b_) / reps
+    pairs = sum(p + 1 for p in range(T))
+    flops = 10.0 * D * pairs * B * Hq
+    return {"workload": "deterministic backward of causal prefill, batch 8 x 2048 tokens, "
+                        "Hq 16, Hkv 4, D 128, block_size 16 (dq and the cache gradients)",
+            "ms_per_call": round(ms, 4), "tflops": round(flops / (ms / 1e3) / 1e12, 2),
+            "algorithmic_flops": flops}
+
+
 def run_ours(args):
     import torch.distributed as dist
     import paged_kv_decode_31_b200 as pkv
@@ -465,6 +515,9 @@ def run_ours(args):
         vl["hbm_frac"] = round(vl["kv_gbs"] / peak, 4)
         vl["frac_of_tensor_peak"] = round(vl["tflops"] / bf16_peak, 4)
         result["varlen"] = vl
+        bw = backward_secondary(dev)
+        bw["frac_of_tensor_peak"] = round(bw["tflops"] / bf16_peak, 4)
+        result["backward"] = bw
     if not args.no_cpu_baseline and world == 1:
         result["cpu_baseline"] = cpu_baseline(di)
     print(json.dumps(result), flush=True)
@@ -522,6 +575,10 @@ def run_reference(args):
 
 def main():
     args = parse_args()
+    if args.backward_only:
+        torch.cuda.set_device(0)
+        print(json.dumps(backward_secondary(torch.device("cuda", 0), reps=max(args.steps, 1))))
+        return
     if args.varlen_only:
         torch.cuda.set_device(0)
         print(json.dumps(varlen_secondary(torch.device("cuda", 0), reps=max(args.steps, 1))))

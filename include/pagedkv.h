@@ -314,6 +314,49 @@ int pkv_merge_partials(const void *partials, int world, int n_splits_local, size
                        int causal, void *out, const int64_t out_strides[3], float *lse,
                        void *stream);
 
+/*
+ * pkv_paged_prefill_attn_bwd: deterministic backward of causal / chunked
+ * prefill (or any seqlen_q) over the paged cache -- the training-side
+ * backward over the same forward graph (RL-Kernel PR #284 "feat(attention):
+ * add CP backward drift validation", Changes: backward reference, dq / dk /
+ * dv, fixed order, fp32 accumulation; decode backward stays unsupported
+ * there, and this call is the prefill form).  Inputs as pkv_paged_prefill_attn
+ * plus the forward's out / lse and dout ([batch, seqlen_q, Hq, D] bf16,
+ * strides dout_strides).  Outputs:
+ *   dq        [batch, seqlen_q, Hq, D] bf16 (strides dq_strides)
+ *   dk_cache / dv_cache  gradient buffers laid out like the caches (views
+ *             [num_blocks, block_size, Hkv, D], strides dk/dv_strides): the
+ *             row of every position < seqlens[b] of every sequence is
+ *             written (a context position with no query row that sees it
+ *             gets zeros); other rows are left untouched.
+ * Every sum (over query rows for dk / dv, over keys for dq) runs in one
+ * fixed ascending order on fp32 accumulators, P and dS enter the tensor
+ * cores as bf16: the result is bitwise reproducible and independent of the
+ * rest of the batch.  Two sequences must not share a cache block.
+ *   workspace >= pkv_bwd_workspace_size(batch, seqlen_q, Hq) bytes.
+ * Errors and device error bits as pkv_paged_prefill_attn (strides of dq,
+ * dout, dk_cache, dv_cache: multiples of 8 elements, bases 16-byte aligned).
+ */
+int pkv_paged_prefill_attn_bwd(const void *q, const int64_t q_strides[3],
+                               const void *k_cache, const int64_t k_strides[3],
+                               const void *v_cache, const int64_t v_strides[3],
+                               int64_t num_blocks,
+                               const int32_t *block_table, int64_t bt_stride,
+                               int max_blocks_per_seq,
+                               const int32_t *seqlens, int max_seqlen_k,
+                               int batch, int seqlen_q, int Hq, int Hkv, int D, int block_size,
+                               float scale, int causal,
+                               const void *out, const int64_t out_strides[3], const float *lse,
+                               const void *dout, const int64_t dout_strides[3],
+                               void *dq, const int64_t dq_strides[3],
+                               void *dk_cache, const int64_t dk_strides[3],
+                               void *dv_cache, const int64_t dv_strides[3],
+                               void *workspace, size_t workspace_bytes,
+                               int32_t *err, void *stream);
+
+/* Workspace bytes pkv_paged_prefill_attn_bwd needs (0 on invalid arguments). */
+size_t pkv_bwd_workspace_size(int batch, int seqlen_q, int Hq);
+
 /* Workspace bytes the attention calls need: fp32 split partials
  * (m, l, acc[D]) for every (batch, query row, query head, split). */
 size_t pkv_workspace_size(int batch, int seqlen_q, int Hq, int D, int max_seqlen_k);

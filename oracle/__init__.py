@@ -219,3 +219,59 @@ def split_partials(q, k_cache, v_cache, block_table, seqlens, scale, causal, spl
                     l[b, i, h, ls] = w.sum()
                     acc[b, i, h, ls] = w @ V[a:e, h // G]
     return m, l, acc
+
+
+def paged_attn_bwd(q, k_cache, v_cache, block_table, seqlens, scale, causal, dout):
+    """fp64 gradients of paged softmax attention (the backward of paged_attn's
+    forward, same masks and bottom-right causal alignment), for the
+    deterministic prefill backward over the same forward graph (RL-Kernel PR
+    #284 "feat(attention): add CP backward drift validation", Changes:
+    backward_reference over the same forward, dq / dk / dv).  With
+    p_ij = exp(s_ij - lse_i), s_ij = scale * q_i.k_j over the visible keys:
+        D_i  = sum_j p_ij (dout_i . v_j)      (= dout_i . out_i)
+        ds_ij = p_ij (dout_i . v_j - D_i)
+        dq_i = scale * sum_j ds_ij k_j
+        dk_j = scale * sum_i ds_ij q_i,   dv_j = sum_i p_ij dout_i
+    summed over every query row (token and query head of the KV head's group)
+    that sees key j.  Plain torch fp64 on the CPU.
+
+    Returns (dq [B, sq, Hq, D], dk [B, Lmax, Hkv, D], dv [B, Lmax, Hkv, D])
+    with dk / dv indexed by token position (zeros past seqlens[b])."""
+    B, sq, Hq, D = q.shape
+    nb, bs, Hkv, _ = k_cache.shape
+    G = Hq // Hkv
+    Lmax = max(int(x) for x in seqlens) if len(seqlens) else 0
+    dq = torch.zeros(B, sq, Hq, D, dtype=torch.float64)
+    dk = torch.zeros(B, max(Lmax, 1), Hkv, D, dtype=torch.float64)
+    dv = torch.zeros(B, max(Lmax, 1), Hkv, D, dtype=torch.float64)
+    for b in range(B):
+        n = max(int(seqlens[b]), 0)
+        if n == 0:
+            continue
+        j = torch.arange(n)
+        blk = block_table[b, j // bs].long()
+        K = k_cache[blk, j % bs].double()    # [n, Hkv, D]
+        V = v_cache[blk, j % bs].double()
+        for h in range(Hq):
+            g = h // G
+            Q = q[b, :, h].double()          # [sq, D]
+            dO = dout[b, :, h].double()
+            S = scale * (Q @ K[:, g].T)      # [sq, n]
+            pos = n - sq + torch.arange(sq)
+            vis = torch.arange(n)[None, :] < n
+            if causal:
+                vis = vis & (torch.arange(n)[None, :] <= pos[:, None])
+            S = S.masked_fill(~vis, float("-inf"))
+            m = S.max(dim=1, keepdim=True).values
+            has = torch.isfinite(m)
+            m = torch.where(has, m, torch.zeros_like(m))
+            E = torch.exp(S - m) * vis
+            P = E / E.sum(dim=1, keepdim=True).clamp_min(1e-300)
+            P = P * has
+            dP = dO @ V[:, g].T              # [sq, n]
+            Dv = (P * dP).sum(dim=1, keepdim=True)
+            dS = P * (dP - Dv)
+            dq[b, :, h] = scale * (dS @ K[:, g])
+            dk[b, :n, g] += scale * (dS.T @ Q)
+            dv[b, :n, g] += P.T @ dO
+    return dq, dk, dv

@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     paged_decode_attn,
     paged_decode_attn_append,
     paged_prefill_attn,
+    paged_prefill_attn_bwd,
     paged_varlen_attn,
     strerror,
     varlen_workspace_size,

@@ -408,6 +408,54 @@ def merge_partials(gathered, world, n_splits_local, seqlens, q_shape, *, causal=
     return out, lse
 
 
+def paged_prefill_attn_bwd(q, k_cache, v_cache, block_table, seqlens, out, lse, dout, *,
+                           max_seqlen_k=None, scale=None, causal=True, dq=None, dk_cache=None,
+                           dv_cache=None, workspace=None, err=None, stream=None):
+    """Deterministic backward of paged attention: returns (dq [B, sq, Hq, D],
+    dk_cache, dv_cache) with the gradients of the cache rows laid out like
+    k_cache / v_cache (new zero-filled buffers unless given)."""
+    L = lib()
+    fn = L.pkv_paged_prefill_attn_bwd
+    if not fn.argtypes:
+        fn.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _P, _I64, _I, _P, _I, _I, _I, _I, _I, _I,
+                       _I, ctypes.c_float, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                       ctypes.c_size_t, _P, _P]
+        fn.restype = _I
+        L.pkv_bwd_workspace_size.argtypes = [_I, _I, _I]
+        L.pkv_bwd_workspace_size.restype = ctypes.c_size_t
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("out", out),
+                    ("dout", dout)):
+        _need_cuda_bf16(name, t)
+    _need_cuda_i32("block_table", block_table)
+    _need_cuda_i32("seqlens", seqlens)
+    B, sq, Hq, D = q.shape
+    num_blocks, bs, Hkv, _ = k_cache.shape
+    if max_seqlen_k is None:
+        max_seqlen_k = int(seqlens.max().item()) if seqlens.numel() else 0
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if dq is None:
+        dq = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if dk_cache is None:
+        dk_cache = torch.zeros(k_cache.shape, dtype=torch.bfloat16, device=q.device)
+    if dv_cache is None:
+        dv_cache = torch.zeros(v_cache.shape, dtype=torch.bfloat16, device=q.device)
+    for name, t in (("dq", dq), ("dk_cache", dk_cache), ("dv_cache", dv_cache)):
+        _need_cuda_bf16(name, t)
+    if workspace is None:
+        workspace = torch.empty(int(L.pkv_bwd_workspace_size(B, sq, Hq)), dtype=torch.uint8,
+                                device=q.device)
+    rc = fn(q.data_ptr(), _st3(q), k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(),
+            _st3(v_cache), num_blocks, block_table.data_ptr(), int(block_table.stride(0)),
+            int(block_table.shape[1]), seqlens.data_ptr(), int(max_seqlen_k), B, sq, Hq, Hkv, D,
+            bs, float(scale), int(bool(causal)), out.data_ptr(), _st3(out), lse.data_ptr(),
+            dout.data_ptr(), _st3(dout), dq.data_ptr(), _st3(dq), dk_cache.data_ptr(),
+            _st3(dk_cache), dv_cache.data_ptr(), _st3(dv_cache), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), _ptr(err), _stream_handle(stream))
+    _check("pkv_paged_prefill_attn_bwd", rc)
+    return dq, dk_cache, dv_cache
+
+
 # Allocation-free decode (see pkv_paged_decode_attn_static_ws in pagedkv.h).
 STATIC_WORKSPACE_BYTES = 8 << 20
 

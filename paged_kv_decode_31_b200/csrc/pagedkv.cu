@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "pagedkv.h"
+#include "attn_bwd.cuh"
 #include "attn_rows.cuh"
 #include "attn_split.cuh"
 #include "kv_append.cuh"
@@ -201,6 +202,29 @@ int launch_rows(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensorM
   }
   const int grid = p.n_units < sm_count(dev) ? p.n_units : sm_count(dev);
   kern<<<grid, pkv::kRowThreads, C::kSmemBytes, s>>>(p, mk, mv, mq);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+// Backward kernels: one CTA per key tile (dK, dV) and per row tile (dQ).
+// Both hold 512 TMEM columns; shared memory is requested at >= 120 KB so that
+// only one CTA of either kernel sits on an SM.
+template <int D>
+int launch_bwd(const pkv::BwdParams &p, int64_t kv_ctas, int64_t q_ctas, cudaStream_t s) {
+  using C = pkv::BwdCfg<D>;
+  constexpr int kSmall = static_cast<int>(sizeof(typename C::Small)) + 1024;
+  constexpr int kKv = 4 * C::kTile + 2 * C::kSq + kSmall;
+  constexpr int kQ0 = 4 * C::kTile + C::kSq + kSmall;
+  constexpr int kQ = kQ0 > 120 * 1024 ? kQ0 : 120 * 1024;
+  constexpr int kKvS = kKv > 120 * 1024 ? kKv : 120 * 1024;
+  static_assert(kKvS <= 232448 && kQ <= 232448, "shared memory budget");
+  if (cudaFuncSetAttribute(pkv::bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kKvS) != cudaSuccess ||
+      cudaFuncSetAttribute(pkv::bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kQ) != cudaSuccess)
+    return PKV_ERR_CUDA;
+  pkv::bwd_kv_kernel<D><<<static_cast<unsigned>(kv_ctas), pkv::kBwdThreads, kKvS, s>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+  pkv::bwd_q_kernel<D><<<static_cast<unsigned>(q_ctas), pkv::kBwdThreads, kQ, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -671,6 +695,129 @@ int pkv_merge_partials(const void *partials, int world, int n_splits_local, size
   m.rank_floats = static_cast<int64_t>(rank_bytes / sizeof(float));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return D == 128 ? launch_merge<128>(m, rows, s) : launch_merge<64>(m, rows, s);
+}
+
+size_t pkv_bwd_workspace_size(int batch, int seqlen_q, int Hq) {
+  if (batch <= 0 || seqlen_q <= 0 || Hq <= 0) return 0;
+  const size_t rows = static_cast<size_t>(batch) * seqlen_q * Hq;
+  return 2 * ((rows * sizeof(float) + 255) & ~static_cast<size_t>(255));
+}
+
+int pkv_paged_prefill_attn_bwd(const void *q, const int64_t q_strides[3], const void *k_cache,
+                               const int64_t k_strides[3], const void *v_cache,
+                               const int64_t v_strides[3], int64_t num_blocks,
+                               const int32_t *block_table, int64_t bt_stride,
+                               int max_blocks_per_seq, const int32_t *seqlens, int max_seqlen_k,
+                               int batch, int seqlen_q, int Hq, int Hkv, int D, int block_size,
+                               float scale, int causal, const void *out,
+                               const int64_t out_strides[3], const float *lse, const void *dout,
+                               const int64_t dout_strides[3], void *dq,
+                               const int64_t dq_strides[3], void *dk_cache,
+                               const int64_t dk_strides[3], void *dv_cache,
+                               const int64_t dv_strides[3], void *workspace,
+                               size_t workspace_bytes, int32_t *err, void *stream) {
+  if (!q || !k_cache || !v_cache || !block_table || !seqlens || !out || !lse || !dout || !dq ||
+      !dk_cache || !dv_cache)
+    return PKV_ERR_ARG;
+  if (batch <= 0 || seqlen_q <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return PKV_ERR_ARG;
+  if (D != 64 && D != 128) return PKV_ERR_ARG;
+  if (!pow2_in(block_size, 16, 256)) return PKV_ERR_ARG;
+  if (num_blocks <= 0 || num_blocks > INT32_MAX || max_blocks_per_seq <= 0 ||
+      bt_stride < max_blocks_per_seq || max_seqlen_k < 0)
+    return PKV_ERR_ARG;
+  if (!strides_ok(q_strides) || !strides_ok(k_strides) || !strides_ok(v_strides) ||
+      !strides_ok(dout_strides) || !strides_ok(dq_strides) || !strides_ok(dk_strides) ||
+      !strides_ok(dv_strides))
+    return PKV_ERR_ARG;
+  if (!out_strides || out_strides[0] <= 0 || out_strides[1] <= 0 || out_strides[2] <= 0)
+    return PKV_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk_cache) || !aligned16(dv_cache))
+    return PKV_ERR_ARG;
+  if (!(scale > 0.f) || !(scale < 3.0e38f)) return PKV_ERR_ARG;
+  const int G = Hq / Hkv;
+  const int64_t rows = static_cast<int64_t>(batch) * seqlen_q * Hq;
+  const int64_t R = static_cast<int64_t>(G) * seqlen_q;
+  if (rows > INT32_MAX || R > INT32_MAX / 2) return PKV_ERR_ARG;
+  const size_t need = pkv_bwd_workspace_size(batch, seqlen_q, Hq);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float *row_d = static_cast<float *>(workspace);
+  float *row_lse2 = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + need / 2);
+
+  pkv::BwdPrepParams pp{};
+  pp.dout = static_cast<const __nv_bfloat16 *>(dout);
+  pp.out = static_cast<const __nv_bfloat16 *>(out);
+  pp.g_sb = dout_strides[0];
+  pp.g_ss = dout_strides[1];
+  pp.g_sh = dout_strides[2];
+  pp.o_sb = out_strides[0];
+  pp.o_ss = out_strides[1];
+  pp.o_sh = out_strides[2];
+  pp.lse = lse;
+  pp.batch = batch;
+  pp.seqlen_q = seqlen_q;
+  pp.Hq = Hq;
+  pp.D = D;
+  pp.row_d = row_d;
+  pp.row_lse2 = row_lse2;
+  pkv::bwd_prep_kernel<<<static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, s>>>(pp);
+  if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+
+  pkv::BwdParams p{};
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.dout = static_cast<const __nv_bfloat16 *>(dout);
+  p.q_sb = q_strides[0];
+  p.q_ss = q_strides[1];
+  p.q_sh = q_strides[2];
+  p.g_sb = dout_strides[0];
+  p.g_ss = dout_strides[1];
+  p.g_sh = dout_strides[2];
+  p.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
+  p.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
+  p.k_sb = k_strides[0];
+  p.k_ss = k_strides[1];
+  p.k_sh = k_strides[2];
+  p.v_sb = v_strides[0];
+  p.v_ss = v_strides[1];
+  p.v_sh = v_strides[2];
+  p.dk_cache = static_cast<__nv_bfloat16 *>(dk_cache);
+  p.dv_cache = static_cast<__nv_bfloat16 *>(dv_cache);
+  p.dk_sb = dk_strides[0];
+  p.dk_ss = dk_strides[1];
+  p.dk_sh = dk_strides[2];
+  p.dv_sb = dv_strides[0];
+  p.dv_ss = dv_strides[1];
+  p.dv_sh = dv_strides[2];
+  p.dq = static_cast<__nv_bfloat16 *>(dq);
+  p.dq_sb = dq_strides[0];
+  p.dq_ss = dq_strides[1];
+  p.dq_sh = dq_strides[2];
+  p.block_table = block_table;
+  p.bt_stride = bt_stride;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
+  p.seqlens = seqlens;
+  p.batch = batch;
+  p.seqlen_q = seqlen_q;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.block_shift = log2i(block_size);
+  p.causal = causal ? 1 : 0;
+  p.n_key_tiles = static_cast<int>(ceil_div(max_seqlen_k > 0 ? max_seqlen_k : 1, pkv::kBwdTile));
+  p.n_row_tiles = static_cast<int>(ceil_div(R, pkv::kBwdTile));
+  p.cscale = scale * 1.4426950408889634f;
+  p.scale = scale;
+  p.row_d = row_d;
+  p.row_lse2 = row_lse2;
+  p.err = err;
+  const int64_t kv_ctas = static_cast<int64_t>(batch) * Hkv * p.n_key_tiles;
+  const int64_t q_ctas = static_cast<int64_t>(batch) * Hkv * p.n_row_tiles;
+  if (kv_ctas > INT32_MAX || q_ctas > INT32_MAX) return PKV_ERR_ARG;
+  return D == 128 ? launch_bwd<128>(p, kv_ctas, q_ctas, s) : launch_bwd<64>(p, kv_ctas, q_ctas, s);
 }
 
 size_t pkv_workspace_size(int batch, int seqlen_q, int Hq, int D, int max_seqlen_k) {

@@ -1,0 +1,116 @@
+"""Deterministic prefill backward (pkv_paged_prefill_attn_bwd) on the GPU:
+dq / dk / dv against the fp64 oracle's gradients, run-to-run and
+batch-composition bit equality, and the cache rows it must leave alone.
+
+Tolerance, derived from the arithmetic: P and dS enter the tensor cores as
+bf16 and the gradients are written as bf16; a CPU simulation of exactly that
+on N(0,1) data puts the max-abs error at 2.5e-3 to 4.3e-3 of max|gradient|.
+The bound here is 1e-2 of max|gradient| per tensor."""
+import pytest
+import torch
+
+import oracle
+import paged_kv_decode_31_b200 as pkv
+from paged_kv_decode_31_b200 import inputs as I
+
+from gpu_helpers import bits_equal
+
+pytestmark = pytest.mark.gpu
+
+REL = 1e-2
+
+
+def _gather(cache_view, table, seqlens, bs):
+    """[B, Lmax, Hkv, D] by token position from a cache-shaped tensor."""
+    B = table.shape[0]
+    Lmax = int(seqlens.max())
+    out = torch.zeros(B, Lmax, cache_view.shape[2], cache_view.shape[3], dtype=torch.float64)
+    for b in range(B):
+        n = int(seqlens[b])
+        j = torch.arange(n)
+        out[b, :n] = cache_view[table[b, j // bs].long(), j % bs].double()
+    return out
+
+
+def _run(di, dout, causal):
+    d = di.to("cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = pkv.paged_prefill_attn(d.q, d.cache.k, d.cache.v, d.block_table, d.seqlens,
+                                      scale=di.scale, causal=causal, err=err)
+    dq, dk, dv = pkv.paged_prefill_attn_bwd(d.q, d.cache.k, d.cache.v, d.block_table, d.seqlens,
+                                            out, lse, dout.cuda(), scale=di.scale, causal=causal,
+                                            err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    return dq.cpu(), dk.cpu(), dv.cpu()
+
+
+def _check(got, ref, name):
+    scale = float(ref.abs().max())
+    e = float((got.double() - ref).abs().max())
+    assert e <= REL * max(scale, 1e-3), f"{name}: max-abs {e:.3e} vs bound {REL * scale:.3e}"
+
+
+CASES = [
+    # (batch, seqlen_q, contexts, Hq, Hkv, D, bs, causal, layout)
+    (2, 40, [300, 160], 16, 4, 128, 16, True, "interleaved"),
+    (2, 130, [700, 130], 8, 2, 64, 32, True, "contiguous"),
+    (1, 64, [5000], 8, 8, 128, 64, False, "contiguous"),      # G = 1, several key tiles
+    (3, 17, [33, 17, 900], 32, 8, 128, 16, True, "interleaved"),
+]
+
+
+@pytest.mark.parametrize("B,sq,ctx,Hq,Hkv,D,bs,causal,layout", CASES)
+def test_backward_matches_oracle(B, sq, ctx, Hq, Hkv, D, bs, causal, layout):
+    di = I.p2_case(B, sq, max(ctx), Hq, Hkv, D, bs, causal=causal, layout=layout,
+                   seed=sum(ctx) + sq, seqlens=ctx)
+    gen = torch.Generator().manual_seed(sq + D)
+    dout = I.randn_bf16((B, sq, Hq, D), gen)
+    dq, dk, dv = _run(di, dout, causal)
+    rq, rk, rv = oracle.paged_attn_bwd(di.q, di.cache.k, di.cache.v, di.block_table, di.seqlens,
+                                       di.scale, causal, dout)
+    _check(dq, rq, "dq")
+    _check(_gather(dk, di.block_table, di.seqlens, bs), rk[:, :max(ctx)], "dk")
+    _check(_gather(dv, di.block_table, di.seqlens, bs), rv[:, :max(ctx)], "dv")
+
+
+def test_backward_is_deterministic_and_batch_invariant():
+    di = I.p2_case(3, 48, 2000, 16, 4, 128, 16, causal=True, layout="contiguous", seed=12,
+                   seqlens=[2000, 900, 1500])
+    gen = torch.Generator().manual_seed(13)
+    dout = I.randn_bf16((3, 48, 16, 128), gen)
+    a = _run(di, dout, True)
+    b = _run(di, dout, True)
+    for x, y in zip(a, b):
+        assert bits_equal(x, y)
+    # sequence 1 alone
+    one = I.DecodeInputs(di.q[1:2].contiguous(), di.cache, di.block_table[1:2].contiguous(),
+                         di.seqlens[1:2].contiguous(), di.Hq, di.Hkv, di.D, di.scale, True)
+    dq1, dk1, dv1 = _run(one, dout[1:2].contiguous(), True)
+    assert bits_equal(dq1[0], a[0][1])
+    n = 900
+    rows = di.block_table[1, :(n + 15) // 16].long()
+    assert bits_equal(dk1[rows], a[1][rows]) and bits_equal(dv1[rows], a[2][rows])
+
+
+def test_backward_leaves_unreferenced_cache_rows_alone():
+    di = I.p2_case(2, 20, 400, 8, 2, 128, 16, causal=True, layout="contiguous", seed=21,
+                   seqlens=[400, 37])
+    d = di.to("cuda")
+    gen = torch.Generator().manual_seed(22)
+    dout = I.randn_bf16((2, 20, 8, 128), gen).cuda()
+    out, lse = pkv.paged_prefill_attn(d.q, d.cache.k, d.cache.v, d.block_table, d.seqlens,
+                                      scale=di.scale, causal=True)
+    sentinel = torch.full(tuple(d.cache.k.shape), 3.0, dtype=torch.bfloat16, device="cuda")
+    dk = sentinel.clone()
+    dv = sentinel.clone()
+    pkv.paged_prefill_attn_bwd(d.q, d.cache.k, d.cache.v, d.block_table, d.seqlens, out, lse,
+                               dout, scale=di.scale, causal=True, dk_cache=dk, dv_cache=dv)
+    torch.cuda.synchronize()
+    used = torch.zeros(d.cache.k.shape[0], d.cache.k.shape[1], dtype=torch.bool)
+    for b, n in enumerate([400, 37]):
+        for j in range(n):
+            used[int(di.block_table[b, j // 16]), j % 16] = True
+    dk, dv = dk.cpu(), dv.cpu()
+    assert torch.all(dk[~used] == 3.0) and torch.all(dv[~used] == 3.0)
+    assert not torch.any(dk[used] == 3.0)
