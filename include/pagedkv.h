@@ -334,8 +334,9 @@ int pkv_merge_partials(const void *partials, int world, int n_splits_local, size
  * cores as bf16: the result is bitwise reproducible and independent of the
  * rest of the batch.  Two sequences must not share a cache block.
  *   workspace >= pkv_bwd_workspace_size(batch, seqlen_q, Hq) bytes.
- * Errors and device error bits as pkv_paged_prefill_attn (strides of dq,
- * dout, dk_cache, dv_cache: multiples of 8 elements, bases 16-byte aligned).
+ * Errors and device error bits as pkv_paged_prefill_attn (strides of out,
+ * dq, dout, dk_cache, dv_cache: multiples of 8 elements, bases 16-byte
+ * aligned).
  */
 int pkv_paged_prefill_attn_bwd(const void *q, const int64_t q_strides[3],
                                const void *k_cache, const int64_t k_strides[3],

@@ -78,9 +78,25 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ B
   const int b = static_cast<int>(bi / p.seqlen_q);
   const __nv_bfloat16 *g = p.dout + b * p.g_sb + i * p.g_ss + h * p.g_sh;
   const __nv_bfloat16 *o = p.out + b * p.o_sb + i * p.o_ss + h * p.o_sh;
+  // lane l: elements [l V, l V + V), V = D / 32, summed in order, then a
+  // fixed xor tree over the lanes
   float acc = 0.f;
-  for (int d = lane; d < p.D; d += 32)
-    acc = __fmaf_rn(__bfloat162float(g[d]), __bfloat162float(o[d]), acc);
+  if (p.D == 128) {  // 8-byte loads: 4 elements per lane
+    const uint2 gv = *reinterpret_cast<const uint2 *>(g + lane * 4);
+    const uint2 ov = *reinterpret_cast<const uint2 *>(o + lane * 4);
+    const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&gv);
+    const __nv_bfloat162 *o2 = reinterpret_cast<const __nv_bfloat162 *>(&ov);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      acc = __fmaf_rn(__low2float(g2[e]), __low2float(o2[e]), acc);
+      acc = __fmaf_rn(__high2float(g2[e]), __high2float(o2[e]), acc);
+    }
+  } else {  // D = 64: 4-byte loads, 2 elements per lane
+    const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162 *>(g + lane * 2);
+    const __nv_bfloat162 o2 = *reinterpret_cast<const __nv_bfloat162 *>(o + lane * 2);
+    acc = __fmaf_rn(__low2float(g2), __low2float(o2), acc);
+    acc = __fmaf_rn(__high2float(g2), __high2float(o2), acc);
+  }
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
   if (lane == 0) {
@@ -105,17 +121,27 @@ struct BwdCfg {
   };
 };
 
-// Stage one [128][D] bf16 tile, rows given by `src_row(c)` (nullptr: zeros),
+// Stage [128][D] bf16 tiles, rows given by `src_row(c)` (nullptr: zeros),
 // 128-byte swizzled K-major (row c at c * 128 bytes of its 64-element half).
+// Every load of a thread is issued before its first store, so the tile costs
+// about one memory round trip.
 template <int D, class F>
 __device__ __forceinline__ void stage_rows(uint8_t *dst, int t, F src_row) {
-  for (int idx = t; idx < kBwdTile * (D / 8); idx += 128) {
+  constexpr int kPer = kBwdTile * (D / 8) / 128;  // 16-byte chunks per thread
+  uint4 v[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = t + k * 128;
     const int c = idx / (D / 8), ch = idx % (D / 8);
     const __nv_bfloat16 *s = src_row(c);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (s) v = __ldg(reinterpret_cast<const uint4 *>(s) + ch);
+    v[k] = s ? __ldg(reinterpret_cast<const uint4 *>(s) + ch) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = t + k * 128;
+    const int c = idx / (D / 8), ch = idx % (D / 8);
     const int h = ch >> 3, cc = ch & 7;
-    *reinterpret_cast<uint4 *>(dst + h * BwdCfg<D>::kHalf + c * 128 + ((cc ^ (c & 7)) << 4)) = v;
+    *reinterpret_cast<uint4 *>(dst + h * BwdCfg<D>::kHalf + c * 128 + ((cc ^ (c & 7)) << 4)) = v[k];
   }
 }
 

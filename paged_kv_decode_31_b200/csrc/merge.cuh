@@ -70,14 +70,20 @@ __device__ __forceinline__ float final_lse(float M, float L) {
                  : __int_as_float(0xff800000);
 }
 
-// One warp per output row; lane l owns head_dim elements [l V, l V + V),
-// V = D / 32.  Every element runs the fold above in ascending split order.
-template <int D>
-__global__ void __launch_bounds__(32 * kMergeRowsPerBlock)
+// Two launch shapes, the same per-element arithmetic (every element runs the
+// fold above in ascending split order):
+//   WIDE = false: one warp per output row, 8 rows per block; lane l owns
+//                 head_dim elements [l V, l V + V), V = D / 32 (many rows);
+//   WIDE = true:  one block of D threads per row, V = 1 (few rows, many
+//                 splits: more SMs share the partial reads).
+template <int D, bool WIDE>
+__global__ void __launch_bounds__(WIDE ? D : 32 * kMergeRowsPerBlock)
     merge_kernel(const __grid_constant__ MergeParams p) {
-  constexpr int V = D / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kMergeRowsPerBlock + warp;
+  constexpr int V = WIDE ? 1 : D / 32;
+  const int warp = WIDE ? 0 : threadIdx.x >> 5;
+  const int lane = WIDE ? threadIdx.x : threadIdx.x & 31;
+  const int64_t row = WIDE ? static_cast<int64_t>(blockIdx.x)
+                           : static_cast<int64_t>(blockIdx.x) * kMergeRowsPerBlock + warp;
   if (row >= p.rows) return;  // row = token * Hq + h; token = b * seqlen_q + i, or packed
   const int h = static_cast<int>(row % p.Hq);
   const int64_t tok = row / p.Hq;
@@ -106,7 +112,7 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerBlock)
   for (int j = 0; j < V; ++j) A[j] = 0.f;
   // Partials are fetched kBatch splits at a time (independent loads in
   // flight together) and folded strictly in ascending split order.
-  constexpr int kBatch = 8;
+  constexpr int kBatch = 16;
   for (int s0 = 0; s0 < n_s; s0 += kBatch) {
     float ms[kBatch], ls[kBatch], as[kBatch][V];
 #pragma unroll
@@ -117,7 +123,7 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerBlock)
 #pragma unroll
       for (int j = 0; j < V; ++j) as[k][j] = 0.f;
       if (s < n_s) {
-        const int r = s / p.n_local;
+        const int r = p.rank_floats == 0 ? 0 : s / p.n_local;  // one block: no division
         const int64_t e = r * p.rank_floats;  // this rank's block, in floats
         const int64_t slot = row * p.n_local + (s - r * p.n_local);
         ms[k] = p.ws_ml[e + slot * 2];
@@ -126,9 +132,11 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerBlock)
         if constexpr (V == 4) {
           const float4 v = *reinterpret_cast<const float4 *>(ap);
           as[k][0] = v.x; as[k][1] = v.y; as[k][2] = v.z; as[k][3] = v.w;
-        } else {
+        } else if constexpr (V == 2) {
           const float2 v = *reinterpret_cast<const float2 *>(ap);
           as[k][0] = v.x; as[k][1] = v.y;
+        } else {
+          as[k][0] = *ap;
         }
       }
     }

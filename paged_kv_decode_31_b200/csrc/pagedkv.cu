@@ -228,10 +228,16 @@ int launch_bwd(const pkv::BwdParams &p, int64_t kv_ctas, int64_t q_ctas, cudaStr
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// Few rows (decode: rows x splits partials spread over one block per row)
+// or many (prefill, packed batches: one warp per row).
 template <int D>
 int launch_merge(const pkv::MergeParams &m, int64_t rows, cudaStream_t s) {
+  if (rows <= 4096) {
+    pkv::merge_kernel<D, true><<<static_cast<unsigned>(rows), D, 0, s>>>(m);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+  }
   const int64_t blocks = ceil_div(rows, pkv::kMergeRowsPerBlock);
-  pkv::merge_kernel<D><<<static_cast<unsigned>(blocks), 32 * pkv::kMergeRowsPerBlock, 0, s>>>(m);
+  pkv::merge_kernel<D, false><<<static_cast<unsigned>(blocks), 32 * pkv::kMergeRowsPerBlock, 0, s>>>(m);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -729,9 +735,9 @@ int pkv_paged_prefill_attn_bwd(const void *q, const int64_t q_strides[3], const 
       !strides_ok(dout_strides) || !strides_ok(dq_strides) || !strides_ok(dk_strides) ||
       !strides_ok(dv_strides))
     return PKV_ERR_ARG;
-  if (!out_strides || out_strides[0] <= 0 || out_strides[1] <= 0 || out_strides[2] <= 0)
-    return PKV_ERR_ARG;
+  if (!strides_ok(out_strides)) return PKV_ERR_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(dout) ||
+      !aligned16(out) ||
       !aligned16(dq) || !aligned16(dk_cache) || !aligned16(dv_cache))
     return PKV_ERR_ARG;
   if (!(scale > 0.f) || !(scale < 3.0e38f)) return PKV_ERR_ARG;
