@@ -20,9 +20,11 @@
 // Every sum therefore has one fixed order and the result is bitwise
 // reproducible and independent of the batch around a sequence.
 //
-// 160 threads: warps 0-3 stage operands and do the elementwise work (thread
-// t = TMEM lane t), warp 4 owns TMEM and lane 0 issues the MMAs.  Phases are
-// separated by __syncthreads and MMA-completion mbarriers (bounded waits).
+// 288 threads: warps 0-7 stage operands and do the elementwise work -- warps
+// w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 (thread t = lane t of the
+// 128) and split the columns in halves -- and warp 8 owns TMEM, its lane 0
+// issuing the MMAs.  Phases are separated by __syncthreads and
+// MMA-completion mbarriers (bounded waits).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -32,7 +34,9 @@
 
 namespace pkv {
 
-constexpr int kBwdThreads = 160;
+constexpr int kBwdThreads = 288;
+constexpr int kBwdCompute = 256;  // staging / elementwise threads
+constexpr int kBwdMmaWarp = 8;
 constexpr int kBwdTile = 128;  // keys per key tile and rows per row tile
 
 struct BwdParams {
@@ -127,18 +131,18 @@ struct BwdCfg {
 // about one memory round trip.
 template <int D, class F>
 __device__ __forceinline__ void stage_rows(uint8_t *dst, int t, F src_row) {
-  constexpr int kPer = kBwdTile * (D / 8) / 128;  // 16-byte chunks per thread
+  constexpr int kPer = kBwdTile * (D / 8) / kBwdCompute;  // 16-byte chunks per thread
   uint4 v[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) {
-    const int idx = t + k * 128;
+    const int idx = t + k * kBwdCompute;
     const int c = idx / (D / 8), ch = idx % (D / 8);
     const __nv_bfloat16 *s = src_row(c);
     v[k] = s ? __ldg(reinterpret_cast<const uint4 *>(s) + ch) : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
   for (int k = 0; k < kPer; ++k) {
-    const int idx = t + k * 128;
+    const int idx = t + k * kBwdCompute;
     const int c = idx / (D / 8), ch = idx % (D / 8);
     const int h = ch >> 3, cc = ch & 7;
     *reinterpret_cast<uint4 *>(dst + h * BwdCfg<D>::kHalf + c * 128 + ((cc ^ (c & 7)) << 4)) = v[k];
@@ -222,7 +226,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
   uint8_t *sK = smem, *sV = sK + C::kTile, *sQ = sV + C::kTile, *sG = sQ + C::kTile;
   uint8_t *sP = sG + C::kTile, *sS = sP + C::kSq;
   auto *sm = reinterpret_cast<typename C::Small *>(sS + C::kSq);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, t = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int t = tid & 127, hf = tid >> 7;  // TMEM lane / token, column half (compute threads)
   volatile int *abort_any = &sm->abort_any;
 
   int u = blockIdx.x;
@@ -234,24 +239,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
   const int tok0 = kt * kBwdTile;
   if (tok0 >= seqlen) return;  // uniform: the whole CTA leaves before any barrier
 
-  if (t == 0) {
+  if (tid == 0) {
     mbar_init(&sm->mma_a, 1);
     mbar_init(&sm->mma_b, 1);
     mbar_init(&sm->drain, 1);
     sm->abort_any = 0;
     fence_barrier_init();
   }
-  if (warp == 4) tmem_alloc(&sm->tmem_base, 512);
+  if (warp == kBwdMmaWarp) tmem_alloc(&sm->tmem_base, 512);
   // K and V of this key tile (tokens past the context are zeros)
-  if (t < 128) {
-    stage_rows<D>(sK, t, [&](int c) -> const __nv_bfloat16 * {
+  if (tid < kBwdCompute) {
+    stage_rows<D>(sK, tid, [&](int c) -> const __nv_bfloat16 * {
       const int tok = tok0 + c;
       if (tok >= seqlen) return nullptr;
       const int64_t blk = bwd_block(p, b, tok);
       if (blk < 0) return nullptr;
       return p.k_cache + blk * p.k_sb + (tok & ((1 << p.block_shift) - 1)) * p.k_ss + kvh * p.k_sh;
     });
-    stage_rows<D>(sV, t, [&](int c) -> const __nv_bfloat16 * {
+    stage_rows<D>(sV, tid, [&](int c) -> const __nv_bfloat16 * {
       const int tok = tok0 + c;
       if (tok >= seqlen) return nullptr;
       const int64_t blk = bwd_block(p, b, tok);
@@ -280,7 +285,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
   int it = 0;
   for (int rt = rt0; rt * kBwdTile < R; ++rt, ++it) {
     const int row0 = rt * kBwdTile;
-    if (t < 128) {
+    if (tid < kBwdCompute) {
       auto rowptr = [&](const __nv_bfloat16 *base, int64_t sb, int64_t ss, int64_t sh, int c)
           -> const __nv_bfloat16 * {
         const int r = row0 + c;
@@ -288,38 +293,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
         const int i = r / p.G, g = r - i * p.G;
         return base + b * sb + static_cast<int64_t>(i) * ss + static_cast<int64_t>(kvh * p.G + g) * sh;
       };
-      stage_rows<D>(sQ, t, [&](int c) { return rowptr(p.q, p.q_sb, p.q_ss, p.q_sh, c); });
-      stage_rows<D>(sG, t, [&](int c) { return rowptr(p.dout, p.g_sb, p.g_ss, p.g_sh, c); });
-      const int r = row0 + t;
-      sm->lim[t] = bwd_row_lim(p, seqlen, r);
-      float l2 = 0.f, ds = 0.f;
-      if (r < R) {
-        const int i = r / p.G, g = r - i * p.G;
-        const int64_t row_id = (static_cast<int64_t>(b) * p.seqlen_q + i) * p.Hq + kvh * p.G + g;
-        l2 = p.row_lse2[row_id];
-        ds = p.row_d[row_id];
+      stage_rows<D>(sQ, tid, [&](int c) { return rowptr(p.q, p.q_sb, p.q_ss, p.q_sh, c); });
+      stage_rows<D>(sG, tid, [&](int c) { return rowptr(p.dout, p.g_sb, p.g_ss, p.g_sh, c); });
+      if (hf == 0) {
+        const int r = row0 + t;
+        sm->lim[t] = bwd_row_lim(p, seqlen, r);
+        float l2 = 0.f, ds = 0.f;
+        if (r < R) {
+          const int i = r / p.G, g = r - i * p.G;
+          const int64_t row_id = (static_cast<int64_t>(b) * p.seqlen_q + i) * p.Hq + kvh * p.G + g;
+          l2 = p.row_lse2[row_id];
+          ds = p.row_d[row_id];
+        }
+        sm->lse2[t] = l2;
+        sm->dsum[t] = ds;
       }
-      sm->lse2[t] = l2;
-      sm->dsum[t] = ds;
       fence_proxy_async_smem();
     }
     tc_fence_before_sync();
     __syncthreads();
     if (*abort_any) break;
-    if (warp == 4 && lane == 0) {
+    if (warp == kBwdMmaWarp && lane == 0) {
       tc_fence_after_sync();
       constexpr uint32_t kId = idesc_bf16(128, 128, 0, 0);
       mma_kk<D>(tS, aK, aQ, kId);   // S^T = K Q^T
       mma_kk<D>(tdP, aV, aG, kId);  // dP^T = V dO^T
       umma_commit(&sm->mma_a);
     }
-    if (t < 128) {
+    if (tid < kBwdCompute) {
       mbar_wait(&sm->mma_a, it & 1, abort_any);
       __syncwarp();
       tc_fence_after_sync();
       const int tok = tok0 + t;
 #pragma unroll 1
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int ch = hf * 4; ch < hf * 4 + 4; ++ch) {  // this thread's 64 rows
         float sv[16], dp[16];
         tmem_ld16(tS + lane_off + ch * 16, sv);
         tmem_ld16(tdP + lane_off + ch * 16, dp);
@@ -350,7 +357,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
     tc_fence_before_sync();
     __syncthreads();
     if (*abort_any) break;
-    if (warp == 4 && lane == 0) {
+    if (warp == kBwdMmaWarp && lane == 0) {
       tc_fence_after_sync();
       constexpr uint32_t kId = idesc_bf16(128, D, 0, 1);
       mma_kn<D>(tdV, aP, aG, kId, it > 0);  // dV += P^T dO
@@ -364,14 +371,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
   tc_fence_before_sync();
   __syncthreads();
   const bool ok = !*abort_any;
-  if (t < 128 && ok) {
+  if (tid < kBwdCompute && ok) {
     tc_fence_after_sync();
     const int tok = tok0 + t;
     int64_t blk = -1;
     if (tok < seqlen) blk = bwd_block(p, b, tok);
     const int slot = tok & ((1 << p.block_shift) - 1);
 #pragma unroll 1
-    for (int ch = 0; ch < D / 16; ++ch) {
+    for (int ch = hf * (D / 32); ch < (hf + 1) * (D / 32); ++ch) {  // this thread's half of D
       float vv[16], kv[16];
       tmem_ld16(tdV + lane_off + ch * 16, vv);
       tmem_ld16(tdK + lane_off + ch * 16, kv);
@@ -397,18 +404,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
       }
     }
   }
-  if (!ok && warp == 4 && lane == 0) {
+  if (!ok && warp == kBwdMmaWarp && lane == 0) {
     umma_commit(&sm->drain);
     volatile int no_abort = 0;
     mbar_wait(&sm->drain, 0, &no_abort);
   }
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kBwdMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, 512);
   }
-  if (t == 0 && !ok && p.err) atomicOr(p.err, kErrTimeout);
+  if (tid == 0 && !ok && p.err) atomicOr(p.err, kErrTimeout);
 }
 
 // ---------------------------------------------------------------------------
@@ -425,7 +432,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
   uint8_t *sQ = smem, *sG = sQ + C::kTile, *sK = sG + C::kTile, *sV = sK + C::kTile;
   uint8_t *sS = sV + C::kTile;
   auto *sm = reinterpret_cast<typename C::Small *>(sS + C::kSq);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, t = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int t = tid & 127, hf = tid >> 7;  // TMEM lane / row, column half (compute threads)
   volatile int *abort_any = &sm->abort_any;
 
   int u = blockIdx.x;
@@ -439,19 +447,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
   // keys [0, lim_max) cover every row of the tile
   const int lim_max = bwd_row_lim(p, seqlen, min(row0 + kBwdTile, R) - 1);
 
-  if (t == 0) {
+  if (tid == 0) {
     mbar_init(&sm->mma_a, 1);
     mbar_init(&sm->mma_b, 1);
     mbar_init(&sm->drain, 1);
     sm->abort_any = 0;
     fence_barrier_init();
   }
-  if (warp == 4) tmem_alloc(&sm->tmem_base, 512);
+  if (warp == kBwdMmaWarp) tmem_alloc(&sm->tmem_base, 512);
   const int r_t = row0 + t;
   int my_lim = 0;
   float my_l2 = 0.f, my_d = 0.f;
   int64_t my_row = -1;
-  if (t < 128) {
+  if (tid < kBwdCompute) {
     auto rowptr = [&](const __nv_bfloat16 *base, int64_t sb, int64_t ss, int64_t sh, int c)
         -> const __nv_bfloat16 * {
       const int r = row0 + c;
@@ -459,8 +467,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
       const int i = r / p.G, g = r - i * p.G;
       return base + b * sb + static_cast<int64_t>(i) * ss + static_cast<int64_t>(kvh * p.G + g) * sh;
     };
-    stage_rows<D>(sQ, t, [&](int c) { return rowptr(p.q, p.q_sb, p.q_ss, p.q_sh, c); });
-    stage_rows<D>(sG, t, [&](int c) { return rowptr(p.dout, p.g_sb, p.g_ss, p.g_sh, c); });
+    stage_rows<D>(sQ, tid, [&](int c) { return rowptr(p.q, p.q_sb, p.q_ss, p.q_sh, c); });
+    stage_rows<D>(sG, tid, [&](int c) { return rowptr(p.dout, p.g_sb, p.g_ss, p.g_sh, c); });
     my_lim = bwd_row_lim(p, seqlen, r_t);
     if (r_t < R) {
       const int i = r_t / p.G, g = r_t - i * p.G;
@@ -483,15 +491,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
   int it = 0;
   for (int kt = 0; kt < n_kt; ++kt, ++it) {
     const int tok0 = kt * kBwdTile;
-    if (t < 128) {
-      stage_rows<D>(sK, t, [&](int c) -> const __nv_bfloat16 * {
+    if (tid < kBwdCompute) {
+      stage_rows<D>(sK, tid, [&](int c) -> const __nv_bfloat16 * {
         const int tok = tok0 + c;
         if (tok >= seqlen) return nullptr;
         const int64_t blk = bwd_block(p, b, tok);
         if (blk < 0) return nullptr;
         return p.k_cache + blk * p.k_sb + (tok & ((1 << p.block_shift) - 1)) * p.k_ss + kvh * p.k_sh;
       });
-      stage_rows<D>(sV, t, [&](int c) -> const __nv_bfloat16 * {
+      stage_rows<D>(sV, tid, [&](int c) -> const __nv_bfloat16 * {
         const int tok = tok0 + c;
         if (tok >= seqlen) return nullptr;
         const int64_t blk = bwd_block(p, b, tok);
@@ -503,19 +511,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
     tc_fence_before_sync();
     __syncthreads();
     if (*abort_any) break;
-    if (warp == 4 && lane == 0) {
+    if (warp == kBwdMmaWarp && lane == 0) {
       tc_fence_after_sync();
       constexpr uint32_t kId = idesc_bf16(128, 128, 0, 0);
       mma_kk<D>(tS, aQ, aK, kId);   // S = Q K^T
       mma_kk<D>(tdP, aG, aV, kId);  // dP = dO V^T
       umma_commit(&sm->mma_a);
     }
-    if (t < 128) {
+    if (tid < kBwdCompute) {
       mbar_wait(&sm->mma_a, it & 1, abort_any);
       __syncwarp();
       tc_fence_after_sync();
 #pragma unroll 1
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int ch = hf * 4; ch < hf * 4 + 4; ++ch) {  // this thread's 64 keys
         float sv[16], dp[16];
         tmem_ld16(tS + lane_off + ch * 16, sv);
         tmem_ld16(tdP + lane_off + ch * 16, dp);
@@ -541,7 +549,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
     tc_fence_before_sync();
     __syncthreads();
     if (*abort_any) break;
-    if (warp == 4 && lane == 0) {
+    if (warp == kBwdMmaWarp && lane == 0) {
       tc_fence_after_sync();
       mma_kn<D>(tdQ, aS, aK, idesc_bf16(128, D, 0, 1), it > 0);  // dQ += dS K
       umma_commit(&sm->mma_b);
@@ -552,10 +560,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
   tc_fence_before_sync();
   __syncthreads();
   const bool ok = !*abort_any;
-  if (t < 128 && ok) {
+  if (tid < kBwdCompute && ok) {
     tc_fence_after_sync();
 #pragma unroll 1
-    for (int ch = 0; ch < D / 16; ++ch) {
+    for (int ch = hf * (D / 32); ch < (hf + 1) * (D / 32); ++ch) {  // this thread's half of D
       float qv[16];
       tmem_ld16(tdQ + lane_off + ch * 16, qv);
       tmem_ld_wait_for(qv);
@@ -573,18 +581,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
       }
     }
   }
-  if (!ok && warp == 4 && lane == 0) {
+  if (!ok && warp == kBwdMmaWarp && lane == 0) {
     umma_commit(&sm->drain);
     volatile int no_abort = 0;
     mbar_wait(&sm->drain, 0, &no_abort);
   }
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kBwdMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, 512);
   }
-  if (t == 0 && !ok && p.err) atomicOr(p.err, kErrTimeout);
+  if (tid == 0 && !ok && p.err) atomicOr(p.err, kErrTimeout);
 }
 
 }  // namespace pkv
