@@ -20,10 +20,10 @@
 // Every sum therefore has one fixed order and the result is bitwise
 // reproducible and independent of the batch around a sequence.
 //
-// 288 threads: warps 0-7 stage operands and do the elementwise work -- warps
-// w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 (thread t = lane t of the
-// 128) and split the columns in halves -- and warp 8 owns TMEM, its lane 0
-// issuing the MMAs.  Phases are separated by __syncthreads and
+// 544 threads: warps 0-15 stage operands and do the elementwise work -- warps
+// w, w + 4, w + 8, w + 12 share TMEM lanes 32 (w % 4) .. + 31 (thread t = lane
+// t of the 128) and split the columns in quarters -- and warp 16 owns TMEM,
+// its lane 0 issuing the MMAs.  Phases are separated by __syncthreads and
 // MMA-completion mbarriers (bounded waits).
 #pragma once
 
@@ -34,9 +34,10 @@
 
 namespace pkv {
 
-constexpr int kBwdThreads = 288;
-constexpr int kBwdCompute = 256;  // staging / elementwise threads
-constexpr int kBwdMmaWarp = 8;
+constexpr int kBwdCompute = 512;               // staging / elementwise threads
+constexpr int kBwdGroups = kBwdCompute / 128;  // column groups per TMEM lane
+constexpr int kBwdThreads = kBwdCompute + 32;
+constexpr int kBwdMmaWarp = kBwdCompute / 32;
 constexpr int kBwdTile = 128;  // keys per key tile and rows per row tile
 
 struct BwdParams {
@@ -227,7 +228,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
   uint8_t *sP = sG + C::kTile, *sS = sP + C::kSq;
   auto *sm = reinterpret_cast<typename C::Small *>(sS + C::kSq);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-  const int t = tid & 127, hf = tid >> 7;  // TMEM lane / token, column half (compute threads)
+  const int t = tid & 127, hf = tid >> 7;  // TMEM lane / token, column group (compute threads)
   volatile int *abort_any = &sm->abort_any;
 
   int u = blockIdx.x;
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
       tc_fence_after_sync();
       const int tok = tok0 + t;
 #pragma unroll 1
-      for (int ch = hf * 4; ch < hf * 4 + 4; ++ch) {  // this thread's 64 rows
+      for (int ch = hf * (8 / kBwdGroups); ch < (hf + 1) * (8 / kBwdGroups); ++ch) {  // its rows
         float sv[16], dp[16];
         tmem_ld16(tS + lane_off + ch * 16, sv);
         tmem_ld16(tdP + lane_off + ch * 16, dp);
@@ -378,7 +379,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
     if (tok < seqlen) blk = bwd_block(p, b, tok);
     const int slot = tok & ((1 << p.block_shift) - 1);
 #pragma unroll 1
-    for (int ch = hf * (D / 32); ch < (hf + 1) * (D / 32); ++ch) {  // this thread's half of D
+    for (int ch = hf * (D / 16 / kBwdGroups); ch < (hf + 1) * (D / 16 / kBwdGroups); ++ch) {  // its part of D
       float vv[16], kv[16];
       tmem_ld16(tdV + lane_off + ch * 16, vv);
       tmem_ld16(tdK + lane_off + ch * 16, kv);
@@ -433,7 +434,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
   uint8_t *sS = sV + C::kTile;
   auto *sm = reinterpret_cast<typename C::Small *>(sS + C::kSq);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-  const int t = tid & 127, hf = tid >> 7;  // TMEM lane / row, column half (compute threads)
+  const int t = tid & 127, hf = tid >> 7;  // TMEM lane / row, column group (compute threads)
   volatile int *abort_any = &sm->abort_any;
 
   int u = blockIdx.x;
@@ -523,7 +524,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
       __syncwarp();
       tc_fence_after_sync();
 #pragma unroll 1
-      for (int ch = hf * 4; ch < hf * 4 + 4; ++ch) {  // this thread's 64 keys
+      for (int ch = hf * (8 / kBwdGroups); ch < (hf + 1) * (8 / kBwdGroups); ++ch) {  // its keys
         float sv[16], dp[16];
         tmem_ld16(tS + lane_off + ch * 16, sv);
         tmem_ld16(tdP + lane_off + ch * 16, dp);
@@ -563,7 +564,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
   if (tid < kBwdCompute && ok) {
     tc_fence_after_sync();
 #pragma unroll 1
-    for (int ch = hf * (D / 32); ch < (hf + 1) * (D / 32); ++ch) {  // this thread's half of D
+    for (int ch = hf * (D / 16 / kBwdGroups); ch < (hf + 1) * (D / 16 / kBwdGroups); ++ch) {  // its part of D
       float qv[16];
       tmem_ld16(tdQ + lane_off + ch * 16, qv);
       tmem_ld_wait_for(qv);
