@@ -205,9 +205,11 @@ struct Unit {
   int n_tiles;  // tiles of this split holding keys < lim_max
 };
 
-// Unit u = kvh + Hkv * (s + n_splits * (b + batch * rt)): the row tile varies
-// slowest, so the first row tiles of every sequence (all the work of decode
-// steps in a packed batch) spread over all CTAs of the strided assignment.
+// Unit u = kvh + Hkv * (s + n_splits * (b + batch * (n_row_tiles - 1 - rt))):
+// the row tile varies slowest, so each row tile of every sequence (the only
+// one of a decode step in a packed batch) spreads over all CTAs of the
+// strided assignment, and the last row tiles -- the heaviest under causal
+// masking, and those of the longest requests -- come first.
 template <int N>
 __device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
   Unit x;
@@ -216,7 +218,7 @@ __device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
   x.s = u % p.n_splits;
   u /= p.n_splits;
   x.b = u % p.batch;
-  x.rt = u / p.batch;
+  x.rt = p.n_row_tiles - 1 - u / p.batch;
   const int sl = __ldg(p.seqlens + x.b);
   x.seqlen = sl > 0 ? sl : 0;
   if (p.cu_q) {
