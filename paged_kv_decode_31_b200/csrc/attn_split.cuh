@@ -109,6 +109,9 @@ struct AttnParams {
   // partials are stored by local split.  part_only: every row leaves
   // partials, none is finished in the split kernel.
   int split_base, part_only;
+  // Packed calls may be served by two launches: this launch handles the
+  // sequences with nq_lo <= query count <= nq_hi (dense: all).
+  int nq_lo, nq_hi;
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -229,7 +232,8 @@ __device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
     x.q0 = static_cast<int64_t>(x.b) * p.seqlen_q;
     x.nq = p.seqlen_q;
   }
-  const int R = p.G * x.nq;
+  const bool mine = x.nq >= p.nq_lo && x.nq <= p.nq_hi;  // another launch serves the rest
+  const int R = mine ? p.G * x.nq : 0;
   x.row0 = x.rt * N;
   x.rows = max(min(N, R - x.row0), 0);
   int lim = x.rows > 0 ? x.seqlen : 0;

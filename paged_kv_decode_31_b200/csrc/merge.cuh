@@ -39,7 +39,8 @@ struct MergeParams {
   int64_t fo_sb, fo_sh;
   float *fin_lse;
   int64_t rows;     // output rows (tokens x Hq)
-  int skip_single;  // rows of at most one split were finished by the split kernel
+  int skip_single;  // rows of at most one split were finished by the split kernel ...
+  int skip_min_nq;  // ... for sequences with at least this many queries
   // Partials of global split s live in block r = s / n_local (local split
   // s % n_local) -- one block per context-parallel rank, gathered side by
   // side rank_floats floats apart; a single call has one block (n_local =
@@ -104,7 +105,7 @@ __global__ void __launch_bounds__(WIDE ? D : 32 * kMergeRowsPerBlock)
   if (p.causal) lim = min(lim, n - nq + i + 1);
   lim = max(lim, 0);
   const int n_s = min((lim + 4095) / 4096, p.n_splits);
-  if (p.skip_single && n_s <= 1) return;
+  if (p.skip_single && nq >= p.skip_min_nq && n_s <= 1) return;
   const int d0 = lane * V;
   const float NEG_INF = __int_as_float(0xff800000);
   float M = NEG_INF, L = 0.f, A[V];

@@ -419,6 +419,8 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   p.ws_acc = ws_acc;
   p.ws_ml = ws_ml;
   p.err = err;
+  p.nq_lo = 0;
+  p.nq_hi = INT_MAX;
   if (share) {
     p.split_base = share->split_begin;
     p.part_only = 1;
@@ -468,10 +470,27 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
     p.v_sh = v_strides[2];
   }
 
+  // A packed call whose longest request needs the row-major kernel also
+  // serves its short requests (at most 16 / G queries: one 16-row tile) with
+  // the transposed kernel, which keeps decode steps at memory speed; each
+  // launch skips the other's sequences.
+  const int small_nq = G <= 16 ? 16 / G : 0;
+  const bool split_by_size = pq && N == pkv::kRowsPerTile && small_nq > 0;
+  if (split_by_size) {
+    pkv::AttnParams ps = p;
+    ps.nq_lo = 1;
+    ps.nq_hi = small_nq;
+    ps.n_row_tiles = 1;
+    ps.n_units = static_cast<int>(static_cast<int64_t>(batch) * S * Hkv);
+    rc = D == 128 ? launch_split<128, 16>(ps, mk, mv, s, dev) : launch_split<64, 16>(ps, mk, mv, s, dev);
+    if (rc != PKV_OK) return rc;
+    p.nq_lo = small_nq + 1;
+  }
   if (N == pkv::kRowsPerTile) {
     // rows of at most one split are finished by the split kernel itself; the
-    // merge (needed only with more than one split) skips them
-    p.direct = (S == 1 && !share) ? 1 : 0;
+    // merge (needed with more than one split, or for the short requests of a
+    // packed call) skips them
+    p.direct = (S == 1 && !share && !split_by_size) ? 1 : 0;
     if (!share) {
       p.out = static_cast<__nv_bfloat16 *>(out);
       p.o_sb = out_strides[0];
@@ -514,6 +533,7 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   m.fin_lse = p.fin_lse;
   m.rows = rows;
   m.skip_single = N == pkv::kRowsPerTile ? 1 : 0;
+  m.skip_min_nq = split_by_size ? small_nq + 1 : 0;
   m.n_local = static_cast<int>(S);
   m.rank_floats = 0;
   return D == 128 ? launch_merge<128>(m, rows, s) : launch_merge<64>(m, rows, s);
