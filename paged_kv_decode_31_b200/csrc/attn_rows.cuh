@@ -10,9 +10,10 @@
 //   softmax one thread per ROW: all of a row's reductions are in-thread
 //           (the row sum replays the 32-key shuffle-down trees and the
 //           four-warp combine of attn_split.cuh element for element),
-//   P      = bf16(p) written back over the front of the S buffer in TMEM,
-//   O      = P * V with P read from TMEM (A operand) and V from shared memory
-//           (MN-major),
+//   P      = [bf16(p) | bf16(p - bf16(p))] written back over S in TMEM,
+//   O      = P_hi * V + P_lo * V (per 16-key step the hi MMA, then the lo MMA,
+//           into one accumulator) with P read from TMEM (A operand) and V
+//           from shared memory (MN-major),
 //   update acc = fma(O, b, acc * a) per row in the correction warpgroup,
 //           which owns the row's (m, l, acc[D]) in registers.
 // The tensor cores give every output element the same bits whichever operand
@@ -28,8 +29,8 @@
 //
 // TMEM (512 columns): three S/P buffers at columns 0, 128 and 256 (tile gi
 // uses buffer gi % 3, so the QK of tile gi waits only for the P.V of tile
-// gi - 3; P of keys [32 g, 32 g + 32) goes to columns [16 g, 16 g + 16), whose
-// scores are already read), O at 384.
+// gi - 3; P of keys [32 g, 32 g + 32) goes over those keys' own S columns:
+// hi in the first 16, lo in the next 16), O at 384.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -203,10 +204,13 @@ __global__ void __launch_bounds__(kRowThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kTileTokens / 16; ++kk) {
           // V: MN-major (N = head_dim), 128-byte swizzle; 64-wide d groups
-          // kHalfBytes apart, 8-key groups 1024 bytes apart.  P of keys
-          // [16 kk, 16 kk + 16): TMEM columns [8 kk, 8 kk + 8).
+          // kHalfBytes apart, 8-key groups 1024 bytes apart.  P_hi of keys
+          // [16 kk, 16 kk + 16): TMEM columns 32 (kk / 2) + 8 (kk % 2) + [0, 8),
+          // P_lo 16 columns further.  Hi, then lo, into the one accumulator.
           const uint64_t b = smem_desc(vaddr + kk * 2048, C::kHalfBytes, 1024, kLayoutSw128);
-          umma_bf16_ts(tmem + C::kColO, pcol + kk * 8, b, kIdescPV, kk > 0 ? 1u : 0u);
+          const uint32_t a = pcol + (kk >> 1) * 32 + (kk & 1) * 8;
+          umma_bf16_ts(tmem + C::kColO, a, b, kIdescPV, kk > 0 ? 1u : 0u);
+          umma_bf16_ts(tmem + C::kColO, a + 16, b, kIdescPV, 1u);
         }
         umma_commit(&sm->o_full);
         umma_commit(&sm->empty_v[st]);
@@ -268,8 +272,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     // ------------------------------------------------------------------
     // Softmax warpgroups: warpgroup wg takes the tiles with gi % 2 == wg;
     // thread t owns row t.  tmax = exact max of the row's masked scores,
-    // p = 2^(s - tmax), P = bf16(p) over S in TMEM, L = the row's sum of the
-    // fp32 p in the contract's fixed tree.
+    // p = 2^(s - tmax), P = [bf16(p) | bf16(p - bf16(p))] over S in TMEM,
+    // L = the row's sum of the fp32 p in the contract's fixed tree.
     // ------------------------------------------------------------------
     regs_dec<kRowsSoftmaxRegs>();
     const int wg = warp >> 2, wq = warp & 3, t = threadIdx.x & 127;
@@ -361,15 +365,19 @@ __global__ void __launch_bounds__(kRowThreads, 1)
               vb[e] = (sb == NEG_INF) ? 0.f : ex2(__fsub_rn(sb, mx));
             }
           }
-          uint32_t w[16];
+          uint32_t whi[16], wlo[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             const float x0 = k < 8 ? va[2 * k] : vb[2 * k - 16];
             const float x1 = k < 8 ? va[2 * k + 1] : vb[2 * k - 15];
             __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
-            w[k] = *reinterpret_cast<uint32_t *>(&h2);
+            __nv_bfloat162 l2 = __floats2bfloat162_rn(__fsub_rn(x0, __low2float(h2)),
+                                                      __fsub_rn(x1, __high2float(h2)));
+            whi[k] = *reinterpret_cast<uint32_t *>(&h2);
+            wlo[k] = *reinterpret_cast<uint32_t *>(&l2);
           }
-          tmem_st16(srow + grp * 16, w);
+          tmem_st16(srow + grp * 32, whi);
+          tmem_st16(srow + grp * 32 + 16, wlo);
           // the shuffle-down tree of one warp's 32 keys: offsets 16, 8, 4, 2, 1
 #pragma unroll
           for (int e = 0; e < 16; ++e) va[e] = __fadd_rn(va[e], vb[e]);

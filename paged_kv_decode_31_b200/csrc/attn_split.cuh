@@ -20,10 +20,13 @@
 //            N = rows, K = head_dim, fp32 accumulation in TMEM);
 //   softmax  one thread per token: mask (key < row limit), scale to base 2,
 //            the tile's column max over its 128 tokens (exact, order-free),
-//            p = 2^(s - tmax); P^T = bf16(p); the fp32 p of each row are summed
-//            in one fixed shuffle tree (so the row sum l never sees the bf16
-//            rounding of P);
-//   O^T      = V^T * P^T on the tensor cores (fresh accumulator each tile);
+//            p = 2^(s - tmax); P^T holds p as two bf16 parts side by side,
+//            hi = bf16(p) and lo = bf16(p - hi), so the tensor cores see p to
+//            ~16 bits; the fp32 p of each row are summed in one fixed
+//            shuffle tree (the row sum l never sees P's rounding);
+//   O^T      = V^T * P_hi^T + V^T * P_lo^T on the tensor cores: per 16-token
+//            step the hi MMA, then the lo MMA, into one fresh fp32
+//            accumulator per tile;
 //   update   m' = max(m, tmax), acc = fma(O, 2^(tmax - m'), acc * 2^(m - m')),
 //            l likewise with the tile's row sum; skipped for rows the tile
 //            does not reach.
@@ -171,7 +174,7 @@ struct Cfg {
   static constexpr int kKVBytes = (D / 64) * kHalfBytes;  // one K (or V) tile
   static constexpr int kQHalfBytes = N * 128;
   static constexpr int kQBytes = (D / 64) * kQHalfBytes;
-  static constexpr int kPCols = N;                        // P^T columns: one per row
+  static constexpr int kPCols = 2 * N;                    // P^T columns: N hi, then N lo
   static constexpr int kPBytes = kTileTokens * kPCols * 2;
   static constexpr int kPKGroup = (kPCols / 8) * 128;     // P^T stride between 8-token groups
   static constexpr int kOffK = 0;
@@ -557,11 +560,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           // (D = 64: both M halves read the same 64 columns; lanes 64..127 are unused).
           const uint64_t a = smem_desc(vaddr + kk * 2048, D == 128 ? C::kHalfBytes : 0, 1024,
                                        kLayoutSw128);
-          // P^T: MN-major, no swizzle; 8-column groups 128 B apart, 8-token
-          // groups kPKGroup apart.
-          const uint64_t b = smem_desc(paddr + kk * 2 * C::kPKGroup, C::kPKGroup, 128,
-                                       kLayoutInterleave);
-          umma_bf16(tO + bb * N, a, b, kIdescPV, kk > 0 ? 1u : 0u);
+          // P^T = [P_hi | P_lo]: MN-major, no swizzle; 8-column groups 128 B
+          // apart (the lo columns start N / 8 groups in), 8-token groups
+          // kPKGroup apart.  Hi, then lo, into the one accumulator.
+          const uint64_t bh = smem_desc(paddr + kk * 2 * C::kPKGroup, C::kPKGroup, 128,
+                                        kLayoutInterleave);
+          const uint64_t bl = smem_desc(paddr + kk * 2 * C::kPKGroup + (N / 8) * 128,
+                                        C::kPKGroup, 128, kLayoutInterleave);
+          umma_bf16(tO + bb * N, a, bh, kIdescPV, kk > 0 ? 1u : 0u);
+          umma_bf16(tO + bb * N, a, bl, kIdescPV, 1u);
         }
         umma_commit(&sm->o_full[bb]);
         umma_commit(&sm->empty_v[st]);
@@ -614,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Softmax warpgroups: warpgroup wg takes the tiles with gi % 2 == wg.
     // Thread t <-> TMEM lane t <-> token t of the tile.  Per tile and row:
     // tmax = exact max of the masked scores, p = 2^(s - tmax) written as
-    // P^T = bf16(p), per-warp sums of the fp32 p.
+    // P^T = [bf16(p) | bf16(p - bf16(p))], per-warp sums of the fp32 p.
     // ------------------------------------------------------------------
     const int wg = warp >> 2, wq = warp & 3, t = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -692,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *prow = smem + C::kOffP + bb * C::kPBytes + (t >> 3) * C::kPKGroup + (t & 7) * 16;
 #pragma unroll
         for (int grp = 0; grp < N / 8; ++grp) {
-          uint32_t w[4] = {0u, 0u, 0u, 0u};
+          uint32_t whi[4] = {0u, 0u, 0u, 0u}, wlo[4] = {0u, 0u, 0u, 0u};
           if (grp * 8 < x.rows) {  // groups of padded rows keep p = 0
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -705,10 +712,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               sv[c0] = p0;
               sv[c0 + 1] = p1;
               __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-              w[e] = *reinterpret_cast<uint32_t *>(&h2);
+              __nv_bfloat162 l2 = __floats2bfloat162_rn(__fsub_rn(p0, __low2float(h2)),
+                                                        __fsub_rn(p1, __high2float(h2)));
+              whi[e] = *reinterpret_cast<uint32_t *>(&h2);
+              wlo[e] = *reinterpret_cast<uint32_t *>(&l2);
             }
           }
-          *reinterpret_cast<uint4 *>(prow + grp * 128) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4 *>(prow + grp * 128) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
+          *reinterpret_cast<uint4 *>(prow + (N / 8 + grp) * 128) =
+              make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
         }
 #pragma unroll
         for (int q4 = 0; q4 < N / 4; ++q4) {

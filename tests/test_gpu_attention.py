@@ -7,6 +7,8 @@ on the interleaved non-contiguous cache with every unused slot NaN, through
 both entry points.  Edge cases: one-token contexts, split boundaries, rows with
 no visible key, empty sequences, many splits with a ragged tail.
 """
+import zlib
+
 import pytest
 import torch
 
@@ -36,7 +38,7 @@ def test_p2_grid_matches_oracle(mha, causal, bs, sqk, d, entry):
     sq, sk = sqk
     Hkv = 6 if mha == "mha" else 3
     di = I.p2_case(2, sq, sk, 6, Hkv, d, bs, causal=causal, layout="interleaved",
-                   seed=hash((mha, causal, bs, sq, d)) % 1000, poison=True)
+                   seed=zlib.crc32(repr((mha, causal, bs, sq, d)).encode()) % 1000, poison=True)
     fn = pkv.paged_decode_attn if entry == "decode" else pkv.paged_prefill_attn
     out, lse = run_gpu(di, entry=fn)
     ref_out, ref_lse = oracle_of(di)
@@ -158,3 +160,21 @@ def test_table_too_narrow_sets_the_error_flag():
                           err=err)
     torch.cuda.synchronize()
     assert int(err.item()) & pkv.binding.DEVERR_TABLE_WIDTH
+
+
+@pytest.mark.parametrize("entry", ["decode", "prefill"])
+def test_short_contexts_stay_in_bounds_over_seeds(entry):
+    """Short causal contexts where one or two keys carry most of the weight:
+    the case where bf16 rounding of P alone (without its low part) pushed
+    out past the 1e-2 bound.  24 seeds of the (gqa, causal, block_size 256,
+    seqlen_q 17, contexts <= 156, D 128) grid case."""
+    fn = pkv.paged_decode_attn if entry == "decode" else pkv.paged_prefill_attn
+    worst = 0.0
+    for seed in range(24):
+        di = I.p2_case(2, 17, 156, 6, 3, 128, 256, causal=True, layout="interleaved",
+                       seed=500 + seed, poison=True)
+        out, lse = run_gpu(di, entry=fn)
+        ref_out, ref_lse = oracle_of(di)
+        d_out, _ = assert_close_to_oracle(out, lse, ref_out, ref_lse)
+        worst = max(worst, d_out)
+    assert worst <= 1e-2

@@ -17,6 +17,8 @@ import math
 import os
 
 import numpy as np
+import zlib
+
 import pytest
 import torch
 import torch.nn.functional as F
@@ -191,7 +193,7 @@ def test_matches_torch_sdpa_fp64_on_p2_grid(mha, causal, bs, sqk, d):
     Hq = 6
     Hkv = 6 if mha == "mha" else 3
     di = I.p2_case(2, sq, sk, Hq, Hkv, d, bs, causal=causal, layout="interleaved",
-                   seed=hash((mha, causal, bs, sq, d)) % 1000, poison=True)
+                   seed=zlib.crc32(repr((mha, causal, bs, sq, d)).encode()) % 1000, poison=True)
     out, lse = run_oracle(di)
     ref_out, ref_lse = sdpa_reference(di)
     finite = torch.isfinite(ref_lse)
