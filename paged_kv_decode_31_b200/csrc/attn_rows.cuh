@@ -11,15 +11,14 @@
 //           (the row sum replays the 32-key shuffle-down trees and the
 //           four-warp combine of attn_split.cuh element for element),
 //   P      = [bf16(p) | bf16(p - bf16(p))] written back over S in TMEM,
-//   O      = P_hi * V + P_lo * V (per 16-key step the hi MMA, then the lo MMA,
-//           into one accumulator) with P read from TMEM (A operand) and V
-//           from shared memory (MN-major),
-//   update acc = fma(O, b, acc * a) per row in the correction warpgroup,
+//   O      = P_hi * V and P_lo * V into two accumulators, with P read from
+//           TMEM (A operand) and V from shared memory (MN-major),
+//   update acc = fma(O_hi + O_lo, b, acc * a) per row in the correction warpgroup,
 //           which owns the row's (m, l, acc[D]) in registers.
 // The tensor cores give every output element the same bits whichever operand
 // is A and whichever is B (the per-element dot products do not depend on the
-// orientation or on N), so S and O here equal the transposed kernel's S^T and
-// O^T bit for bit, and so does every row's result.
+// orientation or on N), so S, O_hi and O_lo here equal the transposed
+// kernel's S^T, O_hi^T and O_lo^T bit for bit, and so does every row's result.
 //
 // Roles (512 threads): warps 0-3 / 4-7 softmax warpgroups (even / odd tiles;
 // thread t = TMEM lane t = row t of the tile), 8-11 correction + epilogue,
@@ -27,10 +26,11 @@
 // 15 idle.  Registers are rebalanced per warpgroup (setmaxnreg): the
 // correction warpgroup holds a row's D fp32 accumulators.
 //
-// TMEM (512 columns): three S/P buffers at columns 0, 128 and 256 (tile gi
-// uses buffer gi % 3, so the QK of tile gi waits only for the P.V of tile
-// gi - 3; P of keys [32 g, 32 g + 32) goes over those keys' own S columns:
-// hi in the first 16, lo in the next 16), O at 384.
+// TMEM (512 columns): kSB S/P buffers of 128 columns (tile gi uses buffer
+// gi % kSB, so the QK of tile gi waits only for the P.V of tile gi - kSB; P
+// of keys [32 g, 32 g + 32) goes over those keys' own S columns: hi in the
+// first 16, lo in the next 16), then O_hi and O_lo (D columns each).  kSB = 2
+// at head_dim 128, 3 at 64.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -76,7 +76,9 @@ struct RowCfg {
   };
   static constexpr int kSmemBytes = kOffSmall + static_cast<int>(sizeof(Small)) + 1024;
   static constexpr int kTmemCols = 512;
-  static constexpr uint32_t kColO = 384;
+  static constexpr int kSB = (512 - 2 * D) / 128;  // S/P buffers next to O_hi and O_lo
+  static_assert(kSB == 2 || kSB == 3, "S/P buffers");
+  static constexpr uint32_t kColOhi = kSB * 128, kColOlo = kSB * 128 + D;
 };
 
 // Row t of a 128-row tile: out / lse through the merge's fold of one split.
@@ -149,7 +151,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       mbar_init(&sm->full_v[i], 1);
       mbar_init(&sm->empty_v[i], 1);
     }
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < C::kSB; ++i) {
       mbar_init(&sm->s_full[i], 1);
       mbar_init(&sm->p_full[i], 4);     // one arrival per softmax warp
       mbar_init(&sm->s_free[i], 1);
@@ -183,19 +185,20 @@ __global__ void __launch_bounds__(kRowThreads, 1)
                  false, lane, abort_any);
     } else if (warp == kMmaWarp && lane == 0) {
       // ----------------------------------------------------------------
-      // MMA issuer.  Per tile gi: S[gi % 3] = Q K^T once the K stage has
-      // landed and P.V of tile gi - 3 (which read P from the same columns)
-      // is done; then P.V of tile gi - 2, so that the softmax of two tiles
-      // can run while the tensor cores work.
+      // MMA issuer.  Per tile gi: S[gi % kSB] = Q K^T once the K stage has
+      // landed and P.V of tile gi - kSB (which read P from the same columns)
+      // is done; then P.V of tile gi - (kSB - 1), so that the softmax of
+      // kSB - 1 tiles can run while the tensor cores work.
       // ----------------------------------------------------------------
       constexpr uint32_t kIdescQK = idesc_bf16(128, 128, 0, 0);  // A = Q, B = K (K-major)
       constexpr uint32_t kIdescPV = idesc_bf16(128, D, 0, 1);    // A = P (TMEM), B = V (MN-major)
-      // (phase parity of the k-th use of buffer gi % 3 is k & 1, k = gi / 3)
+      // (phase parity of the k-th use of buffer gi % kSB is k & 1, k = gi / kSB)
+      constexpr int SB = C::kSB;
       int gi = 0, ui = 0, pend0 = -1, pend1 = -1;  // tiles whose P.V is not issued yet
       bool failed = false;
       auto pv_step = [&](int g) -> bool {
-        const int st = g % NS, bb = g % 3;
-        if (!mbar_wait(&sm->p_full[bb], (g / 3) & 1, abort_any)) return false;
+        const int st = g % NS, bb = g % SB;
+        if (!mbar_wait(&sm->p_full[bb], (g / SB) & 1, abort_any)) return false;
         if (!mbar_wait(&sm->o_free, (g & 1) ^ 1, abort_any)) return false;
         if (!mbar_wait(&sm->full_v[st], (g / NS) & 1, abort_any)) return false;
         tc_fence_after_sync();
@@ -206,11 +209,11 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           // V: MN-major (N = head_dim), 128-byte swizzle; 64-wide d groups
           // kHalfBytes apart, 8-key groups 1024 bytes apart.  P_hi of keys
           // [16 kk, 16 kk + 16): TMEM columns 32 (kk / 2) + 8 (kk % 2) + [0, 8),
-          // P_lo 16 columns further.  Hi, then lo, into the one accumulator.
+          // P_lo 16 columns further.
           const uint64_t b = smem_desc(vaddr + kk * 2048, C::kHalfBytes, 1024, kLayoutSw128);
           const uint32_t a = pcol + (kk >> 1) * 32 + (kk & 1) * 8;
-          umma_bf16_ts(tmem + C::kColO, a, b, kIdescPV, kk > 0 ? 1u : 0u);
-          umma_bf16_ts(tmem + C::kColO, a + 16, b, kIdescPV, 1u);
+          umma_bf16_ts(tmem + C::kColOhi, a, b, kIdescPV, kk > 0 ? 1u : 0u);
+          umma_bf16_ts(tmem + C::kColOlo, a + 16, b, kIdescPV, kk > 0 ? 1u : 0u);
         }
         umma_commit(&sm->o_full);
         umma_commit(&sm->empty_v[st]);
@@ -227,9 +230,9 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         }
         const uint32_t qaddr = sbase + C::kOffQ + qb * C::kQBytes;
         for (int j = 0; j < x.n_tiles; ++j, ++gi) {
-          const int st = gi % NS, bb = gi % 3;
+          const int st = gi % NS, bb = gi % SB;
           if (!mbar_wait(&sm->full_k[st], (gi / NS) & 1, abort_any) ||
-              !mbar_wait(&sm->s_free[bb], ((gi / 3) & 1) ^ 1, abort_any)) {
+              !mbar_wait(&sm->s_free[bb], ((gi / SB) & 1) ^ 1, abort_any)) {
             failed = true;
             break;
           }
@@ -245,7 +248,14 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           umma_commit(&sm->s_full[bb]);
           umma_commit(&sm->empty_k[st]);
           if (j == x.n_tiles - 1) umma_commit(&sm->q_empty[qb]);
-          if (pend1 >= 0) {
+          // keep at most kSB - 1 tiles whose P.V is not issued yet
+          if (SB == 2 && pend0 >= 0) {
+            if (!pv_step(pend0)) {
+              failed = true;
+              break;
+            }
+            pend0 = gi;
+          } else if (SB == 3 && pend1 >= 0) {
             if (!pv_step(pend0)) {
               failed = true;
               break;
@@ -294,7 +304,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       for (int j = 0; j < x.n_tiles; ++j) {
         const int gi = gbase + j;
         if ((gi & 1) != wg) continue;
-        const int bb = gi % 3, st = gi % NS, par = (gi / 3) & 1;
+        const int bb = gi % C::kSB, st = gi % NS, par = (gi / C::kSB) & 1;
         bool ok = mbar_wait(&sm->s_full[bb], par, abort_any);
         ok = mbar_wait(&sm->stat_free[bb], par ^ 1, abort_any) && ok;
         tc_fence_after_sync();
@@ -427,8 +437,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     // ------------------------------------------------------------------
     // Correction + epilogue warpgroup: thread t owns row t's running
     // (m, l, acc[D]).  Per tile, in order: m' = max(m, tmax), a = 2^(m - m'),
-    // b = 2^(tmax - m'), acc = fma(O, b, acc * a), l = fma(L, b, l * a); a
-    // tile the row does not reach (tmax = -inf) leaves it untouched.
+    // b = 2^(tmax - m'), acc = fma(O_hi + O_lo, b, acc * a), l = fma(L, b,
+    // l * a); a tile the row does not reach (tmax = -inf) leaves it untouched.
     // ------------------------------------------------------------------
     regs_inc<kRowsCorrRegs>();
     const int wq = warp & 3, t = threadIdx.x & 127;
@@ -454,7 +464,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       for (int c = 0; c < D; ++c) acc[c] = 0.f;
       float m_run = NEG_INF, l_run = 0.f;
       for (int j = 0; j < x.n_tiles; ++j) {
-        const int gi = gbase + j, bb = gi % 3, par = (gi / 3) & 1;
+        const int gi = gbase + j, bb = gi % C::kSB, par = (gi / C::kSB) & 1;
         bool ok = mbar_wait(&sm->p_full[bb], par, abort_any);  // the tile's row statistics
         ok = mbar_wait(&sm->o_full, gi & 1, abort_any) && ok;    // its P.V
         tc_fence_after_sync();
@@ -479,18 +489,16 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         const uint32_t orow = tmem + lane_off;
         __syncwarp();
 #pragma unroll
-        for (int ch = 0; ch < D / 16; ch += 2) {
-          float o0[16], o1[16];
-          tmem_ld16(orow + C::kColO + ch * 16, o0);
-          tmem_ld16(orow + C::kColO + ch * 16 + 16, o1);
-          tmem_ld_wait_for(o0);
-          tmem_ld_wait_for(o1);
+        for (int ch = 0; ch < D / 16; ++ch) {
+          float hi[16], lo[16];
+          tmem_ld16(orow + C::kColOhi + ch * 16, hi);
+          tmem_ld16(orow + C::kColOlo + ch * 16, lo);
+          tmem_ld_wait_for(hi);
+          tmem_ld_wait_for(lo);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {  // branch-free: the loop's TMEM loads are warp-wide
-            const float n0 = __fmaf_rn(o0[e], b, __fmul_rn(acc[ch * 16 + e], a));
-            const float n1 = __fmaf_rn(o1[e], b, __fmul_rn(acc[ch * 16 + 16 + e], a));
-            acc[ch * 16 + e] = skip ? acc[ch * 16 + e] : n0;
-            acc[ch * 16 + 16 + e] = skip ? acc[ch * 16 + 16 + e] : n1;
+            const float nv = __fmaf_rn(__fadd_rn(hi[e], lo[e]), b, __fmul_rn(acc[ch * 16 + e], a));
+            acc[ch * 16 + e] = skip ? acc[ch * 16 + e] : nv;
           }
         }
         tc_fence_before_sync();

@@ -24,9 +24,8 @@
 //            hi = bf16(p) and lo = bf16(p - hi), so the tensor cores see p to
 //            ~16 bits; the fp32 p of each row are summed in one fixed
 //            shuffle tree (the row sum l never sees P's rounding);
-//   O^T      = V^T * P_hi^T + V^T * P_lo^T on the tensor cores: per 16-token
-//            step the hi MMA, then the lo MMA, into one fresh fp32
-//            accumulator per tile;
+//   O^T      = V^T * [P_hi | P_lo]^T on the tensor cores (fresh accumulators
+//            each tile), O = O_hi + O_lo in fp32 on the CUDA cores;
 //   update   m' = max(m, tmax), acc = fma(O, 2^(tmax - m'), acc * 2^(m - m')),
 //            l likewise with the tile's row sum; skipped for rows the tile
 //            does not reach.
@@ -197,8 +196,8 @@ struct Cfg {
     int tab[2][2][kSplitTokens / 16];      // [producer][unit parity]: block-table entries
   };
   static constexpr int kSmemBytes = kOffSmall + static_cast<int>(sizeof(Small)) + 1024;
-  // TMEM: S^T (N columns) x 2 buffers, then O^T (N columns) x 2 buffers
-  static constexpr int kTmemCols = (4 * N <= 128) ? 128 : (4 * N <= 256) ? 256 : 512;
+  // TMEM: S^T (N columns) x 2 buffers, then O^T (hi and lo, 2N columns) x 2 buffers
+  static constexpr int kTmemCols = (6 * N <= 128) ? 128 : (6 * N <= 256) ? 256 : 512;
 };
 
 struct Unit {
@@ -542,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------
     if (lane == 0) {
       constexpr uint32_t kIdescQK = idesc_bf16(128, N, 0, 0);           // A = K tile, B = Q (K-major)
-      constexpr uint32_t kIdescPV = idesc_bf16(128, N, 1, 1);  // A = V^T, B = P^T (MN-major)
+      constexpr uint32_t kIdescPV = idesc_bf16(128, C::kPCols, 1, 1);  // A = V^T, B = P^T (MN-major)
       const uint32_t tS = tmem, tO = tmem + 2 * N;
       int gi = 0, ui = 0, prev = -1;
       bool failed = false;
@@ -561,14 +560,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t a = smem_desc(vaddr + kk * 2048, D == 128 ? C::kHalfBytes : 0, 1024,
                                        kLayoutSw128);
           // P^T = [P_hi | P_lo]: MN-major, no swizzle; 8-column groups 128 B
-          // apart (the lo columns start N / 8 groups in), 8-token groups
-          // kPKGroup apart.  Hi, then lo, into the one accumulator.
-          const uint64_t bh = smem_desc(paddr + kk * 2 * C::kPKGroup, C::kPKGroup, 128,
-                                        kLayoutInterleave);
-          const uint64_t bl = smem_desc(paddr + kk * 2 * C::kPKGroup + (N / 8) * 128,
-                                        C::kPKGroup, 128, kLayoutInterleave);
-          umma_bf16(tO + bb * N, a, bh, kIdescPV, kk > 0 ? 1u : 0u);
-          umma_bf16(tO + bb * N, a, bl, kIdescPV, 1u);
+          // apart, 8-token groups kPKGroup apart.  O_hi and O_lo side by side.
+          const uint64_t b = smem_desc(paddr + kk * 2 * C::kPKGroup, C::kPKGroup, 128,
+                                       kLayoutInterleave);
+          umma_bf16(tO + bb * C::kPCols, a, b, kIdescPV, kk > 0 ? 1u : 0u);
         }
         umma_commit(&sm->o_full[bb]);
         umma_commit(&sm->empty_v[st]);
@@ -746,8 +741,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Correction + epilogue warpgroup: thread t <-> TMEM lane t <-> output
     // column d of O^T; thread r (< rows) owns row r's running (m, l).
     // Per tile, in order: m' = max(m, tmax), a = 2^(m - m'), b = 2^(tmax - m'),
-    // acc = fma(O, b, acc * a), l = fma(sum p, b, l * a); a tile a row does
-    // not reach (tmax = -inf) leaves the row untouched.
+    // acc = fma(O_hi + O_lo, b, acc * a), l = fma(sum p, b, l * a); a tile a
+    // row does not reach (tmax = -inf) leaves the row untouched.
     // ------------------------------------------------------------------
     const int wq = warp & 3, t = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -796,14 +791,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int ch = 0; ch < N / 16; ++ch) {
           if (ch * 16 < x.rows) {  // warp-uniform
-            float o[16];
-            tmem_ld16(tmem + lane_off + 2 * N + bb * N + ch * 16, o);
-            tmem_ld_wait_for(o);
+            float hi[16], lo[16];
+            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + ch * 16, hi);
+            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + N + ch * 16, lo);
+            tmem_ld_wait_for(hi);
+            tmem_ld_wait_for(lo);
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int c = ch * 16 + e;
               if (c < x.rows && !sm->coef_skip[c])
-                acc[c] = __fmaf_rn(o[e], sm->coef_b[c], __fmul_rn(acc[c], sm->coef_a[c]));
+                acc[c] = __fmaf_rn(__fadd_rn(hi[e], lo[e]), sm->coef_b[c],
+                                   __fmul_rn(acc[c], sm->coef_a[c]));
             }
           }
         }
