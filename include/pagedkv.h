@@ -22,11 +22,13 @@
  * starting at absolute position 0, each split into tiles of PKV_TILE_TOKENS
  * tokens.  Within a split, tiles are folded in ascending order with an online
  * softmax in fp32: scores and P.V on the tensor cores with fp32 accumulation
- * (P entering P.V as bf16), each tile's max and row sums of the fp32
- * probabilities on the CUDA cores in fixed reduction trees, and the running
- * rescale in fp32 with the tile's own max.  Split partials are
- * merged in ascending split index (= global block index) order in fp32, and
- * out is rounded to bf16 once, at the final write.  Source: RL-Kernel PR #284
+ * (each probability entering P.V as a bf16 part and a bf16 remainder, ~16
+ * significant bits, into two accumulators added in fp32), each tile's max
+ * and row sums of the fp32 probabilities on the CUDA cores in fixed reduction
+ * trees, and the running rescale in fp32 with the tile's own max.  Split
+ * partials are merged in ascending split index (= global block index) order
+ * in fp32, and out is rounded to bf16 once, at the final write.  Source:
+ * RL-Kernel PR #284
  * "feat(attention): add CP backward drift validation", Changes ("fixed
  * global_block_index merge order, fp32 accumulation, final-write downcast"),
  * and the [WS1] "KV-cache path consistency (prefill & decode)" issue, Notes
