@@ -17,6 +17,7 @@ from .binding import (  # noqa: F401
     partials_size,
     paged_decode_attn,
     paged_decode_attn_append,
+    paged_decode_attn_static_ws,
     paged_prefill_attn,
     paged_prefill_attn_bwd,
     paged_varlen_attn,
