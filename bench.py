@@ -352,6 +352,50 @@ def backward_secondary(dev, reps: int = 5):
             "algorithmic_flops": flops}
 
 
+def decode_workload_secondary(dev, name: str, reps: int = 200, warmup: int = 20):
+    """The other timed decode workloads: `gqa_shard` (batch 32 x 4096, Hq 32 /
+    Hkv 8, D 128, block_size 16, contiguous) and `ragged` (batch 64, contexts
+    U[1, 32768], Hq 16 / Hkv 4, D 128, block_size 256, interleaved, NaN tails
+    and spare blocks).  One paged_decode_attn call per step, 20 warm-up and
+    200 timed steps with CUDA events per call; K/V bytes per call /
+    device time (mean, median, best).  Inputs are larger than L2."""
+    import paged_kv_decode_31_b200 as pkv
+    from paged_kv_decode_31_b200 import inputs as I
+    # drawn on the host (the generators are CPU ones), then moved
+    di = (I.config_gqa_shard if name == "gqa_shard" else I.config_ragged)().to(dev)
+    msk = int(di.seqlens.max().item())
+    ws = torch.empty(pkv.workspace_size(di.q.shape[0], 1, di.Hq, di.D, msk), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty(tuple(di.q.shape), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(di.q.shape[0], di.Hq, 1, dtype=torch.float32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def call():
+        pkv.paged_decode_attn(di.q, di.cache.k, di.cache.v, di.block_table, di.seqlens,
+                              max_seqlen_k=msk, scale=di.scale, causal=False, out=out, lse=lse,
+                              workspace=ws, err=err)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for a, b in ev:
+        a.record()
+        call()
+        b.record()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(err.item())}")
+    t = sorted(a.elapsed_time(b) for a, b in ev)
+    kv = di.kv_bytes()
+    mean = sum(t) / len(t)
+    return {"workload": name, "kv_bytes": kv, "ms_mean": round(mean, 5),
+            "ms_median": round(t[len(t) // 2], 5), "ms_best": round(t[0], 5),
+            "gbs_mean": round(kv / (mean / 1e3) / 1e9, 2),
+            "gbs_best": round(kv / (t[0] / 1e3) / 1e9, 2)}
+
+
 def run_ours(args):
     import torch.distributed as dist
     import paged_kv_decode_31_b200 as pkv
@@ -518,6 +562,13 @@ def run_ours(args):
         bw = backward_secondary(dev)
         bw["frac_of_tensor_peak"] = round(bw["tflops"] / bf16_peak, 4)
         result["backward"] = bw
+        for name in ("gqa_shard", "ragged"):
+            try:
+                dw = decode_workload_secondary(dev, name)
+                dw["hbm_frac"] = round(dw["gbs_mean"] / peak, 4)
+            except Exception as exc:  # the headline line is printed regardless
+                dw = {"workload": name, "error": str(exc)[:200]}
+            result[name] = dw
     if not args.no_cpu_baseline and world == 1:
         result["cpu_baseline"] = cpu_baseline(di)
     print(json.dumps(result), flush=True)
