@@ -535,6 +535,7 @@ def run_ours(args):
                      "kernel": "paged_decode_attn_append (attn_split_kernel<128,16,3,2> + merge_kernel<128>)",
                      "algorithmic_bytes_per_launch": kv_bytes,
                      "launch_ms_mean": round(dec_ms, 5),
+                     "launch_ms_median": round(statistics.median(decode_ms), 5),
                      "launch_ms_min": round(min(decode_ms), 5),
                      "peak_basis": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s"},
         "gpu_launches": 2 * args.steps,
