@@ -136,3 +136,17 @@ def test_context_parallel_exchange_and_ascending_merge_with_gloo(world):
         assert shares == (rank * n_local, n_local)
         assert d_out < 1e-12 and d_lse < 1e-12 and same_empty
     assert pdist.cp_split_share(20000, 2, 3) == (4, 2)
+
+
+@pytest.mark.parametrize("ctx,world", [(1, 1), (4096, 1), (4097, 2), (20000, 3), (8192, 8), (0, 4)])
+def test_cp_shares_cover_every_split_once_in_rank_order(ctx, world):
+    """Contiguous equal shares of the S = ceil(ctx / 4096) splits (S >= 1): every
+    split belongs to exactly one rank, rank r's share starts where rank r-1's
+    ends, and shares past S only happen at the end (more ranks than splits)."""
+    S = max(1, -(-ctx // 4096))
+    shares = [pdist.cp_split_share(ctx, r, world) for r in range(world)]
+    n = shares[0][1]
+    assert all(nl == n for _, nl in shares) and n >= 1
+    assert [b for b, _ in shares] == [r * n for r in range(world)]
+    covered = [s for b, nl in shares for s in range(b, b + nl) if s < S]
+    assert covered == list(range(S))
