@@ -7,8 +7,13 @@ into ``liboracle.so`` and loaded with ctypes.
 
 The arithmetic and the passages it follows are documented at the top of
 ``pkv_oracle.c``.  This module only marshals torch CPU tensors into the C
-calls.  Parity of every function here is pinned by ``tests/test_oracle_pins.py``
-(closed forms, invariants, and a library routine on special cases).
+calls.  Every function here is pinned against something other than itself
+(closed forms, invariants, brute force on tiny inputs, a library routine on
+special cases): ``paged_attn`` and ``kv_append`` in
+``tests/test_oracle_pins.py``, the packed forms in
+``tests/test_oracle_varlen_pins.py``, ``split_partials`` in
+``tests/test_oracle_split_pins.py`` and ``paged_attn_bwd`` in
+``tests/test_oracle_bwd_pins.py``.
 """
 from __future__ import annotations
 
