@@ -109,6 +109,54 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+# The library sees pointers, strides and the sizes passed beside them, nothing
+# else: a tensor smaller than those sizes say would be read or written out of
+# bounds on the device.  These checks tie every tensor to the sizes passed.
+
+def _need_err(err: Optional[torch.Tensor]) -> None:
+    if err is not None and (not err.is_cuda or err.dtype != torch.int32 or err.numel() < 1):
+        raise TypeError("err must be an int32 CUDA tensor with at least one element")
+
+
+def _need_cache_and_table(B: int, Hkv: Optional[int], D: int, k_cache: torch.Tensor,
+                          v_cache: torch.Tensor, block_table: torch.Tensor,
+                          seqlens: torch.Tensor) -> None:
+    """k_cache and v_cache of one shape [num_blocks, block_size, Hkv, D]; a
+    2-D block table of at least B rows with a unit column stride; at least B
+    contiguous sequence lengths."""
+    if tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError(f"k_cache {tuple(k_cache.shape)} and v_cache {tuple(v_cache.shape)} "
+                         "must have the same shape")
+    if int(k_cache.shape[3]) != D or (Hkv is not None and int(k_cache.shape[2]) != Hkv):
+        raise ValueError(f"the caches {tuple(k_cache.shape)} disagree with Hkv {Hkv}, D {D}")
+    if block_table.dim() != 2 or block_table.shape[0] < B:
+        raise ValueError(f"block_table must be 2-D with at least batch = {B} rows")
+    if block_table.stride(1) != 1:
+        raise ValueError("block_table must have a unit column stride")
+    if seqlens.dim() != 1 or seqlens.shape[0] < B or not seqlens.is_contiguous():
+        raise ValueError(f"seqlens must be a contiguous 1-D tensor of at least batch = {B} "
+                         "entries")
+
+
+def _need_one_device(*tensors: Optional[torch.Tensor]) -> None:
+    dev = tensors[0].device
+    for t in tensors:
+        if t is not None and t.device != dev:
+            raise ValueError(f"every tensor must be on {dev} (found one on {t.device})")
+
+
+def _need_rows(name: str, t: torch.Tensor, shape: tuple) -> None:
+    """A bf16 tensor of exactly `shape` with a unit last stride."""
+    if t.dtype != torch.bfloat16 or tuple(t.shape) != tuple(shape) or t.stride(-1) != 1:
+        raise ValueError(f"{name} must be bf16 {list(shape)} with a unit last stride "
+                         f"(got {t.dtype} {list(t.shape)})")
+
+
+def _need_lse(name: str, t: torch.Tensor, shape: tuple) -> None:
+    if t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be a contiguous fp32 {list(shape)} tensor")
+
+
 def workspace_size(batch: int, seqlen_q: int, Hq: int, D: int, max_seqlen_k: int) -> int:
     return int(lib().pkv_workspace_size(batch, seqlen_q, Hq, D, max_seqlen_k))
 
@@ -122,9 +170,12 @@ def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
         _need_cuda_bf16(name, t)
     _need_cuda_i32("block_table", block_table)
     _need_cuda_i32("seqlens", seqlens)
-    if block_table.stride(1) != 1:
-        raise ValueError("block_table must have a unit column stride")
+    _need_err(err)
     B, n, Hkv, D = k_new.shape
+    if tuple(v_new.shape) != tuple(k_new.shape):
+        raise ValueError("k_new and v_new must have the same shape")
+    _need_cache_and_table(B, Hkv, D, k_cache, v_cache, block_table, seqlens)
+    _need_one_device(k_new, v_new, k_cache, v_cache, block_table, seqlens, err)
     rc = lib().pkv_kv_append(
         k_new.data_ptr(), _st3(k_new), v_new.data_ptr(), _st3(v_new),
         k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(), _st3(v_cache),
@@ -141,12 +192,10 @@ def _attn(fn_name: str, q, k_cache, v_cache, block_table, seqlens, max_seqlen_k,
     _need_cuda_bf16("v_cache", v_cache)
     _need_cuda_i32("block_table", block_table)
     _need_cuda_i32("seqlens", seqlens)
-    if block_table.stride(1) != 1:
-        raise ValueError("block_table must have a unit column stride")
+    _need_err(err)
     B, sq, Hq, D = q.shape
-    num_blocks, bs, Hkv, D2 = k_cache.shape
-    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape):
-        raise ValueError("q / k_cache / v_cache shapes disagree")
+    num_blocks, bs, Hkv, _ = k_cache.shape
+    _need_cache_and_table(B, None, D, k_cache, v_cache, block_table, seqlens)
     if max_seqlen_k is None:
         max_seqlen_k = int(seqlens.max().item()) if seqlens.numel() else 0
     if scale is None:
@@ -155,13 +204,12 @@ def _attn(fn_name: str, q, k_cache, v_cache, block_table, seqlens, max_seqlen_k,
         out = torch.empty(B, sq, Hq, D, dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty(B, Hq, sq, dtype=torch.float32, device=q.device)
-    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, sq):
-        raise ValueError("lse must be a contiguous fp32 [B, Hq, seqlen_q] tensor")
-    if out.dtype != torch.bfloat16 or tuple(out.shape) != (B, sq, Hq, D) or out.stride(-1) != 1:
-        raise ValueError("out must be bf16 [B, seqlen_q, Hq, D] with a unit last stride")
+    _need_lse("lse", lse, (B, Hq, sq))
+    _need_rows("out", out, (B, sq, Hq, D))
     need = workspace_size(B, sq, Hq, D, max_seqlen_k)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _need_one_device(q, k_cache, v_cache, block_table, seqlens, out, lse, workspace, err)
     rc = getattr(lib(), fn_name)(
         q.data_ptr(), _st3(q), k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(),
         _st3(v_cache), num_blocks, block_table.data_ptr(), int(block_table.stride(0)),
@@ -202,10 +250,13 @@ def paged_decode_attn_append(q, k_new, v_new, k_cache, v_cache, block_table, seq
     _need_cuda_bf16("v_cache", v_cache)
     _need_cuda_i32("block_table", block_table)
     _need_cuda_i32("seqlens", seqlens)
-    if block_table.stride(1) != 1:
-        raise ValueError("block_table must have a unit column stride")
+    _need_err(err)
     B, sq, Hq, D = q.shape
     num_blocks, bs, Hkv, _ = k_cache.shape
+    _need_cache_and_table(B, None, D, k_cache, v_cache, block_table, seqlens)
+    if tuple(v_new.shape) != tuple(k_new.shape) or int(k_new.shape[0]) != B or \
+            tuple(k_new.shape[2:]) != (Hkv, D):
+        raise ValueError(f"k_new and v_new must both be [{B}, n_new, {Hkv}, {D}]")
     if max_seqlen_k is None:
         max_seqlen_k = int(seqlens.max().item()) if seqlens.numel() else 0
     if scale is None:
@@ -214,9 +265,13 @@ def paged_decode_attn_append(q, k_new, v_new, k_cache, v_cache, block_table, seq
         out = torch.empty(B, sq, Hq, D, dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty(B, Hq, sq, dtype=torch.float32, device=q.device)
+    _need_lse("lse", lse, (B, Hq, sq))
+    _need_rows("out", out, (B, sq, Hq, D))
     if workspace is None:
         workspace = torch.empty(workspace_size(B, sq, Hq, D, max_seqlen_k), dtype=torch.uint8,
                                 device=q.device)
+    _need_one_device(q, k_new, v_new, k_cache, v_cache, block_table, seqlens, out, lse,
+                     workspace, err)
     rc = fn(q.data_ptr(), _st3(q), k_new.data_ptr(), _st3(k_new), v_new.data_ptr(), _st3(v_new),
             int(k_new.shape[1]), k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(),
             _st3(v_cache), num_blocks, block_table.data_ptr(), int(block_table.stride(0)),
@@ -266,15 +321,13 @@ def paged_varlen_attn(q, k_cache, v_cache, block_table, seqlens, cu_seqlens_q, m
     _need_cuda_i32("block_table", block_table)
     _need_cuda_i32("seqlens", seqlens)
     _need_cuda_i32("cu_seqlens_q", cu_seqlens_q)
-    if block_table.stride(1) != 1:
-        raise ValueError("block_table must have a unit column stride")
+    _need_err(err)
     total_q, Hq, D = q.shape
     B = int(seqlens.shape[0])
-    if tuple(cu_seqlens_q.shape) != (B + 1,):
-        raise ValueError("cu_seqlens_q must have batch + 1 entries")
-    num_blocks, bs, Hkv, D2 = k_cache.shape
-    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape):
-        raise ValueError("q / k_cache / v_cache shapes disagree")
+    if tuple(cu_seqlens_q.shape) != (B + 1,) or not cu_seqlens_q.is_contiguous():
+        raise ValueError("cu_seqlens_q must be a contiguous tensor of batch + 1 entries")
+    num_blocks, bs, Hkv, _ = k_cache.shape
+    _need_cache_and_table(B, None, D, k_cache, v_cache, block_table, seqlens)
     if max_seqlen_k is None:
         max_seqlen_k = int(seqlens.max().item()) if seqlens.numel() else 0
     if scale is None:
@@ -295,11 +348,14 @@ def paged_varlen_attn(q, k_cache, v_cache, block_table, seqlens, cu_seqlens_q, m
     if final_out is not None:
         _need_packed_bf16("final_out", final_out)
         if tuple(final_out.shape) != (B, Hq, D) or final_lse is None or \
-                tuple(final_lse.shape) != (B, Hq) or not final_lse.is_contiguous():
+                tuple(final_lse.shape) != (B, Hq) or not final_lse.is_contiguous() or \
+                final_lse.dtype != torch.float32:
             raise ValueError("final_out must be [B, Hq, D] and final_lse a contiguous [B, Hq]")
     need = varlen_workspace_size(total_q, Hq, D, max_seqlen_k)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _need_one_device(q, k_cache, v_cache, block_table, seqlens, cu_seqlens_q, out, lse,
+                     final_out, final_lse, workspace, err)
     rc = lib().pkv_paged_varlen_attn(
         q.data_ptr(), _st2(q), cu_seqlens_q.data_ptr(), total_q, int(max_seqlen_q),
         k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(), _st3(v_cache), num_blocks,
@@ -326,10 +382,15 @@ def kv_append_varlen(k_new, v_new, k_cache, v_cache, block_table, seqlens, cu_se
     _need_cuda_i32("block_table", block_table)
     _need_cuda_i32("seqlens", seqlens)
     _need_cuda_i32("cu_seqlens_new", cu_seqlens_new)
-    if block_table.stride(1) != 1:
-        raise ValueError("block_table must have a unit column stride")
+    _need_err(err)
     total, Hkv, D = k_new.shape
     B = int(seqlens.shape[0])
+    if tuple(v_new.shape) != tuple(k_new.shape):
+        raise ValueError("k_new and v_new must have the same shape")
+    if tuple(cu_seqlens_new.shape) != (B + 1,) or not cu_seqlens_new.is_contiguous():
+        raise ValueError("cu_seqlens_new must be a contiguous tensor of batch + 1 entries")
+    _need_cache_and_table(B, Hkv, D, k_cache, v_cache, block_table, seqlens)
+    _need_one_device(k_new, v_new, k_cache, v_cache, block_table, seqlens, cu_seqlens_new, err)
     rc = lib().pkv_kv_append_varlen(
         k_new.data_ptr(), _st2(k_new), v_new.data_ptr(), _st2(v_new), cu_seqlens_new.data_ptr(),
         total, k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(), _st3(v_cache),
@@ -364,15 +425,16 @@ def paged_attn_partials(q, k_cache, v_cache, block_table, seqlens, split_begin, 
         _need_cuda_bf16(name, t)
     _need_cuda_i32("block_table", block_table)
     _need_cuda_i32("seqlens", seqlens)
-    if block_table.stride(1) != 1:
-        raise ValueError("block_table must have a unit column stride")
+    _need_err(err)
     B, sq, Hq, D = q.shape
     num_blocks, bs, Hkv, _ = k_cache.shape
+    _need_cache_and_table(B, None, D, k_cache, v_cache, block_table, seqlens)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     need = partials_size(B, sq, Hq, D, n_splits_local)
     if partials is None:
         partials = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _need_one_device(q, k_cache, v_cache, block_table, seqlens, partials, err)
     rc = fn(q.data_ptr(), _st3(q), k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(),
             _st3(v_cache), num_blocks, block_table.data_ptr(), int(block_table.stride(0)),
             int(block_table.shape[1]), seqlens.data_ptr(), B, sq, Hq, Hkv, D, bs, float(scale),
@@ -393,7 +455,12 @@ def merge_partials(gathered, world, n_splits_local, seqlens, q_shape, *, causal=
         fn.argtypes = [_P, _I, _I, ctypes.c_size_t, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]
         fn.restype = _I
     _need_cuda_i32("seqlens", seqlens)
+    if not gathered.is_cuda or not gathered.is_contiguous():
+        raise TypeError("gathered must be a contiguous CUDA tensor")
     B, sq, Hq, D = q_shape
+    if seqlens.dim() != 1 or seqlens.shape[0] < B or not seqlens.is_contiguous():
+        raise ValueError(f"seqlens must be a contiguous 1-D tensor of at least batch = {B} "
+                         "entries")
     nbytes = gathered.numel() * gathered.element_size()
     if nbytes % world != 0:
         raise ValueError("gathered buffer is not world equal blocks")
@@ -401,6 +468,9 @@ def merge_partials(gathered, world, n_splits_local, seqlens, q_shape, *, causal=
         out = torch.empty(B, sq, Hq, D, dtype=torch.bfloat16, device=gathered.device)
     if lse is None:
         lse = torch.empty(B, Hq, sq, dtype=torch.float32, device=gathered.device)
+    _need_rows("out", out, (B, sq, Hq, D))
+    _need_lse("lse", lse, (B, Hq, sq))
+    _need_one_device(gathered, seqlens, out, lse)
     rc = fn(gathered.data_ptr(), int(world), int(n_splits_local), nbytes // world,
             seqlens.data_ptr(), B, sq, Hq, D, int(bool(causal)), out.data_ptr(), _st3(out),
             lse.data_ptr(), _stream_handle(stream))
@@ -428,8 +498,13 @@ def paged_prefill_attn_bwd(q, k_cache, v_cache, block_table, seqlens, out, lse, 
         _need_cuda_bf16(name, t)
     _need_cuda_i32("block_table", block_table)
     _need_cuda_i32("seqlens", seqlens)
+    _need_err(err)
     B, sq, Hq, D = q.shape
     num_blocks, bs, Hkv, _ = k_cache.shape
+    _need_cache_and_table(B, None, D, k_cache, v_cache, block_table, seqlens)
+    _need_rows("out", out, (B, sq, Hq, D))
+    _need_rows("dout", dout, (B, sq, Hq, D))
+    _need_lse("lse", lse, (B, Hq, sq))
     if max_seqlen_k is None:
         max_seqlen_k = int(seqlens.max().item()) if seqlens.numel() else 0
     if scale is None:
@@ -442,9 +517,14 @@ def paged_prefill_attn_bwd(q, k_cache, v_cache, block_table, seqlens, out, lse, 
         dv_cache = torch.zeros(v_cache.shape, dtype=torch.bfloat16, device=q.device)
     for name, t in (("dq", dq), ("dk_cache", dk_cache), ("dv_cache", dv_cache)):
         _need_cuda_bf16(name, t)
+    _need_rows("dq", dq, (B, sq, Hq, D))
+    _need_rows("dk_cache", dk_cache, tuple(k_cache.shape))
+    _need_rows("dv_cache", dv_cache, tuple(v_cache.shape))
     if workspace is None:
         workspace = torch.empty(int(L.pkv_bwd_workspace_size(B, sq, Hq)), dtype=torch.uint8,
                                 device=q.device)
+    _need_one_device(q, k_cache, v_cache, block_table, seqlens, out, lse, dout, dq, dk_cache,
+                     dv_cache, workspace, err)
     rc = fn(q.data_ptr(), _st3(q), k_cache.data_ptr(), _st3(k_cache), v_cache.data_ptr(),
             _st3(v_cache), num_blocks, block_table.data_ptr(), int(block_table.stride(0)),
             int(block_table.shape[1]), seqlens.data_ptr(), int(max_seqlen_k), B, sq, Hq, Hkv, D,
@@ -479,10 +559,13 @@ def paged_decode_attn_static_ws(q, k_cache, v_cache, block_table, seqlens, *, ma
         _need_cuda_bf16(name, t)
     _need_cuda_i32("block_table", block_table)
     _need_cuda_i32("seqlens", seqlens)
+    _need_err(err)
     B, sq, Hq, D = q.shape
     num_blocks, bs, Hkv, _ = k_cache.shape
-    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, sq):
-        raise ValueError("lse must be a contiguous fp32 [B, Hq, seqlen_q] tensor")
+    _need_cache_and_table(B, None, D, k_cache, v_cache, block_table, seqlens)
+    _need_lse("lse", lse, (B, Hq, sq))
+    _need_rows("out", out, (B, sq, Hq, D))
+    _need_one_device(q, k_cache, v_cache, block_table, seqlens, out, lse, err)
     need = workspace_size(B, sq, Hq, D, max_seqlen_k)
     if need > STATIC_WORKSPACE_BYTES:
         raise PagedKVError(f"this problem needs {need} bytes of scratch; the library's static "
