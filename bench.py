@@ -48,6 +48,7 @@ WORKLOAD = ("long-context split-K decode: batch 4, seqlen_q 1, context 131072, H
             "[4, 8192], split chunk 4096 tokens")
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+L2_BYTES = 126 * 1024 * 1024  # B200 L2
 
 
 def parse_args():
@@ -524,14 +525,18 @@ def run_ours(args):
                    "Hq": Hq, "Hkv": Hkv, "head_dim": D, "block_size": 16,
                    "split_tokens": pkv.SPLIT_TOKENS,
                    "step": "paged_decode_attn_append: kv_append of 1 token/sequence fused into the decode call",
-                   "l2": "inputs larger than L2 (2.15 GB of K/V per rank), no flush",
+                   "l2": (f"inputs larger than L2 ({kv_bytes / 1e9:.3g} GB of K/V per rank), no flush"
+                          if kv_bytes > L2_BYTES else
+                          f"inputs NOT larger than L2 ({kv_bytes / 1e9:.3g} GB of K/V per rank): "
+                          "a profiling size, not a bench number"),
                    "parallelism": f"dp{world}"},
         "tokens_per_s": round(B * world * args.steps / (ms_total / 1e3), 1),
         "hbm_frac": round(value / world / peak, 4),
         "hbm_frac_basis": f"{peak_kind} HBM copy bandwidth {peak} GB/s",
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(),
+                     # the ncu figure belongs to the full-size workload only
+                     "traffic": profiled_traffic() if (args.context, args.batch) == (131072, 4) else None,
                      "kernel": "paged_decode_attn_append (attn_split_kernel<128,16,3,2> + merge_kernel<128>)",
                      "algorithmic_bytes_per_launch": kv_bytes,
                      "launch_ms_mean": round(dec_ms, 5),
@@ -546,30 +551,43 @@ def run_ours(args):
         result["config"]["workload"] = (f"profiling size: batch {B}, context {ctx} "
                                         "(otherwise as the long-context workload)")
     if world == 1 and (args.context, args.batch) == (131072, 4):
-        pre = prefill_secondary(dev)
         bf16_peak = None
         try:
             with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
                 bf16_peak = float(json.load(f)["bf16_tflops"])
         except Exception:
             bf16_peak = 1590.0
-        pre["tensor_peak_tflops"] = bf16_peak
-        pre["frac_of_tensor_peak"] = round(pre["tflops"] / bf16_peak, 4)
-        result["prefill"] = pre
-        vl = varlen_secondary(dev)
-        vl["hbm_frac"] = round(vl["kv_gbs"] / peak, 4)
-        vl["frac_of_tensor_peak"] = round(vl["tflops"] / bf16_peak, 4)
-        result["varlen"] = vl
-        bw = backward_secondary(dev)
-        bw["frac_of_tensor_peak"] = round(bw["tflops"] / bf16_peak, 4)
-        result["backward"] = bw
-        for name in ("gqa_shard", "ragged"):
+
+        def prefill_obj():
+            pre = prefill_secondary(dev)
+            pre["tensor_peak_tflops"] = bf16_peak
+            pre["frac_of_tensor_peak"] = round(pre["tflops"] / bf16_peak, 4)
+            return pre
+
+        def varlen_obj():
+            vl = varlen_secondary(dev)
+            vl["hbm_frac"] = round(vl["kv_gbs"] / peak, 4)
+            vl["frac_of_tensor_peak"] = round(vl["tflops"] / bf16_peak, 4)
+            return vl
+
+        def backward_obj():
+            bw = backward_secondary(dev)
+            bw["frac_of_tensor_peak"] = round(bw["tflops"] / bf16_peak, 4)
+            return bw
+
+        def decode_obj(name):
+            dw = decode_workload_secondary(dev, name)
+            dw["hbm_frac"] = round(dw["gbs_mean"] / peak, 4)
+            return dw
+
+        secondary = [("prefill", prefill_obj), ("varlen", varlen_obj), ("backward", backward_obj),
+                     ("gqa_shard", lambda: decode_obj("gqa_shard")),
+                     ("ragged", lambda: decode_obj("ragged"))]
+        for key, fn in secondary:
             try:
-                dw = decode_workload_secondary(dev, name)
-                dw["hbm_frac"] = round(dw["gbs_mean"] / peak, 4)
+                result[key] = fn()
             except Exception as exc:  # the headline line is printed regardless
-                dw = {"workload": name, "error": str(exc)[:200]}
-            result[name] = dw
+                result[key] = {"error": f"{type(exc).__name__}: {str(exc)[:200]}"}
     if not args.no_cpu_baseline and world == 1:
         result["cpu_baseline"] = cpu_baseline(di)
     print(json.dumps(result), flush=True)
