@@ -16,7 +16,8 @@ value   = algorithmic KV bytes (every visible token read once per KV head, K
           flush is needed between steps.
 e2e     = the same metric through the public API with pinned host buffers:
           each step copies q, the new K/V, the sequence lengths and the block
-          table host->device and the output and lse device->host.
+          table host->device (packed in one pinned buffer, one copy) and the
+          output and lse device->host (one copy).
 roofline: the decode call's KV bytes / its mean CUDA-event duration, against
           the measured HBM copy bandwidth.
 cpu_baseline: the CPU fp64 oracle on a bounded sample of the same workload.
@@ -397,6 +398,23 @@ def decode_workload_secondary(dev, name: str, reps: int = 200, warmup: int = 20)
             "gbs_best": round(kv / (t[0] / 1e3) / 1e9, 2)}
 
 
+def packed_layout(tensors):
+    """Byte offsets of `tensors` laid end to end in one buffer, each start
+    16-byte aligned, and the buffer's size."""
+    offs, off = [], 0
+    for t in tensors:
+        offs.append(off)
+        off += (t.numel() * t.element_size() + 15) // 16 * 16
+    return offs, off
+
+
+def packed_views(buf, like, offs):
+    """Views of the uint8 buffer `buf` with the dtypes and shapes of `like`
+    (contiguous), at the offsets of packed_layout."""
+    return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(tuple(t.shape))
+            for t, o in zip(like, offs)]
+
+
 def run_ours(args):
     import torch.distributed as dist
     import paged_kv_decode_31_b200 as pkv
@@ -458,28 +476,31 @@ def run_ours(args):
     if int(err.item()) != 0:
         raise RuntimeError(f"device error bits {int(err.item())}")
 
-    # e2e through the public API with pinned host buffers
+    # e2e through the public API with pinned host buffers: the step's inputs
+    # (q, the new K/V, the lengths, the block table) travel in one pinned
+    # buffer and its results (out, lse) come back in another -- one copy each
+    # way per step, the call itself taking views of the device buffers.
     e2e = None
     if not args.no_e2e:
-        h_q = di.q.cpu().pin_memory()
-        h_kn, h_vn = k_new.cpu().pin_memory(), v_new.cpu().pin_memory()
-        h_s = seq.cpu().pin_memory()
-        h_bt = di.block_table.cpu().pin_memory()
-        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        d_q, d_kn, d_vn = torch.empty_like(di.q), torch.empty_like(k_new), torch.empty_like(v_new)
-        d_s, d_bt = torch.empty_like(seq), torch.empty_like(di.block_table)
-        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_s, h_bt))
-        d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+        ins = (di.q, k_new, v_new, seq, di.block_table)
+        in_offs, h2d = packed_layout(ins)
+        h_in = torch.empty(h2d, dtype=torch.uint8).pin_memory()
+        for t, hv in zip(ins, packed_views(h_in, ins, in_offs)):
+            hv.copy_(t.cpu())
+        d_in = torch.empty(h2d, dtype=torch.uint8, device=dev)
+        d_q, d_kn, d_vn, d_s, d_bt = packed_views(d_in, ins, in_offs)
+        res = (out, lse)
+        res_offs, d2h = packed_layout(res)
+        d_res = torch.empty(d2h, dtype=torch.uint8, device=dev)
+        e_out, e_lse = packed_views(d_res, res, res_offs)
+        h_res = torch.empty(d2h, dtype=torch.uint8).pin_memory()
 
         def e2e_step():
-            for d, h in ((d_q, h_q), (d_kn, h_kn), (d_vn, h_vn), (d_s, h_s), (d_bt, h_bt)):
-                d.copy_(h, non_blocking=True)
+            d_in.copy_(h_in, non_blocking=True)
             pkv.paged_decode_attn_append(d_q, d_kn, d_vn, di.cache.k, di.cache.v, d_bt, d_s,
-                                         max_seqlen_k=ctx, scale=di.scale, causal=False, out=out,
-                                         lse=lse, workspace=ws, err=err)
-            h_out.copy_(out, non_blocking=True)
-            h_lse.copy_(lse, non_blocking=True)
+                                         max_seqlen_k=ctx, scale=di.scale, causal=False,
+                                         out=e_out, lse=e_lse, workspace=ws, err=err)
+            h_res.copy_(d_res, non_blocking=True)
 
         for _ in range(max(3, args.warmup)):
             e2e_step()
