@@ -110,3 +110,29 @@ def test_kv_append_places_every_token_at_its_position(c, n_new):
     # nothing else changed
     assert torch.equal(k[~touched].view(torch.int16), k0[~touched].view(torch.int16))
     assert torch.equal(v[~touched].view(torch.int16), v0[~touched].view(torch.int16))
+
+
+@settings(max_examples=40, deadline=None)
+@given(SHAPES, st.sampled_from([1, 2, 3, 5, 8, 16]), st.integers(1, 4))
+def test_rank_shares_of_split_partials_fold_to_the_whole_context(c, split_tokens, world):
+    """Context parallelism on the oracle side: the splits cut into `world`
+    contiguous shares of ceil(S / world) (the last ones may run past the
+    context), each share's partials computed alone, laid side by side and
+    folded in ascending split order equal the whole-context result."""
+    from test_oracle_split_pins import _fold
+
+    q, k, v, table, seqlens, scale = _problem(c)
+    S = max(1, math.ceil(c["max_ctx"] / split_tokens))
+    n_local = math.ceil(S / world)
+    parts = [oracle.split_partials(q, k, v, table, seqlens, scale, c["causal"], r * n_local,
+                                   n_local, split_tokens=split_tokens) for r in range(world)]
+    m = torch.cat([p[0] for p in parts], -1)
+    l = torch.cat([p[1] for p in parts], -1)
+    acc = torch.cat([p[2] for p in parts], -2)
+    out, lse = _fold(m, l, acc)
+    ref_out, ref_lse = oracle.paged_attn(q, k, v, table, seqlens, scale, c["causal"])
+    assert torch.allclose(out, ref_out, rtol=1e-12, atol=1e-12)
+    lse = lse.permute(0, 2, 1)
+    fin = torch.isfinite(ref_lse)
+    assert torch.equal(torch.isfinite(lse), fin)
+    assert torch.allclose(lse[fin], ref_lse[fin], rtol=1e-12, atol=1e-12)
