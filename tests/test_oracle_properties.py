@@ -136,3 +136,29 @@ def test_rank_shares_of_split_partials_fold_to_the_whole_context(c, split_tokens
     fin = torch.isfinite(ref_lse)
     assert torch.equal(torch.isfinite(lse), fin)
     assert torch.allclose(lse[fin], ref_lse[fin], rtol=1e-12, atol=1e-12)
+
+
+@settings(max_examples=30, deadline=None)
+@given(SHAPES)
+def test_backward_oracle_equals_autograd_on_random_problems(c):
+    """The fp64 backward oracle against torch autograd through the dense
+    definition, on the same random problems (rows that see no key included:
+    they get no gradient)."""
+    from test_oracle_bwd_pins import _dense_autograd
+
+    from paged_kv_decode_31_b200 import inputs as I
+
+    q, k, v, table, seqlens, scale = _problem(c)
+    Hq, Hkv, D = q.shape[2], k.shape[2], q.shape[3]
+    layout = "interleaved" if c["interleaved"] else "contiguous"
+    cache = I.PagedCache(k, v, (k, v), layout)
+    di = I.DecodeInputs(q, cache, table, seqlens, Hq, Hkv, D, scale, c["causal"])
+    g = torch.Generator().manual_seed(c["seed"] + 2)
+    dout = torch.randn(tuple(q.shape), generator=g).to(torch.bfloat16)
+    dq, dk, dv = oracle.paged_attn_bwd(q, k, v, table, seqlens, scale, c["causal"], dout)
+    rq, rk, rv = _dense_autograd(di, dout)
+    assert torch.allclose(dq, rq, rtol=1e-12, atol=1e-12)
+    L = rk.shape[1]
+    assert torch.allclose(dk[:, :L], rk, rtol=1e-12, atol=1e-12)
+    assert torch.allclose(dv[:, :L], rv, rtol=1e-12, atol=1e-12)
+    assert not (dk[:, L:].any() or dv[:, L:].any())
