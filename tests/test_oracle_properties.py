@@ -162,3 +162,34 @@ def test_backward_oracle_equals_autograd_on_random_problems(c):
     assert torch.allclose(dk[:, :L], rk, rtol=1e-12, atol=1e-12)
     assert torch.allclose(dv[:, :L], rv, rtol=1e-12, atol=1e-12)
     assert not (dk[:, L:].any() or dv[:, L:].any())
+
+
+@settings(max_examples=40, deadline=None)
+@given(SHAPES, st.lists(st.integers(0, 6), min_size=3, max_size=3))
+def test_packed_oracle_equals_each_request_alone(c, n_q):
+    """Packed queries: request b's n_b rows (rows cu[b] .. cu[b+1]-1 of the
+    packed q) are the last n_b positions of its context; each request's rows
+    equal the plain definition on that request alone, lse is [Hq, total_q],
+    and the final rows are the rows at cu[b+1]-1."""
+    q, k, v, table, seqlens, scale = _problem(c)
+    B, Hq, D = q.shape[0], q.shape[2], q.shape[3]
+    n_q = n_q[:B]
+    if sum(n_q) == 0:
+        n_q[0] = 1
+    g = torch.Generator().manual_seed(c["seed"] + 3)
+    qp = torch.randn(sum(n_q), Hq, D, generator=g).to(torch.bfloat16)
+    cu = torch.tensor([0] + list(torch.tensor(n_q).cumsum(0)), dtype=torch.int32)
+    out, lse, fin_out, fin_lse = oracle.paged_attn_varlen(qp, k, v, table, seqlens, cu, scale,
+                                                          c["causal"])
+    for b in range(B):
+        a, e = int(cu[b]), int(cu[b + 1])
+        if e == a:
+            continue
+        ro, rl = _definition(qp[a:e].unsqueeze(0), k, v, table[b:b + 1], seqlens[b:b + 1],
+                             scale, c["causal"])
+        assert torch.allclose(out[a:e], ro[0], rtol=1e-12, atol=1e-12)
+        fin = torch.isfinite(rl[0])
+        assert torch.equal(torch.isfinite(lse[:, a:e]), fin)
+        assert torch.allclose(lse[:, a:e][fin], rl[0][fin], rtol=1e-12, atol=1e-12)
+        assert torch.equal(fin_out[b], out[e - 1])
+        assert torch.equal(fin_lse[b], lse[:, e - 1])
