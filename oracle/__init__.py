@@ -46,7 +46,7 @@ def _load():
         p = ctypes.c_void_p
         i64 = ctypes.c_int64
         i32 = ctypes.c_int
-        lib.oracle_paged_attn.argtypes = [p, p, p, p, p, p, i64, p, i64, p,
+        lib.oracle_paged_attn.argtypes = [p, p, p, p, p, p, i64, p, i64, i32, p,
                                           i32, i32, i32, i32, i32, i32,
                                           ctypes.c_double, i32,
                                           i32, i32, i32, i32, p, p]
@@ -92,7 +92,9 @@ def paged_attn(q, k_cache, v_cache, block_table, seqlens, scale, causal,
     block_table:  [B, nblk] int32
     seqlens:      [B] int32, context length including the query tokens
     Returns (out [B, sq, Hq, D] fp64, lse [B, Hq, sq] fp64).  Rows outside
-    b_range x kvh_range are left as NaN.
+    b_range x kvh_range are left as NaN.  Raises RuntimeError (status 2) when
+    a selected sequence has a token past the table's nblk columns or a block
+    id outside [0, num_blocks).
     """
     lib = _load()
     B, sq, Hq, D = q.shape
@@ -109,7 +111,7 @@ def paged_attn(q, k_cache, v_cache, block_table, seqlens, scale, causal,
     h0, h1 = kvh_range if kvh_range is not None else (0, Hkv)
     rc = lib.oracle_paged_attn(
         qb.data_ptr(), _strides3(q), kb.data_ptr(), _strides3(k_cache),
-        vb.data_ptr(), _strides3(v_cache), nblocks, bt.data_ptr(), bt.stride(0),
+        vb.data_ptr(), _strides3(v_cache), nblocks, bt.data_ptr(), bt.stride(0), bt.shape[1],
         sl.data_ptr(), B, sq, Hq, Hkv, D, bs, float(scale), int(bool(causal)),
         b0, b1, h0, h1, out.data_ptr(), lse.data_ptr())
     if rc != 0:

@@ -44,8 +44,9 @@
  * like the in-place cache's put + advance in jouleclaw's kv_cache_inplace.rs.
  *
  * Numbers: bf16 inputs are widened exactly to fp64; all arithmetic is fp64.
- * Parallelism: OpenMP over (batch, KV head) tasks; each task gathers its own
- * dense K/V, so results do not depend on the thread count.
+ * Parallelism: OpenMP over query rows (sequence, query head, query token);
+ * each row reads its keys and values through the table itself, so results do
+ * not depend on the thread count, and one sequence can use every host core.
  */
 #include <math.h>
 #include <stdint.h>
@@ -70,24 +71,23 @@ static double bf16_to_f64(uint16_t h)
     return (double)f;
 }
 
-/* Step 1: gather the first n tokens of one KV head of one sequence into a
- * dense row-major [n][D] fp64 array.  Returns ORACLE_ERR_BLOCK if the table
- * names a block outside [0, num_blocks). */
-static int gather_head(const uint16_t *cache, const int64_t st[3],
-                       const int32_t *table_row, int64_t num_blocks,
-                       int block_size, int kvh, int D, int n, double *dense)
+/* Step 1, the dense gather, one token at a time: the row of token j of one
+ * sequence at KV head kvh in a cache view with element strides st = (block,
+ * slot, head).  Token j lives in block table_row[j / block_size], slot
+ * j % block_size.  Returns NULL when the table has no column for j (column
+ * >= max_blocks_per_seq) or names a block outside [0, num_blocks). */
+static const uint16_t *token_row(const uint16_t *cache, const int64_t st[3],
+                                 const int32_t *table_row, int max_blocks_per_seq,
+                                 int64_t num_blocks, int block_size, int kvh, int j)
 {
-    for (int j = 0; j < n; ++j) {
-        int32_t blk = table_row[j / block_size];
-        if (blk < 0 || (int64_t)blk >= num_blocks)
-            return ORACLE_ERR_BLOCK;
-        const uint16_t *src = cache + (int64_t)blk * st[0]
-                                    + (int64_t)(j % block_size) * st[1]
-                                    + (int64_t)kvh * st[2];
-        for (int d = 0; d < D; ++d)
-            dense[(int64_t)j * D + d] = bf16_to_f64(src[d]);
-    }
-    return ORACLE_OK;
+    const int col = j / block_size;
+    if (col >= max_blocks_per_seq)
+        return NULL;
+    const int32_t blk = table_row[col];
+    if (blk < 0 || (int64_t)blk >= num_blocks)
+        return NULL;
+    return cache + (int64_t)blk * st[0] + (int64_t)(j % block_size) * st[1]
+                 + (int64_t)kvh * st[2];
 }
 
 /*
@@ -97,97 +97,105 @@ static int gather_head(const uint16_t *cache, const int64_t st[3],
  *   q        bf16 bits, element strides q_st = (batch, token, head), d-stride 1
  *   k_cache  bf16 bits, element strides k_st = (block, slot, head), d-stride 1
  *   v_cache  same with v_st
- *   block_table int32 [batch][bt_stride]
+ *   block_table int32 [batch][bt_stride]; only the first max_blocks_per_seq
+ *            columns of a row describe that sequence's blocks
  *   seqlens  int32 [batch] (context length including the query tokens)
  *   out      fp64 [batch][seqlen_q][Hq][D] (only the selected rows written)
  *   lse      fp64 [batch][Hq][seqlen_q]
+ *
+ * Returns ORACLE_ERR_BLOCK, with nothing written, if a selected sequence has
+ * a token whose table column is at or past max_blocks_per_seq or whose block
+ * lies outside [0, num_blocks): the table does not describe that context.
+ * Each query row (b, h, i) is an independent task; the work is spread over
+ * the threads by row, and a row's arithmetic does not depend on the thread
+ * count.
  */
 int oracle_paged_attn(const uint16_t *q, const int64_t q_st[3],
                       const uint16_t *k_cache, const int64_t k_st[3],
                       const uint16_t *v_cache, const int64_t v_st[3],
                       int64_t num_blocks, const int32_t *block_table,
-                      int64_t bt_stride, const int32_t *seqlens,
+                      int64_t bt_stride, int max_blocks_per_seq,
+                      const int32_t *seqlens,
                       int batch, int seqlen_q, int Hq, int Hkv, int D,
                       int block_size, double scale, int causal,
                       int b_begin, int b_end, int kvh_begin, int kvh_end,
                       double *out, double *lse)
 {
     if (batch <= 0 || seqlen_q <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 ||
-        block_size <= 0 || Hq % Hkv != 0 || b_begin < 0 || b_end > batch ||
+        block_size <= 0 || max_blocks_per_seq <= 0 || bt_stride < max_blocks_per_seq ||
+        Hq % Hkv != 0 || b_begin < 0 || b_end > batch ||
         kvh_begin < 0 || kvh_end > Hkv)
         return ORACLE_ERR_ARG;
     const int G = Hq / Hkv;
     const int nb = b_end - b_begin, nh = kvh_end - kvh_begin;
-    const int ntask = nb * nh;
-    int status = ORACLE_OK;
 
-#pragma omp parallel for schedule(dynamic, 1)
-    for (int task = 0; task < ntask; ++task) {
-        const int b = b_begin + task / nh;
-        const int kvh = kvh_begin + task % nh;
+    /* step 1's bounds: every token of every selected sequence has a block */
+    for (int b = b_begin; b < b_end; ++b) {
         const int n = seqlens[b] > 0 ? seqlens[b] : 0;
-        double *K = NULL, *V = NULL, *s = NULL;
-        if (n > 0) {
-            K = (double *)malloc(sizeof(double) * (size_t)n * D);
-            V = (double *)malloc(sizeof(double) * (size_t)n * D);
-            s = (double *)malloc(sizeof(double) * (size_t)n);
-            if (!K || !V || !s) {
-#pragma omp critical
-                status = ORACLE_ERR_NOMEM;
-                free(K); free(V); free(s);
-                continue;
-            }
-            const int32_t *row = block_table + (int64_t)b * bt_stride;
-            int e1 = gather_head(k_cache, k_st, row, num_blocks, block_size, kvh, D, n, K);
-            int e2 = gather_head(v_cache, v_st, row, num_blocks, block_size, kvh, D, n, V);
-            if (e1 != ORACLE_OK || e2 != ORACLE_OK) {
-#pragma omp critical
-                status = ORACLE_ERR_BLOCK;
-                free(K); free(V); free(s);
-                continue;
-            }
+        const int32_t *row = block_table + (int64_t)b * bt_stride;
+        for (int j = 0; j < n; j += block_size)
+            if (!token_row(k_cache, k_st, row, max_blocks_per_seq, num_blocks,
+                           block_size, 0, j))
+                return ORACLE_ERR_BLOCK;
+    }
+
+    const int64_t ntask = (int64_t)nb * nh * G * seqlen_q;
+    int status = ORACLE_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t task = 0; task < ntask; ++task) {
+        const int i = (int)(task % seqlen_q);
+        const int g = (int)((task / seqlen_q) % G);
+        const int kvh = kvh_begin + (int)((task / ((int64_t)seqlen_q * G)) % nh);
+        const int b = b_begin + (int)(task / ((int64_t)seqlen_q * G * nh));
+        const int h = kvh * G + g;                             /* step 2 */
+        const int n = seqlens[b] > 0 ? seqlens[b] : 0;
+        const int32_t *row = block_table + (int64_t)b * bt_stride;
+        double *o = out + (((int64_t)b * seqlen_q + i) * Hq + h) * D;
+        double *ls = lse + ((int64_t)b * Hq + h) * seqlen_q + i;
+        const int pos = n - seqlen_q + i;                      /* step 4 */
+        int nvis = n;                                          /* step 3 */
+        if (causal && pos + 1 < nvis)
+            nvis = pos + 1;
+        if (nvis <= 0) {                                       /* step 6 */
+            for (int d = 0; d < D; ++d)
+                o[d] = 0.0;
+            *ls = -INFINITY;
+            continue;
         }
-        for (int g = 0; g < G; ++g) {
-            const int h = kvh * G + g;                       /* step 2 */
-            for (int i = 0; i < seqlen_q; ++i) {
-                double *o = out + (((int64_t)b * seqlen_q + i) * Hq + h) * D;
-                double *ls = lse + ((int64_t)b * Hq + h) * seqlen_q + i;
-                const int pos = n - seqlen_q + i;              /* step 4 */
-                int nvis = n;                                  /* step 3 */
-                if (causal && pos + 1 < nvis)
-                    nvis = pos + 1;
-                if (nvis <= 0) {                               /* step 6 */
-                    for (int d = 0; d < D; ++d)
-                        o[d] = 0.0;
-                    *ls = -INFINITY;
-                    continue;
-                }
-                const uint16_t *qr = q + (int64_t)b * q_st[0] + (int64_t)i * q_st[1]
-                                       + (int64_t)h * q_st[2];
-                double m = -INFINITY;                          /* step 5 */
-                for (int j = 0; j < nvis; ++j) {
-                    double acc = 0.0;
-                    for (int d = 0; d < D; ++d)
-                        acc += bf16_to_f64(qr[d]) * K[(int64_t)j * D + d];
-                    s[j] = scale * acc;
-                    if (s[j] > m)
-                        m = s[j];
-                }
-                double l = 0.0;
-                for (int d = 0; d < D; ++d)
-                    o[d] = 0.0;
-                for (int j = 0; j < nvis; ++j) {
-                    const double p = exp(s[j] - m);
-                    l += p;
-                    for (int d = 0; d < D; ++d)
-                        o[d] += p * V[(int64_t)j * D + d];
-                }
-                for (int d = 0; d < D; ++d)
-                    o[d] /= l;
-                *ls = m + log(l);
-            }
+        double *s = (double *)malloc(sizeof(double) * (size_t)nvis);
+        if (!s) {
+#pragma omp critical
+            status = ORACLE_ERR_NOMEM;
+            continue;
         }
-        free(K); free(V); free(s);
+        const uint16_t *qr = q + (int64_t)b * q_st[0] + (int64_t)i * q_st[1]
+                               + (int64_t)h * q_st[2];
+        double m = -INFINITY;                                  /* step 5 */
+        for (int j = 0; j < nvis; ++j) {
+            const uint16_t *kr = token_row(k_cache, k_st, row, max_blocks_per_seq,
+                                           num_blocks, block_size, kvh, j);
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d)
+                acc += bf16_to_f64(qr[d]) * bf16_to_f64(kr[d]);
+            s[j] = scale * acc;
+            if (s[j] > m)
+                m = s[j];
+        }
+        double l = 0.0;
+        for (int d = 0; d < D; ++d)
+            o[d] = 0.0;
+        for (int j = 0; j < nvis; ++j) {
+            const uint16_t *vr = token_row(v_cache, v_st, row, max_blocks_per_seq,
+                                           num_blocks, block_size, kvh, j);
+            const double p = exp(s[j] - m);
+            l += p;
+            for (int d = 0; d < D; ++d)
+                o[d] += p * bf16_to_f64(vr[d]);
+        }
+        for (int d = 0; d < D; ++d)
+            o[d] /= l;
+        *ls = m + log(l);
+        free(s);
     }
     return status;
 }
@@ -232,8 +240,7 @@ int oracle_kv_append(const uint16_t *k_new, const int64_t kn_st[3],
     return ORACLE_OK;
 }
 
-/* Cap the number of OpenMP threads (each task holds a dense fp64 copy of one
- * KV head of one sequence, so the cap bounds host memory). */
+/* Cap the number of OpenMP threads the oracle runs on (n <= 0: no change). */
 void oracle_set_num_threads(int n)
 {
 #ifdef _OPENMP

@@ -359,3 +359,28 @@ def test_bad_block_id_is_an_error():
     di.block_table[0, 1] = di.cache.num_blocks + 5
     with pytest.raises(RuntimeError):
         run_oracle(di)
+
+
+def test_table_narrower_than_the_context_is_an_error():
+    # Column j of a table row holds tokens [j * bs, (j + 1) * bs) (aiter d293d61,
+    # _generate_interleaved_block_kvcache: randperm reshaped to (batch, nblocks)).
+    # A table whose row is narrower than seqlens[b] / bs does not describe the
+    # context: the oracle refuses instead of reading the next row or past the
+    # end of the tensor.  Here the last sequence's context needs 3 columns, the
+    # table (a column slice, so the row stride stays wider) has 2.
+    di = I.p2_case(2, 1, 40, 2, 1, 64, 16, causal=False, seed=17, seqlens=[32, 40])
+    narrow = I.DecodeInputs(di.q, di.cache, di.block_table[:, :2], di.seqlens, di.Hq,
+                            di.Hkv, di.D, di.scale, di.causal)
+    with pytest.raises(RuntimeError, match="status 2"):
+        run_oracle(narrow)
+    # the same table with both contexts inside its two columns is accepted,
+    # and equals the wide table's result for that sequence bit for bit
+    fits = I.DecodeInputs(di.q, di.cache, di.block_table[:, :2],
+                          torch.tensor([32, 20], dtype=torch.int32), di.Hq, di.Hkv, di.D,
+                          di.scale, di.causal)
+    wide = I.DecodeInputs(di.q, di.cache, di.block_table,
+                          torch.tensor([32, 20], dtype=torch.int32), di.Hq, di.Hkv, di.D,
+                          di.scale, di.causal)
+    o1, l1 = run_oracle(fits)
+    o2, l2 = run_oracle(wide)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
