@@ -98,6 +98,11 @@ extern "C" {
 #define PKV_DEVERR_QUERY_LEN 8   /* packed call: a sequence has more than max_seqlen_q
                                     queries (or cu_seqlens_q decreases); rows past the
                                     bound are not written */
+#define PKV_DEVERR_SEQ_LEN 16    /* a sequence's seqlens[b] exceeds max_seqlen_k: the
+                                    split grid (or the backward's key tiles) was sized
+                                    from max_seqlen_k, so keys past its last split (key
+                                    tile) are not read and the result is not that
+                                    context's attention */
 
 /*
  * pkv_kv_append: for every sequence b and new token t < n_new, copy the bf16
@@ -129,7 +134,9 @@ int pkv_kv_append(const void *k_new, const int64_t kn_strides[3],
  *   num_blocks   number of blocks in the cache (table entries are checked against it)
  *   seqlens      [batch] int32 device, context lengths incl. the query tokens
  *   max_seqlen_k host upper bound of seqlens (sizes the split grid); a sequence
- *                longer than it is an error of the caller (its tail is ignored)
+ *                longer than it is an error of the caller: it sets
+ *                PKV_DEVERR_SEQ_LEN in *err, and keys past the grid's last split
+ *                (ceil(max_seqlen_k / PKV_SPLIT_TOKENS) splits) are not read
  *   scale        softmax scale applied to q.k (e.g. 1/sqrt(D))
  *   causal       0 or 1 (bottom-right aligned)
  *   out          [batch, seqlen_q, Hq, D] bf16, element strides out_strides = (b, s, h)
@@ -283,7 +290,10 @@ int pkv_kv_append_varlen(const void *k_new, const int64_t kn_strides[2],
  * into `partials` (>= pkv_partials_size(batch, seqlen_q, Hq, D,
  * n_splits_local) bytes, 16-byte aligned) the fp32 partials (m, l, acc[D]) of
  * every (row, local split): acc [rows][n_local][D] (256-byte padded), then
- * (m, l) [rows][n_local][2], rows = batch * seqlen_q * Hq.  Partials of
+ * (m, l) [rows][n_local][2], rows = batch * seqlen_q * Hq in (b, i, h) order;
+ * m is the split's max score in base-2 units (scale * log2(e) * q.k), l the
+ * sum of 2^(s - m) and acc the sum of 2^(s - m) v over the split's visible
+ * keys (s in the same units).  Partials of
  * (row, split) pairs the row does not reach are left unwritten (the merge
  * never reads them).  Errors as pkv_paged_decode_attn (PKV_ERR_WORKSPACE if
  * partials is too small).

@@ -23,6 +23,7 @@ DEVERR_BAD_BLOCK = 1
 DEVERR_TABLE_WIDTH = 2
 DEVERR_TIMEOUT = 4
 DEVERR_QUERY_LEN = 8
+DEVERR_SEQ_LEN = 16
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64

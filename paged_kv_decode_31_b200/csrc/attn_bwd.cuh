@@ -70,6 +70,11 @@ struct BwdPrepParams {
   const float *lse;  // [batch, Hq, seqlen_q]
   int batch, seqlen_q, Hq, D;
   float *row_d, *row_lse2;
+  // a context longer than max_seqlen_k (the host bound that sized the key
+  // tiles; keys past it are not read) is flagged once per sequence
+  const int32_t *seqlens;
+  int max_seqlen_k;
+  int32_t *err;
 };
 
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ BwdPrepParams p) {
@@ -105,6 +110,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ B
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
   if (lane == 0) {
+    if (h == 0 && i == 0 && p.err && __ldg(p.seqlens + b) > p.max_seqlen_k)
+      atomicOr(p.err, kErrSeqLen);
     p.row_d[row] = acc;
     const float l = p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.seqlen_q + i];
     p.row_lse2[row] = __fmul_rn(l, 1.4426950408889634f);

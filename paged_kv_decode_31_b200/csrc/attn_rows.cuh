@@ -449,7 +449,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     bool stop = false;
     for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
       const Unit x = unit_at<kRowsPerTile>(p, u);
-      if (t == 0) check_query_count(p, x);
+      if (t == 0) check_sequence(p, x);
       if (x.n_tiles == 0) {
         // rows that see no key: out = 0, lse = -inf (written by the unit of
         // split 0; the merge skips rows of at most one split)

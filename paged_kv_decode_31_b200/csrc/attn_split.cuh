@@ -44,23 +44,17 @@
 
 #include <cuda_bf16.h>
 
+#include "contract.cuh"
 #include "ptx.cuh"
 
 namespace pkv {
 
-constexpr int kSplitTokens = 4096;
-constexpr int kTileTokens = 128;
 constexpr int kThreads = 480;  // 15 warps
 // warps 0-3 and 4-7: softmax warpgroups (even / odd tiles of the CTA's sequence)
 constexpr int kCorrWarp0 = 8;  // warps 8-11: correction + epilogue warpgroup
 constexpr int kKWarp = 12;     // K producer (+ Q staging)
 constexpr int kVWarp = 13;     // V producer
 constexpr int kMmaWarp = 14;   // MMA issuer + TMEM owner
-
-constexpr int kErrBadBlock = 1;
-constexpr int kErrTableWidth = 2;
-constexpr int kErrTimeout = 4;
-constexpr int kErrQueryLen = 8;
 
 struct AttnParams {
   const __nv_bfloat16 *q;
@@ -75,6 +69,7 @@ struct AttnParams {
   int box_slots;        // cache rows per TMA box = min(block_size, 128)
   int map_head_first;   // tensor-map dim order (D, Hkv, slot, block) vs (D, slot, Hkv, block)
   int n_row_tiles, n_splits, n_units;
+  int max_seqlen_k;     // host bound on seqlens (n_splits = ceil(max_seqlen_k / 4096))
   float cscale;         // softmax scale * log2(e)
   int causal;
   float *ws_acc;        // [rows][n_splits][D]
@@ -265,12 +260,18 @@ __device__ __forceinline__ int64_t lse_index(const AttnParams &p, const Unit &x,
                 : (static_cast<int64_t>(x.b) * p.Hq + h) * p.seqlen_q + i;
 }
 
-// Sequences whose query count exceeds the host bound are flagged once (by
-// the unit of their first row tile, KV head 0, split 0).
-__device__ __forceinline__ void check_query_count(const AttnParams &p, const Unit &x) {
-  if (p.cu_q && x.rt == 0 && x.kvh == 0 && x.s == 0 && p.err) {
-    const int n = __ldg(p.cu_q + x.b + 1) - __ldg(p.cu_q + x.b);
-    if (n < 0 || n > p.seqlen_q) atomicOr(p.err, kErrQueryLen);
+// Caller errors the host cannot see, flagged once per sequence (by the unit
+// of its first row tile, KV head 0, split 0): a packed sequence with more
+// queries than the host bound, and a context longer than max_seqlen_k (the
+// host bound that sized the split grid; keys past the grid's last split are
+// not read).
+__device__ __forceinline__ void check_sequence(const AttnParams &p, const Unit &x) {
+  if (x.rt == 0 && x.kvh == 0 && x.s == 0 && p.err) {
+    if (p.cu_q) {
+      const int n = __ldg(p.cu_q + x.b + 1) - __ldg(p.cu_q + x.b);
+      if (n < 0 || n > p.seqlen_q) atomicOr(p.err, kErrQueryLen);
+    }
+    if (!p.part_only && x.seqlen > p.max_seqlen_k) atomicOr(p.err, kErrSeqLen);
   }
 }
 
@@ -754,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool stop = false;
     for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
       const Unit x = unit_at<N>(p, u);
-      if (t == 0) check_query_count(p, x);
+      if (t == 0) check_sequence(p, x);
       if (x.n_tiles == 0) continue;
 #pragma unroll
       for (int c = 0; c < N; ++c) acc[c] = 0.f;

@@ -17,6 +17,7 @@
 
 #include <cuda_bf16.h>
 
+#include "contract.cuh"
 #include "packed.cuh"
 #include "ptx.cuh"
 
@@ -104,7 +105,7 @@ __global__ void __launch_bounds__(WIDE ? D : 32 * kMergeRowsPerBlock)
   int lim = n;
   if (p.causal) lim = min(lim, n - nq + i + 1);
   lim = max(lim, 0);
-  const int n_s = min((lim + 4095) / 4096, p.n_splits);
+  const int n_s = min(splits_for(lim), p.n_splits);
   if (p.skip_single && nq >= p.skip_min_nq && n_s <= 1) return;
   const int d0 = lane * V;
   const float NEG_INF = __int_as_float(0xff800000);

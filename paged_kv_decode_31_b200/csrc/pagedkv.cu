@@ -24,6 +24,7 @@ static_assert(PKV_DEVERR_BAD_BLOCK == pkv::kErrBadBlock, "error bits");
 static_assert(PKV_DEVERR_TABLE_WIDTH == pkv::kErrTableWidth, "error bits");
 static_assert(PKV_DEVERR_TIMEOUT == pkv::kErrTimeout, "error bits");
 static_assert(PKV_DEVERR_QUERY_LEN == pkv::kErrQueryLen, "error bits");
+static_assert(PKV_DEVERR_SEQ_LEN == pkv::kErrSeqLen, "error bits");
 
 namespace {
 
@@ -414,6 +415,7 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   p.n_row_tiles = static_cast<int>(RT);
   p.n_splits = static_cast<int>(S);
   p.n_units = static_cast<int>(units);
+  p.max_seqlen_k = max_seqlen_k;
   p.cscale = scale * 1.4426950408889634f;  // host IEEE multiply, one rounding
   p.causal = causal ? 1 : 0;
   p.ws_acc = ws_acc;
@@ -789,6 +791,9 @@ int pkv_paged_prefill_attn_bwd(const void *q, const int64_t q_strides[3], const 
   pp.D = D;
   pp.row_d = row_d;
   pp.row_lse2 = row_lse2;
+  pp.seqlens = seqlens;
+  pp.max_seqlen_k = max_seqlen_k;
+  pp.err = err;
   pkv::bwd_prep_kernel<<<static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, s>>>(pp);
   if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
 

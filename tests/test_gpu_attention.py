@@ -178,3 +178,33 @@ def test_short_contexts_stay_in_bounds_over_seeds(entry):
         d_out, _ = assert_close_to_oracle(out, lse, ref_out, ref_lse)
         worst = max(worst, d_out)
     assert worst <= 1e-2
+
+
+@pytest.mark.parametrize("sq", [1, 64])          # transposed kernel / row-major kernel
+def test_context_longer_than_max_seqlen_k_sets_the_error_flag(sq):
+    """max_seqlen_k sizes the split grid on the host; a sequence longer than
+    it is a caller error the device reports (PKV_DEVERR_SEQ_LEN) instead of
+    returning a silently truncated attention.  A bound that covers every
+    context leaves the error word at zero."""
+    di = I.p2_case(2, sq, 9000, 16, 4, 128, 16, causal=True, layout="contiguous", seed=26,
+                   seqlens=[9000, 3000])
+    d = di.to("cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for fn in (pkv.paged_decode_attn, pkv.paged_prefill_attn):
+        err.zero_()
+        fn(d.q, d.cache.k, d.cache.v, d.block_table, d.seqlens, max_seqlen_k=5000,
+           scale=di.scale, causal=True, err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == pkv.binding.DEVERR_SEQ_LEN
+        err.zero_()
+        out, lse = fn(d.q, d.cache.k, d.cache.v, d.block_table, d.seqlens, max_seqlen_k=9000,
+                      scale=di.scale, causal=True, err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+    # the backward sizes its key tiles from the same bound and flags the same way
+    dout = torch.randn(out.shape, dtype=torch.bfloat16, device="cuda")
+    err.zero_()
+    pkv.paged_prefill_attn_bwd(d.q, d.cache.k, d.cache.v, d.block_table, d.seqlens, out, lse, dout,
+                               max_seqlen_k=5000, scale=di.scale, causal=True, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == pkv.binding.DEVERR_SEQ_LEN

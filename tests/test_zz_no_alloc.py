@@ -64,12 +64,25 @@ def test_static_workspace_rejects_problems_beyond_its_size():
             q, di.cache.k, di.cache.v, di.block_table.expand(64, -1).contiguous(),
             di.seqlens.expand(64).contiguous(), max_seqlen_k=16384, out=torch.empty_like(q),
             lse=torch.empty(64, 32, 64, dtype=torch.float32, device="cuda"))
-    # the C entry point itself returns PKV_ERR_WORKSPACE and launches nothing
+    # the C entry point itself returns PKV_ERR_WORKSPACE and launches nothing;
+    # every pointer is a real device buffer of the sizes passed, so even a call
+    # that got past the size check could only touch memory it owns
     import ctypes
     fn = binding.lib().pkv_paged_decode_attn_static_ws
     assert fn.argtypes  # set by the binding call above
-    st = (ctypes.c_int64 * 3)(64 * 32 * 128, 32 * 128, 128)
-    kst = (ctypes.c_int64 * 3)(16 * 2 * 128, 2 * 128, 128)
-    rc = fn(0x10000, st, 0x20000, kst, 0x30000, kst, 64, 0x40000, 1024, 1024, 0x50000, 16384,
-            64, 64, 32, 2, 128, 16, 0.088, 0, 0x60000, st, 0x70000, None, None)
+    table = di.block_table.expand(64, -1).contiguous()
+    seqlens = di.seqlens.expand(64).contiguous()
+    out = torch.empty_like(q)
+    lse = torch.empty(64, 32, 64, dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = (ctypes.c_int64 * 3)(*q.stride()[:3])
+    kst = (ctypes.c_int64 * 3)(*di.cache.k.stride()[:3])
+    vst = (ctypes.c_int64 * 3)(*di.cache.v.stride()[:3])
+    ost = (ctypes.c_int64 * 3)(*out.stride()[:3])
+    rc = fn(q.data_ptr(), st, di.cache.k.data_ptr(), kst, di.cache.v.data_ptr(), vst,
+            di.cache.k.shape[0], table.data_ptr(), table.stride(0), table.shape[1],
+            seqlens.data_ptr(), 16384, 64, 64, 32, 2, 128, 16, 0.088, 0, out.data_ptr(), ost,
+            lse.data_ptr(), err.data_ptr(), None)
+    torch.cuda.synchronize()
     assert rc == 2  # PKV_ERR_WORKSPACE
+    assert int(err.item()) == 0
