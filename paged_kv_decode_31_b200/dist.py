@@ -69,12 +69,39 @@ def cp_split_share(max_seqlen_k: int, rank: int, world: int) -> Tuple[int, int]:
     return rank * n_local, n_local
 
 
+def partials_bytes(batch: int, seqlen_q: int, Hq: int, D: int, n_splits_local: int) -> int:
+    """Bytes of one rank's partial buffer (what pkv_partials_size returns),
+    computed on the host without the library: see partials_views."""
+    rows = batch * seqlen_q * Hq
+    return -(-(rows * n_splits_local * D * 4) // 256) * 256 + rows * n_splits_local * 2 * 4
+
+
+def partials_views(buf: torch.Tensor, batch: int, seqlen_q: int, Hq: int, D: int,
+                   n_splits_local: int) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The two arrays inside one rank's partial buffer (a uint8 tensor of
+    partials_size(batch, seqlen_q, Hq, D, n_splits_local) bytes, the layout
+    pkv_paged_attn_partials writes and pkv_merge_partials reads): acc fp32
+    [rows, n_local, D], then, after padding to a multiple of 256 bytes, (m, l)
+    fp32 [rows, n_local, 2], rows = batch * seqlen_q * Hq in (b, i, h) order.
+    m is the split's max score in base-2 units (scale * log2(e) * q.k), l the
+    sum of 2^(s - m) and acc the sum of 2^(s - m) v over the split's visible
+    keys.  Views, not copies; usable on any device."""
+    rows = batch * seqlen_q * Hq
+    acc_bytes = -(-(rows * n_splits_local * D * 4) // 256) * 256
+    need = partials_bytes(batch, seqlen_q, Hq, D, n_splits_local)
+    flat = buf.reshape(-1)
+    if flat.dtype != torch.uint8 or flat.numel() < need:
+        raise ValueError(f"partial buffer must be uint8 with at least {need} bytes")
+    acc = flat[:rows * n_splits_local * D * 4].view(torch.float32).view(rows, n_splits_local, D)
+    ml = flat[acc_bytes:need].view(torch.float32).view(rows, n_splits_local, 2)
+    return acc, ml
+
+
 def cp_exchange(partials: torch.Tensor, group=None) -> torch.Tensor:
     """All-gather every rank's partial buffer (equal sizes) side by side, rank
-    0's first: the layout pkv_merge_partials reads."""
+    0's first: the layout pkv_merge_partials reads.  Every rank takes this
+    collective step, whatever the world size."""
     world = dist.get_world_size(group)
-    if world == 1:
-        return partials
     flat = partials.reshape(-1)
     if dist.get_backend(group) == "nccl":
         out = torch.empty(world * flat.numel(), dtype=flat.dtype, device=flat.device)

@@ -59,50 +59,62 @@ def test_shard_sizes_and_rate():
 
 
 def _cp_worker(rank, world, port, q):
-    """One CP rank on CPU: fp64 partials of its split share (the oracle's), the
-    gloo exchange of the packed buffers, then the ascending fold over all
-    global splits from the gathered blocks."""
+    """One CP rank on CPU: fp64 partials of its split share (the oracle's),
+    written into the library's partial-buffer layout (dist.partials_views:
+    fp32 acc [rows][n_local][D] padded to 256 bytes, then (m, l) with m in
+    base-2 units), the product exchange (dist.cp_exchange over gloo), then the
+    merge's ascending fold over all global splits read back out of the
+    gathered rank blocks through the same views."""
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
     import math
     import torch
-    import torch.distributed as dist
     import oracle
     from paged_kv_decode_31_b200 import inputs as I
     pdist.init("gloo", timeout_s=60)
     split = 64   # small splits so a short context spans several
-    di = I.p2_case(2, 3, 300, 4, 2, 64, 16, causal=True, seed=31, seqlens=[300, 141])
+    B, sq, Hq, Hkv, D = 2, 3, 4, 2, 64
+    di = I.p2_case(B, sq, 300, Hq, Hkv, D, 16, causal=True, seed=31, seqlens=[300, 141])
     S = -(-300 // split)
     n_local = -(-S // world)
     begin = rank * n_local
     m, l, acc = oracle.split_partials(di.q, di.cache.k, di.cache.v, di.block_table, di.seqlens,
                                       di.scale, True, begin, n_local, split_tokens=split)
-    block = torch.cat([acc.reshape(-1), m.reshape(-1), l.reshape(-1)])
-    gathered = pdist.cp_exchange(block, None).reshape(world, -1)
-    B, sq, Hq, D = di.q.shape
-    na = B * sq * Hq * n_local * D
-    nm = B * sq * Hq * n_local
+    rows = B * sq * Hq
+    rank_bytes = pdist.partials_bytes(B, sq, Hq, D, n_local)
+    buf = torch.full((rank_bytes,), 0xFF, dtype=torch.uint8)   # unreached partials: garbage
+    acc_v, ml_v = pdist.partials_views(buf, B, sq, Hq, D, n_local)
+    log2e = 1.0 / math.log(2.0)
+    reached = torch.isfinite(m.reshape(rows, n_local))
+    acc_v[reached] = acc.reshape(rows, n_local, D)[reached].float()
+    ml_v[..., 0][reached] = (m.reshape(rows, n_local)[reached] * log2e).float()
+    ml_v[..., 1][reached] = l.reshape(rows, n_local)[reached].float()
+    gathered = pdist.cp_exchange(buf, None)
+    assert gathered.dtype == torch.uint8 and gathered.numel() == world * rank_bytes
+    views = [pdist.partials_views(gathered[r * rank_bytes:(r + 1) * rank_bytes], B, sq, Hq, D,
+                                  n_local) for r in range(world)]
     out = torch.zeros(B, sq, Hq, D, dtype=torch.float64)
     lse = torch.zeros(B, Hq, sq, dtype=torch.float64)
     for b in range(B):
+        n = int(di.seqlens[b])
         for i in range(sq):
+            lim = max(min(n, n - sq + i + 1), 0)
+            n_s = -(-lim // split)            # the merge reads splits [0, n_s) only
             for h in range(Hq):
+                row = (b * sq + i) * Hq + h
                 M, Lsum, A = -math.inf, 0.0, torch.zeros(D, dtype=torch.float64)
-                for s in range(world * n_local):          # ascending global split
+                for s in range(n_s):          # ascending global split
                     r, ls = divmod(s, n_local)
-                    blk = gathered[r]
-                    idx = ((b * sq + i) * Hq + h) * n_local + ls
-                    ms, lsv = float(blk[na + idx]), float(blk[na + nm + idx])
-                    if ms == -math.inf:
-                        continue
-                    a_s = blk[idx * D:(idx + 1) * D]
+                    a_v, m_v = views[r]
+                    ms, lsv = float(m_v[row, ls, 0]), float(m_v[row, ls, 1])
                     Mn = max(M, ms)
-                    ca, cs = math.exp(M - Mn) if M > -math.inf else 0.0, math.exp(ms - Mn)
+                    ca = 2.0 ** (M - Mn) if M > -math.inf else 0.0
+                    cs = 2.0 ** (ms - Mn)
                     Lsum = Lsum * ca + lsv * cs
-                    A = A * ca + a_s * cs
+                    A = A * ca + a_v[row, ls].double() * cs
                     M = Mn
                 out[b, i, h] = A / Lsum if Lsum > 0 else 0.0
-                lse[b, h, i] = M + math.log(Lsum) if Lsum > 0 else -math.inf
+                lse[b, h, i] = (M + math.log2(Lsum)) * math.log(2.0) if Lsum > 0 else -math.inf
     ro, rl = oracle.paged_attn(di.q, di.cache.k, di.cache.v, di.block_table, di.seqlens,
                                di.scale, True)
     ok_out = float((out - ro).abs().max())
@@ -110,16 +122,17 @@ def _cp_worker(rank, world, port, q):
     ok_lse = float((lse[fin] - rl[fin]).abs().max())
     same_empty = bool(torch.equal(torch.isneginf(lse), torch.isneginf(rl)))
     shares = (begin, n_local)
-    dist.barrier()
-    dist.destroy_process_group()
-    q.put((rank, ok_out, ok_lse, same_empty, shares))
+    torch.distributed.barrier()
+    torch.distributed.destroy_process_group()
+    q.put((rank, ok_out, ok_lse, same_empty, shares, rank_bytes))
 
 
 @pytest.mark.parametrize("world", [2, 3])
 def test_context_parallel_exchange_and_ascending_merge_with_gloo(world):
-    """The split shares cover every split once, in rank order; the exchanged
-    blocks land side by side; folding them in ascending global split order
-    reproduces the whole-context attention (fp64, CPU)."""
+    """The split shares cover every split once, in rank order; partial buffers
+    in the library's layout go through the product exchange and land side by
+    side; folding them in ascending global split order, read through the same
+    layout, reproduces the whole-context attention (fp32 partials: 1e-5)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -132,10 +145,30 @@ def test_context_parallel_exchange_and_ascending_merge_with_gloo(world):
         assert p.exitcode == 0
     S = -(-300 // 64)
     n_local = -(-S // world)
-    for rank, d_out, d_lse, same_empty, shares in res:
+    for rank, d_out, d_lse, same_empty, shares, rank_bytes in res:
         assert shares == (rank * n_local, n_local)
-        assert d_out < 1e-12 and d_lse < 1e-12 and same_empty
+        assert d_out < 1e-5 and d_lse < 1e-5 and same_empty
     assert pdist.cp_split_share(20000, 2, 3) == (4, 2)
+
+
+def test_partials_views_match_the_library_size():
+    """dist.partials_views describes the buffer pkv_partials_size sizes: the
+    (m, l) block ends exactly at the library's byte count, after an acc block
+    padded to 256 bytes."""
+    import torch
+    from paged_kv_decode_31_b200 import binding
+    from paged_kv_decode_31_b200 import build as pkv_build
+    pkv_build.build()
+    for (B, sq, Hq, D, n) in [(2, 3, 4, 64, 3), (4, 1, 32, 128, 32), (1, 7, 6, 64, 1)]:
+        need = binding.partials_size(B, sq, Hq, D, n)
+        assert pdist.partials_bytes(B, sq, Hq, D, n) == need
+        buf = torch.zeros(need, dtype=torch.uint8)
+        acc, ml = pdist.partials_views(buf, B, sq, Hq, D, n)
+        assert acc.shape == (B * sq * Hq, n, D) and ml.shape == (B * sq * Hq, n, 2)
+        assert ml.data_ptr() - buf.data_ptr() == -(-(acc.numel() * 4) // 256) * 256
+        assert ml.data_ptr() + ml.numel() * 4 == buf.data_ptr() + need
+        with pytest.raises(ValueError):
+            pdist.partials_views(buf[:need - 4], B, sq, Hq, D, n)
 
 
 @pytest.mark.parametrize("ctx,world", [(1, 1), (4096, 1), (4097, 2), (20000, 3), (8192, 8), (0, 4)])
