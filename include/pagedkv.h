@@ -181,6 +181,31 @@ int pkv_paged_prefill_attn(const void *q, const int64_t q_strides[3],
                            int32_t *err, void *stream);
 
 /*
+ * pkv_debug_paged_decode_attn: pkv_paged_decode_attn (same arguments, same
+ * results) with every internal pipeline wait limited to wait_limit_ns instead
+ * of the 2 s every other call uses.  It has no counterpart on the pages: it
+ * exists to exercise the library's own failure handling (every pipeline wait
+ * is bounded and a stuck pipeline ends the call with an error bit instead of a
+ * hung GPU).  A wait that runs out makes the
+ * kernel give up: each CTA waits (with the full 2 s limit) for its own copies
+ * and tensor-core operations in flight, releases its tensor memory, sets
+ * PKV_DEVERR_TIMEOUT in *err and returns; out / lse then hold no result, and
+ * the device stays usable for the next call.  wait_limit_ns may be 0 (any wait
+ * not satisfied at once gives up); more than 2e9 is PKV_ERR_ARG.
+ */
+int pkv_debug_paged_decode_attn(const void *q, const int64_t q_strides[3],
+                                const void *k_cache, const int64_t k_strides[3],
+                                const void *v_cache, const int64_t v_strides[3],
+                                int64_t num_blocks,
+                                const int32_t *block_table, int64_t bt_stride,
+                                int max_blocks_per_seq, const int32_t *seqlens, int max_seqlen_k,
+                                int batch, int seqlen_q, int Hq, int Hkv, int D, int block_size,
+                                float scale, int causal,
+                                void *out, const int64_t out_strides[3], float *lse,
+                                void *workspace, size_t workspace_bytes,
+                                int32_t *err, void *stream, uint64_t wait_limit_ns);
+
+/*
  * pkv_paged_decode_attn_append: kv_append fused into the attention call --
  * the "new_kv" form of flash_attn_with_kvcache in the aiter test grid.  The
  * n_new tokens of k_new/v_new ([batch, n_new, Hkv, D] bf16, element strides

@@ -187,7 +187,8 @@ def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
 
 
 def _attn(fn_name: str, q, k_cache, v_cache, block_table, seqlens, max_seqlen_k, scale,
-          causal, out, lse, workspace, err, stream) -> Tuple[torch.Tensor, torch.Tensor]:
+          causal, out, lse, workspace, err, stream,
+          extra=()) -> Tuple[torch.Tensor, torch.Tensor]:
     _need_cuda_bf16("q", q)
     _need_cuda_bf16("k_cache", k_cache)
     _need_cuda_bf16("v_cache", v_cache)
@@ -217,7 +218,7 @@ def _attn(fn_name: str, q, k_cache, v_cache, block_table, seqlens, max_seqlen_k,
         int(block_table.shape[1]), seqlens.data_ptr(), int(max_seqlen_k), B, sq, Hq, Hkv, D, bs,
         float(scale), int(bool(causal)), out.data_ptr(), _st3(out), lse.data_ptr(),
         workspace.data_ptr(), workspace.numel() * workspace.element_size(), _ptr(err),
-        _stream_handle(stream))
+        _stream_handle(stream), *extra)
     _check(fn_name, rc)
     return out, lse
 
@@ -229,6 +230,22 @@ def paged_decode_attn(q, k_cache, v_cache, block_table, seqlens, *, max_seqlen_k
     (out [B, sq, Hq, D] bf16, lse [B, Hq, sq] fp32).  See include/pagedkv.h."""
     return _attn("pkv_paged_decode_attn", q, k_cache, v_cache, block_table, seqlens,
                  max_seqlen_k, scale, causal, out, lse, workspace, err, stream)
+
+
+def debug_paged_decode_attn(q, k_cache, v_cache, block_table, seqlens, *, wait_limit_ns,
+                            max_seqlen_k=None, scale=None, causal=False, out=None, lse=None,
+                            workspace=None, err=None, stream=None):
+    """paged_decode_attn with every internal pipeline wait limited to
+    wait_limit_ns (at most the library's 2 s): the failure path under test.
+    A wait that runs out makes the call give up: it returns, PKV_DEVERR_TIMEOUT
+    is set in err and out / lse hold no result."""
+    fn = lib().pkv_debug_paged_decode_attn
+    if not fn.argtypes:
+        fn.argtypes = _ATTN_ARGS + [ctypes.c_uint64]
+        fn.restype = _I
+    return _attn("pkv_debug_paged_decode_attn", q, k_cache, v_cache, block_table, seqlens,
+                 max_seqlen_k, scale, causal, out, lse, workspace, err, stream,
+                 extra=(int(wait_limit_ns),))
 
 
 def paged_decode_attn_append(q, k_new, v_new, k_cache, v_cache, block_table, seqlens, *,

@@ -73,6 +73,10 @@ struct RowCfg {
     float tmax[3][kRowsPerTile];  // [buffer][row]: the tile's max (base-2 units)
     float lsum[3][kRowsPerTile];  // [buffer][row]: the tile's sum of p
     int tab[2][2][kSplitTokens / 16];
+    int sched_list[kSchedMaxMine];     // this CTA's units (balanced schedule)
+    int sched_meta[kSchedMaxMine][3];  // their sequence length and query range
+    int sched_hist[kSchedBuckets + 2], sched_start[kSchedBuckets];
+    int sched_count;
   };
   static constexpr int kSmemBytes = kOffSmall + static_cast<int>(sizeof(Small)) + 1024;
   static constexpr int kTmemCols = 512;
@@ -174,15 +178,23 @@ __global__ void __launch_bounds__(kRowThreads, 1)
   const uint32_t tmem = sm->tmem_base;
   const uint32_t sbase = smem_u32(smem);
   const float NEG_INF = neg_inf();
+  // the Q buffers are not in use yet: one byte per unit of scratch
+  static_assert(C::kQB * C::kQBytes >= kSchedMaxUnits, "schedule scratch");
+  Sched sc = strided_sched(p);
+  if (p.sched) {
+    build_schedule<kRowsPerTile>(p, smem + C::kOffQ, sm->sched_hist, sm->sched_start,
+                                 sm->sched_list, sm->sched_meta, &sm->sched_count);
+    if (sm->sched_count >= 0) sc = Sched{sm->sched_list, sm->sched_meta, sm->sched_count};
+  }
 
   if (warp >= kKWarp) {
     regs_dec<kRowsAuxRegs>();
     if (warp == kKWarp) {
       produce<C>(p, &map_k, &map_q, smem, sm, sm->full_k, sm->empty_k, sm->tab[0], C::kOffK, true,
-                 lane, abort_any);
+                 lane, abort_any, sc);
     } else if (warp == kVWarp) {
       produce<C>(p, &map_v, nullptr, smem, sm, sm->full_v, sm->empty_v, sm->tab[1], C::kOffV,
-                 false, lane, abort_any);
+                 false, lane, abort_any, sc);
     } else if (warp == kMmaWarp && lane == 0) {
       // ----------------------------------------------------------------
       // MMA issuer.  Per tile gi: S[gi % kSB] = Q K^T once the K stage has
@@ -198,9 +210,9 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       bool failed = false;
       auto pv_step = [&](int g) -> bool {
         const int st = g % NS, bb = g % SB;
-        if (!mbar_wait(&sm->p_full[bb], (g / SB) & 1, abort_any)) return false;
-        if (!mbar_wait(&sm->o_free, (g & 1) ^ 1, abort_any)) return false;
-        if (!mbar_wait(&sm->full_v[st], (g / NS) & 1, abort_any)) return false;
+        if (!mbar_wait(&sm->p_full[bb], (g / SB) & 1, abort_any, p.wait_ns)) return false;
+        if (!mbar_wait(&sm->o_free, (g & 1) ^ 1, abort_any, p.wait_ns)) return false;
+        if (!mbar_wait(&sm->full_v[st], (g / NS) & 1, abort_any, p.wait_ns)) return false;
         tc_fence_after_sync();
         const uint32_t vaddr = sbase + C::kOffV + st * C::kKVBytes;
         const uint32_t pcol = tmem + bb * 128;
@@ -220,19 +232,19 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         umma_commit(&sm->s_free[bb]);
         return true;
       };
-      for (int u = blockIdx.x; u < p.n_units && !failed; u += gridDim.x) {
-        const Unit x = unit_at<kRowsPerTile>(p, u);
+      for (int k = 0; k < sc.count && !failed; ++k) {
+        const Unit x = sc.get<kRowsPerTile>(p, k);
         if (x.n_tiles == 0) continue;
         const int qb = ui & 1;
-        if (!mbar_wait(&sm->q_full[qb], (ui >> 1) & 1, abort_any)) {
+        if (!mbar_wait(&sm->q_full[qb], (ui >> 1) & 1, abort_any, p.wait_ns)) {
           failed = true;
           break;
         }
         const uint32_t qaddr = sbase + C::kOffQ + qb * C::kQBytes;
         for (int j = 0; j < x.n_tiles; ++j, ++gi) {
           const int st = gi % NS, bb = gi % SB;
-          if (!mbar_wait(&sm->full_k[st], (gi / NS) & 1, abort_any) ||
-              !mbar_wait(&sm->s_free[bb], ((gi / SB) & 1) ^ 1, abort_any)) {
+          if (!mbar_wait(&sm->full_k[st], (gi / NS) & 1, abort_any, p.wait_ns) ||
+              !mbar_wait(&sm->s_free[bb], ((gi / SB) & 1) ^ 1, abort_any, p.wait_ns)) {
             failed = true;
             break;
           }
@@ -272,11 +284,12 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       }
       if (!failed && pend0 >= 0) failed = !pv_step(pend0);
       if (!failed && pend1 >= 0) failed = !pv_step(pend1);
-      if (failed) {
-        umma_commit(&sm->drain);
-        volatile int no_abort = 0;
-        mbar_wait(&sm->drain, 0, &no_abort);
-      }
+      // every MMA this thread issued completes before TMEM is released, also
+      // when the consumers gave up (bounded wait, default limit)
+      (void)failed;
+      umma_commit(&sm->drain);
+      volatile int no_abort = 0;
+      mbar_wait(&sm->drain, 0, &no_abort);
     }
   } else if (warp < kCorrWarp0) {
     // ------------------------------------------------------------------
@@ -291,8 +304,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     const uint32_t bar_id = 1 + wg;
     int gbase = 0;
     bool stop = false;
-    for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
-      const Unit x = unit_at<kRowsPerTile>(p, u);
+    for (int k = 0; k < sc.count && !stop; ++k) {
+      const Unit x = sc.get<kRowsPerTile>(p, k);
       if (x.n_tiles == 0) continue;
       int nlim = 0;  // keys [0, nlim) are visible to row t
       if (t < x.rows) {
@@ -305,8 +318,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         const int gi = gbase + j;
         if ((gi & 1) != wg) continue;
         const int bb = gi % C::kSB, st = gi % NS, par = (gi / C::kSB) & 1;
-        bool ok = mbar_wait(&sm->s_full[bb], par, abort_any);
-        ok = mbar_wait(&sm->stat_free[bb], par ^ 1, abort_any) && ok;
+        bool ok = mbar_wait(&sm->s_full[bb], par, abort_any, p.wait_ns);
+        ok = mbar_wait(&sm->stat_free[bb], par ^ 1, abort_any, p.wait_ns) && ok;
         tc_fence_after_sync();
         const int tok0 = x.tok0 + j * kTileTokens;
         const int nvis = min(max(nlim - tok0, 0), kTileTokens);
@@ -407,7 +420,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           // The last tile: keys past the loaded range hold stale bytes or the
           // cache's NaN tails; once V has landed, zero those V rows so that
           // 0 * V stays 0 in P.V.
-          ok = mbar_wait(&sm->full_v[st], (gi / NS) & 1, abort_any) && ok;
+          ok = mbar_wait(&sm->full_v[st], (gi / NS) & 1, abort_any, p.wait_ns) && ok;
           if (ok && tok0 + t >= x.lim_max) {
             uint8_t *vrow = smem + C::kOffV + st * C::kKVBytes + t * 128;
 #pragma unroll
@@ -447,8 +460,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     float acc[D];
     int gbase = 0;
     bool stop = false;
-    for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
-      const Unit x = unit_at<kRowsPerTile>(p, u);
+    for (int k = 0; k < sc.count && !stop; ++k) {
+      const Unit x = sc.get<kRowsPerTile>(p, k);
       if (t == 0) check_sequence(p, x);
       if (x.n_tiles == 0) {
         // rows that see no key: out = 0, lse = -inf (written by the unit of
@@ -465,8 +478,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       float m_run = NEG_INF, l_run = 0.f;
       for (int j = 0; j < x.n_tiles; ++j) {
         const int gi = gbase + j, bb = gi % C::kSB, par = (gi / C::kSB) & 1;
-        bool ok = mbar_wait(&sm->p_full[bb], par, abort_any);  // the tile's row statistics
-        ok = mbar_wait(&sm->o_full, gi & 1, abort_any) && ok;    // its P.V
+        bool ok = mbar_wait(&sm->p_full[bb], par, abort_any, p.wait_ns);  // the tile's row statistics
+        ok = mbar_wait(&sm->o_full, gi & 1, abort_any, p.wait_ns) && ok;    // its P.V
         tc_fence_after_sync();
         __syncwarp();  // the waits above spin per thread; the TMEM loads below are warp-wide
         const float tm = sm->tmax[bb][t];
@@ -488,17 +501,26 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         }
         const uint32_t orow = tmem + lane_off;
         __syncwarp();
+        // two 16-column chunks of O_hi and O_lo per wait (tcgen05.wait::ld
+        // waits for every load in flight, so loads are batched, not pipelined)
 #pragma unroll
-        for (int ch = 0; ch < D / 16; ++ch) {
-          float hi[16], lo[16];
-          tmem_ld16(orow + C::kColOhi + ch * 16, hi);
-          tmem_ld16(orow + C::kColOlo + ch * 16, lo);
-          tmem_ld_wait_for(hi);
-          tmem_ld_wait_for(lo);
+        for (int ch = 0; ch < D / 16; ch += 2) {
+          float hi0[16], lo0[16], hi1[16], lo1[16];
+          tmem_ld16(orow + C::kColOhi + ch * 16, hi0);
+          tmem_ld16(orow + C::kColOlo + ch * 16, lo0);
+          tmem_ld16(orow + C::kColOhi + ch * 16 + 16, hi1);
+          tmem_ld16(orow + C::kColOlo + ch * 16 + 16, lo1);
+          tmem_ld_wait_for(hi0);
+          tmem_ld_wait_for(lo0);
+          tmem_ld_wait_for(hi1);
+          tmem_ld_wait_for(lo1);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {  // branch-free: the loop's TMEM loads are warp-wide
-            const float nv = __fmaf_rn(__fadd_rn(hi[e], lo[e]), b, __fmul_rn(acc[ch * 16 + e], a));
-            acc[ch * 16 + e] = skip ? acc[ch * 16 + e] : nv;
+            const float nv0 = __fmaf_rn(__fadd_rn(hi0[e], lo0[e]), b, __fmul_rn(acc[ch * 16 + e], a));
+            acc[ch * 16 + e] = skip ? acc[ch * 16 + e] : nv0;
+            const float nv1 =
+                __fmaf_rn(__fadd_rn(hi1[e], lo1[e]), b, __fmul_rn(acc[ch * 16 + 16 + e], a));
+            acc[ch * 16 + 16 + e] = skip ? acc[ch * 16 + 16 + e] : nv1;
           }
         }
         tc_fence_before_sync();

@@ -45,6 +45,7 @@
 #include <cuda_bf16.h>
 
 #include "contract.cuh"
+#include "merge.cuh"
 #include "ptx.cuh"
 
 namespace pkv {
@@ -55,6 +56,12 @@ constexpr int kCorrWarp0 = 8;  // warps 8-11: correction + epilogue warpgroup
 constexpr int kKWarp = 12;     // K producer (+ Q staging)
 constexpr int kVWarp = 13;     // V producer
 constexpr int kMmaWarp = 14;   // MMA issuer + TMEM owner
+
+// Balanced schedule limits (see build_schedule): units per call, units per
+// CTA, and the tile-count buckets of the sort.
+constexpr int kSchedMaxUnits = 16384;
+constexpr int kSchedMaxMine = 128;
+constexpr int kSchedBuckets = kSplitTokens / kTileTokens + 1;  // tile counts 0 .. 32
 
 struct AttnParams {
   const __nv_bfloat16 *q;
@@ -70,6 +77,7 @@ struct AttnParams {
   int map_head_first;   // tensor-map dim order (D, Hkv, slot, block) vs (D, slot, Hkv, block)
   int n_row_tiles, n_splits, n_units;
   int max_seqlen_k;     // host bound on seqlens (n_splits = ceil(max_seqlen_k / 4096))
+  uint64_t wait_ns;     // limit of every pipeline wait (kWaitTimeoutNs unless a debug call lowers it)
   float cscale;         // softmax scale * log2(e)
   int causal;
   float *ws_acc;        // [rows][n_splits][D]
@@ -86,6 +94,10 @@ struct AttnParams {
   // lse written with the merge's arithmetic.  direct: every row of the call
   // has at most one split (host side: no merge launch).
   int direct, out_vec;
+  // sched: the split kernel builds the balanced unit order (host: at most
+  // kSchedMaxUnits units and kSchedMaxMine per CTA); otherwise units are dealt
+  // with stride gridDim.x
+  int sched;
   __nv_bfloat16 *out;
   int64_t o_sb, o_ss, o_sh;
   float *lse;
@@ -187,6 +199,11 @@ struct Cfg {
     float tmax[2][N];                      // [buffer][row]: the tile's max (base-2 units)
     float coef_a[N], coef_b[N];            // correction factors of the current tile
     int coef_skip[N];
+    float fin_m[N], fin_l[N];              // each row's (m, l) for the direct final write
+    int sched_list[kSchedMaxMine];         // this CTA's units (balanced schedule)
+    int sched_meta[kSchedMaxMine][3];      // their sequence length and query range
+    int sched_hist[kSchedBuckets + 2], sched_start[kSchedBuckets];
+    int sched_count;
     int lim[2][N];                         // [softmax warpgroup][row]: key limit
     int tab[2][2][kSplitTokens / 16];      // [producer][unit parity]: block-table entries
   };
@@ -210,8 +227,15 @@ struct Unit {
 // one of a decode step in a packed batch) spreads over all CTAs of the
 // strided assignment, and the last row tiles -- the heaviest under causal
 // masking, and those of the longest requests -- come first.
+// Sequence of unit u.
+__device__ __forceinline__ int unit_seq(const AttnParams &p, int u) {
+  return (u / p.Hkv / p.n_splits) % p.batch;
+}
+
+// Unit u given its sequence's length sl and (packed calls) query range
+// [a, e) -- arithmetic only.
 template <int N>
-__device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
+__device__ __forceinline__ Unit unit_make(const AttnParams &p, int u, int sl, int a, int e) {
   Unit x;
   x.kvh = u % p.Hkv;
   u /= p.Hkv;
@@ -219,10 +243,8 @@ __device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
   u /= p.n_splits;
   x.b = u % p.batch;
   x.rt = p.n_row_tiles - 1 - u / p.batch;
-  const int sl = __ldg(p.seqlens + x.b);
   x.seqlen = sl > 0 ? sl : 0;
   if (p.cu_q) {
-    const int a = __ldg(p.cu_q + x.b), e = __ldg(p.cu_q + x.b + 1);
     x.q0 = a;
     x.nq = min(max(e - a, 0), p.seqlen_q);  // more than the bound: flagged, rows past it unwritten
   } else {
@@ -243,6 +265,14 @@ __device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
   const int ntok = min(kSplitTokens, x.lim_max - x.tok0);
   x.n_tiles = ntok > 0 ? (ntok + kTileTokens - 1) / kTileTokens : 0;
   return x;
+}
+
+template <int N>
+__device__ __forceinline__ Unit unit_at(const AttnParams &p, int u) {
+  const int b = unit_seq(p, u);
+  const int sl = __ldg(p.seqlens + b);
+  const int a = p.cu_q ? __ldg(p.cu_q + b) : 0, e = p.cu_q ? __ldg(p.cu_q + b + 1) : 0;
+  return unit_make<N>(p, u, sl, a, e);
 }
 
 constexpr int kPastWidth = static_cast<int>(0x80000000u);
@@ -275,14 +305,132 @@ __device__ __forceinline__ void check_sequence(const AttnParams &p, const Unit &
   }
 }
 
-// First unit at or after `from` (stride gridDim.x) with work, or -1.
+// The units this CTA runs, in order: the k-th is list[k] (a balanced order
+// built at kernel start, see build_schedule) or, without a list, unit
+// blockIdx.x + k gridDim.x.  Which CTA runs a unit never changes its
+// arithmetic, so the order only moves the makespan.
+// With a list, each entry's sequence length and packed query range were
+// loaded into shared memory with the list (meta[k] = {seqlen, a, e}), so no
+// role reads global memory to learn its next unit -- under a saturated memory
+// system such a read costs microseconds at every unit boundary.
+struct Sched {
+  const int *list;
+  const int (*meta)[3];
+  int count;
+  __device__ __forceinline__ int unit(int k) const {
+    return list ? list[k] : static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+  }
+  template <int N>
+  __device__ __forceinline__ Unit get(const AttnParams &p, int k) const {
+    if (list) return unit_make<N>(p, list[k], meta[k][0], meta[k][1], meta[k][2]);
+    return unit_at<N>(p, unit(k));
+  }
+};
+
+__device__ __forceinline__ Sched strided_sched(const AttnParams &p) {
+  const int g = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+  return Sched{nullptr, nullptr, p.n_units > b ? (p.n_units - b + g - 1) / g : 0};
+}
+
+// First schedule slot at or after `from` whose unit has work, or -1.
 template <int N>
-__device__ __forceinline__ int next_unit(const AttnParams &p, int from, Unit &out) {
-  for (int v = from; v < p.n_units; v += gridDim.x) {
-    out = unit_at<N>(p, v);
-    if (out.n_tiles > 0) return v;
+__device__ __forceinline__ int next_unit(const AttnParams &p, const Sched &sc, int from,
+                                         Unit &out) {
+  for (int k = from; k < sc.count; ++k) {
+    out = sc.get<N>(p, k);
+    if (out.n_tiles > 0) return k;
   }
   return -1;
+}
+
+// Balanced schedule (decode-shaped calls of at most kSchedMaxUnits units):
+// every CTA sorts all units by tile count, largest first -- a stable counting
+// sort, so every CTA computes the same order -- and takes the positions of a
+// snake deal over the grid: round r hands positions r G .. r G + G - 1 to CTAs
+// 0 .. G - 1 when r is even and to CTAs G - 1 .. 0 when r is odd.  The CTA's
+// k-th unit is the one at its position of round k.  With contexts of mixed
+// lengths this evens out the tiles per CTA (a stride-G deal leaves some CTAs
+// with far more).  When every unit with work has the same tile count there is
+// nothing to balance: *count is set to -1 and the caller keeps the stride-G
+// deal.  All threads of the CTA take part; `scratch` holds one byte per unit
+// (free shared memory at kernel start); hist has kSchedBuckets + 2 entries.
+
+template <int N>
+__device__ __forceinline__ void build_schedule(const AttnParams &p, uint8_t *scratch, int *hist,
+                                               int *start, int *list, int (*meta)[3],
+                                               int *count) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  int *nt_min = hist + kSchedBuckets, *nt_max = hist + kSchedBuckets + 1;
+  for (int i = tid; i < kSchedBuckets; i += nthr) hist[i] = 0;
+  if (tid == 0) {
+    *nt_min = kSchedBuckets;
+    *nt_max = 0;
+  }
+  __syncthreads();
+  int lo = kSchedBuckets, hi = 0;
+  for (int u = tid; u < p.n_units; u += nthr) {
+    const int nt = unit_at<N>(p, u).n_tiles;
+    scratch[u] = static_cast<uint8_t>(nt);
+    atomicAdd(&hist[nt], 1);
+    if (nt > 0) {
+      lo = min(lo, nt);
+      hi = max(hi, nt);
+    }
+  }
+  if (lo <= hi) {
+    atomicMin(nt_min, lo);
+    atomicMax(nt_max, hi);
+  }
+  __syncthreads();
+  if (*nt_min >= *nt_max) {  // uniform (or no work): keep the stride-G deal
+    __syncthreads();         // every thread has read nt_min / nt_max
+    if (tid == 0) *count = -1;
+    __syncthreads();
+    return;
+  }
+  if (tid == 0) {  // bucket starts, largest tile count first
+    int acc = 0;
+    for (int nt = kSchedBuckets - 1; nt >= 0; --nt) {
+      start[nt] = acc;
+      acc += hist[nt];
+      hist[nt] = 0;  // from here on: units of the bucket placed so far
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const int G = static_cast<int>(gridDim.x), me = static_cast<int>(blockIdx.x);
+    const int lane = tid;
+    for (int base = 0; base < p.n_units; base += 32) {
+      const int u = base + lane;
+      const int nt = u < p.n_units ? scratch[u] : -1;
+      const unsigned same = __match_any_sync(0xffffffffu, nt);
+      const int rank = __popc(same & ((1u << lane) - 1u));
+      const int placed = nt >= 0 ? hist[nt] : 0;
+      __syncwarp();
+      if (nt >= 0) {
+        if (rank == 0) hist[nt] = placed + __popc(same);
+        const int pos = start[nt] + placed + rank;
+        const int r = pos / G, i = pos - r * G;
+        if (((r & 1) ? G - 1 - i : i) == me) list[r] = u;
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {
+      // rounds in which this CTA has a position below n_units
+      const int full_rounds = p.n_units / G, rem = p.n_units - full_rounds * G;
+      const int pos_last = (full_rounds & 1) ? G - 1 - me : me;  // its position in the partial round
+      *count = full_rounds + (pos_last < rem ? 1 : 0);
+    }
+  }
+  __syncthreads();
+  // the listed units' sequence lengths and query ranges, read once
+  for (int k = tid; k < *count; k += nthr) {
+    const int b = unit_seq(p, list[k]);
+    meta[k][0] = __ldg(p.seqlens + b);
+    meta[k][1] = p.cu_q ? __ldg(p.cu_q + b) : 0;
+    meta[k][2] = p.cu_q ? __ldg(p.cu_q + b + 1) : 0;
+  }
+  __syncthreads();
 }
 
 // Stage the Q rows of unit x (the B operand of S^T = K Q^T, 128-byte
@@ -363,12 +511,24 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
                                         const CUtensorMap *map_q, uint8_t *smem,
                                         typename C::Small *sm, uint64_t *full, uint64_t *empty,
                                         int (*tabs)[kSplitTokens / 16], uint32_t dst_off,
-                                        bool with_q, int lane, volatile int *abort_any) {
+                                        bool with_q, int lane, volatile int *abort_any,
+                                        const Sched &sc) {
   constexpr int D = C::kD, N = C::kN, NS = C::kNS, QB = C::kQB;
-  // Q of unit u into buffer qb: TMA (completing on q_full[qb]) or plain loads
-  auto put_q = [&](const Unit &u, int qb) {
+  // Q copies by TMA still to be accounted for at exit (lane 0): per buffer,
+  // the ordinal of the last unit whose Q went there, and whether its q_full
+  // arrival is still to come (the copy was issued, the unit boundary not yet
+  // reached)
+  int q_last[QB];
+#pragma unroll
+  for (int i = 0; i < QB; ++i) q_last[i] = -1;
+  int q_pending = -1, q_pending_ord = -1;
+  // Q of unit u (the warp's ord-th unit) into buffer qb: TMA (completing on
+  // q_full[qb]) or plain loads
+  auto put_q = [&](const Unit &u, int qb, int ord) {
     if constexpr (C::kQTma) {
       if (lane == 0) {
+        q_pending = qb;
+        q_pending_ord = ord;
         mbar_expect_tx(&sm->q_full[qb], static_cast<uint32_t>(C::kQBytes));
         const int i0 = u.row0 / p.G;
         // dense map (D, Hq, seqlen_q, batch); packed map (D, Hq, total_q, 1)
@@ -390,20 +550,26 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
   for (int i = 0; i < NS; ++i) last_gi[i] = -1;
   bool failed = false;
   Unit cur;
-  int cu = next_unit<N>(p, blockIdx.x, cur);
+  int cu = next_unit<N>(p, sc, 0, cur);
   if (cu >= 0) {
     const int bmask = (1 << p.block_shift) - 1;
     int ui = 0, gi = 0;
     // the first unit (Q buffer 0 is free)
     stage_tab(p, cur, tabs[0], lane);
-    if (with_q) put_q(cur, 0);
+    if (with_q) put_q(cur, 0, 0);
     if (with_q) fence_proxy_async_smem();
     __syncwarp();
-    if (with_q && lane == 0) mbar_arrive(&sm->q_full[0]);
+    if (with_q && lane == 0) {
+      mbar_arrive(&sm->q_full[0]);
+      if constexpr (C::kQTma) {
+        q_last[0] = 0;
+        q_pending = -1;
+      }
+    }
     while (true) {
       // stage the next unit while this one's tiles are issued
       Unit nxt;
-      const int nu = next_unit<N>(p, cu + gridDim.x, nxt);
+      const int nu = next_unit<N>(p, sc, cu + 1, nxt);
       bool q_early = false;
       if (nu >= 0) stage_tab(p, nxt, tabs[(ui + 1) & 1], lane);
       const int *tab = tabs[ui & 1];
@@ -414,17 +580,17 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
           // QKs are done by the time this unit's last tile is issued
           const int qb = (ui + 1) % QB;
           bool okq = true;
-          if (lane == 0) okq = mbar_wait(&sm->q_empty[qb], (((ui + 1) / QB) & 1) ^ 1, abort_any);
+          if (lane == 0) okq = mbar_wait(&sm->q_empty[qb], (((ui + 1) / QB) & 1) ^ 1, abort_any, p.wait_ns);
           if (!__shfl_sync(0xffffffffu, okq ? 1 : 0, 0)) {
             failed = true;
             break;
           }
-          put_q(nxt, qb);
+          put_q(nxt, qb, ui + 1);
           q_early = true;
         }
         const int st = gi % NS;
         bool okw = true;
-        if (lane == 0) okw = mbar_wait(&empty[st], ((gi / NS) & 1) ^ 1, abort_any);
+        if (lane == 0) okw = mbar_wait(&empty[st], ((gi / NS) & 1) ^ 1, abort_any, p.wait_ns);
         if (!__shfl_sync(0xffffffffu, okw ? 1 : 0, 0)) {
           failed = true;
           break;
@@ -463,27 +629,92 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
       if (with_q && !q_early) {  // one Q buffer: wait until this unit's QKs are done
         const int qb = (ui + 1) % QB;
         bool okq = true;
-        if (lane == 0) okq = mbar_wait(&sm->q_empty[qb], (((ui + 1) / QB) & 1) ^ 1, abort_any);
+        if (lane == 0) okq = mbar_wait(&sm->q_empty[qb], (((ui + 1) / QB) & 1) ^ 1, abort_any, p.wait_ns);
         if (!__shfl_sync(0xffffffffu, okq ? 1 : 0, 0)) {
           failed = true;
           break;
         }
-        put_q(nxt, qb);
+        put_q(nxt, qb, ui + 1);
       }
       if (with_q) fence_proxy_async_smem();
       __syncwarp();
-      if (with_q && lane == 0) mbar_arrive(&sm->q_full[(ui + 1) % QB]);
+      if (with_q && lane == 0) {
+        mbar_arrive(&sm->q_full[(ui + 1) % QB]);
+        if constexpr (C::kQTma) {
+          q_last[(ui + 1) % QB] = ui + 1;
+          q_pending = -1;
+        }
+      }
       ++ui;
       cur = nxt;
       cu = nu;
     }
   }
-  if (failed && lane == 0) {
-    // wait (bounded, ignoring the abort flag) for this warp's copies in flight
+  if (lane == 0) {
+    // Whatever ended the loop, wait (bounded, ignoring the abort flag) until
+    // every copy this warp issued has landed, so that none is in flight when
+    // the CTA exits even if its consumers gave up.  After a normal run these
+    // phases have long completed and the waits return at once.  A Q copy whose
+    // q_full arrival was still to come gets it now, so its phase can complete.
     volatile int no_abort = 0;
 #pragma unroll
     for (int i = 0; i < NS; ++i)
       if (last_gi[i] >= 0) mbar_wait(&full[i], (last_gi[i] / NS) & 1, &no_abort);
+    if constexpr (C::kQTma) {
+      if (with_q && q_pending >= 0) {
+        mbar_arrive(&sm->q_full[q_pending]);
+        q_last[q_pending] = q_pending_ord;
+      }
+#pragma unroll
+      for (int i = 0; i < QB; ++i)
+        if (with_q && q_last[i] >= 0) mbar_wait(&sm->q_full[i], (q_last[i] / QB) & 1, &no_abort);
+    }
+  }
+}
+
+// Direct final write (calls whose every row has at most one split, no merge
+// launch): row c of unit x gets out / lse through the merge's fold of that one
+// partial, so the bits are those the merge would write.  Thread t < D writes
+// column t of every row (acc[c] = the row's unnormalised column t); thread
+// t < rows also writes row t's lse.  m / l of every row come from shared
+// memory (fin_m / fin_l), published before the call.
+template <int D, int N>
+__device__ __forceinline__ void write_final_cols(const AttnParams &p, const Unit &x, int t,
+                                                 const float (&acc)[N], const float *fin_m,
+                                                 const float *fin_l) {
+  const float NEG_INF = neg_inf();
+#pragma unroll
+  for (int c = 0; c < N; ++c) {
+    if (c < x.rows && t < D) {
+      const int r = x.row0 + c;
+      const int i = r / p.G, g = r - i * p.G;
+      const int h = x.kvh * p.G + g;
+      const float m = fin_m[c];
+      float L = 0.f, A = 0.f;
+      if (m != NEG_INF) {
+        const FoldCoef kc = fold_coef(NEG_INF, m);
+        L = fold_val(0.f, fin_l[c], kc);
+        A = fold_val(0.f, acc[c], kc);
+      }
+      const __nv_bfloat16 ob = __float2bfloat16_rn(final_out(A, L));
+      p.out[o_tok_off(p, x, i) + h * p.o_sh + t] = ob;
+      if (p.fin_out != nullptr && i == x.nq - 1) p.fin_out[x.b * p.fo_sb + h * p.fo_sh + t] = ob;
+    }
+  }
+  if (t < x.rows) {
+    const int r = x.row0 + t;
+    const int i = r / p.G, g = r - i * p.G;
+    const int h = x.kvh * p.G + g;
+    const float m = fin_m[t];
+    float M = NEG_INF, L = 0.f;
+    if (m != NEG_INF) {
+      const FoldCoef kc = fold_coef(NEG_INF, m);
+      L = fold_val(0.f, fin_l[t], kc);
+      M = kc.Mn;
+    }
+    const float ls = final_lse(M, L);
+    p.lse[lse_index(p, x, i, h)] = ls;
+    if (p.fin_out != nullptr && i == x.nq - 1) p.fin_lse[static_cast<int64_t>(x.b) * p.Hq + h] = ls;
   }
 }
 
@@ -529,13 +760,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = sm->tmem_base;
   const uint32_t sbase = smem_u32(smem);
+  // the P^T buffers are not in use yet: one byte per unit of scratch
+  static_assert(2 * C::kPBytes >= kSchedMaxUnits, "schedule scratch");
+  Sched sc = strided_sched(p);
+  if (p.sched) {
+    build_schedule<N>(p, smem + C::kOffP, sm->sched_hist, sm->sched_start, sm->sched_list,
+                      sm->sched_meta, &sm->sched_count);
+    if (sm->sched_count >= 0) sc = Sched{sm->sched_list, sm->sched_meta, sm->sched_count};
+  }
 
   if (warp == kKWarp) {
     produce<C>(p, &map_k, nullptr, smem, sm, sm->full_k, sm->empty_k, sm->tab[0], C::kOffK, true,
-               lane, abort_any);
+               lane, abort_any, sc);
   } else if (warp == kVWarp) {
     produce<C>(p, &map_v, nullptr, smem, sm, sm->full_v, sm->empty_v, sm->tab[1], C::kOffV, false,
-               lane, abort_any);
+               lane, abort_any, sc);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------
     // MMA issuer (one thread)
@@ -544,13 +783,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kIdescQK = idesc_bf16(128, N, 0, 0);           // A = K tile, B = Q (K-major)
       constexpr uint32_t kIdescPV = idesc_bf16(128, C::kPCols, 1, 1);  // A = V^T, B = P^T (MN-major)
       const uint32_t tS = tmem, tO = tmem + 2 * N;
+      // QK^T of tile gi, then P.V of tile gi - 1
       int gi = 0, ui = 0, prev = -1;
       bool failed = false;
       auto pv_step = [&](int g) -> bool {
         const int st = g % NS, bb = g & 1;
-        if (!mbar_wait(&sm->p_full[bb], (g >> 1) & 1, abort_any)) return false;
-        if (!mbar_wait(&sm->o_free[bb], ((g >> 1) & 1) ^ 1, abort_any)) return false;
-        if (!mbar_wait(&sm->full_v[st], (g / NS) & 1, abort_any)) return false;
+        if (!mbar_wait(&sm->p_full[bb], (g >> 1) & 1, abort_any, p.wait_ns)) return false;
+        if (!mbar_wait(&sm->o_free[bb], ((g >> 1) & 1) ^ 1, abort_any, p.wait_ns)) return false;
+        if (!mbar_wait(&sm->full_v[st], (g / NS) & 1, abort_any, p.wait_ns)) return false;
         tc_fence_after_sync();
         const uint32_t vaddr = sbase + C::kOffV + st * C::kKVBytes;
         const uint32_t paddr = sbase + C::kOffP + bb * C::kPBytes;
@@ -570,18 +810,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&sm->empty_v[st]);
         return true;
       };
-      for (int u = blockIdx.x; u < p.n_units && !failed; u += gridDim.x) {
-        const Unit x = unit_at<N>(p, u);
+      for (int k = 0; k < sc.count && !failed; ++k) {
+        const Unit x = sc.get<N>(p, k);
         if (x.n_tiles == 0) continue;
         const int qb = ui % QB;
-        if (!mbar_wait(&sm->q_full[qb], (ui / QB) & 1, abort_any)) {
+        if (!mbar_wait(&sm->q_full[qb], (ui / QB) & 1, abort_any, p.wait_ns)) {
           failed = true;
           break;
         }
         const uint32_t qaddr = sbase + C::kOffQ + qb * C::kQBytes;
         for (int j = 0; j < x.n_tiles; ++j, ++gi) {
           const int st = gi % NS, bb = gi & 1;
-          if (!mbar_wait(&sm->full_k[st], (gi / NS) & 1, abort_any)) {
+          if (!mbar_wait(&sm->full_k[st], (gi / NS) & 1, abort_any, p.wait_ns)) {
             failed = true;
             break;
           }
@@ -606,11 +846,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++ui;
       }
       if (!failed && prev >= 0) failed = !pv_step(prev);
-      if (failed) {
-        umma_commit(&sm->drain);
-        volatile int no_abort = 0;
-        mbar_wait(&sm->drain, 0, &no_abort);
-      }
+      // every MMA this thread issued completes before TMEM is released, also
+      // when the consumers gave up (bounded wait, default limit)
+      (void)failed;
+      umma_commit(&sm->drain);
+      volatile int no_abort = 0;
+      mbar_wait(&sm->drain, 0, &no_abort);
     }
   } else if (warp < kCorrWarp0) {
     // ------------------------------------------------------------------
@@ -625,8 +866,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float NEG_INF = neg_inf();
     int gbase = 0;
     bool stop = false;
-    for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
-      const Unit x = unit_at<N>(p, u);
+    for (int k = 0; k < sc.count && !stop; ++k) {
+      const Unit x = sc.get<N>(p, k);
       if (x.n_tiles == 0) continue;
       if (t < N) {
         int lim = 0;
@@ -646,11 +887,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int gi = gbase + j;
         if ((gi & 1) != wg) continue;
         const int bb = wg, st = gi % NS, par = (gi >> 1) & 1;
-        bool ok = mbar_wait(&sm->s_full[bb], par, abort_any);
+        bool ok = mbar_wait(&sm->s_full[bb], par, abort_any, p.wait_ns);
         // P^T[bb] is free once P.V of tile gi - 2 is done, the row statistics
         // once the correction of tile gi - 2 has read them
-        ok = mbar_wait(&sm->o_full[bb], par ^ 1, abort_any) && ok;
-        ok = mbar_wait(&sm->stat_free[bb], par ^ 1, abort_any) && ok;
+        ok = mbar_wait(&sm->o_full[bb], par ^ 1, abort_any, p.wait_ns) && ok;
+        ok = mbar_wait(&sm->stat_free[bb], par ^ 1, abort_any, p.wait_ns) && ok;
         tc_fence_after_sync();
         float sv[N];
 #pragma unroll
@@ -667,8 +908,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // The last tile: keys past the loaded range hold stale bytes or the
           // cache's NaN tails; once V has landed, zero those V rows so that
           // 0 * V stays 0 in P.V.
-          ok = mbar_wait(&sm->full_v[st], (gi / NS) & 1, abort_any) && ok;
-          if (tok >= x.lim_max) {
+          ok = mbar_wait(&sm->full_v[st], (gi / NS) & 1, abort_any, p.wait_ns) && ok;
+          if (ok && tok >= x.lim_max) {
             uint8_t *vrow = smem + C::kOffV + st * C::kKVBytes + t * 128;
 #pragma unroll
             for (int h = 0; h < D / 64; ++h)
@@ -753,18 +994,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = NEG_INF, l_run = 0.f;
     int gbase = 0;
     bool stop = false;
-    for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
-      const Unit x = unit_at<N>(p, u);
+    for (int k = 0; k < sc.count && !stop; ++k) {
+      const Unit x = sc.get<N>(p, k);
       if (t == 0) check_sequence(p, x);
-      if (x.n_tiles == 0) continue;
+      if (x.n_tiles == 0) {
+        // direct write: rows of this unit see no key (out = 0, lse = -inf)
+        if (p.direct && x.rows > 0) {
+#pragma unroll
+          for (int c = 0; c < N; ++c) acc[c] = 0.f;
+          float none[N];
+#pragma unroll
+          for (int c = 0; c < N; ++c) none[c] = NEG_INF;
+          write_final_cols<D, N>(p, x, t, acc, none, none);
+        }
+        continue;
+      }
 #pragma unroll
       for (int c = 0; c < N; ++c) acc[c] = 0.f;
       m_run = NEG_INF;
       l_run = 0.f;
       for (int j = 0; j < x.n_tiles; ++j) {
         const int gi = gbase + j, bb = gi & 1, par = (gi >> 1) & 1;
-        bool ok = mbar_wait(&sm->p_full[bb], par, abort_any);  // the tile's row statistics
-        ok = mbar_wait(&sm->o_full[bb], par, abort_any) && ok;  // its P.V
+        bool ok = mbar_wait(&sm->p_full[bb], par, abort_any, p.wait_ns);  // the tile's row statistics
+        ok = mbar_wait(&sm->o_full[bb], par, abort_any, p.wait_ns) && ok;  // its P.V
         tc_fence_after_sync();
         if (t < x.rows) {
           const float tm = sm->tmax[bb][t];
@@ -813,6 +1065,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sm->o_free[bb]);
       }
       if (stop) break;
+      if (p.direct) {
+        // every row of the call has at most one split: out / lse here
+        if (t < x.rows) {
+          sm->fin_m[t] = m_run;
+          sm->fin_l[t] = l_run;
+        }
+        wg_bar_or(bar_id, false);
+        write_final_cols<D, N>(p, x, t, acc, sm->fin_m, sm->fin_l);
+        gbase += x.n_tiles;
+        continue;
+      }
       // epilogue: unnormalised split partial of every real row
       const int64_t S = p.n_splits;
 #pragma unroll

@@ -177,7 +177,11 @@ int launch_split(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensor
     if (dev >= 0 && dev < kMaxDevices) attr_set[dev].store(true, std::memory_order_release);
   }
   const int grid = p.n_units < sm_count(dev) ? p.n_units : sm_count(dev);
-  kern<<<grid, pkv::kThreads, C::kSmemBytes, s>>>(p, mk, mv);
+  // balanced unit order when it fits the kernel's schedule arrays
+  pkv::AttnParams pp = p;
+  pp.sched = (p.n_units <= pkv::kSchedMaxUnits &&
+              ceil_div(p.n_units, grid) <= pkv::kSchedMaxMine) ? 1 : 0;
+  kern<<<grid, pkv::kThreads, C::kSmemBytes, s>>>(pp, mk, mv);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -202,7 +206,10 @@ int launch_rows(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensorM
     if (dev >= 0 && dev < kMaxDevices) attr_set[dev].store(true, std::memory_order_release);
   }
   const int grid = p.n_units < sm_count(dev) ? p.n_units : sm_count(dev);
-  kern<<<grid, pkv::kRowThreads, C::kSmemBytes, s>>>(p, mk, mv, mq);
+  pkv::AttnParams pp = p;
+  pp.sched = (p.n_units <= pkv::kSchedMaxUnits &&
+              ceil_div(p.n_units, grid) <= pkv::kSchedMaxMine) ? 1 : 0;
+  kern<<<grid, pkv::kRowThreads, C::kSmemBytes, s>>>(pp, mk, mv, mq);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -229,6 +236,8 @@ int launch_bwd(const pkv::BwdParams &p, int64_t kv_ctas, int64_t q_ctas, cudaStr
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// Few rows (decode: rows x splits partials spread over one block per row)
+// or many (prefill, packed batches: one warp per row).
 // Few rows (decode: rows x splits partials spread over one block per row)
 // or many (prefill, packed batches: one warp per row).
 template <int D>
@@ -338,7 +347,7 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
                void *out, const int64_t out_strides[3], float *lse, void *workspace,
                size_t workspace_bytes, int32_t *err, void *stream,
                const FusedAppend *app = nullptr, const PackedQ *pq = nullptr,
-               const SplitShare *share = nullptr) {
+               const SplitShare *share = nullptr, uint64_t wait_ns = pkv::kWaitTimeoutNs) {
   if (!q || !k_cache || !v_cache || !block_table || !seqlens) return PKV_ERR_ARG;
   if (!share && (!out || !lse)) return PKV_ERR_ARG;
   if (share && (pq || app || share->split_begin < 0 || share->n_local <= 0)) return PKV_ERR_ARG;
@@ -416,6 +425,7 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
   p.n_splits = static_cast<int>(S);
   p.n_units = static_cast<int>(units);
   p.max_seqlen_k = max_seqlen_k;
+  p.wait_ns = wait_ns;
   p.cscale = scale * 1.4426950408889634f;  // host IEEE multiply, one rounding
   p.causal = causal ? 1 : 0;
   p.ws_acc = ws_acc;
@@ -472,6 +482,22 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
     p.v_sh = v_strides[2];
   }
 
+  // Every row of a call with one split is finished by the kernel that computed
+  // it, with the merge's fold of one partial (the same bits): no merge launch.
+  // With more splits the row-major kernel still finishes rows of at most one
+  // split and the merge skips them.
+  p.direct = (S == 1 && !share) ? 1 : 0;
+  if (!share) {
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.o_sb = out_strides[0];
+    p.o_ss = out_strides[1];
+    p.o_sh = out_strides[2];
+    p.lse = lse;
+    p.out_vec = (aligned16(out) && out_strides[0] % 8 == 0 && out_strides[1] % 8 == 0 &&
+                 out_strides[2] % 8 == 0)
+                    ? 1
+                    : 0;
+  }
   // A packed call whose longest request needs the row-major kernel also
   // serves its short requests (at most 16 / G queries: one 16-row tile) with
   // the transposed kernel, which keeps decode steps at memory speed; each
@@ -489,29 +515,13 @@ int attn_entry(const void *q, const int64_t q_strides[3], const void *k_cache,
     p.nq_lo = small_nq + 1;
   }
   if (N == pkv::kRowsPerTile) {
-    // rows of at most one split are finished by the split kernel itself; the
-    // merge (needed with more than one split, or for the short requests of a
-    // packed call) skips them
-    p.direct = (S == 1 && !share && !split_by_size) ? 1 : 0;
-    if (!share) {
-      p.out = static_cast<__nv_bfloat16 *>(out);
-      p.o_sb = out_strides[0];
-      p.o_ss = out_strides[1];
-      p.o_sh = out_strides[2];
-      p.lse = lse;
-      p.out_vec = (aligned16(out) && out_strides[0] % 8 == 0 && out_strides[1] % 8 == 0 &&
-                   out_strides[2] % 8 == 0)
-                      ? 1
-                      : 0;
-    }
     rc = D == 128 ? launch_rows<128>(p, mk, mv, mq, s, dev) : launch_rows<64>(p, mk, mv, mq, s, dev);
-    if (rc != PKV_OK || p.direct || share) return rc;
   } else if (D == 128) {
     rc = N == 16 ? launch_split<128, 16>(p, mk, mv, s, dev) : launch_split<128, 64>(p, mk, mv, s, dev);
   } else {
     rc = N == 16 ? launch_split<64, 16>(p, mk, mv, s, dev) : launch_split<64, 64>(p, mk, mv, s, dev);
   }
-  if (rc != PKV_OK || share) return rc;
+  if (rc != PKV_OK || share || p.direct) return rc;
 
   pkv::MergeParams m{};
   m.seqlens = seqlens;
@@ -593,6 +603,22 @@ int pkv_paged_prefill_attn(const void *q, const int64_t q_strides[3], const void
                     bt_stride, max_blocks_per_seq, seqlens, max_seqlen_k, batch, seqlen_q, Hq, Hkv,
                     D, block_size, scale, causal, out, out_strides, lse, workspace,
                     workspace_bytes, err, stream);
+}
+
+int pkv_debug_paged_decode_attn(const void *q, const int64_t q_strides[3], const void *k_cache,
+                                const int64_t k_strides[3], const void *v_cache,
+                                const int64_t v_strides[3], int64_t num_blocks,
+                                const int32_t *block_table, int64_t bt_stride,
+                                int max_blocks_per_seq, const int32_t *seqlens, int max_seqlen_k,
+                                int batch, int seqlen_q, int Hq, int Hkv, int D, int block_size,
+                                float scale, int causal, void *out, const int64_t out_strides[3],
+                                float *lse, void *workspace, size_t workspace_bytes, int32_t *err,
+                                void *stream, uint64_t wait_limit_ns) {
+  if (wait_limit_ns > pkv::kWaitTimeoutNs) return PKV_ERR_ARG;
+  return attn_entry(q, q_strides, k_cache, k_strides, v_cache, v_strides, num_blocks, block_table,
+                    bt_stride, max_blocks_per_seq, seqlens, max_seqlen_k, batch, seqlen_q, Hq, Hkv,
+                    D, block_size, scale, causal, out, out_strides, lse, workspace,
+                    workspace_bytes, err, stream, nullptr, nullptr, nullptr, wait_limit_ns);
 }
 
 int pkv_paged_decode_attn_append(const void *q, const int64_t q_strides[3], const void *k_new,

@@ -60,20 +60,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Every pipeline wait in this library is bounded: after kWaitTimeoutNs of
-// wall time (or as soon as *abort is set by another thread of the CTA) the
-// wait gives up, sets *abort and returns false.  No correct run comes within
-// orders of magnitude of the limit; it exists so that a logic error can never
-// hang the GPU.
+// Every pipeline wait in this library is bounded: after limit_ns of wall time
+// (kWaitTimeoutNs unless the call asked for less) or as soon as *abort is set
+// by another thread of the CTA, the wait gives up, sets *abort and returns
+// false.  No correct run comes within orders of magnitude of the default
+// limit; it exists so that a logic error can never hang the GPU.  The waits
+// of the abort path itself (a thread's own copies and MMAs in flight) always
+// take the default limit.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
 
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort = 1;
       return false;
     }

@@ -45,6 +45,8 @@ def test_constants_agree_with_header(lib):
     assert m["PKV_DEVERR_BAD_BLOCK"] == binding.DEVERR_BAD_BLOCK
     assert m["PKV_DEVERR_TABLE_WIDTH"] == binding.DEVERR_TABLE_WIDTH
     assert m["PKV_DEVERR_TIMEOUT"] == binding.DEVERR_TIMEOUT
+    assert m["PKV_DEVERR_QUERY_LEN"] == binding.DEVERR_QUERY_LEN
+    assert m["PKV_DEVERR_SEQ_LEN"] == binding.DEVERR_SEQ_LEN
 
 
 def test_strerror_covers_every_status(lib):
@@ -229,3 +231,14 @@ def test_backward_and_packed_append_reject_bad_arguments(lib):
     assert app(D=96) == E["PKV_ERR_ARG"]
     assert app(total=-1) == E["PKV_ERR_ARG"]
     assert app(total=0) == 0   # nothing to append: no launch
+
+
+def test_debug_wait_limit_above_the_default_is_rejected_before_any_cuda_call(lib):
+    # the debug entry point may only lower the 2 s limit of every pipeline wait
+    fn = lib.pkv_debug_paged_decode_attn
+    fn.argtypes = binding._ATTN_ARGS + [ctypes.c_uint64]
+    fn.restype = ctypes.c_int
+    assert fn(*_attn_args(), 2_000_000_001) == header_macros()["PKV_ERR_ARG"]
+    # and it checks every other argument like pkv_paged_decode_attn
+    assert fn(*_attn_args(D=96), 0) == header_macros()["PKV_ERR_ARG"]
+    assert fn(*_attn_args(ws_bytes=100), 0) == header_macros()["PKV_ERR_WORKSPACE"]
