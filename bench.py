@@ -63,6 +63,9 @@ def parse_args():
     ap.add_argument("--context", type=int, default=131072,
                     help="tokens per sequence (a smaller workload for profiling captures)")
     ap.add_argument("--batch", type=int, default=4)
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the secondary objects (prefill, varlen, backward, other decode "
+                         "workloads): the decode step alone, for launch-list captures")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only the prefill backward and print its result object")
     ap.add_argument("--varlen-only", action="store_true",
@@ -574,7 +577,7 @@ def run_ours(args):
     if (args.context, args.batch) != (131072, 4):
         result["config"]["workload"] = (f"profiling size: batch {B}, context {ctx} "
                                         "(otherwise as the long-context workload)")
-    if world == 1 and (args.context, args.batch) == (131072, 4):
+    if world == 1 and (args.context, args.batch) == (131072, 4) and not args.no_secondary:
         bf16_peak = None
         try:
             with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:

@@ -56,6 +56,9 @@ struct RowCfg {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static constexpr int kD = D, kN = kRowsPerTile, kNS = NS, kQB = 2;
   static constexpr bool kQTma = true;  // Q rows arrive by TMA
+  // a unit's Q buffer is released by its last QK^T alone, so the next unit's
+  // Q may be loaded before the current unit's last tile is issued
+  static constexpr bool kEarlyQ = true;
   static constexpr int kHalfBytes = kTileTokens * 128;  // 128 keys x 64 head_dim x bf16
   static constexpr int kKVBytes = (D / 64) * kHalfBytes;
   static constexpr int kQHalfBytes = kRowsPerTile * 128;

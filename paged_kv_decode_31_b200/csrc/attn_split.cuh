@@ -176,6 +176,10 @@ struct Cfg {
   static_assert(QB == 1 || QB == 2, "Q buffers");
   static constexpr int kD = D, kN = N, kNS = NS, kQB = QB;
   static constexpr bool kQTma = false;  // Q rows staged with plain loads
+  // Two Q buffers: the epilogue of a unit is staged in its Q buffer, so the
+  // next unit's Q is loaded only after the current unit's last tile is issued
+  // (see produce()).
+  static constexpr bool kEarlyQ = false;
   static constexpr int kHalfBytes = kTileTokens * 128;   // 128 tokens x 64 head_dim x bf16
   static constexpr int kKVBytes = (D / 64) * kHalfBytes;  // one K (or V) tile
   static constexpr int kQHalfBytes = N * 128;
@@ -575,7 +579,7 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
       const int *tab = tabs[ui & 1];
       if (p.n_new > 0) append_new_tokens<D>(p, cur, tab, with_q, lane);
       for (int j = 0; j < cur.n_tiles && !failed; ++j, ++gi) {
-        if (with_q && QB == 2 && nu >= 0 && j == cur.n_tiles - 1) {
+        if (C::kEarlyQ && with_q && QB == 2 && nu >= 0 && j == cur.n_tiles - 1) {
           // the next unit's Q goes to the buffer of the previous unit, whose
           // QKs are done by the time this unit's last tile is issued
           const int qb = (ui + 1) % QB;
@@ -626,7 +630,13 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
       }
       if (failed || nu < 0) break;
       // unit boundary: the next unit's entries (and Q) are in shared memory
-      if (with_q && !q_early) {  // one Q buffer: wait until this unit's QKs are done
+      // The next unit's Q goes into the buffer of the unit before this one,
+      // once that unit has released it.  Without kEarlyQ the release also
+      // waits for that unit's epilogue, which needs the P.V of its last
+      // tile, which the MMA warp issues after the QK^T of this unit's first
+      // tile: the wait then comes after every tile of this unit is issued
+      // (waiting earlier would close a cycle when this unit has one tile).
+      if (with_q && !q_early) {
         const int qb = (ui + 1) % QB;
         bool okq = true;
         if (lane == 0) okq = mbar_wait(&sm->q_empty[qb], (((ui + 1) / QB) & 1) ^ 1, abort_any, p.wait_ns);
@@ -677,11 +687,13 @@ __device__ __forceinline__ void produce(const AttnParams &p, const CUtensorMap *
 // partial, so the bits are those the merge would write.  Thread t < D writes
 // column t of every row (acc[c] = the row's unnormalised column t); thread
 // t < rows also writes row t's lse.  m / l of every row come from shared
-// memory (fin_m / fin_l), published before the call.
+// memory (fin_m / fin_l), published before the call.  With `stage` (shared
+// memory, [rows][D] bf16) the out rows go there instead, for bulk stores.
 template <int D, int N>
 __device__ __forceinline__ void write_final_cols(const AttnParams &p, const Unit &x, int t,
                                                  const float (&acc)[N], const float *fin_m,
-                                                 const float *fin_l) {
+                                                 const float *fin_l,
+                                                 __nv_bfloat16 *stage = nullptr) {
   const float NEG_INF = neg_inf();
 #pragma unroll
   for (int c = 0; c < N; ++c) {
@@ -697,7 +709,10 @@ __device__ __forceinline__ void write_final_cols(const AttnParams &p, const Unit
         A = fold_val(0.f, acc[c], kc);
       }
       const __nv_bfloat16 ob = __float2bfloat16_rn(final_out(A, L));
-      p.out[o_tok_off(p, x, i) + h * p.o_sh + t] = ob;
+      if (stage)
+        stage[c * D + t] = ob;
+      else
+        p.out[o_tok_off(p, x, i) + h * p.o_sh + t] = ob;
       if (p.fin_out != nullptr && i == x.nq - 1) p.fin_out[x.b * p.fo_sb + h * p.fo_sh + t] = ob;
     }
   }
@@ -748,7 +763,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < QB; ++i) {
       mbar_init(&sm->q_full[i], 1);
-      mbar_init(&sm->q_empty[i], 1);
+      // two Q buffers: the buffer is free once the unit's last QK^T is done
+      // (MMA commit) and the correction warpgroup has staged that unit's
+      // epilogue through it (one arrival)
+      mbar_init(&sm->q_empty[i], QB == 2 ? 2 : 1);
     }
     mbar_init(&sm->drain, 1);
     sm->abort_any = 0;
@@ -992,7 +1010,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float NEG_INF = neg_inf();
     float acc[N];
     float m_run = NEG_INF, l_run = 0.f;
-    int gbase = 0;
+    int gbase = 0, cui = 0;  // cui: ordinal of the unit among this CTA's units with work
+    bool bulk_out = false;   // thread 0 has bulk stores to complete before exit
     bool stop = false;
     for (int k = 0; k < sc.count && !stop; ++k) {
       const Unit x = sc.get<N>(p, k);
@@ -1072,30 +1091,90 @@ __global__ void __launch_bounds__(kThreads, 1)
           sm->fin_l[t] = l_run;
         }
         wg_bar_or(bar_id, false);
-        write_final_cols<D, N>(p, x, t, acc, sm->fin_m, sm->fin_l);
-        gbase += x.n_tiles;
-        continue;
-      }
-      // epilogue: unnormalised split partial of every real row
-      const int64_t S = p.n_splits;
+        if constexpr (QB == 2) {
+          if (p.out_vec) {
+            // the out rows go through this unit's Q buffer and bulk stores
+            // (at most N rows of D bf16: the buffer's size)
+            __nv_bfloat16 *stage =
+                reinterpret_cast<__nv_bfloat16 *>(smem + C::kOffQ + (cui % QB) * C::kQBytes);
+            write_final_cols<D, N>(p, x, t, acc, sm->fin_m, sm->fin_l, stage);
+            fence_proxy_async_smem();
+            wg_bar_or(bar_id, false);
+            if (t == 0) {
+              for (int c = 0; c < x.rows; ++c) {
+                const int r = x.row0 + c;
+                const int i = r / p.G, g = r - i * p.G;
+                bulk_store(p.out + o_tok_off(p, x, i) + (x.kvh * p.G + g) * p.o_sh, stage + c * D,
+                           D * 2);
+              }
+              bulk_commit();
+              bulk_out = true;
+            }
+          } else {
+            write_final_cols<D, N>(p, x, t, acc, sm->fin_m, sm->fin_l);
+          }
+        } else {
+          write_final_cols<D, N>(p, x, t, acc, sm->fin_m, sm->fin_l);
+        }
+      } else {
+        // epilogue: unnormalised split partial of every real row.  With two Q
+        // buffers, this unit's (its QK^T are done) stages the rows and the
+        // TMA engine stores them, so no thread waits on global stores while
+        // the SM streams the cache.
+        const int64_t S = p.n_splits;
+        if constexpr (QB == 2) {
+          float *stage = reinterpret_cast<float *>(smem + C::kOffQ + (cui % QB) * C::kQBytes);
+          constexpr int kRowsStaged = C::kQBytes / (D * 4);
+          for (int c0 = 0; c0 < x.rows; c0 += kRowsStaged) {
+            if (c0 > 0 && t == 0) bulk_wait_read<0>();  // the previous round has read the stage
+            if (c0 > 0) wg_bar_or(bar_id, false);
 #pragma unroll
-      for (int c = 0; c < N; ++c) {
-        if (c < x.rows && t < D) {
-          const int r = x.row0 + c;
+            for (int c = 0; c < N; ++c)
+              if (c >= c0 && c < min(x.rows, c0 + kRowsStaged) && t < D)
+                stage[(c - c0) * D + t] = acc[c];
+            fence_proxy_async_smem();
+            wg_bar_or(bar_id, false);
+            if (t == 0) {
+              for (int c = c0; c < min(x.rows, c0 + kRowsStaged); ++c) {
+                const int r = x.row0 + c;
+                const int i = r / p.G, g = r - i * p.G;
+                const int64_t row_id = (x.q0 + i) * p.Hq + x.kvh * p.G + g;
+                bulk_store(p.ws_acc + (row_id * S + x.s) * D, stage + (c - c0) * D, D * 4);
+              }
+              bulk_commit();
+              bulk_out = true;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < N; ++c) {
+            if (c < x.rows && t < D) {
+              const int r = x.row0 + c;
+              const int i = r / p.G, g = r - i * p.G;
+              const int64_t row_id = (x.q0 + i) * p.Hq + x.kvh * p.G + g;
+              p.ws_acc[(row_id * S + x.s) * D + t] = acc[c];
+            }
+          }
+        }
+        if (t < x.rows) {
+          const int r = x.row0 + t;
           const int i = r / p.G, g = r - i * p.G;
           const int64_t row_id = (x.q0 + i) * p.Hq + x.kvh * p.G + g;
-          p.ws_acc[(row_id * S + x.s) * D + t] = acc[c];
+          *reinterpret_cast<float2 *>(p.ws_ml + (row_id * S + x.s) * 2) = make_float2(m_run, l_run);
         }
       }
-      if (t < x.rows) {
-        const int r = x.row0 + t;
-        const int i = r / p.G, g = r - i * p.G;
-        const int64_t row_id = (x.q0 + i) * p.Hq + x.kvh * p.G + g;
-        p.ws_ml[(row_id * S + x.s) * 2 + 0] = m_run;
-        p.ws_ml[(row_id * S + x.s) * 2 + 1] = l_run;
+      if constexpr (QB == 2) {
+        // the stage has been read: the producer may load a later unit's Q here
+        if (t == 0) {
+          if (bulk_out) bulk_wait_read<0>();
+          mbar_arrive(&sm->q_empty[cui % QB]);
+        }
       }
+      ++cui;
       gbase += x.n_tiles;
     }
+    // the partials are complete in global memory before the CTA leaves
+    if (bulk_out) bulk_wait<0>();
     (void)stop;
   }
 
