@@ -23,8 +23,15 @@
 // 544 threads: warps 0-15 stage operands and do the elementwise work -- warps
 // w, w + 4, w + 8, w + 12 share TMEM lanes 32 (w % 4) .. + 31 (thread t = lane
 // t of the 128) and split the columns in quarters -- and warp 16 owns TMEM,
-// its lane 0 issuing the MMAs.  Phases are separated by __syncthreads and
-// MMA-completion mbarriers (bounded waits).
+// its lane 0 issuing the MMAs.  The second operand pair of each product (P^T
+// and dS^T, or dS) never touches shared memory: the elementwise pass packs it
+// as bf16 into the TMEM columns its S / dP values came from, and the next MMAs
+// read it from there as their A operand.  The shared memory this frees holds a
+// second buffer of the streamed tiles (Q and dO, or K and V), filled with
+// cp.async while the current tile's MMAs and elementwise pass run; one
+// barrier per tile hands both the packed TMEM operands and the next tile to
+// the MMA warp, whose tensor pipe executes the previous tile's accumulation
+// and the current tile's S / dP products back to back.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -120,48 +127,36 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ B
 
 template <int D>
 struct BwdCfg {
-  static constexpr int kHalf = kBwdTile * 128;          // 128 rows x 64 elements x bf16
-  static constexpr int kTile = (D / 64) * kHalf;        // a [128][D] operand
-  static constexpr int kSq = 2 * kHalf;                 // a [128][128] operand
+  static constexpr int kHalf = kBwdTile * 128;    // 128 rows x 64 elements x bf16
+  static constexpr int kTile = (D / 64) * kHalf;  // a [128][D] operand
+  static constexpr int kTiles = 6;                // two fixed + two double-buffered
   struct Small {
-    uint64_t mma_a, mma_b, drain;
+    uint64_t mma_a, mma_b, mma_bv, drain;
     uint32_t tmem_base;
-    int abort_any;
-    int lim[kBwdTile];       // key limit of each row of the current row tile
-    float lse2[kBwdTile];
-    float dsum[kBwdTile];
+    int lim[2][kBwdTile];  // key limit of each row of the row tile in buffer j
+    float lse2[2][kBwdTile];
+    float dsum[2][kBwdTile];
   };
+  static constexpr int kSmem = kTiles * kTile + static_cast<int>(sizeof(Small)) + 1024;
 };
 
-// Stage [128][D] bf16 tiles, rows given by `src_row(c)` (nullptr: zeros),
-// 128-byte swizzled K-major (row c at c * 128 bytes of its 64-element half).
-// Every load of a thread is issued before its first store, so the tile costs
-// about one memory round trip.
+// cp.async a [128][D] bf16 tile, rows given by `src_row(c)` (nullptr: zeros),
+// into the 128-byte swizzled K-major layout of the MMA operands (row c at
+// c * 128 bytes of its 64-element half, 16-byte chunk cc at (cc ^ (c % 8)) * 16).
+// `any` is a valid global address for the zero-filled chunks, of which nothing
+// is read.  The caller commits the group.
 template <int D, class F>
-__device__ __forceinline__ void stage_rows(uint8_t *dst, int t, F src_row) {
+__device__ __forceinline__ void async_rows(uint8_t *dst, int t, const void *any, F src_row) {
   constexpr int kPer = kBwdTile * (D / 8) / kBwdCompute;  // 16-byte chunks per thread
-  uint4 v[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) {
     const int idx = t + k * kBwdCompute;
     const int c = idx / (D / 8), ch = idx % (D / 8);
     const __nv_bfloat16 *s = src_row(c);
-    v[k] = s ? __ldg(reinterpret_cast<const uint4 *>(s) + ch) : make_uint4(0u, 0u, 0u, 0u);
-  }
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int idx = t + k * kBwdCompute;
-    const int c = idx / (D / 8), ch = idx % (D / 8);
     const int h = ch >> 3, cc = ch & 7;
-    *reinterpret_cast<uint4 *>(dst + h * BwdCfg<D>::kHalf + c * 128 + ((cc ^ (c & 7)) << 4)) = v[k];
+    cp_async16(dst + h * BwdCfg<D>::kHalf + c * 128 + ((cc ^ (c & 7)) << 4),
+               s ? static_cast<const void *>(s + ch * 8) : any, s ? 16u : 0u);
   }
-}
-
-// Eight bf16 (one 16-byte chunk) into row `row` of a [128][128] K-major
-// swizzled operand, columns [col8 * 8, col8 * 8 + 8).
-__device__ __forceinline__ void put8(uint8_t *dst, int row, int col8, uint4 v) {
-  const int h = col8 >> 3, cc = col8 & 7;
-  *reinterpret_cast<uint4 *>(dst + h * (kBwdTile * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -178,8 +173,8 @@ __device__ __forceinline__ int bwd_row_lim(const BwdParams &p, int seqlen, int r
   return lim > 0 ? lim : 0;
 }
 
-// Cache row of token `tok` of sequence b (nullptr past the table or the
-// cache, with the error bits set as in the forward).
+// Cache row of token `tok` of sequence b (-1 past the table or the cache,
+// with the error bits set as in the forward).
 __device__ __forceinline__ int64_t bwd_block(const BwdParams &p, int b, int tok) {
   const int col = tok >> p.block_shift;
   if (col >= p.max_blocks_per_seq) {
@@ -194,7 +189,28 @@ __device__ __forceinline__ int64_t bwd_block(const BwdParams &p, int b, int tok)
   return blk;
 }
 
-// Issue D[tmem] = A[128 x K] * B^T for two K-major [128][K] operands.
+// Row of token tok0 + c of one cache (nullptr past the context or the table).
+__device__ __forceinline__ const __nv_bfloat16 *bwd_cache_row(const BwdParams &p, const __nv_bfloat16 *cache,
+                                                              int64_t sb, int64_t ss, int64_t sh, int b,
+                                                              int kvh, int seqlen, int tok) {
+  if (tok >= seqlen) return nullptr;
+  const int64_t blk = bwd_block(p, b, tok);
+  if (blk < 0) return nullptr;
+  return cache + blk * sb + (tok & ((1 << p.block_shift) - 1)) * ss + kvh * sh;
+}
+
+// Row r = i G + g of the row tiles of (b, kvh) in a [batch][seqlen_q][Hq][D]
+// tensor (nullptr for padded rows).
+__device__ __forceinline__ const __nv_bfloat16 *bwd_query_row(const BwdParams &p, const __nv_bfloat16 *base,
+                                                              int64_t sb, int64_t ss, int64_t sh, int b,
+                                                              int kvh, int r) {
+  if (r >= p.G * p.seqlen_q) return nullptr;
+  const int i = r / p.G, g = r - i * p.G;
+  return base + b * sb + static_cast<int64_t>(i) * ss + static_cast<int64_t>(kvh * p.G + g) * sh;
+}
+
+// Issue D[tmem] = A[128 x K] * B^T for two K-major [128][K] operands in
+// shared memory.
 template <int K>
 __device__ __forceinline__ void mma_kk(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc) {
 #pragma unroll
@@ -206,37 +222,51 @@ __device__ __forceinline__ void mma_kk(uint32_t d, uint32_t a, uint32_t b, uint3
   }
 }
 
-// Issue D[tmem] (+)= A[128 x 128] * B[128 x N], A K-major, B MN-major (a
-// [128][N] tile read along its rows).
+// Issue D[tmem] (+)= A[128 x 128] * B[128 x N]: A packed bf16 in TMEM, its
+// K steps of 16 at columns a + 16 kk .. + 8 (where the elementwise pass wrote
+// them over the 16 fp32 columns they came from); B a [128][N] tile in shared
+// memory read along its rows (MN-major).
 template <int N>
-__device__ __forceinline__ void mma_kn(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc,
+__device__ __forceinline__ void mma_tn(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc,
                                        bool accumulate) {
 #pragma unroll
-  for (int kk = 0; kk < kBwdTile / 16; ++kk) {
-    const int h = kk >> 2, off = (kk & 3) * 32;
-    umma_bf16(d, smem_desc(a + h * (kBwdTile * 128) + off, 16, 1024, kLayoutSw128),
-              smem_desc(b + kk * 2048, kBwdTile * 128, 1024, kLayoutSw128), idesc,
-              (accumulate || kk > 0) ? 1u : 0u);
-  }
+  for (int kk = 0; kk < kBwdTile / 16; ++kk)
+    umma_bf16_ts(d, a + kk * 16, smem_desc(b + kk * 2048, kBwdTile * 128, 1024, kLayoutSw128), idesc,
+                 (accumulate || kk > 0) ? 1u : 0u);
+}
+
+__device__ __forceinline__ uint8_t *bwd_smem_base(uint8_t *raw) {
+  return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
+                                     ~static_cast<uintptr_t>(1023));
 }
 
 // ---------------------------------------------------------------------------
 // dK / dV: one CTA per (b, kvh, key tile).
-// smem: K, V, Q, dO tiles ([128][D]), P^T and dS^T ([128 keys][128 rows]).
-// TMEM: S^T [0,128), dP^T [128,256), dV [256, 256 + D), dK [256 + D, 256 + 2D).
+// smem: K, V, then Q and dO of row tile j (j = it % 2) at (2 + 2 j) and
+// (3 + 2 j) tiles.
+// TMEM: S^T [0,128) (P^T packed over it), dP^T [128,256) (dS^T packed over
+// it), dV [256, 256 + D), dK [256 + D, 256 + 2D).
+// Tile it: barrier; MMA warp: dV += P^T(it - 1) dO, dK += dS^T(it - 1) Q,
+// then S^T = K Q(it)^T, dP^T = V dO(it)^T; compute warps: once the first
+// pair is done, cp.async row tile it + 1 into the other buffer; once the
+// second is, P^T / dS^T of it into TMEM.  MMAs into different accumulators
+// carry no ordering guarantee among themselves, so S^T(it), which overwrites
+// the P^T that dV(it - 1) reads, is issued once dV(it - 1) has completed (its
+// own commit, `mma_bv`, landing while dK(it - 1) runs), and dP^T(it) once
+// dK(it - 1) has (`mma_b`, landing while S^T(it) runs).
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *sK = smem, *sV = sK + C::kTile, *sQ = sV + C::kTile, *sG = sQ + C::kTile;
-  uint8_t *sP = sG + C::kTile, *sS = sP + C::kSq;
-  auto *sm = reinterpret_cast<typename C::Small *>(sS + C::kSq);
+  uint8_t *smem = bwd_smem_base(smem_raw);
+  auto *sm = reinterpret_cast<typename C::Small *>(smem + C::kTiles * C::kTile);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-  const int t = tid & 127, hf = tid >> 7;  // TMEM lane / token, column group (compute threads)
-  volatile int *abort_any = &sm->abort_any;
+  const int t = tid & 127, hf = tid >> 7;  // TMEM lane / key, column group (compute threads)
+  const bool compute = tid < kBwdCompute;
+  const bool issuer = warp == kBwdMmaWarp && lane == 0;
+  int abort_flag = 0;  // the waits' abort word; agreement goes through the barriers
+  volatile int *abort_any = &abort_flag;
 
   int u = blockIdx.x;
   const int kt = u % p.n_key_tiles;
@@ -246,142 +276,171 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
   const int seqlen = max(__ldg(p.seqlens + b), 0);
   const int tok0 = kt * kBwdTile;
   if (tok0 >= seqlen) return;  // uniform: the whole CTA leaves before any barrier
-
-  if (tid == 0) {
-    mbar_init(&sm->mma_a, 1);
-    mbar_init(&sm->mma_b, 1);
-    mbar_init(&sm->drain, 1);
-    sm->abort_any = 0;
-    fence_barrier_init();
-  }
-  if (warp == kBwdMmaWarp) tmem_alloc(&sm->tmem_base, 512);
-  // K and V of this key tile (tokens past the context are zeros)
-  if (tid < kBwdCompute) {
-    stage_rows<D>(sK, tid, [&](int c) -> const __nv_bfloat16 * {
-      const int tok = tok0 + c;
-      if (tok >= seqlen) return nullptr;
-      const int64_t blk = bwd_block(p, b, tok);
-      if (blk < 0) return nullptr;
-      return p.k_cache + blk * p.k_sb + (tok & ((1 << p.block_shift) - 1)) * p.k_ss + kvh * p.k_sh;
-    });
-    stage_rows<D>(sV, tid, [&](int c) -> const __nv_bfloat16 * {
-      const int tok = tok0 + c;
-      if (tok >= seqlen) return nullptr;
-      const int64_t blk = bwd_block(p, b, tok);
-      if (blk < 0) return nullptr;
-      return p.v_cache + blk * p.v_sb + (tok & ((1 << p.block_shift) - 1)) * p.v_ss + kvh * p.v_sh;
-    });
-  }
-  tc_fence_before_sync();
-  __syncthreads();
-  tc_fence_after_sync();
-  const uint32_t tmem = sm->tmem_base;
-  const uint32_t sbase = smem_u32(smem);
-  const uint32_t aK = sbase, aV = aK + C::kTile, aQ = aV + C::kTile, aG = aQ + C::kTile;
-  const uint32_t aP = aG + C::kTile, aS = aP + C::kSq;
-  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
-  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const float NEG_INF = neg_inf();
   const int R = p.G * p.seqlen_q;
-
   // first row tile with a row that sees key tok0: rows r with i >= tok0 - (seqlen - sq)
   int rt0 = 0;
   if (p.causal) {
     const int i_min = tok0 - (seqlen - p.seqlen_q);
     rt0 = i_min > 0 ? (i_min * p.G) / kBwdTile : 0;
   }
-  int it = 0;
-  for (int rt = rt0; rt * kBwdTile < R; ++rt, ++it) {
+  const int n = (R + kBwdTile - 1) / kBwdTile - rt0;  // row tiles, >= 1
+
+  if (tid == 0) {
+    mbar_init(&sm->mma_a, 1);
+    mbar_init(&sm->mma_b, 1);
+    mbar_init(&sm->mma_bv, 1);
+    mbar_init(&sm->drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == kBwdMmaWarp) tmem_alloc(&sm->tmem_base, 512);
+
+  // Q / dO rows of row tile rt into buffer j, with the row statistics
+  // loaded into registers (stored by the caller once the tile's elementwise
+  // pass no longer reads that buffer).
+  int n_lim = 0;
+  float n_l2 = 0.f, n_ds = 0.f;
+  auto stage_rows_of = [&](int rt, int j) {
     const int row0 = rt * kBwdTile;
-    if (tid < kBwdCompute) {
-      auto rowptr = [&](const __nv_bfloat16 *base, int64_t sb, int64_t ss, int64_t sh, int c)
-          -> const __nv_bfloat16 * {
-        const int r = row0 + c;
-        if (r >= R) return nullptr;
+    async_rows<D>(smem + (2 + 2 * j) * C::kTile, tid, p.q, [&](int c) {
+      return bwd_query_row(p, p.q, p.q_sb, p.q_ss, p.q_sh, b, kvh, row0 + c);
+    });
+    async_rows<D>(smem + (3 + 2 * j) * C::kTile, tid, p.q, [&](int c) {
+      return bwd_query_row(p, p.dout, p.g_sb, p.g_ss, p.g_sh, b, kvh, row0 + c);
+    });
+    cp_async_commit();
+    if (hf == 0) {
+      const int r = row0 + t;
+      n_lim = bwd_row_lim(p, seqlen, r);
+      n_l2 = 0.f;
+      n_ds = 0.f;
+      if (r < R) {
         const int i = r / p.G, g = r - i * p.G;
-        return base + b * sb + static_cast<int64_t>(i) * ss + static_cast<int64_t>(kvh * p.G + g) * sh;
-      };
-      stage_rows<D>(sQ, tid, [&](int c) { return rowptr(p.q, p.q_sb, p.q_ss, p.q_sh, c); });
-      stage_rows<D>(sG, tid, [&](int c) { return rowptr(p.dout, p.g_sb, p.g_ss, p.g_sh, c); });
-      if (hf == 0) {
-        const int r = row0 + t;
-        sm->lim[t] = bwd_row_lim(p, seqlen, r);
-        float l2 = 0.f, ds = 0.f;
-        if (r < R) {
-          const int i = r / p.G, g = r - i * p.G;
-          const int64_t row_id = (static_cast<int64_t>(b) * p.seqlen_q + i) * p.Hq + kvh * p.G + g;
-          l2 = p.row_lse2[row_id];
-          ds = p.row_d[row_id];
-        }
-        sm->lse2[t] = l2;
-        sm->dsum[t] = ds;
+        const int64_t row_id = (static_cast<int64_t>(b) * p.seqlen_q + i) * p.Hq + kvh * p.G + g;
+        n_l2 = p.row_lse2[row_id];
+        n_ds = p.row_d[row_id];
       }
-      fence_proxy_async_smem();
     }
-    tc_fence_before_sync();
-    __syncthreads();
-    if (*abort_any) break;
-    if (warp == kBwdMmaWarp && lane == 0) {
-      tc_fence_after_sync();
-      constexpr uint32_t kId = idesc_bf16(128, 128, 0, 0);
-      mma_kk<D>(tS, aK, aQ, kId);   // S^T = K Q^T
-      mma_kk<D>(tdP, aV, aG, kId);  // dP^T = V dO^T
-      umma_commit(&sm->mma_a);
+  };
+  auto store_stats = [&](int j) {
+    if (hf == 0) {
+      sm->lim[j][t] = n_lim;
+      sm->lse2[j][t] = n_l2;
+      sm->dsum[j][t] = n_ds;
     }
-    if (tid < kBwdCompute) {
-      mbar_wait(&sm->mma_a, it & 1, abort_any);
-      __syncwarp();
-      tc_fence_after_sync();
-      const int tok = tok0 + t;
-#pragma unroll 1
-      for (int ch = hf * (8 / kBwdGroups); ch < (hf + 1) * (8 / kBwdGroups); ++ch) {  // its rows
-        float sv[16], dp[16];
-        tmem_ld16(tS + lane_off + ch * 16, sv);
-        tmem_ld16(tdP + lane_off + ch * 16, dp);
-        tmem_ld_wait_for(sv);
-        tmem_ld_wait_for(dp);
-        uint32_t pw[8], sw[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int c = ch * 16 + e + k;
-            const bool vis = tok < sm->lim[c];
-            const float pr = vis ? ex2(__fsub_rn(__fmul_rn(sv[e + k], p.cscale), sm->lse2[c])) : 0.f;
-            pv[k] = pr;
-            dv[k] = __fmul_rn(pr, __fsub_rn(dp[e + k], sm->dsum[c]));
-          }
-          pw[e / 2] = pack_bf16(pv[0], pv[1]);
-          sw[e / 2] = pack_bf16(dv[0], dv[1]);
-        }
-        put8(sP, t, ch * 2, make_uint4(pw[0], pw[1], pw[2], pw[3]));
-        put8(sP, t, ch * 2 + 1, make_uint4(pw[4], pw[5], pw[6], pw[7]));
-        put8(sS, t, ch * 2, make_uint4(sw[0], sw[1], sw[2], sw[3]));
-        put8(sS, t, ch * 2 + 1, make_uint4(sw[4], sw[5], sw[6], sw[7]));
-      }
-      fence_proxy_async_smem();
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    if (*abort_any) break;
-    if (warp == kBwdMmaWarp && lane == 0) {
-      tc_fence_after_sync();
-      constexpr uint32_t kId = idesc_bf16(128, D, 0, 1);
-      mma_kn<D>(tdV, aP, aG, kId, it > 0);  // dV += P^T dO
-      mma_kn<D>(tdK, aS, aQ, kId, it > 0);  // dK += dS^T Q
-      umma_commit(&sm->mma_b);
-    }
-    // operands are overwritten by the next row tile only after these MMAs
-    mbar_wait(&sm->mma_b, it & 1, abort_any);
-    __syncwarp();
+  };
+
+  // K and V of this key tile (tokens past the context are zeros), row tile rt0
+  if (compute) {
+    async_rows<D>(smem, tid, p.q, [&](int c) {
+      return bwd_cache_row(p, p.k_cache, p.k_sb, p.k_ss, p.k_sh, b, kvh, seqlen, tok0 + c);
+    });
+    async_rows<D>(smem + C::kTile, tid, p.q, [&](int c) {
+      return bwd_cache_row(p, p.v_cache, p.v_sb, p.v_ss, p.v_sh, b, kvh, seqlen, tok0 + c);
+    });
+    stage_rows_of(rt0, 0);
+    store_stats(0);
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
   }
   tc_fence_before_sync();
   __syncthreads();
-  const bool ok = !*abort_any;
-  if (tid < kBwdCompute && ok) {
+  tc_fence_after_sync();
+  const uint32_t tmem = sm->tmem_base;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const int tok = tok0 + t;
+
+  bool ok = true, failed = false;
+  for (int it = 0; it < n; ++it) {
+    const int j = it & 1;
+    if (issuer) {
+      tc_fence_after_sync();
+      if (it > 0) {
+        constexpr uint32_t kIdB = idesc_bf16(128, D, 0, 1);
+        const uint32_t aQ = sbase + (2 + 2 * (j ^ 1)) * C::kTile, aG = aQ + C::kTile;
+        mma_tn<D>(tdV, tS, aG, kIdB, it > 1);   // dV += P^T dO
+        umma_commit(&sm->mma_bv);
+        mma_tn<D>(tdK, tdP, aQ, kIdB, it > 1);  // dK += dS^T Q
+        umma_commit(&sm->mma_b);
+      }
+      constexpr uint32_t kIdA = idesc_bf16(128, 128, 0, 0);
+      const uint32_t aQ = sbase + (2 + 2 * j) * C::kTile, aG = aQ + C::kTile;
+      if (it > 0) ok = mbar_wait(&sm->mma_bv, (it - 1) & 1, abort_any);
+      if (ok) {
+        tc_fence_after_sync();
+        mma_kk<D>(tS, sbase, aQ, kIdA);  // S^T = K Q^T
+      }
+      if (ok && it > 0) ok = mbar_wait(&sm->mma_b, (it - 1) & 1, abort_any);
+      if (ok) {
+        tc_fence_after_sync();
+        mma_kk<D>(tdP, sbase + C::kTile, aG, kIdA);  // dP^T = V dO^T
+        umma_commit(&sm->mma_a);
+      }
+    }
+    if (compute) {
+      // buffer j ^ 1 is free once the accumulation of tile it - 1 is done
+      if (it > 0) ok = ok && mbar_wait(&sm->mma_b, (it - 1) & 1, abort_any);
+      const bool next = ok && it + 1 < n;
+      if (next) stage_rows_of(rt0 + it + 1, j ^ 1);
+      ok = ok && mbar_wait(&sm->mma_a, it & 1, abort_any);
+      if (ok) {
+        __syncwarp();
+        tc_fence_after_sync();
+#pragma unroll 1
+        for (int ch = hf * (8 / kBwdGroups); ch < (hf + 1) * (8 / kBwdGroups); ++ch) {  // its rows
+          float sv[16], dp[16];
+          tmem_ld16(tS + lane_off + ch * 16, sv);
+          tmem_ld16(tdP + lane_off + ch * 16, dp);
+          tmem_ld_wait_for(sv);
+          tmem_ld_wait_for(dp);
+          uint32_t pw[8], sw[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float pv[2], dv[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int c = ch * 16 + e + k;
+              const bool vis = tok < sm->lim[j][c];
+              const float pr =
+                  vis ? ex2(__fsub_rn(__fmul_rn(sv[e + k], p.cscale), sm->lse2[j][c])) : 0.f;
+              pv[k] = pr;
+              dv[k] = __fmul_rn(pr, __fsub_rn(dp[e + k], sm->dsum[j][c]));
+            }
+            pw[e / 2] = pack_bf16(pv[0], pv[1]);
+            sw[e / 2] = pack_bf16(dv[0], dv[1]);
+          }
+          tmem_st8(tS + lane_off + ch * 16, pw);
+          tmem_st8(tdP + lane_off + ch * 16, sw);
+        }
+        tmem_st_wait();
+      }
+      if (next) store_stats(j ^ 1);
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+    }
+    tc_fence_before_sync();
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+  }
+  if (!failed) {
+    if (issuer) {
+      tc_fence_after_sync();
+      const uint32_t aQ = sbase + (2 + 2 * ((n - 1) & 1)) * C::kTile, aG = aQ + C::kTile;
+      constexpr uint32_t kIdB = idesc_bf16(128, D, 0, 1);
+      mma_tn<D>(tdV, tS, aG, kIdB, n > 1);
+      umma_commit(&sm->mma_bv);
+      mma_tn<D>(tdK, tdP, aQ, kIdB, n > 1);
+      umma_commit(&sm->mma_b);
+    }
+    if (compute) ok = mbar_wait(&sm->mma_b, (n - 1) & 1, abort_any);
+    tc_fence_before_sync();
+    failed = __syncthreads_or(!ok);
+  }
+  if (compute && !failed) {
     tc_fence_after_sync();
-    const int tok = tok0 + t;
     int64_t blk = -1;
     if (tok < seqlen) blk = bwd_block(p, b, tok);
     const int slot = tok & ((1 << p.block_shift) - 1);
@@ -396,12 +455,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
         uint32_t wv[8], wk[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          // a tile no row reached leaves zeros (it = 0: accumulators unwritten)
-          const float v0 = it > 0 ? vv[2 * e] : 0.f, v1 = it > 0 ? vv[2 * e + 1] : 0.f;
-          const float k0 = it > 0 ? __fmul_rn(kv[2 * e], p.scale) : 0.f;
-          const float k1 = it > 0 ? __fmul_rn(kv[2 * e + 1], p.scale) : 0.f;
-          wv[e] = pack_bf16(v0, v1);
-          wk[e] = pack_bf16(k0, k1);
+          wv[e] = pack_bf16(vv[2 * e], vv[2 * e + 1]);
+          wk[e] = pack_bf16(__fmul_rn(kv[2 * e], p.scale), __fmul_rn(kv[2 * e + 1], p.scale));
         }
         uint4 *dv = reinterpret_cast<uint4 *>(p.dv_cache + blk * p.dv_sb + slot * p.dv_ss + kvh * p.dv_sh + ch * 16);
         uint4 *dk = reinterpret_cast<uint4 *>(p.dk_cache + blk * p.dk_sb + slot * p.dk_ss + kvh * p.dk_sh + ch * 16);
@@ -412,9 +467,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
       }
     }
   }
-  if (!ok && warp == kBwdMmaWarp && lane == 0) {
+  if (failed && issuer) {
     umma_commit(&sm->drain);
-    volatile int no_abort = 0;
+    int no_abort = 0;
     mbar_wait(&sm->drain, 0, &no_abort);
   }
   tc_fence_before_sync();
@@ -423,26 +478,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
     tc_fence_after_sync();
     tmem_dealloc(tmem, 512);
   }
-  if (tid == 0 && !ok && p.err) atomicOr(p.err, kErrTimeout);
+  if (tid == 0 && failed && p.err) atomicOr(p.err, kErrTimeout);
 }
 
 // ---------------------------------------------------------------------------
 // dQ: one CTA per (b, kvh, row tile).
-// smem: Q, dO, K, V tiles ([128][D]), dS ([128 rows][128 keys]).
-// TMEM: S [0,128), dP [128,256), dQ [256, 256 + D).
+// smem: Q, dO, then K and V of key tile j (j = it % 2) at (2 + 2 j) and
+// (3 + 2 j) tiles.
+// TMEM: S of tile it (dS packed over it) at [0,128) for even it and
+// [384,512) for odd it, dP [128,256), dQ [256, 256 + D).
+// Tile it: barrier; MMA warp: dQ += dS(it - 1) K, then S = Q K(it)^T,
+// dP = dO V(it)^T; compute warps: cp.async key tile it + 1 into the other
+// buffer once the accumulation of it - 1 is done, then dS of it into TMEM.
+// S(it) never lands on the dS(it - 1) that the accumulation reads (MMAs
+// into different accumulators are not ordered among themselves), and dP(it)
+// overwrites values only the elementwise pass read.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *sQ = smem, *sG = sQ + C::kTile, *sK = sG + C::kTile, *sV = sK + C::kTile;
-  uint8_t *sS = sV + C::kTile;
-  auto *sm = reinterpret_cast<typename C::Small *>(sS + C::kSq);
+  uint8_t *smem = bwd_smem_base(smem_raw);
+  auto *sm = reinterpret_cast<typename C::Small *>(smem + C::kTiles * C::kTile);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const int t = tid & 127, hf = tid >> 7;  // TMEM lane / row, column group (compute threads)
-  volatile int *abort_any = &sm->abort_any;
+  const bool compute = tid < kBwdCompute;
+  const bool issuer = warp == kBwdMmaWarp && lane == 0;
+  int abort_flag = 0;
+  volatile int *abort_any = &abort_flag;
 
   int u = blockIdx.x;
   const int rt = u % p.n_row_tiles;
@@ -454,29 +517,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
   const int row0 = rt * kBwdTile;
   // keys [0, lim_max) cover every row of the tile
   const int lim_max = bwd_row_lim(p, seqlen, min(row0 + kBwdTile, R) - 1);
+  const int n = (lim_max + kBwdTile - 1) / kBwdTile;
 
   if (tid == 0) {
     mbar_init(&sm->mma_a, 1);
     mbar_init(&sm->mma_b, 1);
+    mbar_init(&sm->mma_bv, 1);
     mbar_init(&sm->drain, 1);
-    sm->abort_any = 0;
     fence_barrier_init();
   }
   if (warp == kBwdMmaWarp) tmem_alloc(&sm->tmem_base, 512);
+  auto stage_keys_of = [&](int kt, int j) {
+    const int k0 = kt * kBwdTile;
+    async_rows<D>(smem + (2 + 2 * j) * C::kTile, tid, p.q, [&](int c) {
+      return bwd_cache_row(p, p.k_cache, p.k_sb, p.k_ss, p.k_sh, b, kvh, seqlen, k0 + c);
+    });
+    async_rows<D>(smem + (3 + 2 * j) * C::kTile, tid, p.q, [&](int c) {
+      return bwd_cache_row(p, p.v_cache, p.v_sb, p.v_ss, p.v_sh, b, kvh, seqlen, k0 + c);
+    });
+    cp_async_commit();
+  };
   const int r_t = row0 + t;
   int my_lim = 0;
   float my_l2 = 0.f, my_d = 0.f;
   int64_t my_row = -1;
-  if (tid < kBwdCompute) {
-    auto rowptr = [&](const __nv_bfloat16 *base, int64_t sb, int64_t ss, int64_t sh, int c)
-        -> const __nv_bfloat16 * {
-      const int r = row0 + c;
-      if (r >= R) return nullptr;
-      const int i = r / p.G, g = r - i * p.G;
-      return base + b * sb + static_cast<int64_t>(i) * ss + static_cast<int64_t>(kvh * p.G + g) * sh;
-    };
-    stage_rows<D>(sQ, tid, [&](int c) { return rowptr(p.q, p.q_sb, p.q_ss, p.q_sh, c); });
-    stage_rows<D>(sG, tid, [&](int c) { return rowptr(p.dout, p.g_sb, p.g_ss, p.g_sh, c); });
+  if (compute) {
+    async_rows<D>(smem, tid, p.q, [&](int c) {
+      return bwd_query_row(p, p.q, p.q_sb, p.q_ss, p.q_sh, b, kvh, row0 + c);
+    });
+    async_rows<D>(smem + C::kTile, tid, p.q, [&](int c) {
+      return bwd_query_row(p, p.dout, p.g_sb, p.g_ss, p.g_sh, b, kvh, row0 + c);
+    });
+    cp_async_commit();
+    if (n > 0) stage_keys_of(0, 0);
     my_lim = bwd_row_lim(p, seqlen, r_t);
     if (r_t < R) {
       const int i = r_t / p.G, g = r_t - i * p.G;
@@ -484,91 +557,85 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
       my_l2 = p.row_lse2[my_row];
       my_d = p.row_d[my_row];
     }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = sm->tmem_base;
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t aQ = sbase, aG = aQ + C::kTile, aK = aG + C::kTile, aV = aK + C::kTile;
-  const uint32_t aS = aV + C::kTile;
-  const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+  const uint32_t tS0 = tmem, tdP = tmem + 128, tdQ = tmem + 256;
   const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  constexpr uint32_t kIdB = idesc_bf16(128, D, 0, 1);
+  static_assert(256 + D <= 384, "dQ below the second S range");
 
-  const int n_kt = (lim_max + kBwdTile - 1) / kBwdTile;
-  int it = 0;
-  for (int kt = 0; kt < n_kt; ++kt, ++it) {
-    const int tok0 = kt * kBwdTile;
-    if (tid < kBwdCompute) {
-      stage_rows<D>(sK, tid, [&](int c) -> const __nv_bfloat16 * {
-        const int tok = tok0 + c;
-        if (tok >= seqlen) return nullptr;
-        const int64_t blk = bwd_block(p, b, tok);
-        if (blk < 0) return nullptr;
-        return p.k_cache + blk * p.k_sb + (tok & ((1 << p.block_shift) - 1)) * p.k_ss + kvh * p.k_sh;
-      });
-      stage_rows<D>(sV, tid, [&](int c) -> const __nv_bfloat16 * {
-        const int tok = tok0 + c;
-        if (tok >= seqlen) return nullptr;
-        const int64_t blk = bwd_block(p, b, tok);
-        if (blk < 0) return nullptr;
-        return p.v_cache + blk * p.v_sb + (tok & ((1 << p.block_shift) - 1)) * p.v_ss + kvh * p.v_sh;
-      });
-      fence_proxy_async_smem();
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    if (*abort_any) break;
-    if (warp == kBwdMmaWarp && lane == 0) {
+  bool ok = true, failed = false;
+  for (int it = 0; it < n; ++it) {
+    const int j = it & 1;
+    const int k0 = it * kBwdTile;
+    const uint32_t tS = tS0 + j * 384;
+    if (issuer) {
       tc_fence_after_sync();
-      constexpr uint32_t kId = idesc_bf16(128, 128, 0, 0);
-      mma_kk<D>(tS, aQ, aK, kId);   // S = Q K^T
-      mma_kk<D>(tdP, aG, aV, kId);  // dP = dO V^T
+      if (it > 0) {
+        mma_tn<D>(tdQ, tS0 + (j ^ 1) * 384, sbase + (2 + 2 * (j ^ 1)) * C::kTile, kIdB, it > 1);  // dQ += dS K
+        umma_commit(&sm->mma_b);
+      }
+      constexpr uint32_t kIdA = idesc_bf16(128, 128, 0, 0);
+      mma_kk<D>(tS, sbase, sbase + (2 + 2 * j) * C::kTile, kIdA);                  // S = Q K^T
+      mma_kk<D>(tdP, sbase + C::kTile, sbase + (3 + 2 * j) * C::kTile, kIdA);      // dP = dO V^T
       umma_commit(&sm->mma_a);
     }
-    if (tid < kBwdCompute) {
-      mbar_wait(&sm->mma_a, it & 1, abort_any);
-      __syncwarp();
-      tc_fence_after_sync();
+    if (compute) {
+      if (it > 0) ok = ok && mbar_wait(&sm->mma_b, (it - 1) & 1, abort_any);
+      if (ok && it + 1 < n) stage_keys_of(it + 1, j ^ 1);
+      ok = ok && mbar_wait(&sm->mma_a, it & 1, abort_any);
+      if (ok) {
+        __syncwarp();
+        tc_fence_after_sync();
 #pragma unroll 1
-      for (int ch = hf * (8 / kBwdGroups); ch < (hf + 1) * (8 / kBwdGroups); ++ch) {  // its keys
-        float sv[16], dp[16];
-        tmem_ld16(tS + lane_off + ch * 16, sv);
-        tmem_ld16(tdP + lane_off + ch * 16, dp);
-        tmem_ld_wait_for(sv);
-        tmem_ld_wait_for(dp);
-        uint32_t sw[8];
+        for (int ch = hf * (8 / kBwdGroups); ch < (hf + 1) * (8 / kBwdGroups); ++ch) {  // its keys
+          float sv[16], dp[16];
+          tmem_ld16(tS + lane_off + ch * 16, sv);
+          tmem_ld16(tdP + lane_off + ch * 16, dp);
+          tmem_ld_wait_for(sv);
+          tmem_ld_wait_for(dp);
+          uint32_t sw[8];
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          float dv[2];
+          for (int e = 0; e < 16; e += 2) {
+            float dv[2];
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int tok = tok0 + ch * 16 + e + k;
-            const float pr = tok < my_lim ? ex2(__fsub_rn(__fmul_rn(sv[e + k], p.cscale), my_l2)) : 0.f;
-            dv[k] = __fmul_rn(pr, __fsub_rn(dp[e + k], my_d));
+            for (int k = 0; k < 2; ++k) {
+              const int tok = k0 + ch * 16 + e + k;
+              const float pr = tok < my_lim ? ex2(__fsub_rn(__fmul_rn(sv[e + k], p.cscale), my_l2)) : 0.f;
+              dv[k] = __fmul_rn(pr, __fsub_rn(dp[e + k], my_d));
+            }
+            sw[e / 2] = pack_bf16(dv[0], dv[1]);
           }
-          sw[e / 2] = pack_bf16(dv[0], dv[1]);
+          tmem_st8(tS + lane_off + ch * 16, sw);
         }
-        put8(sS, t, ch * 2, make_uint4(sw[0], sw[1], sw[2], sw[3]));
-        put8(sS, t, ch * 2 + 1, make_uint4(sw[4], sw[5], sw[6], sw[7]));
+        tmem_st_wait();
       }
+      cp_async_wait<0>();
       fence_proxy_async_smem();
     }
     tc_fence_before_sync();
-    __syncthreads();
-    if (*abort_any) break;
-    if (warp == kBwdMmaWarp && lane == 0) {
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+  }
+  if (!failed && n > 0) {
+    if (issuer) {
       tc_fence_after_sync();
-      mma_kn<D>(tdQ, aS, aK, idesc_bf16(128, D, 0, 1), it > 0);  // dQ += dS K
+      mma_tn<D>(tdQ, tS0 + ((n - 1) & 1) * 384, sbase + (2 + 2 * ((n - 1) & 1)) * C::kTile, kIdB, n > 1);
       umma_commit(&sm->mma_b);
     }
-    mbar_wait(&sm->mma_b, it & 1, abort_any);
-    __syncwarp();
+    if (compute) ok = mbar_wait(&sm->mma_b, (n - 1) & 1, abort_any);
+    tc_fence_before_sync();
+    failed = __syncthreads_or(!ok);
   }
-  tc_fence_before_sync();
-  __syncthreads();
-  const bool ok = !*abort_any;
-  if (tid < kBwdCompute && ok) {
+  if (compute && !failed) {
     tc_fence_after_sync();
 #pragma unroll 1
     for (int ch = hf * (D / 16 / kBwdGroups); ch < (hf + 1) * (D / 16 / kBwdGroups); ++ch) {  // its part of D
@@ -578,10 +645,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
       if (my_row >= 0) {
         const int i = r_t / p.G, g = r_t - i * p.G;
         uint32_t w[8];
+        // rows that see no key (n = 0) leave zeros: the accumulator is unwritten
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          w[e] = pack_bf16(it > 0 ? __fmul_rn(qv[2 * e], p.scale) : 0.f,
-                           it > 0 ? __fmul_rn(qv[2 * e + 1], p.scale) : 0.f);
+          w[e] = pack_bf16(n > 0 ? __fmul_rn(qv[2 * e], p.scale) : 0.f,
+                           n > 0 ? __fmul_rn(qv[2 * e + 1], p.scale) : 0.f);
         uint4 *dst = reinterpret_cast<uint4 *>(p.dq + b * p.dq_sb + static_cast<int64_t>(i) * p.dq_ss +
                                                static_cast<int64_t>(kvh * p.G + g) * p.dq_sh + ch * 16);
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -589,9 +657,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
       }
     }
   }
-  if (!ok && warp == kBwdMmaWarp && lane == 0) {
+  if (failed && issuer) {
     umma_commit(&sm->drain);
-    volatile int no_abort = 0;
+    int no_abort = 0;
     mbar_wait(&sm->drain, 0, &no_abort);
   }
   tc_fence_before_sync();
@@ -600,7 +668,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
     tc_fence_after_sync();
     tmem_dealloc(tmem, 512);
   }
-  if (tid == 0 && !ok && p.err) atomicOr(p.err, kErrTimeout);
+  if (tid == 0 && failed && p.err) atomicOr(p.err, kErrTimeout);
 }
 
 }  // namespace pkv

@@ -218,21 +218,16 @@ int launch_rows(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensorM
 // only one CTA of either kernel sits on an SM.
 template <int D>
 int launch_bwd(const pkv::BwdParams &p, int64_t kv_ctas, int64_t q_ctas, cudaStream_t s) {
-  using C = pkv::BwdCfg<D>;
-  constexpr int kSmall = static_cast<int>(sizeof(typename C::Small)) + 1024;
-  constexpr int kKv = 4 * C::kTile + 2 * C::kSq + kSmall;
-  constexpr int kQ0 = 4 * C::kTile + C::kSq + kSmall;
-  constexpr int kQ = kQ0 > 120 * 1024 ? kQ0 : 120 * 1024;
-  constexpr int kKvS = kKv > 120 * 1024 ? kKv : 120 * 1024;
-  static_assert(kKvS <= 232448 && kQ <= 232448, "shared memory budget");
+  constexpr int kSmem = pkv::BwdCfg<D>::kSmem > 120 * 1024 ? pkv::BwdCfg<D>::kSmem : 120 * 1024;
+  static_assert(kSmem <= 232448, "shared memory budget");
   if (cudaFuncSetAttribute(pkv::bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kKvS) != cudaSuccess ||
+                           kSmem) != cudaSuccess ||
       cudaFuncSetAttribute(pkv::bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kQ) != cudaSuccess)
+                           kSmem) != cudaSuccess)
     return PKV_ERR_CUDA;
-  pkv::bwd_kv_kernel<D><<<static_cast<unsigned>(kv_ctas), pkv::kBwdThreads, kKvS, s>>>(p);
+  pkv::bwd_kv_kernel<D><<<static_cast<unsigned>(kv_ctas), pkv::kBwdThreads, kSmem, s>>>(p);
   if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
-  pkv::bwd_q_kernel<D><<<static_cast<unsigned>(q_ctas), pkv::kBwdThreads, kQ, s>>>(p);
+  pkv::bwd_q_kernel<D><<<static_cast<unsigned>(q_ctas), pkv::kBwdThreads, kSmem, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
