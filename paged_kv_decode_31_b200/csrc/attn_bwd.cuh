@@ -133,9 +133,9 @@ struct BwdCfg {
   struct Small {
     uint64_t mma_a, mma_b, mma_bv, drain;
     uint32_t tmem_base;
-    int lim[2][kBwdTile];  // key limit of each row of the row tile in buffer j
-    float lse2[2][kBwdTile];
-    float dsum[2][kBwdTile];
+    alignas(16) int lim[2][kBwdTile];  // key limit of each row of the row tile in buffer j
+    alignas(16) float lse2[2][kBwdTile];
+    alignas(16) float dsum[2][kBwdTile];
   };
   static constexpr int kSmem = kTiles * kTile + static_cast<int>(sizeof(Small)) + 1024;
 };
@@ -268,9 +268,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
   int abort_flag = 0;  // the waits' abort word; agreement goes through the barriers
   volatile int *abort_any = &abort_flag;
 
+  // key tiles in ascending order across the grid: under causal masking the
+  // first ones meet the most row tiles, and CTAs start roughly in index
+  // order, so the longest run first and the short ones fill the tail
   int u = blockIdx.x;
-  const int kt = u % p.n_key_tiles;
-  u /= p.n_key_tiles;
+  const int kt = u / (p.batch * p.Hkv);
+  u -= kt * (p.batch * p.Hkv);
   const int kvh = u % p.Hkv;
   const int b = u / p.Hkv;
   const int seqlen = max(__ldg(p.seqlens + b), 0);
@@ -507,9 +510,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
   int abort_flag = 0;
   volatile int *abort_any = &abort_flag;
 
+  // row tiles in descending order across the grid (the last rows see the
+  // most keys under causal masking): longest runs first
   int u = blockIdx.x;
-  const int rt = u % p.n_row_tiles;
-  u /= p.n_row_tiles;
+  const int rt = p.n_row_tiles - 1 - u / (p.batch * p.Hkv);
+  u %= p.batch * p.Hkv;
   const int kvh = u % p.Hkv;
   const int b = u / p.Hkv;
   const int seqlen = max(__ldg(p.seqlens + b), 0);
