@@ -20,18 +20,23 @@
 // Every sum therefore has one fixed order and the result is bitwise
 // reproducible and independent of the batch around a sequence.
 //
-// 544 threads: warps 0-15 stage operands and do the elementwise work -- warps
-// w, w + 4, w + 8, w + 12 share TMEM lanes 32 (w % 4) .. + 31 (thread t = lane
-// t of the 128) and split the columns in quarters -- and warp 16 owns TMEM,
-// its lane 0 issuing the MMAs.  The second operand pair of each product (P^T
-// and dS^T, or dS) never touches shared memory: the elementwise pass packs it
-// as bf16 into the TMEM columns its S / dP values came from, and the next MMAs
-// read it from there as their A operand.  The shared memory this frees holds a
-// second buffer of the streamed tiles (Q and dO, or K and V), filled with
-// cp.async while the current tile's MMAs and elementwise pass run; one
-// barrier per tile hands both the packed TMEM operands and the next tile to
-// the MMA warp, whose tensor pipe executes the previous tile's accumulation
-// and the current tile's S / dP products back to back.
+// 576 threads: warps 0-15 do the elementwise work -- warps w, w + 4, w + 8,
+// w + 12 share TMEM lanes 32 (w % 4) .. + 31 (thread t = lane t of the 128)
+// and split the columns in quarters --, warp 16 owns TMEM, its lane 0
+// issuing the MMAs, and warp 17 loads every operand tile with TMA (the
+// cache's K / V rows in boxes addressed through the block table, as the
+// forward does; Q and dO in boxes of 128 / G tokens x G heads).  The second
+// operand pair of each product (P^T and dS^T, or dS) never touches shared
+// memory: the elementwise pass packs it as bf16 into the TMEM columns its
+// S / dP values came from and the next MMAs read it from there as their A
+// operand.  The shared memory this frees holds a second buffer of the
+// streamed tiles (Q and dO, or K and V), which the load warp fills while the
+// current tile's MMAs and elementwise pass run; one named barrier per tile
+// (compute and MMA warps) hands the packed TMEM operands to the MMA warp,
+// whose tensor pipe executes the previous tile's accumulation and the
+// current tile's S / dP products back to back.  Where a row tile cannot be
+// one Q box (G not dividing 128, or fewer than 128 / G query tokens), the
+// compute threads stage the Q / dO tiles with cp.async instead.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -41,11 +46,14 @@
 
 namespace pkv {
 
-constexpr int kBwdCompute = 512;               // staging / elementwise threads
+constexpr int kBwdCompute = 512;               // elementwise threads
 constexpr int kBwdGroups = kBwdCompute / 128;  // column groups per TMEM lane
-constexpr int kBwdThreads = kBwdCompute + 32;
 constexpr int kBwdMmaWarp = kBwdCompute / 32;
+constexpr int kBwdLoadWarp = kBwdMmaWarp + 1;
+constexpr int kBwdThreads = kBwdCompute + 64;
 constexpr int kBwdTile = 128;  // keys per key tile and rows per row tile
+constexpr uint32_t kBwdBar = 1;                   // named barrier of compute + MMA warps
+constexpr uint32_t kBwdBarThreads = kBwdCompute + 32;
 
 struct BwdParams {
   const __nv_bfloat16 *q, *dout;
@@ -63,6 +71,8 @@ struct BwdParams {
   const int32_t *seqlens;
   int batch, seqlen_q, Hq, Hkv, G, block_shift, causal;
   int n_key_tiles, n_row_tiles;
+  int box_slots;       // cache rows per K / V box = min(block_size, 128)
+  int map_head_first;  // K / V map dimension order (D, Hkv, slot, block) vs (D, slot, Hkv, block)
   float cscale, scale;
   const float *row_d;     // [rows] dout . out
   const float *row_lse2;  // [rows] lse * log2 e
@@ -131,6 +141,8 @@ struct BwdCfg {
   static constexpr int kTile = (D / 64) * kHalf;  // a [128][D] operand
   static constexpr int kTiles = 6;                // two fixed + two double-buffered
   struct Small {
+    uint64_t full[2], empty[2];  // streamed tile buffers: loaded / free again
+    uint64_t fixed;              // the fixed tiles loaded
     uint64_t mma_a, mma_b, mma_bv, drain;
     uint32_t tmem_base;
     alignas(16) int lim[2][kBwdTile];  // key limit of each row of the row tile in buffer j
@@ -142,9 +154,10 @@ struct BwdCfg {
 
 // cp.async a [128][D] bf16 tile, rows given by `src_row(c)` (nullptr: zeros),
 // into the 128-byte swizzled K-major layout of the MMA operands (row c at
-// c * 128 bytes of its 64-element half, 16-byte chunk cc at (cc ^ (c % 8)) * 16).
-// `any` is a valid global address for the zero-filled chunks, of which nothing
-// is read.  The caller commits the group.
+// c * 128 bytes of its 64-element half, 16-byte chunk cc at (cc ^ (c % 8)) * 16,
+// the layout a 128-byte-swizzled TMA box writes).  `any` is a valid global
+// address for the zero-filled chunks, of which nothing is read.  The caller
+// commits the group.
 template <int D, class F>
 __device__ __forceinline__ void async_rows(uint8_t *dst, int t, const void *any, F src_row) {
   constexpr int kPer = kBwdTile * (D / 8) / kBwdCompute;  // 16-byte chunks per thread
@@ -189,16 +202,6 @@ __device__ __forceinline__ int64_t bwd_block(const BwdParams &p, int b, int tok)
   return blk;
 }
 
-// Row of token tok0 + c of one cache (nullptr past the context or the table).
-__device__ __forceinline__ const __nv_bfloat16 *bwd_cache_row(const BwdParams &p, const __nv_bfloat16 *cache,
-                                                              int64_t sb, int64_t ss, int64_t sh, int b,
-                                                              int kvh, int seqlen, int tok) {
-  if (tok >= seqlen) return nullptr;
-  const int64_t blk = bwd_block(p, b, tok);
-  if (blk < 0) return nullptr;
-  return cache + blk * sb + (tok & ((1 << p.block_shift) - 1)) * ss + kvh * sh;
-}
-
 // Row r = i G + g of the row tiles of (b, kvh) in a [batch][seqlen_q][Hq][D]
 // tensor (nullptr for padded rows).
 __device__ __forceinline__ const __nv_bfloat16 *bwd_query_row(const BwdParams &p, const __nv_bfloat16 *base,
@@ -207,6 +210,76 @@ __device__ __forceinline__ const __nv_bfloat16 *bwd_query_row(const BwdParams &p
   if (r >= p.G * p.seqlen_q) return nullptr;
   const int i = r / p.G, g = r - i * p.G;
   return base + b * sb + static_cast<int64_t>(i) * ss + static_cast<int64_t>(kvh * p.G + g) * sh;
+}
+
+// Load warp: the K and V rows of tokens [tok0, tok0 + 128) of sequence b,
+// KV head kvh, as TMA boxes of box_slots cache rows (lane l: box l) into
+// dk / dv, completing on `bar` (count 1: lane 0 arrives after every lane has
+// announced its bytes).  Boxes of tokens past the context, past the table or
+// of an invalid block read a block coordinate outside the map and land as
+// zeros (the latter two set the error bits as in the forward); rows past the
+// context inside a loaded block keep the cache's bytes and are zeroed by the
+// consumer.
+template <int D>
+__device__ __forceinline__ void load_kv_tile(const BwdParams &p, const CUtensorMap *mk, const CUtensorMap *mv,
+                                             uint8_t *dk, uint8_t *dv, uint64_t *bar, int b, int kvh,
+                                             int seqlen, int tok0, int lane) {
+  const int nbox = kBwdTile / p.box_slots;
+  int errs = 0;
+  if (lane < nbox) {
+    const int r = lane * p.box_slots;
+    const int tok = tok0 + r;
+    int blk = static_cast<int>(p.num_blocks);
+    if (tok < seqlen) {
+      const int col = tok >> p.block_shift;
+      if (col >= p.max_blocks_per_seq) {
+        errs = kErrTableWidth;
+      } else {
+        const int id = __ldg(p.block_table + b * p.bt_stride + col);
+        if (id < 0 || static_cast<int64_t>(id) >= p.num_blocks)
+          errs = kErrBadBlock;
+        else
+          blk = id;
+      }
+    }
+    const int slot = tok & ((1 << p.block_shift) - 1);
+    const int c1 = p.map_head_first ? kvh : slot;
+    const int c2 = p.map_head_first ? slot : kvh;
+    mbar_expect_tx(bar, static_cast<uint32_t>(2 * (D / 64) * p.box_slots * 128));
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h) {
+      tma_load_4d(dk + h * BwdCfg<D>::kHalf + r * 128, mk, bar, h * 64, c1, c2, blk);
+      tma_load_4d(dv + h * BwdCfg<D>::kHalf + r * 128, mv, bar, h * 64, c1, c2, blk);
+    }
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  if (errs && p.err) atomicOr(p.err, errs);
+}
+
+// Load warp, lane 0: the Q and dO rows of row tile rt of (b, kvh) -- one box
+// of 128 / G tokens x G heads per 64-element half -- into dq / dg.
+template <int D>
+__device__ __forceinline__ void load_row_tile(const BwdParams &p, const CUtensorMap *mq, const CUtensorMap *mg,
+                                              uint8_t *dq, uint8_t *dg, uint64_t *bar, int b, int kvh, int rt) {
+  mbar_expect_tx(bar, static_cast<uint32_t>(2 * BwdCfg<D>::kTile));
+  const int i0 = rt * (kBwdTile / p.G);
+#pragma unroll
+  for (int h = 0; h < D / 64; ++h) {
+    tma_load_4d(dq + h * BwdCfg<D>::kHalf, mq, bar, h * 64, kvh * p.G, i0, b);
+    tma_load_4d(dg + h * BwdCfg<D>::kHalf, mg, bar, h * 64, kvh * p.G, i0, b);
+  }
+  mbar_arrive(bar);
+}
+
+// Zero rows [from, 128) of a K tile and of a V tile (compute threads; thread
+// (t, hf) takes row t of tensor hf % 2, half hf / 2).
+template <int D>
+__device__ __forceinline__ void zero_rows_from(uint8_t *dk, uint8_t *dv, int from, int t, int hf) {
+  if (t < from || hf / 2 >= D / 64) return;
+  uint8_t *row = ((hf & 1) ? dv : dk) + (hf / 2) * BwdCfg<D>::kHalf + t * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(row + c * 16) = make_uint4(0u, 0u, 0u, 0u);
 }
 
 // Issue D[tmem] = A[128 x K] * B^T for two K-major [128][K] operands in
@@ -226,9 +299,7 @@ __device__ __forceinline__ void mma_kk(uint32_t d, uint32_t a, uint32_t b, uint3
 // K steps of 16 at columns a + 16 kk .. + 8 (where the elementwise pass wrote
 // them over the 16 fp32 columns they came from); B a [128][N] tile in shared
 // memory read along its rows (MN-major).
-template <int N>
-__device__ __forceinline__ void mma_tn(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc,
-                                       bool accumulate) {
+__device__ __forceinline__ void mma_tn(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < kBwdTile / 16; ++kk)
     umma_bf16_ts(d, a + kk * 16, smem_desc(b + kk * 2048, kBwdTile * 128, 1024, kLayoutSw128), idesc,
@@ -240,6 +311,20 @@ __device__ __forceinline__ uint8_t *bwd_smem_base(uint8_t *raw) {
                                      ~static_cast<uintptr_t>(1023));
 }
 
+template <class Small>
+__device__ __forceinline__ void bwd_init_barriers(Small *sm) {
+  for (int j = 0; j < 2; ++j) {
+    mbar_init(&sm->full[j], 1);
+    mbar_init(&sm->empty[j], 1);
+  }
+  mbar_init(&sm->fixed, 1);
+  mbar_init(&sm->mma_a, 1);
+  mbar_init(&sm->mma_b, 1);
+  mbar_init(&sm->mma_bv, 1);
+  mbar_init(&sm->drain, 1);
+  fence_barrier_init();
+}
+
 // ---------------------------------------------------------------------------
 // dK / dV: one CTA per (b, kvh, key tile).
 // smem: K, V, then Q and dO of row tile j (j = it % 2) at (2 + 2 j) and
@@ -247,16 +332,20 @@ __device__ __forceinline__ uint8_t *bwd_smem_base(uint8_t *raw) {
 // TMEM: S^T [0,128) (P^T packed over it), dP^T [128,256) (dS^T packed over
 // it), dV [256, 256 + D), dK [256 + D, 256 + 2D).
 // Tile it: barrier; MMA warp: dV += P^T(it - 1) dO, dK += dS^T(it - 1) Q,
-// then S^T = K Q(it)^T, dP^T = V dO(it)^T; compute warps: once the first
-// pair is done, cp.async row tile it + 1 into the other buffer; once the
-// second is, P^T / dS^T of it into TMEM.  MMAs into different accumulators
-// carry no ordering guarantee among themselves, so S^T(it), which overwrites
-// the P^T that dV(it - 1) reads, is issued once dV(it - 1) has completed (its
-// own commit, `mma_bv`, landing while dK(it - 1) runs), and dP^T(it) once
-// dK(it - 1) has (`mma_b`, landing while S^T(it) runs).
+// then S^T = K Q(it)^T, dP^T = V dO(it)^T; compute warps: P^T / dS^T of it
+// into TMEM once the second pair is done; load warp: row tile it + 2 into
+// buffer j once the first pair of it is done.  MMAs into different
+// accumulators carry no ordering guarantee among themselves, so S^T(it),
+// which overwrites the P^T that dV(it - 1) reads, is issued once dV(it - 1)
+// has completed (its own commit, `mma_bv`, landing while dK(it - 1) runs),
+// and dP^T(it) once dK(it - 1) has (`mma_b`, landing while S^T(it) runs).
+// kRowsTma false: the compute threads stage the row tiles with cp.async.
 // ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_constant__ BwdParams p) {
+template <int D, bool kRowsTma>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_kv_kernel(const __grid_constant__ BwdParams p, const __grid_constant__ CUtensorMap map_k,
+                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q,
+                  const __grid_constant__ CUtensorMap map_g) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = bwd_smem_base(smem_raw);
@@ -287,41 +376,68 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
     rt0 = i_min > 0 ? (i_min * p.G) / kBwdTile : 0;
   }
   const int n = (R + kBwdTile - 1) / kBwdTile - rt0;  // row tiles, >= 1
+  uint8_t *sK = smem, *sV = smem + C::kTile;
+  auto sQ = [&](int j) { return smem + (2 + 2 * j) * C::kTile; };
+  auto sG = [&](int j) { return smem + (3 + 2 * j) * C::kTile; };
 
-  if (tid == 0) {
-    mbar_init(&sm->mma_a, 1);
-    mbar_init(&sm->mma_b, 1);
-    mbar_init(&sm->mma_bv, 1);
-    mbar_init(&sm->drain, 1);
-    fence_barrier_init();
-  }
+  if (tid == 0) bwd_init_barriers(sm);
   if (warp == kBwdMmaWarp) tmem_alloc(&sm->tmem_base, 512);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
 
-  // Q / dO rows of row tile rt into buffer j, with the row statistics
-  // loaded into registers (stored by the caller once the tile's elementwise
-  // pass no longer reads that buffer).
+  if (warp == kBwdLoadWarp) {
+    // ---------------- load warp ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      if (kRowsTma) {
+        tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(&map_g);
+      }
+    }
+    load_kv_tile<D>(p, &map_k, &map_v, sK, sV, &sm->fixed, b, kvh, seqlen, tok0, lane);
+    if constexpr (kRowsTma) {
+      bool okl = true;
+      for (int it = 0; it < n && okl; ++it) {
+        const int j = it & 1;
+        if (lane == 0) {
+          if (it >= 2) okl = mbar_wait(&sm->empty[j], ((it >> 1) - 1) & 1, abort_any);
+          if (okl) load_row_tile<D>(p, &map_q, &map_g, sQ(j), sG(j), &sm->full[j], b, kvh, rt0 + it);
+        }
+        okl = __shfl_sync(0xffffffffu, okl ? 1 : 0, 0) != 0;
+      }
+      // nothing of ours may still be landing when the CTA exits
+      if (lane == 0) {
+        for (int it = max(n - 2, 0); it < n; ++it) {
+          int no_abort = 0;
+          mbar_wait(&sm->full[it & 1], (it >> 1) & 1, &no_abort);
+        }
+      }
+    }
+    if (lane == 0) {
+      int no_abort = 0;
+      mbar_wait(&sm->fixed, 0, &no_abort);
+    }
+    __syncwarp();
+    __syncthreads();  // the final barrier below
+    return;
+  }
+
+  // ---------------- compute + MMA warps ----------------
   int n_lim = 0;
   float n_l2 = 0.f, n_ds = 0.f;
-  auto stage_rows_of = [&](int rt, int j) {
-    const int row0 = rt * kBwdTile;
-    async_rows<D>(smem + (2 + 2 * j) * C::kTile, tid, p.q, [&](int c) {
-      return bwd_query_row(p, p.q, p.q_sb, p.q_ss, p.q_sh, b, kvh, row0 + c);
-    });
-    async_rows<D>(smem + (3 + 2 * j) * C::kTile, tid, p.q, [&](int c) {
-      return bwd_query_row(p, p.dout, p.g_sb, p.g_ss, p.g_sh, b, kvh, row0 + c);
-    });
-    cp_async_commit();
-    if (hf == 0) {
-      const int r = row0 + t;
-      n_lim = bwd_row_lim(p, seqlen, r);
-      n_l2 = 0.f;
-      n_ds = 0.f;
-      if (r < R) {
-        const int i = r / p.G, g = r - i * p.G;
-        const int64_t row_id = (static_cast<int64_t>(b) * p.seqlen_q + i) * p.Hq + kvh * p.G + g;
-        n_l2 = p.row_lse2[row_id];
-        n_ds = p.row_d[row_id];
-      }
+  auto row_stats = [&](int rt) {  // statistics of row t of row tile rt (registers)
+    if (hf != 0) return;
+    const int r = rt * kBwdTile + t;
+    n_lim = bwd_row_lim(p, seqlen, r);
+    n_l2 = 0.f;
+    n_ds = 0.f;
+    if (r < R) {
+      const int i = r / p.G, g = r - i * p.G;
+      const int64_t row_id = (static_cast<int64_t>(b) * p.seqlen_q + i) * p.Hq + kvh * p.G + g;
+      n_l2 = p.row_lse2[row_id];
+      n_ds = p.row_d[row_id];
     }
   };
   auto store_stats = [&](int j) {
@@ -331,45 +447,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
       sm->dsum[j][t] = n_ds;
     }
   };
+  auto async_row_tile = [&](int rt, int j) {  // cp.async staging (kRowsTma false)
+    const int row0 = rt * kBwdTile;
+    async_rows<D>(sQ(j), tid, p.q, [&](int c) {
+      return bwd_query_row(p, p.q, p.q_sb, p.q_ss, p.q_sh, b, kvh, row0 + c);
+    });
+    async_rows<D>(sG(j), tid, p.q, [&](int c) {
+      return bwd_query_row(p, p.dout, p.g_sb, p.g_ss, p.g_sh, b, kvh, row0 + c);
+    });
+    cp_async_commit();
+  };
 
-  // K and V of this key tile (tokens past the context are zeros), row tile rt0
+  bool ok = true, failed = false;
   if (compute) {
-    async_rows<D>(smem, tid, p.q, [&](int c) {
-      return bwd_cache_row(p, p.k_cache, p.k_sb, p.k_ss, p.k_sh, b, kvh, seqlen, tok0 + c);
-    });
-    async_rows<D>(smem + C::kTile, tid, p.q, [&](int c) {
-      return bwd_cache_row(p, p.v_cache, p.v_sb, p.v_ss, p.v_sh, b, kvh, seqlen, tok0 + c);
-    });
-    stage_rows_of(rt0, 0);
+    if constexpr (!kRowsTma) async_row_tile(rt0, 0);
+    row_stats(rt0);
     store_stats(0);
-    cp_async_wait<0>();
+    // key rows past the context: zeros (their cache bytes may be anything)
+    if (tok0 + kBwdTile > seqlen) {
+      ok = mbar_wait(&sm->fixed, 0, abort_any);
+      if (ok) zero_rows_from<D>(sK, sV, seqlen - tok0, t, hf);
+    }
+    if constexpr (!kRowsTma) cp_async_wait<0>();
     fence_proxy_async_smem();
   }
   tc_fence_before_sync();
-  __syncthreads();
+  failed = named_bar_or(kBwdBar, kBwdBarThreads, !ok);
   tc_fence_after_sync();
   const uint32_t tmem = sm->tmem_base;
   const uint32_t sbase = smem_u32(smem);
   const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
   const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const int tok = tok0 + t;
+  constexpr uint32_t kIdA = idesc_bf16(128, 128, 0, 0);
+  constexpr uint32_t kIdB = idesc_bf16(128, D, 0, 1);
 
-  bool ok = true, failed = false;
-  for (int it = 0; it < n; ++it) {
+  for (int it = 0; it < n && !failed; ++it) {
     const int j = it & 1;
     if (issuer) {
       tc_fence_after_sync();
+      if (it == 0) ok = mbar_wait(&sm->fixed, 0, abort_any);
       if (it > 0) {
-        constexpr uint32_t kIdB = idesc_bf16(128, D, 0, 1);
-        const uint32_t aQ = sbase + (2 + 2 * (j ^ 1)) * C::kTile, aG = aQ + C::kTile;
-        mma_tn<D>(tdV, tS, aG, kIdB, it > 1);   // dV += P^T dO
+        const uint32_t aQ = smem_u32(sQ(j ^ 1)), aG = smem_u32(sG(j ^ 1));
+        mma_tn(tdV, tS, aG, kIdB, it > 1);   // dV += P^T dO
         umma_commit(&sm->mma_bv);
-        mma_tn<D>(tdK, tdP, aQ, kIdB, it > 1);  // dK += dS^T Q
+        mma_tn(tdK, tdP, aQ, kIdB, it > 1);  // dK += dS^T Q
         umma_commit(&sm->mma_b);
+        if (kRowsTma) umma_commit(&sm->empty[j ^ 1]);
       }
-      constexpr uint32_t kIdA = idesc_bf16(128, 128, 0, 0);
-      const uint32_t aQ = sbase + (2 + 2 * j) * C::kTile, aG = aQ + C::kTile;
-      if (it > 0) ok = mbar_wait(&sm->mma_bv, (it - 1) & 1, abort_any);
+      if (kRowsTma && ok) ok = mbar_wait(&sm->full[j], (it >> 1) & 1, abort_any);
+      const uint32_t aQ = smem_u32(sQ(j)), aG = smem_u32(sG(j));
+      if (ok && it > 0) ok = mbar_wait(&sm->mma_bv, (it - 1) & 1, abort_any);
       if (ok) {
         tc_fence_after_sync();
         mma_kk<D>(tS, sbase, aQ, kIdA);  // S^T = K Q^T
@@ -382,10 +510,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
       }
     }
     if (compute) {
-      // buffer j ^ 1 is free once the accumulation of tile it - 1 is done
-      if (it > 0) ok = ok && mbar_wait(&sm->mma_b, (it - 1) & 1, abort_any);
-      const bool next = ok && it + 1 < n;
-      if (next) stage_rows_of(rt0 + it + 1, j ^ 1);
+      const bool next = it + 1 < n;
+      if constexpr (!kRowsTma) {
+        // buffer j ^ 1 is free once the accumulation of tile it - 1 is done
+        if (it > 0) ok = ok && mbar_wait(&sm->mma_b, (it - 1) & 1, abort_any);
+        if (ok && next) async_row_tile(rt0 + it + 1, j ^ 1);
+      }
+      if (next) row_stats(rt0 + it + 1);
       ok = ok && mbar_wait(&sm->mma_a, it & 1, abort_any);
       if (ok) {
         __syncwarp();
@@ -419,28 +550,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
         tmem_st_wait();
       }
       if (next) store_stats(j ^ 1);
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
+      if constexpr (!kRowsTma) {
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+      }
     }
     tc_fence_before_sync();
-    if (__syncthreads_or(!ok)) {
-      failed = true;
-      break;
-    }
+    failed = named_bar_or(kBwdBar, kBwdBarThreads, !ok);
   }
   if (!failed) {
     if (issuer) {
       tc_fence_after_sync();
-      const uint32_t aQ = sbase + (2 + 2 * ((n - 1) & 1)) * C::kTile, aG = aQ + C::kTile;
-      constexpr uint32_t kIdB = idesc_bf16(128, D, 0, 1);
-      mma_tn<D>(tdV, tS, aG, kIdB, n > 1);
-      umma_commit(&sm->mma_bv);
-      mma_tn<D>(tdK, tdP, aQ, kIdB, n > 1);
+      const uint32_t aQ = smem_u32(sQ((n - 1) & 1)), aG = smem_u32(sG((n - 1) & 1));
+      mma_tn(tdV, tS, aG, kIdB, n > 1);
+      mma_tn(tdK, tdP, aQ, kIdB, n > 1);
       umma_commit(&sm->mma_b);
     }
+    // every earlier phase of mma_b has completed (the MMA warp waited for
+    // it before the last dP^T), so this parity names the last one
     if (compute) ok = mbar_wait(&sm->mma_b, (n - 1) & 1, abort_any);
     tc_fence_before_sync();
-    failed = __syncthreads_or(!ok);
+    failed = named_bar_or(kBwdBar, kBwdBarThreads, !ok);
   }
   if (compute && !failed) {
     tc_fence_after_sync();
@@ -491,14 +621,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kv_kernel(const __grid_con
 // TMEM: S of tile it (dS packed over it) at [0,128) for even it and
 // [384,512) for odd it, dP [128,256), dQ [256, 256 + D).
 // Tile it: barrier; MMA warp: dQ += dS(it - 1) K, then S = Q K(it)^T,
-// dP = dO V(it)^T; compute warps: cp.async key tile it + 1 into the other
-// buffer once the accumulation of it - 1 is done, then dS of it into TMEM.
-// S(it) never lands on the dS(it - 1) that the accumulation reads (MMAs
-// into different accumulators are not ordered among themselves), and dP(it)
-// overwrites values only the elementwise pass read.
+// dP = dO V(it)^T; compute warps: dS of it into TMEM; load warp: key tile
+// it + 2 into buffer j once the accumulation of it is done.  S(it) never
+// lands on the dS(it - 1) that the accumulation reads (MMAs into different
+// accumulators are not ordered among themselves; S(it) reuses the columns
+// of dS(it - 2), whose accumulation completed before S(it - 1) did), and
+// dP(it) overwrites values only the elementwise pass read.
+// kRowsTma false: the compute threads stage Q and dO with cp.async.
 // ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_constant__ BwdParams p) {
+template <int D, bool kRowsTma>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_q_kernel(const __grid_constant__ BwdParams p, const __grid_constant__ CUtensorMap map_k,
+                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q,
+                 const __grid_constant__ CUtensorMap map_g) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = bwd_smem_base(smem_raw);
@@ -523,38 +658,61 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
   // keys [0, lim_max) cover every row of the tile
   const int lim_max = bwd_row_lim(p, seqlen, min(row0 + kBwdTile, R) - 1);
   const int n = (lim_max + kBwdTile - 1) / kBwdTile;
+  uint8_t *sQ = smem, *sG = smem + C::kTile;
+  auto sK = [&](int j) { return smem + (2 + 2 * j) * C::kTile; };
+  auto sV = [&](int j) { return smem + (3 + 2 * j) * C::kTile; };
 
-  if (tid == 0) {
-    mbar_init(&sm->mma_a, 1);
-    mbar_init(&sm->mma_b, 1);
-    mbar_init(&sm->mma_bv, 1);
-    mbar_init(&sm->drain, 1);
-    fence_barrier_init();
-  }
+  if (tid == 0) bwd_init_barriers(sm);
   if (warp == kBwdMmaWarp) tmem_alloc(&sm->tmem_base, 512);
-  auto stage_keys_of = [&](int kt, int j) {
-    const int k0 = kt * kBwdTile;
-    async_rows<D>(smem + (2 + 2 * j) * C::kTile, tid, p.q, [&](int c) {
-      return bwd_cache_row(p, p.k_cache, p.k_sb, p.k_ss, p.k_sh, b, kvh, seqlen, k0 + c);
-    });
-    async_rows<D>(smem + (3 + 2 * j) * C::kTile, tid, p.q, [&](int c) {
-      return bwd_cache_row(p, p.v_cache, p.v_sb, p.v_ss, p.v_sh, b, kvh, seqlen, k0 + c);
-    });
-    cp_async_commit();
-  };
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+
+  if (warp == kBwdLoadWarp) {
+    // ---------------- load warp ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      if (kRowsTma) {
+        tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(&map_g);
+        load_row_tile<D>(p, &map_q, &map_g, sQ, sG, &sm->fixed, b, kvh, rt);
+      }
+    }
+    bool okl = true;
+    for (int it = 0; it < n && okl; ++it) {
+      const int j = it & 1;
+      if (lane == 0 && it >= 2) okl = mbar_wait(&sm->empty[j], ((it >> 1) - 1) & 1, abort_any);
+      okl = __shfl_sync(0xffffffffu, okl ? 1 : 0, 0) != 0;
+      if (okl) load_kv_tile<D>(p, &map_k, &map_v, sK(j), sV(j), &sm->full[j], b, kvh, seqlen, it * kBwdTile, lane);
+    }
+    // nothing of ours may still be landing when the CTA exits
+    if (lane == 0) {
+      int no_abort = 0;
+      for (int it = max(n - 2, 0); it < n; ++it) mbar_wait(&sm->full[it & 1], (it >> 1) & 1, &no_abort);
+      if (kRowsTma) mbar_wait(&sm->fixed, 0, &no_abort);
+    }
+    __syncwarp();
+    __syncthreads();  // the final barrier below
+    return;
+  }
+
+  // ---------------- compute + MMA warps ----------------
   const int r_t = row0 + t;
   int my_lim = 0;
   float my_l2 = 0.f, my_d = 0.f;
   int64_t my_row = -1;
+  bool ok = true, failed = false;
   if (compute) {
-    async_rows<D>(smem, tid, p.q, [&](int c) {
-      return bwd_query_row(p, p.q, p.q_sb, p.q_ss, p.q_sh, b, kvh, row0 + c);
-    });
-    async_rows<D>(smem + C::kTile, tid, p.q, [&](int c) {
-      return bwd_query_row(p, p.dout, p.g_sb, p.g_ss, p.g_sh, b, kvh, row0 + c);
-    });
-    cp_async_commit();
-    if (n > 0) stage_keys_of(0, 0);
+    if constexpr (!kRowsTma) {
+      async_rows<D>(sQ, tid, p.q, [&](int c) {
+        return bwd_query_row(p, p.q, p.q_sb, p.q_ss, p.q_sh, b, kvh, row0 + c);
+      });
+      async_rows<D>(sG, tid, p.q, [&](int c) {
+        return bwd_query_row(p, p.dout, p.g_sb, p.g_ss, p.g_sh, b, kvh, row0 + c);
+      });
+      cp_async_commit();
+    }
     my_lim = bwd_row_lim(p, seqlen, r_t);
     if (r_t < R) {
       const int i = r_t / p.G, g = r_t - i * p.G;
@@ -562,38 +720,46 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
       my_l2 = p.row_lse2[my_row];
       my_d = p.row_d[my_row];
     }
-    cp_async_wait<0>();
+    // key rows past the context in the first key tile: zeros
+    if (n > 0 && kBwdTile > seqlen) {
+      ok = mbar_wait(&sm->full[0], 0, abort_any);
+      if (ok) zero_rows_from<D>(sK(0), sV(0), seqlen, t, hf);
+    }
+    if constexpr (!kRowsTma) cp_async_wait<0>();
     fence_proxy_async_smem();
   }
   tc_fence_before_sync();
-  __syncthreads();
+  failed = named_bar_or(kBwdBar, kBwdBarThreads, !ok);
   tc_fence_after_sync();
   const uint32_t tmem = sm->tmem_base;
   const uint32_t sbase = smem_u32(smem);
   const uint32_t tS0 = tmem, tdP = tmem + 128, tdQ = tmem + 256;
   const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  constexpr uint32_t kIdA = idesc_bf16(128, 128, 0, 0);
   constexpr uint32_t kIdB = idesc_bf16(128, D, 0, 1);
   static_assert(256 + D <= 384, "dQ below the second S range");
 
-  bool ok = true, failed = false;
-  for (int it = 0; it < n; ++it) {
+  for (int it = 0; it < n && !failed; ++it) {
     const int j = it & 1;
     const int k0 = it * kBwdTile;
     const uint32_t tS = tS0 + j * 384;
     if (issuer) {
       tc_fence_after_sync();
+      if (kRowsTma && it == 0) ok = mbar_wait(&sm->fixed, 0, abort_any);
       if (it > 0) {
-        mma_tn<D>(tdQ, tS0 + (j ^ 1) * 384, sbase + (2 + 2 * (j ^ 1)) * C::kTile, kIdB, it > 1);  // dQ += dS K
+        mma_tn(tdQ, tS0 + (j ^ 1) * 384, smem_u32(sK(j ^ 1)), kIdB, it > 1);  // dQ += dS K
         umma_commit(&sm->mma_b);
+        umma_commit(&sm->empty[j ^ 1]);
       }
-      constexpr uint32_t kIdA = idesc_bf16(128, 128, 0, 0);
-      mma_kk<D>(tS, sbase, sbase + (2 + 2 * j) * C::kTile, kIdA);                  // S = Q K^T
-      mma_kk<D>(tdP, sbase + C::kTile, sbase + (3 + 2 * j) * C::kTile, kIdA);      // dP = dO V^T
-      umma_commit(&sm->mma_a);
+      if (ok) ok = mbar_wait(&sm->full[j], (it >> 1) & 1, abort_any);
+      if (ok) {
+        tc_fence_after_sync();
+        mma_kk<D>(tS, sbase, smem_u32(sK(j)), kIdA);               // S = Q K^T
+        mma_kk<D>(tdP, sbase + C::kTile, smem_u32(sV(j)), kIdA);   // dP = dO V^T
+        umma_commit(&sm->mma_a);
+      }
     }
     if (compute) {
-      if (it > 0) ok = ok && mbar_wait(&sm->mma_b, (it - 1) & 1, abort_any);
-      if (ok && it + 1 < n) stage_keys_of(it + 1, j ^ 1);
       ok = ok && mbar_wait(&sm->mma_a, it & 1, abort_any);
       if (ok) {
         __syncwarp();
@@ -621,24 +787,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_q_kernel(const __grid_cons
         }
         tmem_st_wait();
       }
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
+      // key rows past the context in the next key tile: zeros, before its MMAs
+      const int k1 = k0 + kBwdTile;
+      if (ok && it + 1 < n && k1 + kBwdTile > seqlen) {
+        ok = mbar_wait(&sm->full[j ^ 1], ((it + 1) >> 1) & 1, abort_any);
+        if (ok) zero_rows_from<D>(sK(j ^ 1), sV(j ^ 1), seqlen - k1, t, hf);
+        fence_proxy_async_smem();
+      }
     }
     tc_fence_before_sync();
-    if (__syncthreads_or(!ok)) {
-      failed = true;
-      break;
-    }
+    failed = named_bar_or(kBwdBar, kBwdBarThreads, !ok);
   }
   if (!failed && n > 0) {
     if (issuer) {
       tc_fence_after_sync();
-      mma_tn<D>(tdQ, tS0 + ((n - 1) & 1) * 384, sbase + (2 + 2 * ((n - 1) & 1)) * C::kTile, kIdB, n > 1);
+      mma_tn(tdQ, tS0 + ((n - 1) & 1) * 384, smem_u32(sK((n - 1) & 1)), kIdB, n > 1);
       umma_commit(&sm->mma_b);
     }
+    // every earlier accumulation completed before the last S / dP did
     if (compute) ok = mbar_wait(&sm->mma_b, (n - 1) & 1, abort_any);
     tc_fence_before_sync();
-    failed = __syncthreads_or(!ok);
+    failed = named_bar_or(kBwdBar, kBwdBarThreads, !ok);
   }
   if (compute && !failed) {
     tc_fence_after_sync();

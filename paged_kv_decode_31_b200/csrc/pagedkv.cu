@@ -216,18 +216,19 @@ int launch_rows(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensorM
 // Backward kernels: one CTA per key tile (dK, dV) and per row tile (dQ).
 // Both hold 512 TMEM columns; shared memory is requested at >= 120 KB so that
 // only one CTA of either kernel sits on an SM.
-template <int D>
-int launch_bwd(const pkv::BwdParams &p, int64_t kv_ctas, int64_t q_ctas, cudaStream_t s) {
+template <int D, bool kRowsTma>
+int launch_bwd(const pkv::BwdParams &p, int64_t kv_ctas, int64_t q_ctas, const CUtensorMap &mk,
+               const CUtensorMap &mv, const CUtensorMap &mq, const CUtensorMap &mg, cudaStream_t s) {
   constexpr int kSmem = pkv::BwdCfg<D>::kSmem > 120 * 1024 ? pkv::BwdCfg<D>::kSmem : 120 * 1024;
   static_assert(kSmem <= 232448, "shared memory budget");
-  if (cudaFuncSetAttribute(pkv::bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSmem) != cudaSuccess ||
-      cudaFuncSetAttribute(pkv::bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSmem) != cudaSuccess)
+  auto kv = pkv::bwd_kv_kernel<D, kRowsTma>;
+  auto qk = pkv::bwd_q_kernel<D, kRowsTma>;
+  if (cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess ||
+      cudaFuncSetAttribute(qk, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
     return PKV_ERR_CUDA;
-  pkv::bwd_kv_kernel<D><<<static_cast<unsigned>(kv_ctas), pkv::kBwdThreads, kSmem, s>>>(p);
+  kv<<<static_cast<unsigned>(kv_ctas), pkv::kBwdThreads, kSmem, s>>>(p, mk, mv, mq, mg);
   if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
-  pkv::bwd_q_kernel<D><<<static_cast<unsigned>(q_ctas), pkv::kBwdThreads, kSmem, s>>>(p);
+  qk<<<static_cast<unsigned>(q_ctas), pkv::kBwdThreads, kSmem, s>>>(p, mk, mv, mq, mg);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -869,7 +870,28 @@ int pkv_paged_prefill_attn_bwd(const void *q, const int64_t q_strides[3], const 
   const int64_t kv_ctas = static_cast<int64_t>(batch) * Hkv * p.n_key_tiles;
   const int64_t q_ctas = static_cast<int64_t>(batch) * Hkv * p.n_row_tiles;
   if (kv_ctas > INT32_MAX || q_ctas > INT32_MAX) return PKV_ERR_ARG;
-  return D == 128 ? launch_bwd<128>(p, kv_ctas, q_ctas, s) : launch_bwd<64>(p, kv_ctas, q_ctas, s);
+  // K / V tiles through the same TMA boxes as the forward; Q / dO row tiles
+  // as one box of 128 / G tokens x G heads where that covers the tile.
+  const int box_slots = block_size < pkv::kBwdTile ? block_size : pkv::kBwdTile;
+  alignas(64) CUtensorMap mk, mv, mq, mg;
+  int hf_k = 0, hf_v = 0;
+  int rc = make_kv_map(&mk, k_cache, k_strides, num_blocks, block_size, Hkv, D, box_slots, &hf_k);
+  if (rc != PKV_OK) return rc;
+  rc = make_kv_map(&mv, v_cache, v_strides, num_blocks, block_size, Hkv, D, box_slots, &hf_v);
+  if (rc != PKV_OK) return rc;
+  if (hf_k != hf_v) return PKV_ERR_LAYOUT;
+  p.box_slots = box_slots;
+  p.map_head_first = hf_k;
+  std::memset(&mq, 0, sizeof(mq));
+  std::memset(&mg, 0, sizeof(mg));
+  const bool rows_tma = G <= pkv::kBwdTile && pkv::kBwdTile % G == 0 && pkv::kBwdTile / G <= seqlen_q &&
+                        make_q_map(&mq, q, q_strides, batch, seqlen_q, Hq, D, G) == PKV_OK &&
+                        make_q_map(&mg, dout, dout_strides, batch, seqlen_q, Hq, D, G) == PKV_OK;
+  if (D == 128)
+    return rows_tma ? launch_bwd<128, true>(p, kv_ctas, q_ctas, mk, mv, mq, mg, s)
+                    : launch_bwd<128, false>(p, kv_ctas, q_ctas, mk, mv, mq, mg, s);
+  return rows_tma ? launch_bwd<64, true>(p, kv_ctas, q_ctas, mk, mv, mq, mg, s)
+                  : launch_bwd<64, false>(p, kv_ctas, q_ctas, mk, mv, mq, mg, s);
 }
 
 size_t pkv_workspace_size(int batch, int seqlen_q, int Hq, int D, int max_seqlen_k) {

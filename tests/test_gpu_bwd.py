@@ -58,13 +58,17 @@ CASES = [
     (2, 130, [700, 130], 8, 2, 64, 32, True, "contiguous"),
     (1, 64, [5000], 8, 8, 128, 64, False, "contiguous"),      # G = 1, several key tiles
     (3, 17, [33, 17, 900], 32, 8, 128, 16, True, "interleaved"),
+    (2, 50, [200, 333], 12, 4, 64, 16, True, "contiguous"),    # G = 3: row tiles staged by cp.async
+    (1, 200, [1000], 8, 1, 128, 128, True, "interleaved"),     # one 128-row K / V box per tile
+    (2, 150, [700, 300], 4, 2, 64, 256, False, "contiguous"),  # boxes at slot 0 and 128 of a block
 ]
 
 
 @pytest.mark.parametrize("B,sq,ctx,Hq,Hkv,D,bs,causal,layout", CASES)
 def test_backward_matches_oracle(B, sq, ctx, Hq, Hkv, D, bs, causal, layout):
+    # unused cache slots and spare blocks hold NaN: any read past a context shows
     di = I.p2_case(B, sq, max(ctx), Hq, Hkv, D, bs, causal=causal, layout=layout,
-                   seed=sum(ctx) + sq, seqlens=ctx)
+                   seed=sum(ctx) + sq, seqlens=ctx, poison=True)
     gen = torch.Generator().manual_seed(sq + D)
     dout = I.randn_bf16((B, sq, Hq, D), gen)
     dq, dk, dv = _run(di, dout, causal)
@@ -115,3 +119,29 @@ def test_backward_leaves_unreferenced_cache_rows_alone():
     dk, dv = dk.cpu(), dv.cpu()
     assert torch.all(dk[~used] == 3.0) and torch.all(dv[~used] == 3.0)
     assert not torch.any(dk[used] == 3.0)
+
+
+def test_backward_flags_bad_block_ids_and_short_tables():
+    """Block ids outside the cache and contexts wider than the table set the
+    same device error bits as the forward; the kernels read nothing there."""
+    di = I.p2_case(2, 24, 300, 8, 2, 128, 16, causal=True, layout="contiguous", seed=31,
+                   seqlens=[300, 200])
+    d = di.to("cuda")
+    gen = torch.Generator().manual_seed(32)
+    dout = I.randn_bf16((2, 24, 8, 128), gen).cuda()
+    out, lse = pkv.paged_prefill_attn(d.q, d.cache.k, d.cache.v, d.block_table, d.seqlens,
+                                      scale=di.scale, causal=True)
+    bad = d.block_table.clone()
+    bad[0, 3] = d.cache.k.shape[0] + 5
+    bad[1, 2] = -7
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.paged_prefill_attn_bwd(d.q, d.cache.k, d.cache.v, bad, d.seqlens, out, lse, dout,
+                               scale=di.scale, causal=True, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & pkv.binding.DEVERR_BAD_BLOCK
+    narrow = d.block_table[:, :10].contiguous()  # 160 tokens of table for contexts of 300 / 200
+    err.zero_()
+    pkv.paged_prefill_attn_bwd(d.q, d.cache.k, d.cache.v, narrow, d.seqlens, out, lse, dout,
+                               scale=di.scale, causal=True, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & pkv.binding.DEVERR_TABLE_WIDTH
