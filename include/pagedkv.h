@@ -206,6 +206,18 @@ int pkv_debug_paged_decode_attn(const void *q, const int64_t q_strides[3],
                                 int32_t *err, void *stream, uint64_t wait_limit_ns);
 
 /*
+ * pkv_debug_final_out: out[i] = the library's final division of a folded
+ * row, A[i] / L[i] (0 where L[i] <= 0), computed on the device exactly as the
+ * attention calls compute every out element (the row's reciprocal once, then
+ * residual corrections; see the kernels).  It has no counterpart on the
+ * pages: it exists so that a test can hold that arithmetic to the IEEE
+ * quotient bit for bit.  A, L, out: device arrays of n floats (caller-owned;
+ * out may not alias A or L).  Returns PKV_ERR_ARG for n < 0 or a null
+ * pointer with n > 0, PKV_ERR_CUDA when the launch fails; n = 0 does nothing.
+ */
+int pkv_debug_final_out(const float *A, const float *L, float *out, int64_t n, void *stream);
+
+/*
  * pkv_paged_decode_attn_append: kv_append fused into the attention call --
  * the "new_kv" form of flash_attn_with_kvcache in the aiter test grid.  The
  * n_new tokens of k_new/v_new ([batch, n_new, Hkv, D] bf16, element strides

@@ -248,6 +248,27 @@ def debug_paged_decode_attn(q, k_cache, v_cache, block_table, seqlens, *, wait_l
                  extra=(int(wait_limit_ns),))
 
 
+def debug_final_out(A, L, out=None, stream=None):
+    """The library's final division of a folded row, A / L elementwise (0
+    where L <= 0), on the device: float32 CUDA tensors of one shape."""
+    L_ = lib()
+    fn = L_.pkv_debug_final_out
+    if not fn.argtypes:
+        fn.argtypes = [_P, _P, _P, _I64, _P]
+        fn.restype = _I
+    for name, t in (("A", A), ("L", L)):
+        if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.float32
+                and t.is_contiguous()):
+            raise TypeError(f"{name} must be a contiguous float32 CUDA tensor")
+    if A.shape != L.shape:
+        raise ValueError(f"A {tuple(A.shape)} and L {tuple(L.shape)} must have one shape")
+    if out is None:
+        out = torch.empty_like(A)
+    _check("pkv_debug_final_out",
+           fn(A.data_ptr(), L.data_ptr(), out.data_ptr(), A.numel(), _stream_handle(stream)))
+    return out
+
+
 def paged_decode_attn_append(q, k_new, v_new, k_cache, v_cache, block_table, seqlens, *,
                              max_seqlen_k=None, scale=None, causal=False, out=None, lse=None,
                              workspace=None, err=None, stream=None):

@@ -109,28 +109,39 @@ __device__ __forceinline__ void write_final_row(const AttnParams &p, const Unit 
   __nv_bfloat16 *o = p.out + o_tok_off(p, x, i) + h * p.o_sh;
   const bool fin = p.fin_out != nullptr && i == x.nq - 1;  // the sequence's last query row
   __nv_bfloat16 *fo = fin ? p.fin_out + x.b * p.fo_sb + h * p.fo_sh : nullptr;
+  const float rL = final_rcp(L);
+  auto emit = [&](auto div) {
 #pragma unroll
-  for (int c8 = 0; c8 < D / 8; ++c8) {
-    float v[8];
+    for (int c8 = 0; c8 < D / 8; ++c8) {
+      float v[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float A = seen ? fold_val(0.f, acc[c8 * 8 + e], FoldCoef{M, k_a, k_c}) : 0.f;
-      v[e] = final_out(A, L);
+      for (int e = 0; e < 8; ++e)
+        v[e] = div(seen ? fold_val(0.f, acc[c8 * 8 + e], FoldCoef{M, k_a, k_c}) : 0.f);
+      if (p.out_vec) {
+        __nv_bfloat162 h2[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h2[e] = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+        *reinterpret_cast<uint4 *>(o + c8 * 8) = *reinterpret_cast<uint4 *>(h2);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[c8 * 8 + e] = __float2bfloat16_rn(v[e]);
+      }
+      if (fin) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) fo[c8 * 8 + e] = __float2bfloat16_rn(v[e]);
+      }
     }
-    if (p.out_vec) {
-      __nv_bfloat162 h2[4];
+  };
+  // one check of the whole row, then a loop without any IEEE division in it
+  // (the quotients are the same either way; see final_out).  The fold of one
+  // split multiplies by ex2(0) = 1 and adds 0 * 0, so |A| = |acc|.
+  bool fast = seen && L > 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) h2[e] = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-      *reinterpret_cast<uint4 *>(o + c8 * 8) = *reinterpret_cast<uint4 *>(h2);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[c8 * 8 + e] = __float2bfloat16_rn(v[e]);
-    }
-    if (fin) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) fo[c8 * 8 + e] = __float2bfloat16_rn(v[e]);
-    }
-  }
+  for (int c = 0; c < D; ++c) fast = fast && final_fast_ok(acc[c], L);
+  if (fast)
+    emit([&](float A) { return final_out_fast(A, L, rL); });
+  else
+    emit([&](float A) { return final_out(A, L, rL); });
   const float ls = final_lse(M, L);
   p.lse[lse_index(p, x, i, h)] = ls;
   if (fin) p.fin_lse[static_cast<int64_t>(x.b) * p.Hq + h] = ls;

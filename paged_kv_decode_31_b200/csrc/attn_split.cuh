@@ -708,7 +708,7 @@ __device__ __forceinline__ void write_final_cols(const AttnParams &p, const Unit
         L = fold_val(0.f, fin_l[c], kc);
         A = fold_val(0.f, acc[c], kc);
       }
-      const __nv_bfloat16 ob = __float2bfloat16_rn(final_out(A, L));
+      const __nv_bfloat16 ob = __float2bfloat16_rn(final_out(A, L, final_rcp(L)));
       if (stage)
         stage[c * D + t] = ob;
       else

@@ -63,9 +63,35 @@ __device__ __forceinline__ FoldCoef fold_coef(float M, float m_s) {
 __device__ __forceinline__ float fold_val(float X, float x_s, const FoldCoef &k) {
   return __fmaf_rn(x_s, k.c, __fmul_rn(X, k.a));
 }
-// Final write of a folded row: out element and lse.
-__device__ __forceinline__ float final_out(float A, float L) {
-  return L > 0.f ? __fdiv_rn(A, L) : 0.f;
+// Final write of a folded row: out element and lse.  out = A / L rounded to
+// nearest (the IEEE quotient), from the row's reciprocal rL = final_rcp(L),
+// taken once per row, by two residual corrections:
+//   q0 = A rL,  q1 = q0 + (A - L q0) rL,  out = q1 + (A - L q1) rL
+// (each step one rounding; the residuals by FMA).  rL is the correctly
+// rounded 1 / L and q1 lies within one ulp of A / L, so the residual A - L q1
+// is exact and the last step rounds to the correctly rounded quotient
+// (Markstein's theorem: P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990; J.-M.
+// Muller et al., Handbook of Floating-Point Arithmetic, division with an
+// FMA).  The theorem needs every intermediate in the normal range:
+// final_fast_ok holds for |A| in [2^-90, 2^96] and L in [2^-20, 2^40] (a row
+// that saw a key has L >= 1), and for A = +-0, whose quotient is A rL itself;
+// other operands (subnormal, infinite or NaN A) take the IEEE division.
+// Either way the bits are __fdiv_rn(A, L)'s.
+__device__ __forceinline__ float final_rcp(float L) { return L > 0.f ? __frcp_rn(L) : 0.f; }
+__device__ __forceinline__ bool final_fast_ok(float A, float L) {
+  const float aa = fabsf(A);
+  return (aa == 0.f || (aa >= 0x1p-90f && aa <= 0x1p96f)) && L >= 0x1p-20f && L <= 0x1p40f;
+}
+__device__ __forceinline__ float final_out_fast(float A, float L, float rL) {
+  const float q0 = __fmul_rn(A, rL);
+  const float q1 = __fmaf_rn(__fmaf_rn(-L, q0, A), rL, q0);
+  const float q2 = __fmaf_rn(__fmaf_rn(-L, q1, A), rL, q1);
+  return A == 0.f ? q0 : q2;
+}
+__device__ __forceinline__ float final_out(float A, float L, float rL) {
+  if (!(L > 0.f)) return 0.f;
+  return final_fast_ok(A, L) ? final_out_fast(A, L, rL) : __fdiv_rn(A, L);
 }
 __device__ __forceinline__ float final_lse(float M, float L) {
   return L > 0.f ? __fmul_rn(__fadd_rn(M, log2f(L)), 0.69314718055994531f)
@@ -153,12 +179,13 @@ __global__ void __launch_bounds__(WIDE ? D : 32 * kMergeRowsPerBlock)
     }
   }
   const float ls = final_lse(M, L);
+  const float rL = final_rcp(L);
   __nv_bfloat16 *o = p.cu_q ? p.out + tok * p.o_ss + h * p.o_sh
                             : p.out + b * p.o_sb + i * p.o_ss + h * p.o_sh;
   const bool fin = p.fin_out != nullptr && i == nq - 1;
 #pragma unroll
   for (int j = 0; j < V; ++j) {
-    const __nv_bfloat16 ob = __float2bfloat16_rn(final_out(A[j], L));
+    const __nv_bfloat16 ob = __float2bfloat16_rn(final_out(A[j], L, rL));
     o[d0 + j] = ob;
     if (fin) p.fin_out[b * p.fo_sb + h * p.fo_sh + d0 + j] = ob;
   }

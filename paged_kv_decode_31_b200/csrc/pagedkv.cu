@@ -617,6 +617,22 @@ int pkv_debug_paged_decode_attn(const void *q, const int64_t q_strides[3], const
                     workspace_bytes, err, stream, nullptr, nullptr, nullptr, wait_limit_ns);
 }
 
+namespace {
+__global__ void final_out_kernel(const float *A, const float *L, float *out, int64_t n) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = pkv::final_out(A[i], L[i], pkv::final_rcp(L[i]));
+}
+}  // namespace
+
+int pkv_debug_final_out(const float *A, const float *L, float *out, int64_t n, void *stream) {
+  if (n < 0 || (n > 0 && (!A || !L || !out))) return PKV_ERR_ARG;
+  if (n == 0) return PKV_OK;
+  if (ceil_div(n, 256) > INT32_MAX) return PKV_ERR_ARG;
+  final_out_kernel<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      A, L, out, n);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 int pkv_paged_decode_attn_append(const void *q, const int64_t q_strides[3], const void *k_new,
                                  const int64_t kn_strides[3], const void *v_new,
                                  const int64_t vn_strides[3], int n_new, void *k_cache,

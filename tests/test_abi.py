@@ -242,3 +242,14 @@ def test_debug_wait_limit_above_the_default_is_rejected_before_any_cuda_call(lib
     # and it checks every other argument like pkv_paged_decode_attn
     assert fn(*_attn_args(D=96), 0) == header_macros()["PKV_ERR_ARG"]
     assert fn(*_attn_args(ws_bytes=100), 0) == header_macros()["PKV_ERR_WORKSPACE"]
+
+
+def test_debug_final_out_checks_its_arguments_before_any_cuda_call(lib):
+    fn = lib.pkv_debug_final_out
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                   ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    E = header_macros()
+    assert fn(None, None, None, -1, None) == E["PKV_ERR_ARG"]
+    assert fn(None, None, None, 4, None) == E["PKV_ERR_ARG"]
+    assert fn(None, None, None, 0, None) == 0  # nothing to do: no launch
