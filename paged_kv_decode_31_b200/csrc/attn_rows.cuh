@@ -67,6 +67,7 @@ struct RowCfg {
   static constexpr int kOffV = NS * kKVBytes;
   static constexpr int kOffQ = 2 * NS * kKVBytes;
   static constexpr int kOffSmall = kOffQ + kQB * kQBytes;
+  static constexpr int kSchedScratch = kQB * kQBytes;  // bytes free at kernel start
   struct Small {
     uint64_t full_k[NS], empty_k[NS], full_v[NS], empty_v[NS];
     uint64_t s_full[3], p_full[3], s_free[3], stat_free[3], o_full, o_free;
@@ -78,7 +79,7 @@ struct RowCfg {
     int tab[2][2][kSplitTokens / 16];
     int sched_list[kSchedMaxMine];     // this CTA's units (balanced schedule)
     int sched_meta[kSchedMaxMine][3];  // their sequence length and query range
-    int sched_hist[kSchedBuckets + 2], sched_start[kSchedBuckets];
+    int sched_hist[kSchedHist], sched_start[kSchedBuckets];
     int sched_count;
   };
   static constexpr int kSmemBytes = kOffSmall + static_cast<int>(sizeof(Small)) + 1024;
@@ -192,12 +193,11 @@ __global__ void __launch_bounds__(kRowThreads, 1)
   const uint32_t tmem = sm->tmem_base;
   const uint32_t sbase = smem_u32(smem);
   const float NEG_INF = neg_inf();
-  // the Q buffers are not in use yet: one byte per unit of scratch
-  static_assert(C::kQB * C::kQBytes >= kSchedMaxUnits, "schedule scratch");
+  // the Q buffers are not in use yet: the schedule's scratch
   Sched sc = strided_sched(p);
   if (p.sched) {
-    build_schedule<kRowsPerTile>(p, smem + C::kOffQ, sm->sched_hist, sm->sched_start,
-                                 sm->sched_list, sm->sched_meta, &sm->sched_count);
+    build_schedule<kRowsPerTile>(p, smem + C::kOffQ, C::kSchedScratch, sm->sched_hist,
+                                 sm->sched_start, sm->sched_list, sm->sched_meta, &sm->sched_count);
     if (sm->sched_count >= 0) sc = Sched{sm->sched_list, sm->sched_meta, sm->sched_count};
   }
 
@@ -528,6 +528,13 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           tmem_ld_wait_for(lo0);
           tmem_ld_wait_for(hi1);
           tmem_ld_wait_for(lo1);
+          if (ch + 2 == D / 16) {
+            // all of O is in registers: the next P.V may overwrite it while
+            // the last chunks are folded in
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->o_free);
+          }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {  // branch-free: the loop's TMEM loads are warp-wide
             const float nv0 = __fmaf_rn(__fadd_rn(hi0[e], lo0[e]), b, __fmul_rn(acc[ch * 16 + e], a));
@@ -537,9 +544,6 @@ __global__ void __launch_bounds__(kRowThreads, 1)
             acc[ch * 16 + 16 + e] = skip ? acc[ch * 16 + 16 + e] : nv1;
           }
         }
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->o_free);
       }
       if (stop) break;
       if (t < x.rows) {

@@ -57,11 +57,12 @@ constexpr int kKWarp = 12;     // K producer (+ Q staging)
 constexpr int kVWarp = 13;     // V producer
 constexpr int kMmaWarp = 14;   // MMA issuer + TMEM owner
 
-// Balanced schedule limits (see build_schedule): units per call, units per
-// CTA, and the tile-count buckets of the sort.
-constexpr int kSchedMaxUnits = 16384;
+// Balanced schedule limits (see build_schedule): units with work per CTA,
+// and the tile-count buckets of the sort.  The units per call are bounded by
+// each kernel's scratch (one byte per unit).
 constexpr int kSchedMaxMine = 128;
 constexpr int kSchedBuckets = kSplitTokens / kTileTokens + 1;  // tile counts 0 .. 32
+constexpr int kSchedHist = kSchedBuckets + 3;                  // + min, max, units kept
 
 struct AttnParams {
   const __nv_bfloat16 *q;
@@ -94,8 +95,8 @@ struct AttnParams {
   // lse written with the merge's arithmetic.  direct: every row of the call
   // has at most one split (host side: no merge launch).
   int direct, out_vec;
-  // sched: the split kernel builds the balanced unit order (host: at most
-  // kSchedMaxUnits units and kSchedMaxMine per CTA); otherwise units are dealt
+  // sched: the kernel builds the balanced unit order (host: at most one unit
+  // per byte of the kernel's schedule scratch); otherwise units are dealt
   // with stride gridDim.x
   int sched;
   __nv_bfloat16 *out;
@@ -192,6 +193,7 @@ struct Cfg {
   static constexpr int kOffQ = 2 * NS * kKVBytes;
   static constexpr int kOffP = kOffQ + QB * kQBytes;
   static constexpr int kOffSmall = kOffP + 2 * kPBytes;
+  static constexpr int kSchedScratch = 2 * kPBytes;  // bytes free at kernel start
   struct Small {
     uint64_t full_k[NS], empty_k[NS], full_v[NS], empty_v[NS];
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2], stat_free[2];
@@ -206,7 +208,7 @@ struct Cfg {
     float fin_m[N], fin_l[N];              // each row's (m, l) for the direct final write
     int sched_list[kSchedMaxMine];         // this CTA's units (balanced schedule)
     int sched_meta[kSchedMaxMine][3];      // their sequence length and query range
-    int sched_hist[kSchedBuckets + 2], sched_start[kSchedBuckets];
+    int sched_hist[kSchedHist], sched_start[kSchedBuckets];
     int sched_count;
     int lim[2][N];                         // [softmax warpgroup][row]: key limit
     int tab[2][2][kSplitTokens / 16];      // [producer][unit parity]: block-table entries
@@ -347,47 +349,84 @@ __device__ __forceinline__ int next_unit(const AttnParams &p, const Sched &sc, i
   return -1;
 }
 
-// Balanced schedule (decode-shaped calls of at most kSchedMaxUnits units):
-// every CTA sorts all units by tile count, largest first -- a stable counting
-// sort, so every CTA computes the same order -- and takes the positions of a
-// snake deal over the grid: round r hands positions r G .. r G + G - 1 to CTAs
-// 0 .. G - 1 when r is even and to CTAs G - 1 .. 0 when r is odd.  The CTA's
-// k-th unit is the one at its position of round k.  With contexts of mixed
-// lengths this evens out the tiles per CTA (a stride-G deal leaves some CTAs
-// with far more).  When every unit with work has the same tile count there is
-// nothing to balance: *count is set to -1 and the caller keeps the stride-G
-// deal.  All threads of the CTA take part; `scratch` holds one byte per unit
-// (free shared memory at kernel start); hist has kSchedBuckets + 2 entries.
+// Balanced schedule: every CTA sorts the units that have work by tile count,
+// largest first -- a stable counting sort, so every CTA computes the same
+// order -- and takes the positions of a snake deal over the grid: round r
+// hands positions r G .. r G + G - 1 to CTAs 0 .. G - 1 when r is even and to
+// CTAs G - 1 .. 0 when r is odd.  The CTA's k-th unit is the one at its
+// position of round k.  With contexts of mixed lengths this evens out the
+// tiles per CTA (a stride-G deal leaves some CTAs with far more).  A unit has
+// work when it has a tile, or when it is split 0 of real rows (the rows that
+// see no key get their zero output there); the others -- splits past a short
+// context, row tiles past a short query range, sequences another launch
+// serves -- are left out, so no role walks over them.  When every unit has
+// work and all have the same tile count there is nothing to balance, and when
+// a CTA's share would overflow its list, *count is set to -1 and the caller
+// keeps the stride-G deal.  All threads of the CTA take part; `scratch`
+// (free shared memory at kernel start, `scratch_bytes` >= n_units) holds one
+// byte per unit and, when it fits behind them, each sequence's length and
+// query range; hist has kSchedHist entries.
 
 template <int N>
-__device__ __forceinline__ void build_schedule(const AttnParams &p, uint8_t *scratch, int *hist,
-                                               int *start, int *list, int (*meta)[3],
+__device__ __forceinline__ void build_schedule(const AttnParams &p, uint8_t *scratch, int scratch_bytes,
+                                               int *hist, int *start, int *list, int (*meta)[3],
                                                int *count) {
   const int tid = threadIdx.x, nthr = blockDim.x;
   int *nt_min = hist + kSchedBuckets, *nt_max = hist + kSchedBuckets + 1;
+  int *n_kept = hist + kSchedBuckets + 2;
+  constexpr uint8_t kSkip = 0xFF;
+  // per-sequence (length, query start, query end), cached behind the unit bytes
+  const int seq_off = (p.n_units + 15) & ~15;
+  int *seq = (seq_off + 12 * p.batch <= scratch_bytes) ? reinterpret_cast<int *>(scratch + seq_off) : nullptr;
   for (int i = tid; i < kSchedBuckets; i += nthr) hist[i] = 0;
   if (tid == 0) {
     *nt_min = kSchedBuckets;
     *nt_max = 0;
+    *n_kept = 0;
   }
-  __syncthreads();
-  int lo = kSchedBuckets, hi = 0;
-  for (int u = tid; u < p.n_units; u += nthr) {
-    const int nt = unit_at<N>(p, u).n_tiles;
-    scratch[u] = static_cast<uint8_t>(nt);
-    atomicAdd(&hist[nt], 1);
-    if (nt > 0) {
-      lo = min(lo, nt);
-      hi = max(hi, nt);
+  if (seq) {
+    for (int b = tid; b < p.batch; b += nthr) {
+      seq[3 * b] = __ldg(p.seqlens + b);
+      seq[3 * b + 1] = p.cu_q ? __ldg(p.cu_q + b) : 0;
+      seq[3 * b + 2] = p.cu_q ? __ldg(p.cu_q + b + 1) : 0;
     }
   }
-  if (lo <= hi) {
-    atomicMin(nt_min, lo);
-    atomicMax(nt_max, hi);
+  __syncthreads();
+  auto unit_of = [&](int u) {
+    if (!seq) return unit_at<N>(p, u);
+    const int b = unit_seq(p, u);
+    return unit_make<N>(p, u, seq[3 * b], seq[3 * b + 1], seq[3 * b + 2]);
+  };
+  int lo = kSchedBuckets, hi = 0, kept = 0;
+  for (int u = tid; u < p.n_units; u += nthr) {
+    const Unit x = unit_of(u);
+    const bool keep = x.n_tiles > 0 || (x.rows > 0 && x.s == 0);
+    scratch[u] = keep ? static_cast<uint8_t>(x.n_tiles) : kSkip;
+    if (keep) {
+      atomicAdd(&hist[x.n_tiles], 1);
+      ++kept;
+      if (x.n_tiles > 0) {
+        lo = min(lo, x.n_tiles);
+        hi = max(hi, x.n_tiles);
+      }
+    }
+  }
+  // one lane per warp updates the shared counters
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  kept = __reduce_add_sync(0xffffffffu, kept);
+  if ((tid & 31) == 0) {
+    if (lo <= hi) {
+      atomicMin(nt_min, lo);
+      atomicMax(nt_max, hi);
+    }
+    if (kept) atomicAdd(n_kept, kept);
   }
   __syncthreads();
-  if (*nt_min >= *nt_max) {  // uniform (or no work): keep the stride-G deal
-    __syncthreads();         // every thread has read nt_min / nt_max
+  const int G = static_cast<int>(gridDim.x), me = static_cast<int>(blockIdx.x);
+  const int total = *n_kept;
+  if ((total == p.n_units && *nt_min >= *nt_max) || (total + G - 1) / G > kSchedMaxMine) {
+    __syncthreads();  // every thread has read the counters
     if (tid == 0) *count = -1;
     __syncthreads();
     return;
@@ -402,11 +441,10 @@ __device__ __forceinline__ void build_schedule(const AttnParams &p, uint8_t *scr
   }
   __syncthreads();
   if (tid < 32) {
-    const int G = static_cast<int>(gridDim.x), me = static_cast<int>(blockIdx.x);
     const int lane = tid;
     for (int base = 0; base < p.n_units; base += 32) {
       const int u = base + lane;
-      const int nt = u < p.n_units ? scratch[u] : -1;
+      const int nt = (u < p.n_units && scratch[u] != kSkip) ? scratch[u] : -1;
       const unsigned same = __match_any_sync(0xffffffffu, nt);
       const int rank = __popc(same & ((1u << lane) - 1u));
       const int placed = nt >= 0 ? hist[nt] : 0;
@@ -420,19 +458,19 @@ __device__ __forceinline__ void build_schedule(const AttnParams &p, uint8_t *scr
       __syncwarp();
     }
     if (lane == 0) {
-      // rounds in which this CTA has a position below n_units
-      const int full_rounds = p.n_units / G, rem = p.n_units - full_rounds * G;
+      // rounds in which this CTA has a position below the kept units
+      const int full_rounds = total / G, rem = total - full_rounds * G;
       const int pos_last = (full_rounds & 1) ? G - 1 - me : me;  // its position in the partial round
       *count = full_rounds + (pos_last < rem ? 1 : 0);
     }
   }
   __syncthreads();
-  // the listed units' sequence lengths and query ranges, read once
+  // the listed units' sequence lengths and query ranges
   for (int k = tid; k < *count; k += nthr) {
     const int b = unit_seq(p, list[k]);
-    meta[k][0] = __ldg(p.seqlens + b);
-    meta[k][1] = p.cu_q ? __ldg(p.cu_q + b) : 0;
-    meta[k][2] = p.cu_q ? __ldg(p.cu_q + b + 1) : 0;
+    meta[k][0] = seq ? seq[3 * b] : __ldg(p.seqlens + b);
+    meta[k][1] = seq ? seq[3 * b + 1] : (p.cu_q ? __ldg(p.cu_q + b) : 0);
+    meta[k][2] = seq ? seq[3 * b + 2] : (p.cu_q ? __ldg(p.cu_q + b + 1) : 0);
   }
   __syncthreads();
 }
@@ -708,7 +746,9 @@ __device__ __forceinline__ void write_final_cols(const AttnParams &p, const Unit
         L = fold_val(0.f, fin_l[c], kc);
         A = fold_val(0.f, acc[c], kc);
       }
-      const __nv_bfloat16 ob = __float2bfloat16_rn(final_out(A, L, final_rcp(L)));
+      // one quotient per (row, element) here: the IEEE division itself,
+      // which final_out reproduces bit for bit elsewhere
+      const __nv_bfloat16 ob = __float2bfloat16_rn(L > 0.f ? __fdiv_rn(A, L) : 0.f);
       if (stage)
         stage[c * D + t] = ob;
       else
@@ -778,12 +818,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = sm->tmem_base;
   const uint32_t sbase = smem_u32(smem);
-  // the P^T buffers are not in use yet: one byte per unit of scratch
-  static_assert(2 * C::kPBytes >= kSchedMaxUnits, "schedule scratch");
+  // the P^T buffers are not in use yet: the schedule's scratch
   Sched sc = strided_sched(p);
   if (p.sched) {
-    build_schedule<N>(p, smem + C::kOffP, sm->sched_hist, sm->sched_start, sm->sched_list,
-                      sm->sched_meta, &sm->sched_count);
+    build_schedule<N>(p, smem + C::kOffP, C::kSchedScratch, sm->sched_hist, sm->sched_start,
+                      sm->sched_list, sm->sched_meta, &sm->sched_count);
     if (sm->sched_count >= 0) sc = Sched{sm->sched_list, sm->sched_meta, sm->sched_count};
   }
 

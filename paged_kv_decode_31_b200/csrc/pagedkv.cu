@@ -177,10 +177,11 @@ int launch_split(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensor
     if (dev >= 0 && dev < kMaxDevices) attr_set[dev].store(true, std::memory_order_release);
   }
   const int grid = p.n_units < sm_count(dev) ? p.n_units : sm_count(dev);
-  // balanced unit order when it fits the kernel's schedule arrays
+  // balanced unit order when the units fit the kernel's schedule scratch
+  // (the kernel itself falls back to the stride-grid deal when its share of
+  // the units with work overflows its list)
   pkv::AttnParams pp = p;
-  pp.sched = (p.n_units <= pkv::kSchedMaxUnits &&
-              ceil_div(p.n_units, grid) <= pkv::kSchedMaxMine) ? 1 : 0;
+  pp.sched = p.n_units <= C::kSchedScratch ? 1 : 0;
   kern<<<grid, pkv::kThreads, C::kSmemBytes, s>>>(pp, mk, mv);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
@@ -207,8 +208,7 @@ int launch_rows(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensorM
   }
   const int grid = p.n_units < sm_count(dev) ? p.n_units : sm_count(dev);
   pkv::AttnParams pp = p;
-  pp.sched = (p.n_units <= pkv::kSchedMaxUnits &&
-              ceil_div(p.n_units, grid) <= pkv::kSchedMaxMine) ? 1 : 0;
+  pp.sched = p.n_units <= C::kSchedScratch ? 1 : 0;
   kern<<<grid, pkv::kRowThreads, C::kSmemBytes, s>>>(pp, mk, mv, mq);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
