@@ -38,16 +38,13 @@ struct AppendParams {
   int32_t *err;
 };
 
+// One block per new token (blockIdx.x: b * n_new + t, or the packed index):
+// one thread resolves the token's sequence, cache position and block once,
+// then the block's threads copy its Hkv x (D / 8) 16-byte pieces.
 __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ AppendParams p) {
-  const int64_t tokens = p.cu_new ? static_cast<int64_t>(p.total_new)
-                                  : static_cast<int64_t>(p.batch) * p.n_new;
-  const int64_t total = tokens * p.Hkv * p.chunks;
-  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(idx % p.chunks);
-    int64_t r = idx / p.chunks;
-    const int h = static_cast<int>(r % p.Hkv);
-    r /= p.Hkv;  // token: b * n_new + t, or the packed index
+  __shared__ int64_t s_dst_k, s_dst_v, s_src_k, s_src_v;  // element offsets (-1: skip the token)
+  const int64_t r = blockIdx.x;
+  if (threadIdx.x == 0) {
     int b, t;
     int64_t kn_off, vn_off;
     if (p.cu_new) {
@@ -61,23 +58,39 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ 
       kn_off = b * p.kn_sb + t * p.kn_st;
       vn_off = b * p.vn_sb + t * p.vn_st;
     }
+    int64_t dk = -1, dv = -1;
     const int64_t pos = static_cast<int64_t>(__ldg(p.seqlens + b)) - p.seq_bias + t;
     const int64_t bi = pos >> p.block_shift;
-    if (pos < 0 && p.seq_bias > 0) continue;
-    if (pos < 0 || bi >= p.max_blocks_per_seq) {
+    if (pos < 0 && p.seq_bias > 0) {
+      // before the sequence's start in the fused path: nothing to write
+    } else if (pos < 0 || bi >= p.max_blocks_per_seq) {
       if (p.err) atomicOr(p.err, 2);
-      continue;
+    } else {
+      const int32_t blk = __ldg(p.block_table + b * p.bt_stride + bi);
+      if (blk < 0 || static_cast<int64_t>(blk) >= p.num_blocks) {
+        if (p.err) atomicOr(p.err, 1);
+      } else {
+        const int64_t slot = pos & ((int64_t{1} << p.block_shift) - 1);
+        dk = blk * p.k_sb + slot * p.k_ss;
+        dv = blk * p.v_sb + slot * p.v_ss;
+      }
     }
-    const int32_t blk = __ldg(p.block_table + b * p.bt_stride + bi);
-    if (blk < 0 || static_cast<int64_t>(blk) >= p.num_blocks) {
-      if (p.err) atomicOr(p.err, 1);
-      continue;
-    }
-    const int64_t slot = pos & ((int64_t{1} << p.block_shift) - 1);
-    const uint4 kv = __ldg(reinterpret_cast<const uint4 *>(p.k_new + kn_off + h * p.kn_sh) + c);
-    const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(p.v_new + vn_off + h * p.vn_sh) + c);
-    reinterpret_cast<uint4 *>(p.k_cache + blk * p.k_sb + slot * p.k_ss + h * p.k_sh)[c] = kv;
-    reinterpret_cast<uint4 *>(p.v_cache + blk * p.v_sb + slot * p.v_ss + h * p.v_sh)[c] = vv;
+    s_dst_k = dk;
+    s_dst_v = dv;
+    s_src_k = kn_off;
+    s_src_v = vn_off;
+  }
+  __syncthreads();
+  const int64_t dk = s_dst_k, dv = s_dst_v;
+  if (dk < 0) return;  // uniform over the block
+  const uint16_t *kn = p.k_new + s_src_k, *vn = p.v_new + s_src_v;
+  const int n = p.Hkv * p.chunks;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int h = i / p.chunks, c = i - h * p.chunks;
+    const uint4 kv = __ldg(reinterpret_cast<const uint4 *>(kn + h * p.kn_sh) + c);
+    const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(vn + h * p.vn_sh) + c);
+    reinterpret_cast<uint4 *>(p.k_cache + dk + h * p.k_sh)[c] = kv;
+    reinterpret_cast<uint4 *>(p.v_cache + dv + h * p.v_sh)[c] = vv;
   }
 }
 

@@ -266,8 +266,6 @@ int launch_append(const void *k_new, const int64_t kn_strides[3], const void *v_
                   const int32_t *seqlens, int batch, int n_new, int Hkv, int D, int block_size,
                   int seq_bias, int32_t *err, cudaStream_t stream,
                   const int32_t *cu_new = nullptr, int total_new = 0) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
   pkv::AppendParams p{};
   p.k_new = static_cast<const uint16_t *>(k_new);
   p.v_new = static_cast<const uint16_t *>(v_new);
@@ -299,12 +297,14 @@ int launch_append(const void *k_new, const int64_t kn_strides[3], const void *v_
   p.cu_new = cu_new;
   p.total_new = total_new;
   p.err = err;
+  // one block per new token, a thread per 16-byte piece of its Hkv heads (up
+  // to 256, looping beyond)
   const int64_t tokens = cu_new ? static_cast<int64_t>(total_new) : static_cast<int64_t>(batch) * n_new;
-  const int64_t total = tokens * Hkv * (D / 8);
-  const int64_t want = ceil_div(total, 256);
-  const int64_t cap = static_cast<int64_t>(sm_count(dev)) * 8;
-  const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
-  pkv::kv_append_kernel<<<grid, 256, 0, stream>>>(p);
+  if (tokens <= 0) return PKV_OK;
+  if (tokens > INT32_MAX) return PKV_ERR_ARG;
+  const int pieces = Hkv * (D / 8);
+  const int threads = pieces < 256 ? ((pieces + 31) / 32) * 32 : 256;
+  pkv::kv_append_kernel<<<static_cast<unsigned>(tokens), threads, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
