@@ -51,6 +51,7 @@ constexpr int kBwdGroups = kBwdCompute / 128;  // column groups per TMEM lane
 constexpr int kBwdMmaWarp = kBwdCompute / 32;
 constexpr int kBwdLoadWarp = kBwdMmaWarp + 1;
 constexpr int kBwdThreads = kBwdCompute + 64;
+constexpr int kBwdQThreads = kBwdCompute + 96;  // dQ: a second load warp (K and V boxes in parallel)
 constexpr int kBwdTile = 128;  // keys per key tile and rows per row tile
 constexpr uint32_t kBwdBar = 1;                   // named barrier of compute + MMA warps
 constexpr uint32_t kBwdBarThreads = kBwdCompute + 32;
@@ -148,6 +149,23 @@ struct BwdCfg {
     alignas(16) int lim[2][kBwdTile];  // key limit of each row of the row tile in buffer j
     alignas(16) float lse2[2][kBwdTile];
     alignas(16) float dsum[2][kBwdTile];
+  };
+  static constexpr int kSmem = kTiles * kTile + static_cast<int>(sizeof(Small)) + 1024;
+};
+
+// dQ: Q and dO, then three K buffers and two V buffers (V is free again once
+// a tile's S / dP products are done, K only after its dQ product).
+template <int D>
+struct BwdQCfg {
+  static constexpr int kTile = BwdCfg<D>::kTile;
+  static constexpr int kKBufs = 3, kVBufs = 2;
+  static constexpr int kTiles = 2 + kKBufs + kVBufs;
+  struct Small {
+    uint64_t kfull[kKBufs], kempty[kKBufs], vfull[kVBufs], vempty[kVBufs];
+    uint64_t fixed;  // Q and dO loaded
+    uint64_t mma_a, mma_b, drain;
+    uint64_t dp_free, ds_ready, fin;  // elementwise pass <-> MMA warp hand-offs
+    uint32_t tmem_base;
   };
   static constexpr int kSmem = kTiles * kTile + static_cast<int>(sizeof(Small)) + 1024;
 };
@@ -255,6 +273,55 @@ __device__ __forceinline__ void load_kv_tile(const BwdParams &p, const CUtensorM
   __syncwarp();
   if (lane == 0) mbar_arrive(bar);
   if (errs && p.err) atomicOr(p.err, errs);
+}
+
+// Load warp: lane l's box of the cache rows of tokens [tok0, tok0 + 128) of
+// sequence b (box l covers rows [l box_slots, (l + 1) box_slots)), resolved
+// once per tile for both caches: the block coordinate (outside the map, so
+// the box lands as zeros, past the context, the table or the cache -- the
+// latter two flagged as in the forward) and the slot / head coordinates.
+struct CacheBox {
+  int r, c1, c2, blk;
+  bool on;
+};
+__device__ __forceinline__ CacheBox cache_box(const BwdParams &p, int b, int kvh, int seqlen, int tok0,
+                                              int lane) {
+  CacheBox x{0, 0, 0, static_cast<int>(p.num_blocks), lane < kBwdTile / p.box_slots};
+  if (!x.on) return x;
+  x.r = lane * p.box_slots;
+  const int tok = tok0 + x.r;
+  int errs = 0;
+  if (tok < seqlen) {
+    const int col = tok >> p.block_shift;
+    if (col >= p.max_blocks_per_seq) {
+      errs = kErrTableWidth;
+    } else {
+      const int id = __ldg(p.block_table + b * p.bt_stride + col);
+      if (id < 0 || static_cast<int64_t>(id) >= p.num_blocks)
+        errs = kErrBadBlock;
+      else
+        x.blk = id;
+    }
+  }
+  const int slot = tok & ((1 << p.block_shift) - 1);
+  x.c1 = p.map_head_first ? kvh : slot;
+  x.c2 = p.map_head_first ? slot : kvh;
+  if (errs && p.err) atomicOr(p.err, errs);
+  return x;
+}
+// Issue one cache's boxes of a tile (every lane with a box), completing on
+// `bar` (count 1: lane 0 arrives after every lane has announced its bytes).
+template <int D>
+__device__ __forceinline__ void issue_cache_boxes(const BwdParams &p, const CUtensorMap *map, uint8_t *dst,
+                                                  uint64_t *bar, const CacheBox &x, int lane) {
+  if (x.on) {
+    mbar_expect_tx(bar, static_cast<uint32_t>((D / 64) * p.box_slots * 128));
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h)
+      tma_load_4d(dst + h * BwdCfg<D>::kHalf + x.r * 128, map, bar, h * 64, x.c1, x.c2, x.blk);
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
 }
 
 // Load warp, lane 0: the Q and dO rows of row tile rt of (b, kvh) -- one box
@@ -616,25 +683,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ---------------------------------------------------------------------------
 // dQ: one CTA per (b, kvh, row tile).
-// smem: Q, dO, then K and V of key tile j (j = it % 2) at (2 + 2 j) and
-// (3 + 2 j) tiles.
-// TMEM: S of tile it (dS packed over it) at [0,128) for even it and
+// smem: Q, dO, K buffers k % 3 at 2 + k % 3, V buffers at 5 + k % 2 (tiles).
+// TMEM: S of key tile it (dS packed over it) at [0,128) for even it and
 // [384,512) for odd it, dP [128,256), dQ [256, 256 + D).
-// Tile it: barrier; MMA warp: dQ += dS(it - 1) K, then S = Q K(it)^T,
-// dP = dO V(it)^T; compute warps: dS of it into TMEM; load warp: key tile
-// it + 2 into buffer j once the accumulation of it is done.  S(it) never
-// lands on the dS(it - 1) that the accumulation reads (MMAs into different
-// accumulators are not ordered among themselves; S(it) reuses the columns
-// of dS(it - 2), whose accumulation completed before S(it - 1) did), and
-// dP(it) overwrites values only the elementwise pass read.
+// No per-tile barrier: the elementwise warps and the MMA warp hand off
+// through mbarriers, so the MMAs of the next key tile run while the
+// elementwise pass of this one computes.  Per key tile it:
+//   elementwise warps: wait for S / dP(it) (mma_a), load their dP columns
+//   (and the first S chunk) into registers, arrive dp_free; compute dS(it)
+//   into the S columns; arrive ds_ready.
+//   MMA warp: once K / V(it) have landed, dP(it - 1) has been read
+//   (dp_free) and dQ += dS(it - 2) K has completed (S(it) reuses those
+//   columns; MMAs into different accumulators are not ordered among
+//   themselves), S(it) = Q K(it)^T and dP(it) = dO V(it)^T, which frees
+//   V(it)'s buffer; then, once dS(it - 1) is written (ds_ready),
+//   dQ += dS(it - 1) K(it - 1), which frees K(it - 1)'s buffer.
+// With K three deep and V two deep the load warp's TMA latency stays behind
+// the pipeline.  Rows past the context in the next key tile are zeroed
+// before dp_free.
 // kRowsTma false: the compute threads stage Q and dO with cp.async.
 // ---------------------------------------------------------------------------
 template <int D, bool kRowsTma>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdQThreads, 1)
     bwd_q_kernel(const __grid_constant__ BwdParams p, const __grid_constant__ CUtensorMap map_k,
                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q,
                  const __grid_constant__ CUtensorMap map_g) {
-  using C = BwdCfg<D>;
+  using C = BwdQCfg<D>;
+  constexpr int KB = C::kKBufs, VB = C::kVBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = bwd_smem_base(smem_raw);
   auto *sm = reinterpret_cast<typename C::Small *>(smem + C::kTiles * C::kTile);
@@ -659,38 +734,63 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lim_max = bwd_row_lim(p, seqlen, min(row0 + kBwdTile, R) - 1);
   const int n = (lim_max + kBwdTile - 1) / kBwdTile;
   uint8_t *sQ = smem, *sG = smem + C::kTile;
-  auto sK = [&](int j) { return smem + (2 + 2 * j) * C::kTile; };
-  auto sV = [&](int j) { return smem + (3 + 2 * j) * C::kTile; };
+  auto sK = [&](int k) { return smem + (2 + k % KB) * C::kTile; };
+  auto sV = [&](int k) { return smem + (2 + KB + k % VB) * C::kTile; };
 
-  if (tid == 0) bwd_init_barriers(sm);
+  if (tid == 0) {
+    for (int i = 0; i < KB; ++i) {
+      mbar_init(&sm->kfull[i], 1);
+      mbar_init(&sm->kempty[i], 1);
+    }
+    for (int i = 0; i < VB; ++i) {
+      mbar_init(&sm->vfull[i], 1);
+      mbar_init(&sm->vempty[i], 1);
+    }
+    mbar_init(&sm->fixed, 1);
+    mbar_init(&sm->mma_a, 1);
+    mbar_init(&sm->mma_b, 1);
+    mbar_init(&sm->drain, 1);
+    mbar_init(&sm->dp_free, kBwdCompute / 32);  // one arrival per elementwise warp
+    mbar_init(&sm->ds_ready, kBwdCompute / 32);
+    mbar_init(&sm->fin, 1);
+    fence_barrier_init();
+  }
   if (warp == kBwdMmaWarp) tmem_alloc(&sm->tmem_base, 512);
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
 
-  if (warp == kBwdLoadWarp) {
-    // ---------------- load warp ----------------
+  if (warp >= kBwdLoadWarp) {
+    // ---------------- load warps: K (and Q / dO), V ----------------
+    // A TMA box of a block-size-16 cache costs the issuing warp ~90 cycles,
+    // so K and V each have a warp.  Per key tile: the block coordinates
+    // first (nothing to wait for), then the boxes once the buffer is free
+    // (V: after S / dP of tile it - 2; K: after dQ of tile it - 3).
+    const bool is_v = warp == kBwdLoadWarp + 1;
     if (lane == 0) {
-      tma_prefetch_desc(&map_k);
-      tma_prefetch_desc(&map_v);
-      if (kRowsTma) {
+      tma_prefetch_desc(is_v ? &map_v : &map_k);
+      if (kRowsTma && !is_v) {
         tma_prefetch_desc(&map_q);
         tma_prefetch_desc(&map_g);
         load_row_tile<D>(p, &map_q, &map_g, sQ, sG, &sm->fixed, b, kvh, rt);
       }
     }
+    const int nbuf = is_v ? VB : KB;
+    uint64_t *full = is_v ? sm->vfull : sm->kfull;
+    uint64_t *empty = is_v ? sm->vempty : sm->kempty;
     bool okl = true;
     for (int it = 0; it < n && okl; ++it) {
-      const int j = it & 1;
-      if (lane == 0 && it >= 2) okl = mbar_wait(&sm->empty[j], ((it >> 1) - 1) & 1, abort_any);
+      const CacheBox y = cache_box(p, b, kvh, seqlen, it * kBwdTile, lane);
+      if (lane == 0 && it >= nbuf) okl = mbar_wait(&empty[it % nbuf], ((it / nbuf) - 1) & 1, abort_any);
       okl = __shfl_sync(0xffffffffu, okl ? 1 : 0, 0) != 0;
-      if (okl) load_kv_tile<D>(p, &map_k, &map_v, sK(j), sV(j), &sm->full[j], b, kvh, seqlen, it * kBwdTile, lane);
+      if (!okl) break;
+      issue_cache_boxes<D>(p, is_v ? &map_v : &map_k, is_v ? sV(it) : sK(it), &full[it % nbuf], y, lane);
     }
     // nothing of ours may still be landing when the CTA exits
     if (lane == 0) {
       int no_abort = 0;
-      for (int it = max(n - 2, 0); it < n; ++it) mbar_wait(&sm->full[it & 1], (it >> 1) & 1, &no_abort);
-      if (kRowsTma) mbar_wait(&sm->fixed, 0, &no_abort);
+      for (int it = max(n - nbuf, 0); it < n; ++it) mbar_wait(&full[it % nbuf], (it / nbuf) & 1, &no_abort);
+      if (kRowsTma && !is_v) mbar_wait(&sm->fixed, 0, &no_abort);
     }
     __syncwarp();
     __syncthreads();  // the final barrier below
@@ -722,7 +822,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     // key rows past the context in the first key tile: zeros
     if (n > 0 && kBwdTile > seqlen) {
-      ok = mbar_wait(&sm->full[0], 0, abort_any);
+      ok = mbar_wait(&sm->kfull[0], 0, abort_any) && mbar_wait(&sm->vfull[0], 0, abort_any);
       if (ok) zero_rows_from<D>(sK(0), sV(0), seqlen, t, hf);
     }
     if constexpr (!kRowsTma) cp_async_wait<0>();
@@ -739,76 +839,97 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr uint32_t kIdB = idesc_bf16(128, D, 0, 1);
   static_assert(256 + D <= 384, "dQ below the second S range");
 
-  for (int it = 0; it < n && !failed; ++it) {
-    const int j = it & 1;
-    const int k0 = it * kBwdTile;
-    const uint32_t tS = tS0 + j * 384;
-    if (issuer) {
+  if (!failed && issuer) {
+    // ---------------- MMA warp ----------------
+    tc_fence_after_sync();
+    if (kRowsTma && n > 0) ok = mbar_wait(&sm->fixed, 0, abort_any);
+    for (int it = 0; it < n && ok; ++it) {
+      ok = mbar_wait(&sm->kfull[it % KB], (it / KB) & 1, abort_any) &&
+           mbar_wait(&sm->vfull[it % VB], (it / VB) & 1, abort_any);
+      if (ok && it >= 1) ok = mbar_wait(&sm->dp_free, (it - 1) & 1, abort_any);
+      if (ok && it >= 2) ok = mbar_wait(&sm->mma_b, (it - 2) & 1, abort_any);
+      if (!ok) break;
       tc_fence_after_sync();
-      if (kRowsTma && it == 0) ok = mbar_wait(&sm->fixed, 0, abort_any);
-      if (it > 0) {
-        mma_tn(tdQ, tS0 + (j ^ 1) * 384, smem_u32(sK(j ^ 1)), kIdB, it > 1);  // dQ += dS K
-        umma_commit(&sm->mma_b);
-        umma_commit(&sm->empty[j ^ 1]);
-      }
-      if (ok) ok = mbar_wait(&sm->full[j], (it >> 1) & 1, abort_any);
-      if (ok) {
+      const uint32_t tS = tS0 + (it & 1) * 384;
+      mma_kk<D>(tS, sbase, smem_u32(sK(it)), kIdA);              // S = Q K^T
+      mma_kk<D>(tdP, sbase + C::kTile, smem_u32(sV(it)), kIdA);  // dP = dO V^T
+      umma_commit(&sm->mma_a);
+      umma_commit(&sm->vempty[it % VB]);
+      if (it >= 1) {
+        ok = mbar_wait(&sm->ds_ready, (it - 1) & 1, abort_any);
+        if (!ok) break;
         tc_fence_after_sync();
-        mma_kk<D>(tS, sbase, smem_u32(sK(j)), kIdA);               // S = Q K^T
-        mma_kk<D>(tdP, sbase + C::kTile, smem_u32(sV(j)), kIdA);   // dP = dO V^T
-        umma_commit(&sm->mma_a);
+        mma_tn(tdQ, tS0 + ((it - 1) & 1) * 384, smem_u32(sK(it - 1)), kIdB, it > 1);  // dQ += dS K
+        umma_commit(&sm->mma_b);
+        umma_commit(&sm->kempty[(it - 1) % KB]);
       }
     }
-    if (compute) {
-      ok = ok && mbar_wait(&sm->mma_a, it & 1, abort_any);
+    if (ok && n > 0) {
+      ok = mbar_wait(&sm->ds_ready, (n - 1) & 1, abort_any);
       if (ok) {
-        __syncwarp();
         tc_fence_after_sync();
-#pragma unroll 1
-        for (int ch = hf * (8 / kBwdGroups); ch < (hf + 1) * (8 / kBwdGroups); ++ch) {  // its keys
-          float sv[16], dp[16];
-          tmem_ld16(tS + lane_off + ch * 16, sv);
-          tmem_ld16(tdP + lane_off + ch * 16, dp);
-          tmem_ld_wait_for(sv);
-          tmem_ld_wait_for(dp);
-          uint32_t sw[8];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float dv[2];
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const int tok = k0 + ch * 16 + e + k;
-              const float pr = tok < my_lim ? ex2(__fsub_rn(__fmul_rn(sv[e + k], p.cscale), my_l2)) : 0.f;
-              dv[k] = __fmul_rn(pr, __fsub_rn(dp[e + k], my_d));
-            }
-            sw[e / 2] = pack_bf16(dv[0], dv[1]);
-          }
-          tmem_st8(tS + lane_off + ch * 16, sw);
-        }
-        tmem_st_wait();
+        mma_tn(tdQ, tS0 + ((n - 1) & 1) * 384, smem_u32(sK(n - 1)), kIdB, n > 1);
+        umma_commit(&sm->fin);
       }
+    }
+  } else if (!failed && compute) {
+    // ---------------- elementwise warps ----------------
+    const int ch0 = hf * (8 / kBwdGroups);  // its two 16-key chunks: ch0, ch0 + 1
+    for (int it = 0; it < n && ok; ++it) {
+      const int k0 = it * kBwdTile;
+      const uint32_t tS = tS0 + (it & 1) * 384;
+      ok = mbar_wait(&sm->mma_a, it & 1, abort_any);
+      if (!ok) break;
+      __syncwarp();
+      tc_fence_after_sync();
+      float sv[16], dp0[16], dp1[16];
+      tmem_ld16(tdP + lane_off + ch0 * 16, dp0);
+      tmem_ld16(tdP + lane_off + ch0 * 16 + 16, dp1);
+      tmem_ld16(tS + lane_off + ch0 * 16, sv);
+      tmem_ld_wait_for(dp0);
+      tmem_ld_wait_for(dp1);
+      tmem_ld_wait_for(sv);
       // key rows past the context in the next key tile: zeros, before its MMAs
       const int k1 = k0 + kBwdTile;
-      if (ok && it + 1 < n && k1 + kBwdTile > seqlen) {
-        ok = mbar_wait(&sm->full[j ^ 1], ((it + 1) >> 1) & 1, abort_any);
-        if (ok) zero_rows_from<D>(sK(j ^ 1), sV(j ^ 1), seqlen - k1, t, hf);
+      if (it + 1 < n && k1 + kBwdTile > seqlen) {
+        ok = mbar_wait(&sm->kfull[(it + 1) % KB], ((it + 1) / KB) & 1, abort_any) &&
+             mbar_wait(&sm->vfull[(it + 1) % VB], ((it + 1) / VB) & 1, abort_any);
+        if (ok) zero_rows_from<D>(sK(it + 1), sV(it + 1), seqlen - k1, t, hf);
         fence_proxy_async_smem();
       }
+      // dP of this tile is in registers: the next tile's MMAs may overwrite it
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm->dp_free);
+      auto ds_chunk = [&](int ch, const float (&s16)[16], const float (&d16)[16]) {
+        uint32_t sw[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          float dv[2];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int tok = k0 + ch * 16 + e + k;
+            const float pr = tok < my_lim ? ex2(__fsub_rn(__fmul_rn(s16[e + k], p.cscale), my_l2)) : 0.f;
+            dv[k] = __fmul_rn(pr, __fsub_rn(d16[e + k], my_d));
+          }
+          sw[e / 2] = pack_bf16(dv[0], dv[1]);
+        }
+        tmem_st8(tS + lane_off + ch * 16, sw);
+      };
+      ds_chunk(ch0, sv, dp0);
+      tmem_ld16(tS + lane_off + ch0 * 16 + 16, sv);
+      tmem_ld_wait_for(sv);
+      ds_chunk(ch0 + 1, sv, dp1);
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm->ds_ready);
     }
-    tc_fence_before_sync();
-    failed = named_bar_or(kBwdBar, kBwdBarThreads, !ok);
+    // the last accumulation (and every MMA before it) has completed
+    if (ok && n > 0) ok = mbar_wait(&sm->fin, 0, abort_any);
   }
-  if (!failed && n > 0) {
-    if (issuer) {
-      tc_fence_after_sync();
-      mma_tn(tdQ, tS0 + ((n - 1) & 1) * 384, smem_u32(sK((n - 1) & 1)), kIdB, n > 1);
-      umma_commit(&sm->mma_b);
-    }
-    // every earlier accumulation completed before the last S / dP did
-    if (compute) ok = mbar_wait(&sm->mma_b, (n - 1) & 1, abort_any);
-    tc_fence_before_sync();
-    failed = named_bar_or(kBwdBar, kBwdBarThreads, !ok);
-  }
+  tc_fence_before_sync();
+  failed = named_bar_or(kBwdBar, kBwdBarThreads, failed || !ok);
   if (compute && !failed) {
     tc_fence_after_sync();
 #pragma unroll 1

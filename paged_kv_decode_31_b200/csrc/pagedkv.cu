@@ -219,16 +219,17 @@ int launch_rows(const pkv::AttnParams &p, const CUtensorMap &mk, const CUtensorM
 template <int D, bool kRowsTma>
 int launch_bwd(const pkv::BwdParams &p, int64_t kv_ctas, int64_t q_ctas, const CUtensorMap &mk,
                const CUtensorMap &mv, const CUtensorMap &mq, const CUtensorMap &mg, cudaStream_t s) {
-  constexpr int kSmem = pkv::BwdCfg<D>::kSmem > 120 * 1024 ? pkv::BwdCfg<D>::kSmem : 120 * 1024;
-  static_assert(kSmem <= 232448, "shared memory budget");
+  constexpr int kKvSmem = pkv::BwdCfg<D>::kSmem > 120 * 1024 ? pkv::BwdCfg<D>::kSmem : 120 * 1024;
+  constexpr int kQSmem = pkv::BwdQCfg<D>::kSmem > 120 * 1024 ? pkv::BwdQCfg<D>::kSmem : 120 * 1024;
+  static_assert(kKvSmem <= 232448 && kQSmem <= 232448, "shared memory budget");
   auto kv = pkv::bwd_kv_kernel<D, kRowsTma>;
   auto qk = pkv::bwd_q_kernel<D, kRowsTma>;
-  if (cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess ||
-      cudaFuncSetAttribute(qk, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
+  if (cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem) != cudaSuccess ||
+      cudaFuncSetAttribute(qk, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem) != cudaSuccess)
     return PKV_ERR_CUDA;
-  kv<<<static_cast<unsigned>(kv_ctas), pkv::kBwdThreads, kSmem, s>>>(p, mk, mv, mq, mg);
+  kv<<<static_cast<unsigned>(kv_ctas), pkv::kBwdThreads, kKvSmem, s>>>(p, mk, mv, mq, mg);
   if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
-  qk<<<static_cast<unsigned>(q_ctas), pkv::kBwdThreads, kSmem, s>>>(p, mk, mv, mq, mg);
+  qk<<<static_cast<unsigned>(q_ctas), pkv::kBwdQThreads, kQSmem, s>>>(p, mk, mv, mq, mg);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
