@@ -55,6 +55,7 @@ constexpr int kBwdQThreads = kBwdCompute + 96;  // dQ: a second load warp (K and
 constexpr int kBwdTile = 128;  // keys per key tile and rows per row tile
 constexpr uint32_t kBwdBar = 1;                   // named barrier of compute + MMA warps
 constexpr uint32_t kBwdBarThreads = kBwdCompute + 32;
+constexpr uint32_t kBwdComputeBar = 2;            // named barrier of the elementwise warps
 
 struct BwdParams {
   const __nv_bfloat16 *q, *dout;
@@ -145,6 +146,7 @@ struct BwdCfg {
     uint64_t full[2], empty[2];  // streamed tile buffers: loaded / free again
     uint64_t fixed;              // the fixed tiles loaded
     uint64_t mma_a, mma_b, mma_bv, drain;
+    uint64_t ds_ready, fin;  // elementwise pass -> MMA warp; last accumulation done
     uint32_t tmem_base;
     alignas(16) int lim[2][kBwdTile];  // key limit of each row of the row tile in buffer j
     alignas(16) float lse2[2][kBwdTile];
@@ -389,6 +391,8 @@ __device__ __forceinline__ void bwd_init_barriers(Small *sm) {
   mbar_init(&sm->mma_b, 1);
   mbar_init(&sm->mma_bv, 1);
   mbar_init(&sm->drain, 1);
+  mbar_init(&sm->ds_ready, kBwdCompute / 32);  // one arrival per elementwise warp
+  mbar_init(&sm->fin, 1);
   fence_barrier_init();
 }
 
@@ -398,14 +402,17 @@ __device__ __forceinline__ void bwd_init_barriers(Small *sm) {
 // (3 + 2 j) tiles.
 // TMEM: S^T [0,128) (P^T packed over it), dP^T [128,256) (dS^T packed over
 // it), dV [256, 256 + D), dK [256 + D, 256 + 2D).
-// Tile it: barrier; MMA warp: dV += P^T(it - 1) dO, dK += dS^T(it - 1) Q,
-// then S^T = K Q(it)^T, dP^T = V dO(it)^T; compute warps: P^T / dS^T of it
-// into TMEM once the second pair is done; load warp: row tile it + 2 into
+// Row tile it: MMA warp: once P^T / dS^T(it - 1) are in TMEM (ds_ready),
+// dV += P^T(it - 1) dO, dK += dS^T(it - 1) Q, then S^T = K Q(it)^T,
+// dP^T = V dO(it)^T; elementwise warps: once the second pair is done (mma_a),
+// P^T / dS^T of it into TMEM, then ds_ready; load warp: row tile it + 2 into
 // buffer j once the first pair of it is done.  MMAs into different
 // accumulators carry no ordering guarantee among themselves, so S^T(it),
 // which overwrites the P^T that dV(it - 1) reads, is issued once dV(it - 1)
 // has completed (its own commit, `mma_bv`, landing while dK(it - 1) runs),
 // and dP^T(it) once dK(it - 1) has (`mma_b`, landing while S^T(it) runs).
+// The elementwise warps meet at a barrier of their own at the start of each
+// tile (the row statistics they share); the MMA warp takes no part in it.
 // kRowsTma false: the compute threads stage the row tiles with cp.async.
 // ---------------------------------------------------------------------------
 template <int D, bool kRowsTma>
@@ -549,12 +556,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr uint32_t kIdA = idesc_bf16(128, 128, 0, 0);
   constexpr uint32_t kIdB = idesc_bf16(128, D, 0, 1);
 
-  for (int it = 0; it < n && !failed; ++it) {
-    const int j = it & 1;
-    if (issuer) {
-      tc_fence_after_sync();
-      if (it == 0) ok = mbar_wait(&sm->fixed, 0, abort_any);
+  if (!failed && issuer) {
+    // ---------------- MMA warp ----------------
+    tc_fence_after_sync();
+    ok = mbar_wait(&sm->fixed, 0, abort_any);
+    for (int it = 0; it < n && ok; ++it) {
+      const int j = it & 1;
       if (it > 0) {
+        // P^T / dS^T of tile it - 1 are in TMEM
+        ok = mbar_wait(&sm->ds_ready, (it - 1) & 1, abort_any);
+        if (!ok) break;
+        tc_fence_after_sync();
         const uint32_t aQ = smem_u32(sQ(j ^ 1)), aG = smem_u32(sG(j ^ 1));
         mma_tn(tdV, tS, aG, kIdB, it > 1);   // dV += P^T dO
         umma_commit(&sm->mma_bv);
@@ -576,7 +588,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         umma_commit(&sm->mma_a);
       }
     }
-    if (compute) {
+    if (ok) {
+      ok = mbar_wait(&sm->ds_ready, (n - 1) & 1, abort_any);
+      if (ok) {
+        tc_fence_after_sync();
+        const uint32_t aQ = smem_u32(sQ((n - 1) & 1)), aG = smem_u32(sG((n - 1) & 1));
+        mma_tn(tdV, tS, aG, kIdB, n > 1);
+        mma_tn(tdK, tdP, aQ, kIdB, n > 1);
+        umma_commit(&sm->fin);
+      }
+    }
+  } else if (!failed && compute) {
+    // ---------------- elementwise warps ----------------
+    for (int it = 0; it < n && ok; ++it) {
+      const int j = it & 1;
       const bool next = it + 1 < n;
       if constexpr (!kRowsTma) {
         // buffer j ^ 1 is free once the accumulation of tile it - 1 is done
@@ -585,60 +610,56 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (next) row_stats(rt0 + it + 1);
       ok = ok && mbar_wait(&sm->mma_a, it & 1, abort_any);
-      if (ok) {
-        __syncwarp();
-        tc_fence_after_sync();
-#pragma unroll 1
-        for (int ch = hf * (8 / kBwdGroups); ch < (hf + 1) * (8 / kBwdGroups); ++ch) {  // its rows
-          float sv[16], dp[16];
-          tmem_ld16(tS + lane_off + ch * 16, sv);
-          tmem_ld16(tdP + lane_off + ch * 16, dp);
-          tmem_ld_wait_for(sv);
-          tmem_ld_wait_for(dp);
-          uint32_t pw[8], sw[8];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float pv[2], dv[2];
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const int c = ch * 16 + e + k;
-              const bool vis = tok < sm->lim[j][c];
-              const float pr =
-                  vis ? ex2(__fsub_rn(__fmul_rn(sv[e + k], p.cscale), sm->lse2[j][c])) : 0.f;
-              pv[k] = pr;
-              dv[k] = __fmul_rn(pr, __fsub_rn(dp[e + k], sm->dsum[j][c]));
-            }
-            pw[e / 2] = pack_bf16(pv[0], pv[1]);
-            sw[e / 2] = pack_bf16(dv[0], dv[1]);
-          }
-          tmem_st8(tS + lane_off + ch * 16, pw);
-          tmem_st8(tdP + lane_off + ch * 16, sw);
-        }
-        tmem_st_wait();
+      // the row statistics of tile it (written during tile it - 1) are
+      // visible to every elementwise thread past this barrier, and nobody
+      // reads the other buffer's any more
+      if (named_bar_or(kBwdComputeBar, kBwdCompute, !ok)) {
+        ok = false;
+        break;
       }
+      __syncwarp();
+      tc_fence_after_sync();
+#pragma unroll 1
+      for (int ch = hf * (8 / kBwdGroups); ch < (hf + 1) * (8 / kBwdGroups); ++ch) {  // its rows
+        float sv[16], dp[16];
+        tmem_ld16(tS + lane_off + ch * 16, sv);
+        tmem_ld16(tdP + lane_off + ch * 16, dp);
+        tmem_ld_wait_for(sv);
+        tmem_ld_wait_for(dp);
+        uint32_t pw[8], sw[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int c = ch * 16 + e + k;
+            const bool vis = tok < sm->lim[j][c];
+            const float pr =
+                vis ? ex2(__fsub_rn(__fmul_rn(sv[e + k], p.cscale), sm->lse2[j][c])) : 0.f;
+            pv[k] = pr;
+            dv[k] = __fmul_rn(pr, __fsub_rn(dp[e + k], sm->dsum[j][c]));
+          }
+          pw[e / 2] = pack_bf16(pv[0], pv[1]);
+          sw[e / 2] = pack_bf16(dv[0], dv[1]);
+        }
+        tmem_st8(tS + lane_off + ch * 16, pw);
+        tmem_st8(tdP + lane_off + ch * 16, sw);
+      }
+      tmem_st_wait();
       if (next) store_stats(j ^ 1);
       if constexpr (!kRowsTma) {
         cp_async_wait<0>();
         fence_proxy_async_smem();
       }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm->ds_ready);
     }
-    tc_fence_before_sync();
-    failed = named_bar_or(kBwdBar, kBwdBarThreads, !ok);
+    // the last accumulation (and every MMA before it) has completed
+    if (ok) ok = mbar_wait(&sm->fin, 0, abort_any);
   }
-  if (!failed) {
-    if (issuer) {
-      tc_fence_after_sync();
-      const uint32_t aQ = smem_u32(sQ((n - 1) & 1)), aG = smem_u32(sG((n - 1) & 1));
-      mma_tn(tdV, tS, aG, kIdB, n > 1);
-      mma_tn(tdK, tdP, aQ, kIdB, n > 1);
-      umma_commit(&sm->mma_b);
-    }
-    // every earlier phase of mma_b has completed (the MMA warp waited for
-    // it before the last dP^T), so this parity names the last one
-    if (compute) ok = mbar_wait(&sm->mma_b, (n - 1) & 1, abort_any);
-    tc_fence_before_sync();
-    failed = named_bar_or(kBwdBar, kBwdBarThreads, !ok);
-  }
+  tc_fence_before_sync();
+  failed = named_bar_or(kBwdBar, kBwdBarThreads, failed || !ok);
   if (compute && !failed) {
     tc_fence_after_sync();
     int64_t blk = -1;
