@@ -899,7 +899,7 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
     for (int it = 0; it < n && ok; ++it) {
       const int k0 = it * kBwdTile;
       const uint32_t tS = tS0 + (it & 1) * 384;
-      ok = mbar_wait(&sm->mma_a, it & 1, abort_any);
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm->mma_a, it & 1, abort_any));  // warp-wide
       if (!ok) break;
       __syncwarp();
       tc_fence_after_sync();
