@@ -11,32 +11,30 @@
 // where i runs over the query rows r = i * G + g of the KV head.  No atomics:
 //   bwd_kv_kernel   one CTA per (sequence, KV head, 128-key tile): S^T = K Q^T
 //                   and dP^T = V dO^T on the tensor cores (keys on M), P^T and
-//                   dS^T to shared memory as bf16, dV += P^T dO and dK += dS^T Q
-//                   accumulated in TMEM over the 128-row tiles in ascending
-//                   order, then written once;
+//                   dS^T packed as bf16 into TMEM, dV += P^T dO and
+//                   dK += dS^T Q accumulated in TMEM over the 128-row tiles in
+//                   ascending order, then written once;
 //   bwd_q_kernel    one CTA per (sequence, KV head, 128-row tile): S = Q K^T,
-//                   dP = dO V^T (rows on M), dS to shared memory, dQ += dS K
+//                   dP = dO V^T (rows on M), dS packed into TMEM, dQ += dS K
 //                   accumulated over the key tiles in ascending order.
 // Every sum therefore has one fixed order and the result is bitwise
 // reproducible and independent of the batch around a sequence.
 //
-// 576 threads: warps 0-15 do the elementwise work -- warps w, w + 4, w + 8,
-// w + 12 share TMEM lanes 32 (w % 4) .. + 31 (thread t = lane t of the 128)
-// and split the columns in quarters --, warp 16 owns TMEM, its lane 0
-// issuing the MMAs, and warp 17 loads every operand tile with TMA (the
-// cache's K / V rows in boxes addressed through the block table, as the
-// forward does; Q and dO in boxes of 128 / G tokens x G heads).  The second
-// operand pair of each product (P^T and dS^T, or dS) never touches shared
-// memory: the elementwise pass packs it as bf16 into the TMEM columns its
-// S / dP values came from and the next MMAs read it from there as their A
-// operand.  The shared memory this frees holds a second buffer of the
-// streamed tiles (Q and dO, or K and V), which the load warp fills while the
-// current tile's MMAs and elementwise pass run; one named barrier per tile
-// (compute and MMA warps) hands the packed TMEM operands to the MMA warp,
-// whose tensor pipe executes the previous tile's accumulation and the
-// current tile's S / dP products back to back.  Where a row tile cannot be
-// one Q box (G not dividing 128, or fewer than 128 / G query tokens), the
-// compute threads stage the Q / dO tiles with cp.async instead.
+// Warps 0-15 do the elementwise work -- warps w, w + 4, w + 8, w + 12 share
+// TMEM lanes 32 (w % 4) .. + 31 (thread t = lane t of the 128) and split the
+// columns in quarters --, warp 16 owns TMEM, its lane 0 issuing the MMAs, and
+// the warps after it load every operand tile with TMA (the cache's K / V rows
+// in boxes addressed through the block table, as the forward does; Q and dO
+// in boxes of 128 / G tokens x G heads): one load warp for dK/dV (576
+// threads), one per cache for dQ (608 threads).  The second operand of each
+// accumulating product (P^T and dS^T, or dS) never touches shared memory:
+// the elementwise pass packs it as bf16 into the TMEM columns its S / dP
+// values came from and the next MMAs read it from there as their A operand.
+// The shared memory this frees holds deeper rings of the streamed tiles (Q
+// and dO, or K and V).  The elementwise warps and the MMA warp hand off
+// through mbarriers (no block-wide barrier per tile).  Where a row tile
+// cannot be one Q box (G not dividing 128, or fewer than 128 / G query
+// tokens), the compute threads stage the Q / dO tiles with cp.async instead.
 #pragma once
 
 #include <cuda_bf16.h>
