@@ -194,7 +194,7 @@ def cpu_baseline(di_dev, n_seq: int = 4):
             "tokens_per_s": round(n_seq / dt, 4)}
 
 
-def prefill_secondary(dev, reps: int = 5):
+def prefill_secondary(dev, reps: int = 20):
     """Chunked causal prefill of the parity workload (batch 8, Hq 16 / Hkv 4,
     D 128, block_size 16): 4 chunks of 512 tokens, each appended and attended
     by one paged_decode_attn_append call (an append launch, then the row-major
@@ -312,7 +312,7 @@ def varlen_secondary(dev, reps: int = 10):
             "tflops": round(flops / (ms / 1e3) / 1e12, 2), "algorithmic_flops": flops}
 
 
-def backward_secondary(dev, reps: int = 5):
+def backward_secondary(dev, reps: int = 20):
     """Deterministic backward of the full causal prefill of the parity
     workload (batch 8 x 2048 tokens, Hq 16 / Hkv 4, D 128, block_size 16):
     one forward for out / lse, then paged_prefill_attn_bwd timed alone.
