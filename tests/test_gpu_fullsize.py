@@ -10,7 +10,7 @@ import oracle
 import paged_kv_decode_31_b200 as pkv
 from paged_kv_decode_31_b200 import inputs as I
 
-from gpu_helpers import assert_close_to_oracle, run_gpu
+from gpu_helpers import assert_close_to_oracle, bits_equal, run_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -63,3 +63,33 @@ def test_long_context_full_size_fused_append():
     torch.cuda.empty_cache()
     # the appended token is in the host copy of the cache (copied after the call)
     _sampled_check(host, out.cpu(), lse.cpu(), seqs=[0, 3], kv_heads=[(0, 1), (7, 8)])
+
+
+def test_million_token_contexts():
+    """The longest contexts tested: 2^20 tokens (256 splits per row) and
+    2^20 - 4097 (a last split of 4095 keys), Hq 8 / Hkv 2, D 128, block size
+    16, contiguous cache with a randperm table.  Every (sequence, KV head)
+    group against the oracle; each sequence run alone bitwise equal to its
+    rows of the batch (the 256-split merge does not depend on the batch)."""
+    dev = torch.device("cuda", 0)
+    Hq, Hkv, D, bs, L = 8, 2, 128, 16, 1 << 20
+    gen = torch.Generator(device=dev).manual_seed(4242)
+    num_blocks = 2 * (L // bs)
+    q = I.randn_bf16((2, 1, Hq, D), gen, dev)
+    cache = I.make_cache(num_blocks, bs, Hkv, D, "contiguous", gen, dev)
+    table = I.randperm_table(num_blocks, 2, gen, dev)
+    sl = torch.tensor([L, L - 4097], dtype=torch.int32, device=dev)
+    scale = 1.0 / D ** 0.5
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    out, lse = pkv.paged_decode_attn(q, cache.k, cache.v, table, sl, max_seqlen_k=L, scale=scale,
+                                     causal=False, err=err)
+    for b in range(2):
+        o1, l1 = pkv.paged_decode_attn(q[b:b + 1], cache.k, cache.v, table[b:b + 1], sl[b:b + 1],
+                                       max_seqlen_k=L, scale=scale, causal=False, err=err)
+        assert bits_equal(o1, out[b:b + 1]) and bits_equal(l1, lse[b:b + 1])
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    host = I.DecodeInputs(q.cpu(), cache.to("cpu"), table.cpu(), sl.cpu(), Hq, Hkv, D, scale, False)
+    del cache
+    torch.cuda.empty_cache()
+    _sampled_check(host, out.cpu(), lse.cpu(), seqs=[0, 1], kv_heads=[(0, 1), (1, 2)])
