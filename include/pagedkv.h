@@ -23,9 +23,11 @@
  * tokens.  Within a split, tiles are folded in ascending order with an online
  * softmax in fp32: scores and P.V on the tensor cores with fp32 accumulation
  * (each probability entering P.V as a bf16 part and a bf16 remainder, ~16
- * significant bits, into two accumulators added in fp32), each tile's max
- * and row sums of the fp32 probabilities on the CUDA cores in fixed reduction
- * trees, and the running rescale in fp32 with the tile's own max.  Split
+ * significant bits, into two accumulators kept over the split's tiles and
+ * added in fp32 at its end), each tile's max and row sums of the fp32
+ * probabilities on the CUDA cores in fixed reduction trees, and a running max
+ * that rises only when a tile's max exceeds it by more than 2^8 (the
+ * accumulators and the row sum are then rescaled in fp32).  Split
  * partials are merged in ascending split index (= global block index) order
  * in fp32, and out is rounded to bf16 once, at the final write.  Source:
  * RL-Kernel PR #284

@@ -7,30 +7,35 @@
 // row's bits do not depend on which kernel ran it -- but the tile is laid out
 // the other way round: 128 rows r = i * G + g of one KV head against 128 keys,
 //   S      = Q * K_tile^T on the tensor cores (M = 128 rows, N = 128 keys),
-//   softmax one thread per ROW: all of a row's reductions are in-thread
-//           (the row sum replays the 32-key shuffle-down trees and the
-//           four-warp combine of attn_split.cuh element for element),
+//   softmax one thread per ROW, two warpgroups on every tile (keys
+//           [0, 64) and [64, 128)): the halves' maxima meet in shared
+//           memory, the running max, the O rescale and l follow
+//           attn_split.cuh's rule, and the row sum replays its 32-key
+//           shuffle-down trees and four-warp combine element for element,
 //   P      = [bf16(p) | bf16(p - bf16(p))] written back over S in TMEM,
-//   O      = P_hi * V and P_lo * V into two accumulators, with P read from
-//           TMEM (A operand) and V from shared memory (MN-major),
-//   update acc = fma(O_hi + O_lo, b, acc * a) per row in the correction warpgroup,
-//           which owns the row's (m, l, acc[D]) in registers.
+//   O      += P_hi * V and P_lo * V into two accumulators that stay in TMEM
+//           over the split's tiles, with P read from TMEM (A operand) and V
+//           from shared memory (MN-major); acc = O_hi + O_lo at the split's
+//           end.
 // The tensor cores give every output element the same bits whichever operand
 // is A and whichever is B (the per-element dot products do not depend on the
 // orientation or on N), so S, O_hi and O_lo here equal the transposed
 // kernel's S^T, O_hi^T and O_lo^T bit for bit, and so does every row's result.
 //
-// Roles (512 threads): warps 0-3 / 4-7 softmax warpgroups (even / odd tiles;
-// thread t = TMEM lane t = row t of the tile), 8-11 correction + epilogue,
-// 12 K producer (+ Q by TMA), 13 V producer, 14 MMA issuer + TMEM owner,
-// 15 idle.  Registers are rebalanced per warpgroup (setmaxnreg): the
-// correction warpgroup holds a row's D fp32 accumulators.
+// Roles (512 threads): warps 0-3 / 4-7 softmax warpgroups (thread t = TMEM
+// lane t = row t of the tile; warpgroup 0 keeps the rows' l and rescales
+// O_hi, warpgroup 1 rescales O_lo), 8-11 epilogue (a unit's O out of TMEM
+// once its last P.V is done, then its out / lse or partials, while the next
+// unit's tiles run), 12 K producer (+ Q by TMA), 13 V producer, 14 MMA issuer
+// + TMEM owner, 15 idle.  Registers are rebalanced per warpgroup
+// (setmaxnreg): the epilogue warpgroup holds a row's D fp32 accumulators.
 //
 // TMEM (512 columns): kSB S/P buffers of 128 columns (tile gi uses buffer
 // gi % kSB, so the QK of tile gi waits only for the P.V of tile gi - kSB; P
 // of keys [32 g, 32 g + 32) goes over those keys' own S columns: hi in the
-// first 16, lo in the next 16), then O_hi and O_lo (D columns each).  kSB = 2
-// at head_dim 128, 3 at 64.
+// first 16, lo in the next 16), then O_hi and O_lo (D columns each, one
+// unit at a time: the next unit's first P.V waits until the epilogue has read
+// O out).  kSB = 2 at head_dim 128, 3 at 64.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -70,12 +75,17 @@ struct RowCfg {
   static constexpr int kSchedScratch = kQB * kQBytes;  // bytes free at kernel start
   struct Small {
     uint64_t full_k[NS], empty_k[NS], full_v[NS], empty_v[NS];
-    uint64_t s_full[3], p_full[3], s_free[3], stat_free[3], o_full, o_free;
+    uint64_t s_full[3], p_full[3], s_free[3];
+    uint64_t ml_full[2];  // [unit parity]: the unit's (m, l) rows are published
+    uint64_t ml_free[2];  // [unit parity]: the epilogue has read them
+    uint64_t unit_done;   // a unit's last P.V completed (one phase per unit)
+    uint64_t o_free;      // O is read out: the next unit's P.V may start it afresh
     uint64_t q_full[2], q_empty[2], drain;
     uint32_t tmem_base;
     int abort_any;
-    float tmax[3][kRowsPerTile];  // [buffer][row]: the tile's max (base-2 units)
-    float lsum[3][kRowsPerTile];  // [buffer][row]: the tile's sum of p
+    float xmax[2][2][kRowsPerTile];  // [tile parity][half][row]: the halves' maxima
+    float xsum[2][kRowsPerTile];     // [tile parity][row]: the second half's sum of p
+    float ml[2][2][kRowsPerTile];    // [unit parity][m, l][row]: the unit's final (m, l)
     int tab[2][2][kSplitTokens / 16];
     int sched_list[kSchedMaxMine];     // this CTA's units (balanced schedule)
     int sched_meta[kSchedMaxMine][3];  // their sequence length and query range
@@ -172,16 +182,17 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     }
     for (int i = 0; i < C::kSB; ++i) {
       mbar_init(&sm->s_full[i], 1);
-      mbar_init(&sm->p_full[i], 4);     // one arrival per softmax warp
+      mbar_init(&sm->p_full[i], 8);  // one arrival per softmax warp
       mbar_init(&sm->s_free[i], 1);
-      mbar_init(&sm->stat_free[i], 4);  // one arrival per correction warp
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm->q_full[i], 1);
       mbar_init(&sm->q_empty[i], 1);
+      mbar_init(&sm->ml_full[i], 4);  // one arrival per warp of softmax warpgroup 0
+      mbar_init(&sm->ml_free[i], 4);  // one arrival per epilogue warp
     }
-    mbar_init(&sm->o_full, 1);
-    mbar_init(&sm->o_free, 4);
+    mbar_init(&sm->unit_done, 1);
+    mbar_init(&sm->o_free, 4);  // one arrival per correction warp
     mbar_init(&sm->drain, 1);
     sm->abort_any = 0;
     fence_barrier_init();
@@ -220,12 +231,18 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       constexpr uint32_t kIdescPV = idesc_bf16(128, D, 0, 1);    // A = P (TMEM), B = V (MN-major)
       // (phase parity of the k-th use of buffer gi % kSB is k & 1, k = gi / kSB)
       constexpr int SB = C::kSB;
-      int gi = 0, ui = 0, pend0 = -1, pend1 = -1;  // tiles whose P.V is not issued yet
+      // a tile whose P.V is not issued yet: its index, whether it opens its
+      // unit (P.V starts O afresh) and the unit's ordinal among units with tiles
+      struct Pend {
+        int g, first, last, uo;
+      };
+      int gi = 0, ui = 0, npend = 0;
+      Pend pend[2] = {{-1, 0, 0, 0}, {-1, 0, 0, 0}};
       bool failed = false;
-      auto pv_step = [&](int g) -> bool {
-        const int st = g % NS, bb = g % SB;
+      auto pv_step = [&](const Pend &pd) -> bool {
+        const int g = pd.g, st = g % NS, bb = g % SB;
         if (!mbar_wait(&sm->p_full[bb], (g / SB) & 1, abort_any, p.wait_ns)) return false;
-        if (!mbar_wait(&sm->o_free, (g & 1) ^ 1, abort_any, p.wait_ns)) return false;
+        if (pd.first && !mbar_wait(&sm->o_free, (pd.uo & 1) ^ 1, abort_any, p.wait_ns)) return false;
         if (!mbar_wait(&sm->full_v[st], (g / NS) & 1, abort_any, p.wait_ns)) return false;
         tc_fence_after_sync();
         const uint32_t vaddr = sbase + C::kOffV + st * C::kKVBytes;
@@ -235,15 +252,16 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           // V: MN-major (N = head_dim), 128-byte swizzle; 64-wide d groups
           // kHalfBytes apart, 8-key groups 1024 bytes apart.  P_hi of keys
           // [16 kk, 16 kk + 16): TMEM columns 32 (kk / 2) + 8 (kk % 2) + [0, 8),
-          // P_lo 16 columns further.
+          // P_lo 16 columns further.  O accumulates over the unit's tiles.
           const uint64_t b = smem_desc(vaddr + kk * 2048, C::kHalfBytes, 1024, kLayoutSw128);
           const uint32_t a = pcol + (kk >> 1) * 32 + (kk & 1) * 8;
-          umma_bf16_ts(tmem + C::kColOhi, a, b, kIdescPV, kk > 0 ? 1u : 0u);
-          umma_bf16_ts(tmem + C::kColOlo, a + 16, b, kIdescPV, kk > 0 ? 1u : 0u);
+          const uint32_t acc = (pd.first && kk == 0) ? 0u : 1u;
+          umma_bf16_ts(tmem + C::kColOhi, a, b, kIdescPV, acc);
+          umma_bf16_ts(tmem + C::kColOlo, a + 16, b, kIdescPV, acc);
         }
-        umma_commit(&sm->o_full);
         umma_commit(&sm->empty_v[st]);
         umma_commit(&sm->s_free[bb]);
+        if (pd.last) umma_commit(&sm->unit_done);
         return true;
       };
       for (int k = 0; k < sc.count && !failed; ++k) {
@@ -275,29 +293,19 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           umma_commit(&sm->empty_k[st]);
           if (j == x.n_tiles - 1) umma_commit(&sm->q_empty[qb]);
           // keep at most kSB - 1 tiles whose P.V is not issued yet
-          if (SB == 2 && pend0 >= 0) {
-            if (!pv_step(pend0)) {
+          if (npend == SB - 1) {
+            if (!pv_step(pend[0])) {
               failed = true;
               break;
             }
-            pend0 = gi;
-          } else if (SB == 3 && pend1 >= 0) {
-            if (!pv_step(pend0)) {
-              failed = true;
-              break;
-            }
-            pend0 = pend1;
-            pend1 = gi;
-          } else if (pend0 >= 0) {
-            pend1 = gi;
-          } else {
-            pend0 = gi;
+            pend[0] = pend[1];
+            --npend;
           }
+          pend[npend++] = Pend{gi, j == 0 ? 1 : 0, j == x.n_tiles - 1 ? 1 : 0, ui};
         }
         ++ui;
       }
-      if (!failed && pend0 >= 0) failed = !pv_step(pend0);
-      if (!failed && pend1 >= 0) failed = !pv_step(pend1);
+      for (int i = 0; i < npend && !failed; ++i) failed = !pv_step(pend[i]);
       // every MMA this thread issued completes before TMEM is released, also
       // when the consumers gave up (bounded wait, default limit)
       (void)failed;
@@ -307,16 +315,24 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     }
   } else if (warp < kCorrWarp0) {
     // ------------------------------------------------------------------
-    // Softmax warpgroups: warpgroup wg takes the tiles with gi % 2 == wg;
-    // thread t owns row t.  tmax = exact max of the row's masked scores,
-    // p = 2^(s - tmax), P = [bf16(p) | bf16(p - bf16(p))] over S in TMEM,
-    // L = the row's sum of the fp32 p in the contract's fixed tree.
+    // Softmax warpgroups: both take every tile, warpgroup wg its keys
+    // [64 wg, 64 wg + 64); thread t owns row t.  tmax = exact max of the
+    // row's masked scores (the two halves' maxima exchanged through shared
+    // memory); the running max m rises to tmax only when tmax > m + kMaxSlack
+    // (a unit starts from -inf), and then O (warpgroup 0: O_hi, 1: O_lo) and
+    // l take the factor a = 2^(m - m') before this tile's P.V adds to O;
+    // p = 2^(s - m), P = [bf16(p) | bf16(p - bf16(p))] over S in TMEM; the
+    // row's sum of the fp32 p in the contract's fixed tree (each warpgroup's
+    // two 32-key sums, then the halves), l = fma(l, a, sum).  Both
+    // warpgroups keep m in registers, warpgroup 0 keeps l and publishes the
+    // unit's (m, l) for the epilogue.
     // ------------------------------------------------------------------
     regs_dec<kRowsSoftmaxRegs>();
     const int wg = warp >> 2, wq = warp & 3, t = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t bar_id = 1 + wg;
-    int gbase = 0;
+    const uint32_t ocol = tmem + lane_off + (wg == 0 ? C::kColOhi : C::kColOlo);
+    constexpr uint32_t kXchgBar = 1, kDoneBar = 2;  // named barriers over both warpgroups
+    int gbase = 0, uo = 0;
     bool stop = false;
     for (int k = 0; k < sc.count && !stop; ++k) {
       const Unit x = sc.get<kRowsPerTile>(p, k);
@@ -328,27 +344,26 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         if (p.causal) lim = min(lim, x.seqlen - x.nq + i + 1);
         nlim = lim > 0 ? lim : 0;
       }
+      float m_run = NEG_INF, l_run = 0.f;
       for (int j = 0; j < x.n_tiles; ++j) {
         const int gi = gbase + j;
-        if ((gi & 1) != wg) continue;
         const int bb = gi % C::kSB, st = gi % NS, par = (gi / C::kSB) & 1;
         bool ok = mbar_wait(&sm->s_full[bb], par, abort_any, p.wait_ns);
-        ok = mbar_wait(&sm->stat_free[bb], par ^ 1, abort_any, p.wait_ns) && ok;
         tc_fence_after_sync();
         const int tok0 = x.tok0 + j * kTileTokens;
         const int nvis = min(max(nlim - tok0, 0), kTileTokens);
         const uint32_t srow = tmem + lane_off + bb * 128;  // S of this tile, then its P
-        // pass 1: the row's max.  Scaling by cscale > 0 rounds monotonically,
-        // so on a fully visible tile max(s) * cscale is the max of the scaled
-        // scores exactly.  The branch is taken per WARP (tcgen05.ld is
-        // .sync.aligned: all 32 lanes must issue the same load together).
+        // pass 1: this half's max.  Scaling by cscale > 0 rounds
+        // monotonically, so on fully visible keys max(s) * cscale is the max
+        // of the scaled scores exactly.  The branch is taken per WARP
+        // (tcgen05.ld is .sync.aligned: all 32 lanes issue the same load).
         __syncwarp();
         const bool full = __all_sync(0xffffffffu, nvis == kTileTokens);  // warp-uniform
-        float mx = NEG_INF;
+        float hm = NEG_INF;
         if (full) {
           float raw = NEG_INF;
 #pragma unroll 1
-          for (int ch = 0; ch < 8; ch += 2) {
+          for (int ch = 4 * wg; ch < 4 * wg + 4; ch += 2) {
             float v0[16], v1[16];
             tmem_ld16(srow + ch * 16, v0);
             tmem_ld16(srow + ch * 16 + 16, v1);
@@ -357,10 +372,10 @@ __global__ void __launch_bounds__(kRowThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) raw = fmaxf(raw, fmaxf(v0[e], v1[e]));
           }
-          mx = __fmul_rn(raw, p.cscale);
+          hm = __fmul_rn(raw, p.cscale);
         } else {
 #pragma unroll 1
-          for (int ch = 0; ch < 8; ch += 2) {
+          for (int ch = 4 * wg; ch < 4 * wg + 4; ch += 2) {
             float v0[16], v1[16];
             tmem_ld16(srow + ch * 16, v0);
             tmem_ld16(srow + ch * 16 + 16, v1);
@@ -370,16 +385,55 @@ __global__ void __launch_bounds__(kRowThreads, 1)
             for (int e = 0; e < 16; ++e) {
               const float s0 = (ch * 16 + e < nvis) ? __fmul_rn(v0[e], p.cscale) : NEG_INF;
               const float s1 = (ch * 16 + 16 + e < nvis) ? __fmul_rn(v1[e], p.cscale) : NEG_INF;
-              mx = fmaxf(mx, fmaxf(s0, s1));
+              hm = fmaxf(hm, fmaxf(s0, s1));
             }
           }
         }
-        // pass 2: p, P_hi / P_lo back into TMEM, and the row sum, 32 keys at
-        // a time (one warp's keys in the transposed kernel); the four 32-key
-        // sums combine as (w0 + w1) + (w2 + w3)
-        float w_even = 0.f, s01 = 0.f, s23 = 0.f;
+        sm->xmax[gi & 1][wg][t] = hm;
+        // both halves' maxima are published (and a failed wait is known to
+        // both warpgroups, which then stop together)
+        if (named_bar_or(kXchgBar, 256, !ok)) {
+          stop = true;
+          break;
+        }
+        const float mx = fmaxf(hm, sm->xmax[gi & 1][wg ^ 1][t]);
+        const float m_prev = m_run;
+        const float m_new = (mx > __fadd_rn(m_prev, kMaxSlack)) ? mx : m_prev;
+        m_run = m_new;
+        const float a = (m_prev == NEG_INF || m_new == m_prev) ? 1.f : ex2(__fsub_rn(m_prev, m_new));
+        if (__any_sync(0xffffffffu, a != 1.f)) {
+          // a != 1 only past the unit's first tile: O holds its tiles < gi.
+          // P.V(gi - 1) completes on s_free[(gi - 1) % kSB]; that barrier's
+          // previous phase (tile gi - 1 - kSB) completed before S(gi) could be
+          // written, so this parity wait cannot alias an older phase.
+          ok = mbar_wait(&sm->s_free[(gi - 1) % C::kSB], ((gi - 1) / C::kSB) & 1, abort_any,
+                         p.wait_ns) && ok;
+          if (__all_sync(0xffffffffu, ok)) {
+            tc_fence_after_sync();
 #pragma unroll 1
-        for (int grp = 0; grp < 4; ++grp) {
+            for (int ch = 0; ch < D / 16; ch += 2) {
+              float o0[16], o1[16];
+              tmem_ld16(ocol + ch * 16, o0);
+              tmem_ld16(ocol + ch * 16 + 16, o1);
+              tmem_ld_wait_for(o0);
+              tmem_ld_wait_for(o1);
+              uint32_t w0[16], w1[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                w0[e] = __float_as_uint(__fmul_rn(o0[e], a));
+                w1[e] = __float_as_uint(__fmul_rn(o1[e], a));
+              }
+              tmem_st16(ocol + ch * 16, w0);
+              tmem_st16(ocol + ch * 16 + 16, w1);
+            }
+          }
+        }
+        // pass 2: p, P_hi / P_lo back into TMEM, and this half's sum, 32 keys
+        // at a time (one warp's keys in the transposed kernel); the four
+        // 32-key sums combine as (w0 + w1) + (w2 + w3)
+        float w_even = 0.f, half = 0.f;
+#pragma unroll 1
+        for (int grp = 2 * wg; grp < 2 * wg + 2; ++grp) {
           float va[16], vb[16];  // keys 32 grp + [0, 16) and + [16, 32)
           tmem_ld16(srow + grp * 32, va);
           tmem_ld16(srow + grp * 32 + 16, vb);
@@ -390,28 +444,28 @@ __global__ void __launch_bounds__(kRowThreads, 1)
             for (int e = 0; e < 16; ++e) {
               const float sa = __fmul_rn(va[e], p.cscale);
               const float sb = __fmul_rn(vb[e], p.cscale);
-              va[e] = (sa == NEG_INF) ? 0.f : ex2(__fsub_rn(sa, mx));
-              vb[e] = (sb == NEG_INF) ? 0.f : ex2(__fsub_rn(sb, mx));
+              va[e] = (sa == NEG_INF) ? 0.f : ex2(__fsub_rn(sa, m_new));
+              vb[e] = (sb == NEG_INF) ? 0.f : ex2(__fsub_rn(sb, m_new));
             }
           } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const float sa = (grp * 32 + e < nvis) ? __fmul_rn(va[e], p.cscale) : NEG_INF;
               const float sb = (grp * 32 + 16 + e < nvis) ? __fmul_rn(vb[e], p.cscale) : NEG_INF;
-              va[e] = (sa == NEG_INF) ? 0.f : ex2(__fsub_rn(sa, mx));
-              vb[e] = (sb == NEG_INF) ? 0.f : ex2(__fsub_rn(sb, mx));
+              va[e] = (sa == NEG_INF) ? 0.f : ex2(__fsub_rn(sa, m_new));
+              vb[e] = (sb == NEG_INF) ? 0.f : ex2(__fsub_rn(sb, m_new));
             }
           }
           uint32_t whi[16], wlo[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float x0 = k < 8 ? va[2 * k] : vb[2 * k - 16];
-            const float x1 = k < 8 ? va[2 * k + 1] : vb[2 * k - 15];
+          for (int k2 = 0; k2 < 16; ++k2) {
+            const float x0 = k2 < 8 ? va[2 * k2] : vb[2 * k2 - 16];
+            const float x1 = k2 < 8 ? va[2 * k2 + 1] : vb[2 * k2 - 15];
             __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
             __nv_bfloat162 l2 = __floats2bfloat162_rn(__fsub_rn(x0, __low2float(h2)),
                                                       __fsub_rn(x1, __high2float(h2)));
-            whi[k] = *reinterpret_cast<uint32_t *>(&h2);
-            wlo[k] = *reinterpret_cast<uint32_t *>(&l2);
+            whi[k2] = *reinterpret_cast<uint32_t *>(&h2);
+            wlo[k2] = *reinterpret_cast<uint32_t *>(&l2);
           }
           tmem_st16(srow + grp * 32, whi);
           tmem_st16(srow + grp * 32 + 16, wlo);
@@ -422,15 +476,13 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           for (int off = 8; off >= 1; off >>= 1)
 #pragma unroll
             for (int e = 0; e < off; ++e) va[e] = __fadd_rn(va[e], va[e + off]);
-          if (grp & 1) {
-            const float pair = __fadd_rn(w_even, va[0]);
-            s01 = grp == 1 ? pair : s01;
-            s23 = grp == 3 ? pair : s23;
-          } else {
+          if (grp & 1)
+            half = __fadd_rn(w_even, va[0]);
+          else
             w_even = va[0];
-          }
         }
-        if (tok0 + kTileTokens > x.lim_max) {
+        if (wg == 1) sm->xsum[gi & 1][t] = half;
+        if (wg == 0 && tok0 + kTileTokens > x.lim_max) {
           // The last tile: keys past the loaded range hold stale bytes or the
           // cache's NaN tails; once V has landed, zero those V rows so that
           // 0 * V stays 0 in P.V.
@@ -440,39 +492,53 @@ __global__ void __launch_bounds__(kRowThreads, 1)
 #pragma unroll
             for (int h = 0; h < D / 64; ++h)
 #pragma unroll
-              for (int k = 0; k < 8; ++k)
-                *reinterpret_cast<uint4 *>(vrow + h * C::kHalfBytes + k * 16) = make_uint4(0u, 0u, 0u, 0u);
+              for (int k2 = 0; k2 < 8; ++k2)
+                *reinterpret_cast<uint4 *>(vrow + h * C::kHalfBytes + k2 * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
         }
-        sm->tmax[bb][t] = mx;
-        sm->lsum[bb][t] = __fadd_rn(s01, s23);
-        if (wg_bar_or(bar_id, !ok)) {
+        if (named_bar_or(kDoneBar, 256, !ok)) {
           stop = true;
           break;
+        }
+        const bool last = j == x.n_tiles - 1;
+        if (wg == 0) {
+          l_run = __fmaf_rn(l_run, a, __fadd_rn(half, sm->xsum[gi & 1][t]));
+          if (last) {
+            // the slot of unit uo - 2 has been read by the epilogue (this wait
+            // also keeps ml_full at most one phase ahead of its waiter)
+            ok = mbar_wait(&sm->ml_free[uo & 1], ((uo >> 1) & 1) ^ 1, abort_any, p.wait_ns) && ok;
+            sm->ml[uo & 1][0][t] = m_run;
+            sm->ml[uo & 1][1][t] = l_run;
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->p_full[bb]);
+        if (lane == 0) {
+          mbar_arrive(&sm->p_full[bb]);
+          if (wg == 0 && last) mbar_arrive(&sm->ml_full[uo & 1]);
+        }
       }
       gbase += x.n_tiles;
+      ++uo;
     }
     (void)stop;
   } else {
     // ------------------------------------------------------------------
-    // Correction + epilogue warpgroup: thread t owns row t's running
-    // (m, l, acc[D]).  Per tile, in order: m' = max(m, tmax), a = 2^(m - m'),
-    // b = 2^(tmax - m'), acc = fma(O_hi + O_lo, b, acc * a), l = fma(L, b,
-    // l * a); a tile the row does not reach (tmax = -inf) leaves it untouched.
+    // Epilogue warpgroup: thread t takes row t of each unit once its last
+    // P.V is done: (m, l) from the softmax warpgroups, acc = O_hi + O_lo out
+    // of TMEM (O is then free for the next unit), and the row's out / lse or
+    // split partial -- while the next unit's tiles already run.
     // ------------------------------------------------------------------
     regs_inc<kRowsCorrRegs>();
     const int wq = warp & 3, t = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t orow = tmem + lane_off;
     constexpr uint32_t bar_id = 3;
     float acc[D];
-    int gbase = 0;
+    int gbase = 0, uo = 0;
     bool stop = false;
     for (int k = 0; k < sc.count && !stop; ++k) {
       const Unit x = sc.get<kRowsPerTile>(p, k);
@@ -487,64 +553,44 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         }
         continue;
       }
+      // the unit's (m, l), then its last P.V (one unit_done phase per unit)
+      bool ok = mbar_wait(&sm->ml_full[uo & 1], (uo >> 1) & 1, abort_any, p.wait_ns);
+      const float m_run = sm->ml[uo & 1][0][t];
+      const float l_run = sm->ml[uo & 1][1][t];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm->ml_free[uo & 1]);
+      ok = mbar_wait(&sm->unit_done, uo & 1, abort_any, p.wait_ns) && ok;
+      if (wg_bar_or(bar_id, !ok)) {
+        stop = true;
+        break;
+      }
+      tc_fence_after_sync();
+      // two 16-column chunks of O_hi and O_lo per wait (tcgen05.wait::ld
+      // waits for every load in flight, so loads are batched, not pipelined)
 #pragma unroll
-      for (int c = 0; c < D; ++c) acc[c] = 0.f;
-      float m_run = NEG_INF, l_run = 0.f;
-      for (int j = 0; j < x.n_tiles; ++j) {
-        const int gi = gbase + j, bb = gi % C::kSB, par = (gi / C::kSB) & 1;
-        bool ok = mbar_wait(&sm->p_full[bb], par, abort_any, p.wait_ns);  // the tile's row statistics
-        ok = mbar_wait(&sm->o_full, gi & 1, abort_any, p.wait_ns) && ok;    // its P.V
-        tc_fence_after_sync();
-        __syncwarp();  // the waits above spin per thread; the TMEM loads below are warp-wide
-        const float tm = sm->tmax[bb][t];
-        const float lt = sm->lsum[bb][t];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->stat_free[bb]);
-        if (wg_bar_or(bar_id, !ok)) {
-          stop = true;
-          break;
+      for (int ch = 0; ch < D / 16; ch += 2) {
+        float hi0[16], lo0[16], hi1[16], lo1[16];
+        tmem_ld16(orow + C::kColOhi + ch * 16, hi0);
+        tmem_ld16(orow + C::kColOlo + ch * 16, lo0);
+        tmem_ld16(orow + C::kColOhi + ch * 16 + 16, hi1);
+        tmem_ld16(orow + C::kColOlo + ch * 16 + 16, lo1);
+        tmem_ld_wait_for(hi0);
+        tmem_ld_wait_for(lo0);
+        tmem_ld_wait_for(hi1);
+        tmem_ld_wait_for(lo1);
+        if (ch + 2 == D / 16) {
+          // all of O is in registers: the next unit's P.V may overwrite it
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm->o_free);
         }
-        const bool skip = !(t < x.rows) || tm == NEG_INF;
-        float a = 1.f, b = 0.f;
-        if (!skip) {
-          const float mn = fmaxf(m_run, tm);
-          a = ex2(__fsub_rn(m_run, mn));
-          b = ex2(__fsub_rn(tm, mn));
-          l_run = __fmaf_rn(lt, b, __fmul_rn(l_run, a));
-          m_run = mn;
-        }
-        const uint32_t orow = tmem + lane_off;
-        __syncwarp();
-        // two 16-column chunks of O_hi and O_lo per wait (tcgen05.wait::ld
-        // waits for every load in flight, so loads are batched, not pipelined)
 #pragma unroll
-        for (int ch = 0; ch < D / 16; ch += 2) {
-          float hi0[16], lo0[16], hi1[16], lo1[16];
-          tmem_ld16(orow + C::kColOhi + ch * 16, hi0);
-          tmem_ld16(orow + C::kColOlo + ch * 16, lo0);
-          tmem_ld16(orow + C::kColOhi + ch * 16 + 16, hi1);
-          tmem_ld16(orow + C::kColOlo + ch * 16 + 16, lo1);
-          tmem_ld_wait_for(hi0);
-          tmem_ld_wait_for(lo0);
-          tmem_ld_wait_for(hi1);
-          tmem_ld_wait_for(lo1);
-          if (ch + 2 == D / 16) {
-            // all of O is in registers: the next P.V may overwrite it while
-            // the last chunks are folded in
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm->o_free);
-          }
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {  // branch-free: the loop's TMEM loads are warp-wide
-            const float nv0 = __fmaf_rn(__fadd_rn(hi0[e], lo0[e]), b, __fmul_rn(acc[ch * 16 + e], a));
-            acc[ch * 16 + e] = skip ? acc[ch * 16 + e] : nv0;
-            const float nv1 =
-                __fmaf_rn(__fadd_rn(hi1[e], lo1[e]), b, __fmul_rn(acc[ch * 16 + 16 + e], a));
-            acc[ch * 16 + 16 + e] = skip ? acc[ch * 16 + 16 + e] : nv1;
-          }
+        for (int e = 0; e < 16; ++e) {
+          acc[ch * 16 + e] = __fadd_rn(hi0[e], lo0[e]);
+          acc[ch * 16 + 16 + e] = __fadd_rn(hi1[e], lo1[e]);
         }
       }
+      ++uo;
       if (stop) break;
       if (t < x.rows) {
         // A row whose visible keys all lie in split 0 is finished here, with

@@ -19,27 +19,35 @@
 //   S^T      = K_tile * Q^T on the tensor cores (tcgen05, M = 128 tokens,
 //            N = rows, K = head_dim, fp32 accumulation in TMEM);
 //   softmax  one thread per token: mask (key < row limit), scale to base 2,
-//            the tile's column max over its 128 tokens (exact, order-free),
-//            p = 2^(s - tmax); P^T holds p as two bf16 parts side by side,
+//            the tile's column max tmax over its 128 tokens (exact,
+//            order-free); the row's running max m (-inf at the split's
+//            start) rises to tmax only when tmax > m + kMaxSlack, and then
+//            the row's O^T column takes the factor a = 2^(m - m') in TMEM
+//            (an fp32 multiply) before this tile's P.V adds to it;
+//            p = 2^(s - m); P^T holds p as two bf16 parts side by side,
 //            hi = bf16(p) and lo = bf16(p - hi), so the tensor cores see p to
 //            ~16 bits; the fp32 p of each row are summed in one fixed
-//            shuffle tree (the row sum l never sees P's rounding);
-//   O^T      = V^T * [P_hi | P_lo]^T on the tensor cores (fresh accumulators
-//            each tile), O = O_hi + O_lo in fp32 on the CUDA cores;
-//   update   m' = max(m, tmax), acc = fma(O, 2^(tmax - m'), acc * 2^(m - m')),
-//            l likewise with the tile's row sum; skipped for rows the tile
-//            does not reach.
+//            shuffle tree (the row sum never sees P's rounding), and
+//            l = fma(l, a, sum);
+//   O^T      += V^T * [P_hi | P_lo]^T on the tensor cores: O_hi and O_lo
+//            accumulate in TMEM over the split's tiles (the first tile
+//            starts them afresh), and acc = O_hi + O_lo in fp32 once, at the
+//            split's end.
 // Tiles start at absolute multiples of 128 and rows never influence each
 // other, so a row's arithmetic depends only on its own query, its visible
 // keys and the fixed constants: decode row t and prefill row t, batch 1 and
 // batch N, contiguous and interleaved caches all give the same bits.
 //
-// Roles (224 threads): warps 0-3 softmax + correction + epilogue (thread t =
-// TMEM lane t = token t of the tile = output column d), warp 4 K producer
-// (+ Q staging), warp 5 V producer, warp 6 MMA issuer (+ TMEM owner).  K and V
-// have their own stage rings, so a K stage is refilled as soon as its S^T is
-// computed.  The kernel is persistent: CTA k takes units k, k + gridDim.x,
-// ...; producers and the MMA issuer run ahead across unit boundaries.
+// Roles (480 threads): warps 0-3 / 4-7 softmax warpgroups on alternating
+// tiles (thread t = TMEM lane t = token t of the tile; each passes its
+// tile's running maxima to the other), warps 8-11 correction + epilogue (the
+// rows' l per tile; at a unit's end thread t = output column d), warp 12 K
+// producer (+ Q staging), warp 13 V producer, warp 14 MMA issuer (+ TMEM
+// owner).  K and V have their own stage rings, so a K stage is refilled as
+// soon as its S^T is computed; O^T has a buffer per unit parity, so a unit's
+// read-out overlaps the next unit's tiles.  The kernel is persistent, with
+// its units dealt by a balanced schedule; producers and the MMA issuer run
+// ahead across unit boundaries.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -196,15 +204,18 @@ struct Cfg {
   static constexpr int kSchedScratch = 2 * kPBytes;  // bytes free at kernel start
   struct Small {
     uint64_t full_k[NS], empty_k[NS], full_v[NS], empty_v[NS];
-    uint64_t s_full[2], p_full[2], o_full[2], o_free[2], stat_free[2];
+    uint64_t s_full[2], p_full[2], o_full[2], stat_free[2];
+    uint64_t m_full[2];     // [tile parity]: the tile's running maxima are published
+    uint64_t unit_done[2];  // [O buffer]: a unit's last P.V completed
+    uint64_t o_free[2];     // [O buffer]: the unit's O is read out
     uint64_t q_full[QB], q_empty[QB], drain;
     uint32_t tmem_base;
     int abort_any;
     __align__(16) float wmax[2][2][4][N];  // [softmax warpgroup][tile parity][warp][row]
     __align__(16) float wsum[2][4][N];     // [buffer][warp][row]: per-warp sums of p
-    float tmax[2][N];                      // [buffer][row]: the tile's max (base-2 units)
-    float coef_a[N], coef_b[N];            // correction factors of the current tile
-    int coef_skip[N];
+    float mnew[2][N];                      // [buffer][row]: the running max after the tile
+    float scl[2][N];                       // [buffer][row]: factor O and l take before it
+    float mrun[2][N];                      // [tile parity][row]: mnew for the next tile
     float fin_m[N], fin_l[N];              // each row's (m, l) for the direct final write
     int sched_list[kSchedMaxMine];         // this CTA's units (balanced schedule)
     int sched_meta[kSchedMaxMine][3];      // their sequence length and query range
@@ -214,7 +225,8 @@ struct Cfg {
     int tab[2][2][kSplitTokens / 16];      // [producer][unit parity]: block-table entries
   };
   static constexpr int kSmemBytes = kOffSmall + static_cast<int>(sizeof(Small)) + 1024;
-  // TMEM: S^T (N columns) x 2 buffers, then O^T (hi and lo, 2N columns) x 2 buffers
+  // TMEM: S^T (N columns) x 2 buffers, then O^T (hi and lo, 2N columns) x 2
+  // buffers (alternate units)
   static constexpr int kTmemCols = (6 * N <= 128) ? 128 : (6 * N <= 256) ? 256 : 512;
 };
 
@@ -798,8 +810,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm->s_full[i], 1);
       mbar_init(&sm->p_full[i], 4);   // one arrival per warp of a softmax warpgroup
       mbar_init(&sm->o_full[i], 1);
-      mbar_init(&sm->o_free[i], 4);   // one arrival per correction warp
       mbar_init(&sm->stat_free[i], 4);
+      mbar_init(&sm->m_full[i], 1);
+      mbar_init(&sm->unit_done[i], 1);
+      mbar_init(&sm->o_free[i], 4);   // one arrival per correction warp
     }
     for (int i = 0; i < QB; ++i) {
       mbar_init(&sm->q_full[i], 1);
@@ -840,13 +854,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kIdescQK = idesc_bf16(128, N, 0, 0);           // A = K tile, B = Q (K-major)
       constexpr uint32_t kIdescPV = idesc_bf16(128, C::kPCols, 1, 1);  // A = V^T, B = P^T (MN-major)
       const uint32_t tS = tmem, tO = tmem + 2 * N;
-      // QK^T of tile gi, then P.V of tile gi - 1
-      int gi = 0, ui = 0, prev = -1;
+      // QK^T of tile gi, then P.V of tile gi - 1.  O^T accumulates over a
+      // unit's tiles in the buffer of the unit's parity.
+      struct Pend {
+        int g, first, last, u;
+      };
+      int gi = 0, ui = 0;
+      Pend prev{-1, 0, 0, 0};
       bool failed = false;
-      auto pv_step = [&](int g) -> bool {
-        const int st = g % NS, bb = g & 1;
+      auto pv_step = [&](const Pend &pd) -> bool {
+        const int g = pd.g, st = g % NS, bb = g & 1, ob = pd.u & 1;
         if (!mbar_wait(&sm->p_full[bb], (g >> 1) & 1, abort_any, p.wait_ns)) return false;
-        if (!mbar_wait(&sm->o_free[bb], ((g >> 1) & 1) ^ 1, abort_any, p.wait_ns)) return false;
+        if (pd.first && !mbar_wait(&sm->o_free[ob], ((pd.u >> 1) & 1) ^ 1, abort_any, p.wait_ns))
+          return false;
         if (!mbar_wait(&sm->full_v[st], (g / NS) & 1, abort_any, p.wait_ns)) return false;
         tc_fence_after_sync();
         const uint32_t vaddr = sbase + C::kOffV + st * C::kKVBytes;
@@ -861,9 +881,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           // apart, 8-token groups kPKGroup apart.  O_hi and O_lo side by side.
           const uint64_t b = smem_desc(paddr + kk * 2 * C::kPKGroup, C::kPKGroup, 128,
                                        kLayoutInterleave);
-          umma_bf16(tO + bb * C::kPCols, a, b, kIdescPV, kk > 0 ? 1u : 0u);
+          umma_bf16(tO + ob * C::kPCols, a, b, kIdescPV, (pd.first && kk == 0) ? 0u : 1u);
         }
         umma_commit(&sm->o_full[bb]);
+        if (pd.last) umma_commit(&sm->unit_done[ob]);
         umma_commit(&sm->empty_v[st]);
         return true;
       };
@@ -894,15 +915,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&sm->s_full[bb]);
           umma_commit(&sm->empty_k[st]);
           if (j == x.n_tiles - 1) umma_commit(&sm->q_empty[qb]);
-          if (prev >= 0 && !pv_step(prev)) {
+          if (prev.g >= 0 && !pv_step(prev)) {
             failed = true;
             break;
           }
-          prev = gi;
+          prev = Pend{gi, j == 0 ? 1 : 0, j == x.n_tiles - 1 ? 1 : 0, ui};
         }
         ++ui;
       }
-      if (!failed && prev >= 0) failed = !pv_step(prev);
+      if (!failed && prev.g >= 0) failed = !pv_step(prev);
       // every MMA this thread issued completes before TMEM is released, also
       // when the consumers gave up (bounded wait, default limit)
       (void)failed;
@@ -914,18 +935,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------
     // Softmax warpgroups: warpgroup wg takes the tiles with gi % 2 == wg.
     // Thread t <-> TMEM lane t <-> token t of the tile.  Per tile and row:
-    // tmax = exact max of the masked scores, p = 2^(s - tmax) written as
-    // P^T = [bf16(p) | bf16(p - bf16(p))], per-warp sums of the fp32 p.
+    // tmax = exact max of the masked scores; the running max m (the
+    // previous tile's, published by the other warpgroup; -inf at a unit's
+    // start) rises to tmax only when tmax > m + kMaxSlack, and then the
+    // row's column of O^T (hi and lo) takes the factor a = 2^(m - m') before
+    // this tile's P.V adds to it; p = 2^(s - m) written as P^T = [bf16(p) |
+    // bf16(p - bf16(p))]; per-warp sums of the fp32 p.
     // ------------------------------------------------------------------
     const int wg = warp >> 2, wq = warp & 3, t = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t bar_id = 1 + wg;
     const float NEG_INF = neg_inf();
-    int gbase = 0;
+    int gbase = 0, uo = 0;  // uo: ordinal of the unit among this CTA's units with work
     bool stop = false;
     for (int k = 0; k < sc.count && !stop; ++k) {
       const Unit x = sc.get<N>(p, k);
       if (x.n_tiles == 0) continue;
+      const uint32_t ocol = tmem + lane_off + 2 * N + (uo & 1) * C::kPCols;  // this unit's O^T
       if (t < N) {
         int lim = 0;
         if (t < x.rows) {
@@ -989,6 +1015,58 @@ __global__ void __launch_bounds__(kThreads, 1)
           stop = true;
           break;
         }
+        // the running maxima: the previous tile's (its phase is awaited for
+        // every tile, so the parity waits stay in step), this tile's
+        if (gi > 0)
+          ok = mbar_wait(&sm->m_full[(gi - 1) & 1], ((gi - 1) >> 1) & 1, abort_any, p.wait_ns) && ok;
+        if (t < N) {
+          float m_new = NEG_INF, a = 1.f;
+          if (t < x.rows) {
+            const float tmax = fmaxf(fmaxf(wmax[0][t], wmax[1][t]), fmaxf(wmax[2][t], wmax[3][t]));
+            const float m_prev = j > 0 ? sm->mrun[(gi - 1) & 1][t] : NEG_INF;
+            m_new = (tmax > __fadd_rn(m_prev, kMaxSlack)) ? tmax : m_prev;
+            a = (m_prev == NEG_INF || m_new == m_prev) ? 1.f : ex2(__fsub_rn(m_prev, m_new));
+          }
+          sm->mnew[bb][t] = m_new;
+          sm->scl[bb][t] = a;
+          sm->mrun[gi & 1][t] = m_new;
+        }
+        if (wg_bar_or(bar_id, !ok)) {
+          stop = true;
+          break;
+        }
+        if (t == 0) mbar_arrive(&sm->m_full[gi & 1]);
+        bool resc = false;
+        for (int c = 0; c < x.rows; ++c) resc = resc || sm->scl[bb][c] != 1.f;
+        if (resc) {
+          // O^T holds the unit's tiles < gi once P.V(gi - 1) is done (o_full
+          // of its parity; that barrier's previous phase, tile gi - 3, is done,
+          // since this warpgroup waited for tile gi - 2's P.V above)
+          ok = mbar_wait(&sm->o_full[(gi - 1) & 1], ((gi - 1) >> 1) & 1, abort_any, p.wait_ns) && ok;
+          if (__all_sync(0xffffffffu, ok)) {
+            tc_fence_after_sync();
+#pragma unroll
+            for (int ch = 0; ch < N / 16; ++ch) {
+              if (ch * 16 < x.rows) {  // warp-uniform
+                float hi[16], lo[16];
+                tmem_ld16(ocol + ch * 16, hi);
+                tmem_ld16(ocol + N + ch * 16, lo);
+                tmem_ld_wait_for(hi);
+                tmem_ld_wait_for(lo);
+                uint32_t wh[16], wl[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  const float a = sm->scl[bb][ch * 16 + e];
+                  wh[e] = __float_as_uint(__fmul_rn(hi[e], a));
+                  wl[e] = __float_as_uint(__fmul_rn(lo[e], a));
+                }
+                tmem_st16(ocol + ch * 16, wh);
+                tmem_st16(ocol + N + ch * 16, wl);
+              }
+            }
+            tmem_st_wait();
+          }
+        }
         // P^T row t (MN-major, no swizzle: one 16-byte chunk per 8 columns).
         uint8_t *prow = smem + C::kOffP + bb * C::kPBytes + (t >> 3) * C::kPKGroup + (t & 7) * 16;
 #pragma unroll
@@ -998,9 +1076,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int c0 = grp * 8 + 2 * e;
-              const float m0 = fmaxf(fmaxf(wmax[0][c0], wmax[1][c0]), fmaxf(wmax[2][c0], wmax[3][c0]));
-              const float m1 = fmaxf(fmaxf(wmax[0][c0 + 1], wmax[1][c0 + 1]),
-                                     fmaxf(wmax[2][c0 + 1], wmax[3][c0 + 1]));
+              const float m0 = sm->mnew[bb][c0];
+              const float m1 = sm->mnew[bb][c0 + 1];
               const float p0 = (sv[c0] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0], m0));
               const float p1 = (sv[c0 + 1] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0 + 1], m1));
               sv[c0] = p0;
@@ -1025,23 +1102,22 @@ __global__ void __launch_bounds__(kThreads, 1)
               *reinterpret_cast<float4 *>(&sm->wsum[bb][wq][4 * q4]) = make_float4(v[0], v[1], v[2], v[3]);
           }
         }
-        if (t < x.rows)
-          sm->tmax[bb][t] = fmaxf(fmaxf(wmax[0][t], wmax[1][t]), fmaxf(wmax[2][t], wmax[3][t]));
         fence_proxy_async_smem();
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->p_full[bb]);
       }
       gbase += x.n_tiles;
+      ++uo;
     }
     (void)stop;
   } else if (warp < kCorrWarp0 + 4) {
     // ------------------------------------------------------------------
-    // Correction + epilogue warpgroup: thread t <-> TMEM lane t <-> output
-    // column d of O^T; thread r (< rows) owns row r's running (m, l).
-    // Per tile, in order: m' = max(m, tmax), a = 2^(m - m'), b = 2^(tmax - m'),
-    // acc = fma(O_hi + O_lo, b, acc * a), l = fma(sum p, b, l * a); a tile a
-    // row does not reach (tmax = -inf) leaves the row untouched.
+    // Correction + epilogue warpgroup: thread r (< rows) owns row r's
+    // running l; per tile, in order, l = fma(l, a, sum p) with the factor a
+    // the softmax chose (1 unless the row's max rose).  At the unit's end,
+    // once its last P.V is done, thread t <-> TMEM lane t <-> column d of
+    // O^T: acc = O_hi + O_lo, then the partials or the final rows.
     // ------------------------------------------------------------------
     const int wq = warp & 3, t = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -1073,25 +1149,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       l_run = 0.f;
       for (int j = 0; j < x.n_tiles; ++j) {
         const int gi = gbase + j, bb = gi & 1, par = (gi >> 1) & 1;
-        bool ok = mbar_wait(&sm->p_full[bb], par, abort_any, p.wait_ns);  // the tile's row statistics
-        ok = mbar_wait(&sm->o_full[bb], par, abort_any, p.wait_ns) && ok;  // its P.V
-        tc_fence_after_sync();
+        const bool ok = mbar_wait(&sm->p_full[bb], par, abort_any, p.wait_ns);  // the tile's row statistics
         if (t < x.rows) {
-          const float tm = sm->tmax[bb][t];
-          const int skip = (tm == NEG_INF) ? 1 : 0;
-          float a = 1.f, b = 0.f;
-          if (!skip) {
-            const float mn = fmaxf(m_run, tm);
-            a = ex2(__fsub_rn(m_run, mn));
-            b = ex2(__fsub_rn(tm, mn));
-            const float lt = __fadd_rn(__fadd_rn(sm->wsum[bb][0][t], sm->wsum[bb][1][t]),
-                                       __fadd_rn(sm->wsum[bb][2][t], sm->wsum[bb][3][t]));
-            l_run = __fmaf_rn(lt, b, __fmul_rn(l_run, a));
-            m_run = mn;
-          }
-          sm->coef_a[t] = a;
-          sm->coef_b[t] = b;
-          sm->coef_skip[t] = skip;
+          const float lt = __fadd_rn(__fadd_rn(sm->wsum[bb][0][t], sm->wsum[bb][1][t]),
+                                     __fadd_rn(sm->wsum[bb][2][t], sm->wsum[bb][3][t]));
+          l_run = __fmaf_rn(l_run, sm->scl[bb][t], lt);
+          m_run = sm->mnew[bb][t];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->stat_free[bb]);  // the tile's statistics are read
@@ -1099,28 +1162,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           stop = true;
           break;
         }
+      }
+      if (stop) break;
+      {
+        // the unit's last P.V, then O^T out of TMEM (one unit_done phase per
+        // unit of this buffer's parity)
+        const int ob = cui & 1;
+        const bool ok = mbar_wait(&sm->unit_done[ob], (cui >> 1) & 1, abort_any, p.wait_ns);
+        if (wg_bar_or(bar_id, !ok)) {
+          stop = true;
+          break;
+        }
+        tc_fence_after_sync();
 #pragma unroll
         for (int ch = 0; ch < N / 16; ++ch) {
           if (ch * 16 < x.rows) {  // warp-uniform
             float hi[16], lo[16];
-            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + ch * 16, hi);
-            tmem_ld16(tmem + lane_off + 2 * N + bb * C::kPCols + N + ch * 16, lo);
+            tmem_ld16(tmem + lane_off + 2 * N + ob * C::kPCols + ch * 16, hi);
+            tmem_ld16(tmem + lane_off + 2 * N + ob * C::kPCols + N + ch * 16, lo);
             tmem_ld_wait_for(hi);
             tmem_ld_wait_for(lo);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int c = ch * 16 + e;
-              if (c < x.rows && !sm->coef_skip[c])
-                acc[c] = __fmaf_rn(__fadd_rn(hi[e], lo[e]), sm->coef_b[c],
-                                   __fmul_rn(acc[c], sm->coef_a[c]));
-            }
+            for (int e = 0; e < 16; ++e) acc[ch * 16 + e] = __fadd_rn(hi[e], lo[e]);
           }
         }
         tc_fence_before_sync();
-        // coef_* are rewritten for the next tile only after this barrier
-        wg_bar_or(bar_id, false);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->o_free[bb]);
+        if (lane == 0) mbar_arrive(&sm->o_free[ob]);
       }
       if (stop) break;
       if (p.direct) {

@@ -13,6 +13,12 @@ namespace pkv {
 constexpr int kSplitTokens = 4096;
 constexpr int kTileTokens = 128;
 
+// Within a split, a row's running max m (base-2 units) rises to a tile's max
+// only when that exceeds it by more than kMaxSlack; p = 2^(s - m) then stays
+// below 2^kMaxSlack, and the P.V products, accumulated on the tensor cores
+// over the split's tiles, are rescaled (by 2^(m - m'), in place) only then.
+constexpr float kMaxSlack = 8.f;
+
 // Number of splits that hold keys [0, n): ceil(n / kSplitTokens), 0 for n <= 0.
 __host__ __device__ constexpr int splits_for(int n) {
   return n > 0 ? (n + kSplitTokens - 1) / kSplitTokens : 0;
