@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     // memory); the running max m rises to tmax only when tmax > m + kMaxSlack
     // (a unit starts from -inf), and then O (warpgroup 0: O_hi, 1: O_lo) and
     // l take the factor a = 2^(m - m') before this tile's P.V adds to O;
-    // p = 2^(s - m), P = [bf16(p) | bf16(p - bf16(p))] over S in TMEM; the
+    // p = 2^(raw * scale - m), P = [bf16(p) | bf16(p - bf16(p))] over S in TMEM; the
     // row's sum of the fp32 p in the contract's fixed tree (each warpgroup's
     // two 32-key sums, then the halves), l = fma(l, a, sum).  Both
     // warpgroups keep m in registers, warpgroup 0 keeps l and publishes the
@@ -353,9 +353,9 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         const int tok0 = x.tok0 + j * kTileTokens;
         const int nvis = min(max(nlim - tok0, 0), kTileTokens);
         const uint32_t srow = tmem + lane_off + bb * 128;  // S of this tile, then its P
-        // pass 1: this half's max.  Scaling by cscale > 0 rounds
-        // monotonically, so on fully visible keys max(s) * cscale is the max
-        // of the scaled scores exactly.  The branch is taken per WARP
+        // pass 1: this half's max over the visible keys, scaled once:
+        // scaling by cscale > 0 rounds monotonically, so max(s) * cscale is
+        // the max of the scaled scores exactly.  The branch is taken per WARP
         // (tcgen05.ld is .sync.aligned: all 32 lanes issue the same load).
         __syncwarp();
         const bool full = __all_sync(0xffffffffu, nvis == kTileTokens);  // warp-uniform
@@ -374,6 +374,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           }
           hm = __fmul_rn(raw, p.cscale);
         } else {
+          float raw = NEG_INF;
 #pragma unroll 1
           for (int ch = 4 * wg; ch < 4 * wg + 4; ch += 2) {
             float v0[16], v1[16];
@@ -383,11 +384,12 @@ __global__ void __launch_bounds__(kRowThreads, 1)
             tmem_ld_wait_for(v1);
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float s0 = (ch * 16 + e < nvis) ? __fmul_rn(v0[e], p.cscale) : NEG_INF;
-              const float s1 = (ch * 16 + 16 + e < nvis) ? __fmul_rn(v1[e], p.cscale) : NEG_INF;
-              hm = fmaxf(hm, fmaxf(s0, s1));
+              const float s0 = (ch * 16 + e < nvis) ? v0[e] : NEG_INF;
+              const float s1 = (ch * 16 + 16 + e < nvis) ? v1[e] : NEG_INF;
+              raw = fmaxf(raw, fmaxf(s0, s1));
             }
           }
+          hm = __fmul_rn(raw, p.cscale);
         }
         sm->xmax[gi & 1][wg][t] = hm;
         // both halves' maxima are published (and a failed wait is known to
@@ -439,21 +441,19 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           tmem_ld16(srow + grp * 32 + 16, vb);
           tmem_ld_wait_for(va);
           tmem_ld_wait_for(vb);
+          // p = 2^(raw * cscale - m), one rounding before ex2; masked keys 0
+          const float nm = -m_new;
           if (full) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float sa = __fmul_rn(va[e], p.cscale);
-              const float sb = __fmul_rn(vb[e], p.cscale);
-              va[e] = (sa == NEG_INF) ? 0.f : ex2(__fsub_rn(sa, m_new));
-              vb[e] = (sb == NEG_INF) ? 0.f : ex2(__fsub_rn(sb, m_new));
+              va[e] = ex2(__fmaf_rn(va[e], p.cscale, nm));
+              vb[e] = ex2(__fmaf_rn(vb[e], p.cscale, nm));
             }
           } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float sa = (grp * 32 + e < nvis) ? __fmul_rn(va[e], p.cscale) : NEG_INF;
-              const float sb = (grp * 32 + 16 + e < nvis) ? __fmul_rn(vb[e], p.cscale) : NEG_INF;
-              va[e] = (sa == NEG_INF) ? 0.f : ex2(__fsub_rn(sa, m_new));
-              vb[e] = (sb == NEG_INF) ? 0.f : ex2(__fsub_rn(sb, m_new));
+              va[e] = (grp * 32 + e < nvis) ? ex2(__fmaf_rn(va[e], p.cscale, nm)) : 0.f;
+              vb[e] = (grp * 32 + 16 + e < nvis) ? ex2(__fmaf_rn(vb[e], p.cscale, nm)) : 0.f;
             }
           }
           uint32_t whi[16], wlo[16];

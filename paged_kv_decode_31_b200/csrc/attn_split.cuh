@@ -24,7 +24,8 @@
 //            start) rises to tmax only when tmax > m + kMaxSlack, and then
 //            the row's O^T column takes the factor a = 2^(m - m') in TMEM
 //            (an fp32 multiply) before this tile's P.V adds to it;
-//            p = 2^(s - m); P^T holds p as two bf16 parts side by side,
+//            p = 2^(raw * scale - m) (one fused multiply-add); P^T holds p
+//            as two bf16 parts side by side,
 //            hi = bf16(p) and lo = bf16(p - hi), so the tensor cores see p to
 //            ~16 bits; the fp32 p of each row are summed in one fixed
 //            shuffle tree (the row sum never sees P's rounding), and
@@ -939,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // previous tile's, published by the other warpgroup; -inf at a unit's
     // start) rises to tmax only when tmax > m + kMaxSlack, and then the
     // row's column of O^T (hi and lo) takes the factor a = 2^(m - m') before
-    // this tile's P.V adds to it; p = 2^(s - m) written as P^T = [bf16(p) |
+    // this tile's P.V adds to it; p = 2^(raw * scale - m) written as P^T = [bf16(p) |
     // bf16(p - bf16(p))]; per-warp sums of the fp32 p.
     // ------------------------------------------------------------------
     const int wg = warp >> 2, wq = warp & 3, t = threadIdx.x & 127;
@@ -984,9 +985,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         const int tok0 = x.tok0 + j * kTileTokens;
         const int tok = tok0 + t;
+        // raw scores of the visible keys (masked: -inf); the row's max over
+        // them is scaled once (cscale > 0 rounds monotonically, so that is
+        // the max of the scaled scores exactly), p = 2^(raw * cscale - m)
 #pragma unroll
-        for (int c = 0; c < N; ++c)
-          sv[c] = (c < x.rows && tok < sm->lim[wg][c]) ? __fmul_rn(sv[c], p.cscale) : NEG_INF;
+        for (int c = 0; c < N; ++c) sv[c] = (c < x.rows && tok < sm->lim[wg][c]) ? sv[c] : NEG_INF;
         if (tok0 + kTileTokens > x.lim_max) {
           // The last tile: keys past the loaded range hold stale bytes or the
           // cache's NaN tails; once V has landed, zero those V rows so that
@@ -1022,7 +1025,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t < N) {
           float m_new = NEG_INF, a = 1.f;
           if (t < x.rows) {
-            const float tmax = fmaxf(fmaxf(wmax[0][t], wmax[1][t]), fmaxf(wmax[2][t], wmax[3][t]));
+            const float tmax = __fmul_rn(
+                fmaxf(fmaxf(wmax[0][t], wmax[1][t]), fmaxf(wmax[2][t], wmax[3][t])), p.cscale);
             const float m_prev = j > 0 ? sm->mrun[(gi - 1) & 1][t] : NEG_INF;
             m_new = (tmax > __fadd_rn(m_prev, kMaxSlack)) ? tmax : m_prev;
             a = (m_prev == NEG_INF || m_new == m_prev) ? 1.f : ex2(__fsub_rn(m_prev, m_new));
@@ -1078,8 +1082,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int c0 = grp * 8 + 2 * e;
               const float m0 = sm->mnew[bb][c0];
               const float m1 = sm->mnew[bb][c0 + 1];
-              const float p0 = (sv[c0] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0], m0));
-              const float p1 = (sv[c0 + 1] == NEG_INF) ? 0.f : ex2(__fsub_rn(sv[c0 + 1], m1));
+              const float p0 = (sv[c0] == NEG_INF) ? 0.f : ex2(__fmaf_rn(sv[c0], p.cscale, -m0));
+              const float p1 =
+                  (sv[c0 + 1] == NEG_INF) ? 0.f : ex2(__fmaf_rn(sv[c0 + 1], p.cscale, -m1));
               sv[c0] = p0;
               sv[c0 + 1] = p1;
               __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
