@@ -345,6 +345,10 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         nlim = lim > 0 ? lim : 0;
       }
       float m_run = NEG_INF, l_run = 0.f;
+      // warpgroup 0 folds a tile's row sum into l one tile late (it needs
+      // warpgroup 1's half, published before the next exchange): the factor
+      // and its own half of the tile before
+      float a_prev = 1.f, half_prev = 0.f;
       for (int j = 0; j < x.n_tiles; ++j) {
         const int gi = gbase + j;
         const int bb = gi % C::kSB, st = gi % NS, par = (gi / C::kSB) & 1;
@@ -398,6 +402,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           stop = true;
           break;
         }
+        if (wg == 0 && j > 0)
+          l_run = __fmaf_rn(l_run, a_prev, __fadd_rn(half_prev, sm->xsum[(gi - 1) & 1][t]));
         const float mx = fmaxf(hm, sm->xmax[gi & 1][wg ^ 1][t]);
         const float m_prev = m_run;
         const float m_new = (mx > __fadd_rn(m_prev, kMaxSlack)) ? mx : m_prev;
@@ -482,7 +488,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
             w_even = va[0];
         }
         if (wg == 1) sm->xsum[gi & 1][t] = half;
-        if (wg == 0 && tok0 + kTileTokens > x.lim_max) {
+        const bool last = j == x.n_tiles - 1;
+        if (wg == 0 && tok0 + kTileTokens > x.lim_max) {  // (only a unit's last tile)
           // The last tile: keys past the loaded range hold stale bytes or the
           // cache's NaN tails; once V has landed, zero those V rows so that
           // 0 * V stays 0 in P.V.
@@ -496,20 +503,24 @@ __global__ void __launch_bounds__(kRowThreads, 1)
                 *reinterpret_cast<uint4 *>(vrow + h * C::kHalfBytes + k2 * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
         }
-        if (named_bar_or(kDoneBar, 256, !ok)) {
-          stop = true;
-          break;
-        }
-        const bool last = j == x.n_tiles - 1;
-        if (wg == 0) {
-          l_run = __fmaf_rn(l_run, a, __fadd_rn(half, sm->xsum[gi & 1][t]));
-          if (last) {
+        if (last) {
+          // the unit's last tile: both halves' sums and any failed wait are
+          // known to both warpgroups
+          if (named_bar_or(kDoneBar, 256, !ok)) {
+            stop = true;
+            break;
+          }
+          if (wg == 0) {
+            l_run = __fmaf_rn(l_run, a, __fadd_rn(half, sm->xsum[gi & 1][t]));
             // the slot of unit uo - 2 has been read by the epilogue (this wait
             // also keeps ml_full at most one phase ahead of its waiter)
             ok = mbar_wait(&sm->ml_free[uo & 1], ((uo >> 1) & 1) ^ 1, abort_any, p.wait_ns) && ok;
             sm->ml[uo & 1][0][t] = m_run;
             sm->ml[uo & 1][1][t] = l_run;
           }
+        } else {
+          a_prev = a;
+          half_prev = half;
         }
         fence_proxy_async_smem();
         __syncwarp();
