@@ -208,3 +208,73 @@ def test_context_longer_than_max_seqlen_k_sets_the_error_flag(sq):
                                max_seqlen_k=5000, scale=di.scale, causal=True, err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == pkv.binding.DEVERR_SEQ_LEN
+
+
+def _growing_keys(di, growth):
+    """Scale every cached key at position pos by 1 + growth * (pos // 128), so
+    that each 128-token tile's scores are larger than the last tile's."""
+    k = di.cache.k
+    bs = di.cache.block_size
+    for b, n in enumerate(di.seqlens.tolist()):
+        pos = torch.arange(n)
+        blk = di.block_table[b, pos // bs].long()
+        f = (1.0 + growth * (pos // 128).float()).to(torch.bfloat16)
+        k[blk, pos % bs] = (k[blk, pos % bs].float() * f[:, None, None].float()).to(torch.bfloat16)
+
+
+def _max_rises(di):
+    """How often, over every (sequence, query row, query head), a tile's max
+    score (base 2) exceeds the split's running max by more than 8 after the
+    split's first tile -- the case where the accumulators are rescaled in
+    place (the running max follows the kernels' rule: it rises to a tile's
+    max only past that slack)."""
+    import math
+    G = di.Hq // di.Hkv
+    rises = 0
+    for b, n in enumerate(di.seqlens.tolist()):
+        pos = torch.arange(n)
+        blk = di.block_table[b, pos // di.cache.block_size].long()
+        kk = di.cache.k[blk, pos % di.cache.block_size].double()        # [n, Hkv, D]
+        q = di.q[b].double()                                             # [sq, Hq, D]
+        s = torch.einsum("qhd,nhd->qhn", q, kk.repeat_interleave(G, dim=1)) * di.scale / math.log(2)
+        sq = q.shape[0]
+        for i in range(sq):
+            lim = n - sq + i + 1 if di.causal else n
+            m = torch.full((di.Hq,), float("-inf"), dtype=torch.float64)
+            for t0 in range(0, lim, 128):
+                if t0 % 4096 == 0:
+                    m.fill_(float("-inf"))
+                tm = s[i, :, t0:min(lim, t0 + 128)].max(dim=1).values
+                rises += int(((m > float("-inf")) & (tm > m + 8)).sum())
+                m = torch.where(tm > m + 8, tm, m)
+    return rises
+
+
+@pytest.mark.parametrize("sq,causal,n", [(1, False, 2200), (3, True, 2200), (150, True, 2200),
+                                          (1, False, 9000), (150, True, 9000)])
+def test_rising_maxima_rescale_in_place_and_match_oracle(sq, causal, n):
+    """Keys that grow tile by tile: a row's max rises past the 2^8 slack at
+    almost every tile, so the accumulators are rescaled in TMEM between tiles
+    (transposed kernel at seqlen_q 1 and 3, row-major kernel at 150 x G 4 rows;
+    9000-token contexts: three splits, the running max restarting at each,
+    and the merge).  Against the oracle; the decode row equals the causal
+    prefill's last row.  The softmax here is nearly one-hot, so out is close
+    to a single V row and can exceed 4 in magnitude, where bf16's own rounding
+    of the exact result reaches 2^-6 = 1.6e-2: out is held to 1e-2 plus half
+    a bf16 unit in the last place of the oracle's value (2^-8 |ref|)."""
+    di = I.p2_case(2, sq, n, 16, 4, 128, 16, causal=causal, layout="interleaved", seed=71,
+                   seqlens=[n, (n * 3) // 5])
+    _growing_keys(di, 2.5)
+    assert _max_rises(di) > 0
+    out, lse = run_gpu(di, entry=pkv.paged_prefill_attn)
+    ref_out, ref_lse = oracle_of(di)
+    assert torch.isfinite(ref_lse).all() and torch.isfinite(lse).all()
+    err = (out.double() - ref_out).abs()
+    assert (err <= 1e-2 + ref_out.abs() * 2.0 ** -8).all(), f"out max-abs error {err.max():.3e}"
+    assert (lse.double() - ref_lse).abs().max() <= 1e-3
+    if causal:
+        last = I.DecodeInputs(di.q[:, -1:].contiguous(), di.cache, di.block_table, di.seqlens,
+                              di.Hq, di.Hkv, di.D, di.scale, True)
+        o1, l1 = run_gpu(last, entry=pkv.paged_decode_attn)
+        from gpu_helpers import bits_equal
+        assert bits_equal(o1, out[:, -1:].contiguous()) and bits_equal(l1, lse[:, :, -1:].contiguous())
