@@ -250,19 +250,22 @@ def _max_rises(di):
     return rises
 
 
-@pytest.mark.parametrize("sq,causal,n", [(1, False, 2200), (3, True, 2200), (150, True, 2200),
-                                          (1, False, 9000), (150, True, 9000)])
-def test_rising_maxima_rescale_in_place_and_match_oracle(sq, causal, n):
+@pytest.mark.parametrize("sq,causal,n,d", [(1, False, 2200, 128), (3, True, 2200, 128),
+                                            (16, True, 2200, 128), (150, True, 2200, 128),
+                                            (1, False, 9000, 128), (150, True, 9000, 128),
+                                            (3, True, 2200, 64), (150, True, 2200, 64)])
+def test_rising_maxima_rescale_in_place_and_match_oracle(sq, causal, n, d):
     """Keys that grow tile by tile: a row's max rises past the 2^8 slack at
     almost every tile, so the accumulators are rescaled in TMEM between tiles
-    (transposed kernel at seqlen_q 1 and 3, row-major kernel at 150 x G 4 rows;
-    9000-token contexts: three splits, the running max restarting at each,
-    and the merge).  Against the oracle; the decode row equals the causal
+    (transposed kernel at seqlen_q 1, 3 and 16 -- 64 rows per KV head --,
+    row-major kernel at 150 x G 4 rows; head_dim 64 and 128; 9000-token
+    contexts: three splits, the running max restarting at each, and the
+    merge).  Against the oracle; the decode row equals the causal
     prefill's last row.  The softmax here is nearly one-hot, so out is close
     to a single V row and can exceed 4 in magnitude, where bf16's own rounding
     of the exact result reaches 2^-6 = 1.6e-2: out is held to 1e-2 plus half
     a bf16 unit in the last place of the oracle's value (2^-8 |ref|)."""
-    di = I.p2_case(2, sq, n, 16, 4, 128, 16, causal=causal, layout="interleaved", seed=71,
+    di = I.p2_case(2, sq, n, 16, 4, d, 16, causal=causal, layout="interleaved", seed=71,
                    seqlens=[n, (n * 3) // 5])
     _growing_keys(di, 2.5)
     assert _max_rises(di) > 0
