@@ -368,7 +368,10 @@ def decode_workload_secondary(dev, name: str, reps: int = 200, warmup: int = 20)
     U[1, 32768], Hq 16 / Hkv 4, D 128, block_size 256, interleaved, NaN tails
     and spare blocks).  One paged_decode_attn call per step, 20 warm-up and
     200 timed steps with CUDA events per call; K/V bytes per call /
-    device time (mean, median, best).  Inputs are larger than L2."""
+    device time (mean, median, best); then 200 more steps back to back
+    between one event pair (`gbs_loop`, the steady-state rate the headline
+    `value` measures, without the per-call events in the stream).  Inputs are
+    larger than L2."""
     import paged_kv_decode_31_b200 as pkv
     from paged_kv_decode_31_b200 import inputs as I
     # drawn on the host (the generators are CPU ones), then moved
@@ -398,12 +401,22 @@ def decode_workload_secondary(dev, name: str, reps: int = 200, warmup: int = 20)
     if int(err.item()) != 0:
         raise RuntimeError(f"device error bits {int(err.item())}")
     t = sorted(a.elapsed_time(b) for a, b in ev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(err.item())}")
+    loop = e0.elapsed_time(e1) / reps
     kv = di.kv_bytes()
     mean = sum(t) / len(t)
     return {"workload": name, "kv_bytes": kv, "ms_mean": round(mean, 5),
             "ms_median": round(t[len(t) // 2], 5), "ms_best": round(t[0], 5),
             "gbs_mean": round(kv / (mean / 1e3) / 1e9, 2),
-            "gbs_best": round(kv / (t[0] / 1e3) / 1e9, 2)}
+            "gbs_best": round(kv / (t[0] / 1e3) / 1e9, 2),
+            "ms_loop": round(loop, 5), "gbs_loop": round(kv / (loop / 1e3) / 1e9, 2)}
 
 
 def packed_layout(tensors):
@@ -656,7 +669,8 @@ def run_ours(args):
 
         def decode_obj(name):
             dw = decode_workload_secondary(dev, name)
-            dw["hbm_frac"] = round(dw["gbs_mean"] / peak, 4)
+            dw["hbm_frac"] = round(dw["gbs_loop"] / peak, 4)
+            dw["hbm_frac_basis"] = "gbs_loop"
             return dw
 
         secondary = [("prefill", prefill_obj), ("varlen", varlen_obj), ("backward", backward_obj),
