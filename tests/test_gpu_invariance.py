@@ -175,3 +175,37 @@ def test_kv_append_out_of_table_sets_error_flag():
     pkv.kv_append(kn, kn, di.cache.k, di.cache.v, narrow, di.seqlens, err=err)
     torch.cuda.synchronize()
     assert int(err.item()) & pkv.binding.DEVERR_TABLE_WIDTH
+
+
+def test_short_units_stay_in_step_under_repetition():
+    """Several units per CTA, many of them one or two tiles long (causal
+    512-token chunks: 512 units of 1-16 tiles per call, so the epilogue of
+    one unit overlaps the next units' tiles): repeated chunked prefill equals
+    the full prefill bit for bit, every wait completes (no timeout bit) and
+    every out / lse element is written (NaN-filled first).  A hand-off
+    between the softmax and epilogue warpgroups that could run two units
+    ahead showed up here as a timeout and unwritten rows."""
+    cache, table, q_all, k_all, v_all = I.config_parity_cache(device="cuda")
+    B, Hq, n, c = 8, 16, 2048, 512
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    seq = lambda v: torch.full((B,), v, dtype=torch.int32, device="cuda")
+    pkv.kv_append(k_all[:, :n], v_all[:, :n], cache.k, cache.v, table, seq(0), err=err)
+
+    def attn(q, ctx):
+        out = torch.full_like(q, float("nan"))
+        lse = torch.full((B, Hq, q.shape[1]), float("nan"), dtype=torch.float32, device="cuda")
+        return pkv.paged_prefill_attn(q, cache.k, cache.v, table, seq(ctx), max_seqlen_k=ctx,
+                                      causal=True, out=out, lse=lse, err=err)
+
+    full_o, full_l = attn(q_all[:, :n], n)
+    for rep in range(6):
+        outs, lses = [], []
+        for s in range(0, n, c):
+            o, l = attn(q_all[:, s:s + c], s + c)
+            outs.append(o)
+            lses.append(l)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0, f"repetition {rep}: device error bits {int(err.item())}"
+        co, cl = torch.cat(outs, 1), torch.cat(lses, 2)
+        assert not torch.isnan(co.float()).any() and not torch.isnan(cl).any()
+        assert bits_equal(co.cpu(), full_o.cpu()) and bits_equal(cl.cpu(), full_l.cpu())
