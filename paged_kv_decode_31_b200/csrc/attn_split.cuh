@@ -456,6 +456,24 @@ __device__ __forceinline__ void build_schedule(const AttnParams &p, uint8_t *scr
   if (tid < 32) {
     const int lane = tid;
     for (int base = 0; base < p.n_units; base += 32) {
+      if constexpr (N >= 128) {
+        // (row-major tiles: a call may have far more unit slots than units
+        // with work) skip a run of 128 slots none of which is kept, four
+        // unit bytes per lane
+        if ((base & 127) == 0) {
+          const int w0 = base + 4 * lane;
+          bool any = false;
+          if (w0 + 3 < p.n_units) {
+            any = *reinterpret_cast<const uint32_t *>(scratch + w0) != 0xFFFFFFFFu;
+          } else {
+            for (int k = 0; k < 4; ++k) any = any || (w0 + k < p.n_units && scratch[w0 + k] != kSkip);
+          }
+          if (__ballot_sync(0xffffffffu, any) == 0u) {
+            base += 96;  // with the loop's 32: the next run of 128
+            continue;
+          }
+        }
+      }
       const int u = base + lane;
       const int nt = (u < p.n_units && scratch[u] != kSkip) ? scratch[u] : -1;
       const unsigned same = __match_any_sync(0xffffffffu, nt);
