@@ -104,15 +104,11 @@ __device__ __forceinline__ float final_lse(float M, float L) {
 //                 head_dim elements [l V, l V + V), V = D / 32 (many rows);
 //   WIDE = true:  one block of D threads per row, V = 1 (few rows, many
 //                 splits: more SMs share the partial reads).
+// One output row (row = token * Hq + h; token = b * seqlen_q + i, or packed)
+// by one block (WIDE) or one warp; `lane` is the thread's index in it.
 template <int D, bool WIDE>
-__global__ void __launch_bounds__(WIDE ? D : 32 * kMergeRowsPerBlock)
-    merge_kernel(const __grid_constant__ MergeParams p) {
+__device__ __forceinline__ void merge_row(const MergeParams &p, int64_t row, int lane) {
   constexpr int V = WIDE ? 1 : D / 32;
-  const int warp = WIDE ? 0 : threadIdx.x >> 5;
-  const int lane = WIDE ? threadIdx.x : threadIdx.x & 31;
-  const int64_t row = WIDE ? static_cast<int64_t>(blockIdx.x)
-                           : static_cast<int64_t>(blockIdx.x) * kMergeRowsPerBlock + warp;
-  if (row >= p.rows) return;  // row = token * Hq + h; token = b * seqlen_q + i, or packed
   const int h = static_cast<int>(row % p.Hq);
   const int64_t tok = row / p.Hq;
   int b, i, nq;
@@ -195,6 +191,22 @@ __global__ void __launch_bounds__(WIDE ? D : 32 * kMergeRowsPerBlock)
     else
       p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.seqlen_q + i] = ls;
     if (fin) p.fin_lse[static_cast<int64_t>(b) * p.Hq + h] = ls;
+  }
+}
+
+// WIDE: one block per row.  Otherwise one warp per row, the warps of the grid
+// striding over the rows (a few blocks per SM: most rows of a packed call may
+// only need the check that the row-major kernel finished them).
+template <int D, bool WIDE>
+__global__ void __launch_bounds__(WIDE ? D : 32 * kMergeRowsPerBlock)
+    merge_kernel(const __grid_constant__ MergeParams p) {
+  if constexpr (WIDE) {
+    if (static_cast<int64_t>(blockIdx.x) < p.rows) merge_row<D, true>(p, blockIdx.x, threadIdx.x);
+  } else {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kMergeRowsPerBlock;
+    for (int64_t row = static_cast<int64_t>(blockIdx.x) * kMergeRowsPerBlock + (threadIdx.x >> 5);
+         row < p.rows; row += stride)
+      merge_row<D, false>(p, row, threadIdx.x & 31);
   }
 }
 

@@ -243,7 +243,12 @@ int launch_merge(const pkv::MergeParams &m, int64_t rows, cudaStream_t s) {
     pkv::merge_kernel<D, true><<<static_cast<unsigned>(rows), D, 0, s>>>(m);
     return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
   }
-  const int64_t blocks = ceil_div(rows, pkv::kMergeRowsPerBlock);
+  // the warps stride over the rows: at most 8 blocks of 8 warps per SM
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  const int64_t need = ceil_div(rows, pkv::kMergeRowsPerBlock);
+  const int64_t cap = static_cast<int64_t>(sm_count(dev)) * 8;
+  const int64_t blocks = need < cap ? need : cap;
   pkv::merge_kernel<D, false><<<static_cast<unsigned>(blocks), 32 * pkv::kMergeRowsPerBlock, 0, s>>>(m);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
